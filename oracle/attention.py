@@ -1,0 +1,209 @@
+"""Exact and emulated-quantized attention (TEST INFRASTRUCTURE ONLY).
+
+Shapes: Q, K, V are [B, H, N, d] arrays holding bf16/fp16 values.
+
+``exact_attention`` is the definition O = softmax(Q K^T * sm_scale + mask) V
+evaluated in FP64.
+
+``emulated_sage_attention`` follows the quantized forward pass step by step
+(SageAttention / SageAttention2 / SageAttention3 abstracts on the dblp author
+page; the kernel-comparison blog's "How FlashAttention reduces memory
+traffic" for the tiled online softmax):
+
+  for each query row, over key tiles j = 0, 1, ... of 128 keys, in order
+  (causal: only keys t_k <= t_q):
+    A      = q_codes . k_codes^T                (exact integer / exact FP64)
+    S      = A * s_Q * s_K * sm_scale           (FP4: A * g_Q * g_K * sm_scale,
+                                                 block scales inside A)
+    m_new  = max(m, rowmax S)
+    alpha  = exp(m - m_new)
+    P~     = exp(S - m_new)                     (<= 1)
+    p      = quantize(P~)                       (FP8: e4m3(448 P~);
+                                                 FP4: per-16-key UE4M3 scale
+                                                 with static tile scale 1/2688)
+    partial= p . v_codes                        (level 1: fresh per tile, exact)
+    O      = alpha O + partial * dequant        (level 2: running accumulator)
+    l      = alpha l + rowsum(P~)               (unquantized P~, reading below)
+  O / l
+
+Readings (pages silent): the exponential may be taken in any base inside a
+kernel (exp2 with log2(e) folded in is the same function); one key tile of
+128 keys per level-1 partial; l sums the unquantized P~; the running max is
+exact (no lazy rescaling); the causal mask is top-left aligned with
+N_q == N_k so no row is ever fully masked.
+"""
+
+import numpy as np
+
+from . import prepass as pp
+from .encoders import (e4m3_encode, e4m3_decode, e2m1_encode, e2m1_decode,
+                       ue4m3_encode, ue4m3_decode, round_to_dtype)
+
+BLOCK = pp.BLOCK
+P_FP8_SCALE = 448.0
+P_FP4_G = 1.0 / 2688.0
+
+
+def exact_attention(q, k, v, causal=False, sm_scale=None, row_chunk=1024):
+    """softmax(Q K^T sm_scale + mask) V in FP64, rows in chunks of row_chunk."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, H, N, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(d)
+    out = np.zeros((B, H, N, d), np.float64)
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, N, row_chunk):
+                r1 = min(r0 + row_chunk, N)
+                s = (q[b, h, r0:r1] @ k[b, h].T) * sm_scale
+                if causal:
+                    rows = np.arange(r0, r1)[:, None]
+                    cols = np.arange(N)[None, :]
+                    s = np.where(cols <= rows, s, -np.inf)
+                m = s.max(axis=1, keepdims=True)
+                p = np.exp(s - m)
+                out[b, h, r0:r1] = (p @ v[b, h]) / p.sum(axis=1, keepdims=True)
+    return out
+
+
+# --------------------------------------------------------------------------
+# P~ quantizers (per key tile, rows x 128 keys, values in [0, 1])
+# --------------------------------------------------------------------------
+
+def quant_p_fp8(pt):
+    """p = e4m3(P~ * 448); returns the dequantized-without-scale codes' values.
+
+    The value returned is the E4M3 value of the code (i.e. 448 P~ rounded);
+    the caller multiplies by 1/448 at the fold.
+    """
+    return e4m3_decode(e4m3_encode(pt * P_FP8_SCALE))
+
+
+def quant_p_fp4(pt):
+    """FP4 P~ with the static tile scale g = 1/2688 and per-16-key UE4M3 scales.
+
+    s16 = ue4m3(amax16 * 448); code = e2m1(P~ / (s16 * g)).  Returns the
+    value code * s16 (the caller multiplies by g at the fold).  Requires the
+    key axis to be a multiple of 16.
+    """
+    R, C = pt.shape
+    blk = pt.reshape(R, C // 16, 16)
+    a16 = blk.max(axis=-1)
+    s16 = ue4m3_decode(ue4m3_encode(a16 * P_FP8_SCALE))
+    den = s16 * P_FP4_G
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.where(den[..., None] > 0, blk / np.where(den > 0, den, 1.0)[..., None], 0.0)
+    codes = e2m1_decode(e2m1_encode(t))
+    return (codes * s16[..., None]).reshape(R, C)
+
+
+# --------------------------------------------------------------------------
+# The tile loop
+# --------------------------------------------------------------------------
+
+def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale):
+    """Online softmax + two-level P~V accumulation for one (b, h).
+
+    qd [N, d], kd [N, d]: decoded code values (exact FP64).
+    vd [N, d]: decoded V code values (exact FP64).
+    s_row [N]: per-row dequant factor of A (s_Q of the row's block).
+    s_key [N]: per-key dequant factor of A (s_K of the key's block).
+    v_fold [ntiles, d]: factor applied to a tile's level-1 partial at the fold.
+    p_quant: P~ -> quantized P~ values (scaled as the partial expects).
+    Returns O [N, d] in FP64 (before the output rounding).
+    """
+    N, d = qd.shape
+    O = np.zeros((N, d))
+    m = np.full(N, -np.inf)
+    l = np.zeros(N)
+    for j, (ks, ke) in enumerate(pp._blocks(N)):
+        r0 = ks if causal else 0                  # rows before ks see no key of tile j
+        rows = np.arange(r0, N)
+        A = qd[r0:] @ kd[ks:ke].T                 # exact
+        S = A * s_row[r0:, None] * s_key[None, ks:ke] * sm_scale
+        if causal:
+            S = np.where(np.arange(ks, ke)[None, :] <= rows[:, None], S, -np.inf)
+        m_new = np.maximum(m[r0:], S.max(axis=1))
+        alpha = np.exp(m[r0:] - m_new)            # exp(-inf) = 0 on the first tile
+        Pt = np.exp(S - m_new[:, None])
+        p = p_quant(Pt)
+        partial = p @ vd[ks:ke]                   # level 1: exact
+        O[r0:] = alpha[:, None] * O[r0:] + partial * v_fold[j][None, :]
+        l[r0:] = alpha * l[r0:] + Pt.sum(axis=1)
+        m[r0:] = m_new
+    return O / l[:, None]
+
+
+def _identity(x):
+    return x
+
+
+def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8",
+                            quantizers="faithful"):
+    """Step-by-step emulation of the quantized forward pass, FP64 O [B,H,N,d].
+
+    mode: "int8_fp8" (INT8 Q/K, FP8 P~ and V) or "fp4" (FP4 Q/K/P~/V).
+    quantizers="identity" replaces every quantizer by the identity (codes =
+    the values, scales = 1, P~ unrounded); the result must then equal
+    ``exact_attention`` up to FP64 rounding.
+    """
+    q = np.asarray(q, np.float32)
+    k = np.asarray(k, np.float32)
+    v = np.asarray(v, np.float32)
+    B, H, N, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(d)
+    out = np.zeros((B, H, N, d))
+    ntiles = -(-N // BLOCK)
+    tile_of = np.arange(N) // BLOCK
+
+    if quantizers == "identity":
+        for b in range(B):
+            for h in range(H):
+                ones_n = np.ones(N)
+                out[b, h] = _tile_loop(q[b, h].astype(np.float64), k[b, h].astype(np.float64),
+                                       v[b, h].astype(np.float64), ones_n, ones_n,
+                                       np.ones((ntiles, d)), _identity, causal, sm_scale)
+        return out
+    if quantizers != "faithful":
+        raise ValueError(quantizers)
+
+    if mode == "int8_fp8":
+        qk = pp.quant_qk_int8(q, k)
+        vc, vs = pp.quant_v_fp8(v)
+        for b in range(B):
+            for h in range(H):
+                qd = qk["q_codes"][b, h].astype(np.float64)
+                kd = qk["k_codes"][b, h].astype(np.float64)
+                vd = e4m3_decode(vc[b, h]).T                      # [N, d]
+                s_row = qk["q_scales"][b, h].astype(np.float64)[tile_of]
+                s_key = qk["k_scales"][b, h].astype(np.float64)[tile_of]
+                v_fold = np.broadcast_to(vs[b, h].astype(np.float64) / P_FP8_SCALE, (ntiles, d))
+                out[b, h] = _tile_loop(qd, kd, vd, s_row, s_key, v_fold, quant_p_fp8,
+                                       causal, sm_scale)
+        return out
+
+    if mode == "fp4":
+        qk = pp.quant_qk_fp4(q, k)
+        vc, vsf, vg = pp.quant_v_fp4(v)
+        for b in range(B):
+            for h in range(H):
+                qd = e2m1_decode(qk["q_codes"][b, h]) * np.repeat(
+                    ue4m3_decode(qk["q_sf"][b, h]), 16, axis=1)
+                kd = e2m1_decode(qk["k_codes"][b, h]) * np.repeat(
+                    ue4m3_decode(qk["k_sf"][b, h]), 16, axis=1)
+                vdt = e2m1_decode(vc[b, h]) * np.repeat(ue4m3_decode(vsf[b, h]), 16, axis=1)
+                s_row = qk["q_g"][b, h].astype(np.float64)[tile_of]
+                s_key = qk["k_g"][b, h].astype(np.float64)[tile_of]
+                v_fold = (vg[b, h].astype(np.float64) * P_FP4_G)[:, None] * np.ones((1, d))
+                out[b, h] = _tile_loop(qd, kd, vdt.T, s_row, s_key, v_fold, quant_p_fp4,
+                                       causal, sm_scale)
+        return out
+    raise ValueError(mode)
+
+
+def sage_attention_output(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", dtype="bf16"):
+    """Emulated O rounded to the input dtype ('bf16' or 'f16'), as float32."""
+    return round_to_dtype(emulated_sage_attention(q, k, v, causal, sm_scale, mode), dtype)

@@ -1,0 +1,311 @@
+"""Pins of the oracle's pre-pass and attention (CPU only).
+
+Exact attention is pinned against a pure-Python triple loop, closed forms
+and invariants; the emulated path is pinned by reducing to exact attention
+with identity quantizers, by closed forms whose every quantizer step is
+exact, and by exact scaling laws.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention as att
+from oracle import encoders as enc
+from oracle import prepass as pp
+
+
+def rnd(shape, seed, scale=1.0, dtype="bf16"):
+    x = np.random.default_rng(seed).standard_normal(shape).astype(np.float32) * np.float32(scale)
+    return enc.bf16_round(x) if dtype == "bf16" else enc.f16_round(x)
+
+
+def brute_attention(q, k, v, causal, sm_scale):
+    """softmax(q k^T sm_scale) v with Python scalars, one (b, h)."""
+    N, d = len(q), len(q[0])
+    out = []
+    for i in range(N):
+        keys = [j for j in range(N) if (j <= i or not causal)]
+        s = [sum(float(q[i][c]) * float(k[j][c]) for c in range(d)) * sm_scale for j in keys]
+        mx = max(s)
+        w = [math.exp(x - mx) for x in s]
+        z = math.fsum(w)
+        out.append([math.fsum(w[t] * float(v[j][c]) for t, j in enumerate(keys)) / z
+                    for c in range(d)])
+    return np.array(out)
+
+
+# ---------------------------------------------------------------- exact ----
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_matches_bruteforce(causal):
+    q, k, v = rnd((1, 2, 13, 5), 1), rnd((1, 2, 13, 5), 2), rnd((1, 2, 13, 5), 3)
+    o = att.exact_attention(q, k, v, causal, 0.37)
+    for h in range(2):
+        ref = brute_attention(q[0, h].tolist(), k[0, h].tolist(), v[0, h].tolist(), causal, 0.37)
+        assert np.max(np.abs(o[0, h] - ref)) <= 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_rows_sum_to_one(causal):
+    q, k = rnd((2, 1, 300, 16), 4, 3.0), rnd((2, 1, 300, 16), 5, 3.0)
+    o = att.exact_attention(q, k, np.ones((2, 1, 300, 16)), causal, 0.25, row_chunk=97)
+    assert np.max(np.abs(o - 1.0)) <= 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_zero_q_gives_visible_mean(causal):
+    v = rnd((1, 1, 50, 8), 6)
+    o = att.exact_attention(np.zeros((1, 1, 50, 8)), rnd((1, 1, 50, 8), 7), v, causal, 1.0)
+    v64 = v[0, 0].astype(np.float64)
+    if causal:
+        want = np.cumsum(v64, axis=0) / np.arange(1, 51)[:, None]
+    else:
+        want = np.broadcast_to(v64.mean(axis=0), (50, 8))
+    assert np.max(np.abs(o[0, 0] - want)) <= 1e-12
+
+
+def test_exact_dominant_key_selects_its_value():
+    N, d = 40, 8
+    k = rnd((1, 1, N, d), 8, 0.01)
+    q = np.zeros((1, 1, N, d), np.float32)
+    q[..., 0] = 1.0
+    k[0, 0, 17, 0] = 1000.0
+    v = rnd((1, 1, N, d), 9)
+    o = att.exact_attention(q, k, v, False, 1.0)
+    assert np.max(np.abs(o[0, 0] - v[0, 0, 17][None, :].astype(np.float64))) <= 1e-12
+
+
+def test_exact_key_permutation_equivariance():
+    q, k, v = rnd((1, 2, 64, 16), 10), rnd((1, 2, 64, 16), 11), rnd((1, 2, 64, 16), 12)
+    perm = np.random.default_rng(0).permutation(64)
+    a = att.exact_attention(q, k, v, False, 0.25)
+    b = att.exact_attention(q, k[:, :, perm], v[:, :, perm], False, 0.25)
+    assert np.max(np.abs(a - b)) <= 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_k_shift_invariance(causal):
+    # the smoothing invariant: K + 1 c^T leaves O unchanged
+    q, k, v = rnd((1, 1, 96, 16), 13), rnd((1, 1, 96, 16), 14), rnd((1, 1, 96, 16), 15)
+    c = np.random.default_rng(1).standard_normal(16) * 5
+    a = att.exact_attention(q, k, v, causal, 0.25)
+    b = att.exact_attention(q, k.astype(np.float64) + c, v, causal, 0.25)
+    assert np.max(np.abs(a - b)) <= 1e-12
+
+
+# ------------------------------------------------------------- pre-pass ----
+
+def test_k_mean_is_the_mean():
+    k = rnd((2, 3, 300, 32), 16, 4.0)
+    mu = pp.k_channel_mean(k)
+    for b in range(2):
+        for h in range(3):
+            for c in range(0, 32, 7):
+                exact = math.fsum(float(x) for x in k[b, h, :, c]) / 300
+                assert abs(float(mu[b, h, c]) - exact) <= abs(exact) * 2.0 ** -24 + 1e-30
+
+
+def test_k_mean_chunk_order():
+    # the FP64 sum is taken per 128-token chunk in token order, then over
+    # chunks; a set of values whose sum depends on the order pins that order
+    N = 256
+    k = np.zeros((1, 1, N, 1), np.float64)
+    k[0, 0, 0, 0] = 2.0 ** 60
+    k[0, 0, 1, 0] = 1.0
+    k[0, 0, 128, 0] = -(2.0 ** 60)
+    # in token order over all N the 1.0 is absorbed; chunk-wise it is too
+    # (2^60 + 1 rounds to 2^60 inside chunk 0), so the mean is 0
+    assert pp.k_channel_mean(k)[0, 0, 0] == 0.0
+    k[0, 0, 1, 0] = 0.0
+    k[0, 0, 129, 0] = 1.0
+    # chunk 1 sums to -2^60 exactly (+1 absorbed), total 0
+    assert pp.k_channel_mean(k)[0, 0, 0] == 0.0
+    k[0, 0, 129, 0] = 0.0
+    k[0, 0, 130, 0] = 2.0 ** 60
+    k[0, 0, 131, 0] = 3.0
+    # chunk 1: -2^60 + 2^60 + 3 = 3 exactly; chunk 0: 2^60; total 2^60 + 3 -> 2^60
+    assert pp.k_channel_mean(k)[0, 0, 0] == np.float32(2.0 ** 60 / N)
+
+
+def test_int8_blocks_properties():
+    x = rnd((1, 2, 300, 64), 17, 2.0)
+    x[0, 1, 128:256] = 0.0                               # an all-zero block
+    codes, scales = pp.quant_int8_blocks(x)
+    assert scales.shape == (1, 2, 3)
+    assert scales[0, 1, 1] == 0 and np.all(codes[0, 1, 128:256] == 0)
+    for h in range(2):
+        for i, (s, e) in enumerate([(0, 128), (128, 256), (256, 300)]):
+            blk = x[0, h, s:e].astype(np.float64)
+            sc = float(scales[0, h, i])
+            if sc == 0:
+                continue
+            assert np.abs(codes[0, h, s:e]).max() == 127
+            assert np.all(np.abs(blk - codes[0, h, s:e] * sc) <= sc * (0.5 + 1e-6))
+            assert scales[0, h, i] == np.float32(np.float32(np.abs(blk).max()) / np.float32(127))
+
+
+def test_quant_qk_smooths_k_only():
+    q, k = rnd((1, 1, 256, 32), 18), rnd((1, 1, 256, 32), 19) + np.float32(10)
+    r = pp.quant_qk_int8(q, k)
+    c2, s2 = pp.quant_int8_blocks(q)
+    assert np.array_equal(r["q_codes"], c2) and np.array_equal(r["q_scales"], s2)
+    kc, ks = pp.quant_int8_blocks(k.astype(np.float32) - r["k_mean"][:, :, None, :])
+    assert np.array_equal(r["k_codes"], kc) and np.array_equal(r["k_scales"], ks)
+    assert np.all(np.abs(r["k_mean"] - 10) < 0.5)
+
+
+def test_fp8_v_properties():
+    v = rnd((1, 2, 256, 32), 20, 3.0)
+    v[0, 0, :, 5] = 0.0
+    codes, s = pp.quant_v_fp8(v)
+    assert codes.shape == (1, 2, 32, 256) and s.shape == (1, 2, 32)
+    assert s[0, 0, 5] == 0 and np.all(codes[0, 0, 5] == 0)
+    vt = v.transpose(0, 1, 3, 2).astype(np.float64)
+    deq = enc.e4m3_decode(codes) * s[..., None]
+    for h in range(2):
+        for c in range(32):
+            if s[0, h, c] == 0:
+                continue
+            row = np.abs(vt[0, h, c])
+            j = row.argmax()
+            assert codes[0, h, c, j] & 0x7F == 0x7E          # the channel max hits 448
+            big = row >= float(s[0, h, c]) * 2.0 ** -6
+            err = np.abs(deq[0, h, c] - vt[0, h, c])
+            assert np.all(err[big] <= row[big] * 2.0 ** -4 * (1 + 1e-6))
+
+
+def test_fp4_tokens_properties():
+    x = rnd((1, 1, 256, 64), 21, 2.0)
+    codes, sf, g = pp.quant_fp4_tokens(x)
+    assert codes.shape == (1, 1, 256, 64) and sf.shape == (1, 1, 256, 4) and g.shape == (1, 1, 2)
+    for t in range(2):
+        blk = x[0, 0, t * 128:(t + 1) * 128].astype(np.float64)
+        r, c = np.unravel_index(np.abs(blk).argmax(), blk.shape)
+        assert codes[0, 0, t * 128 + r, c] & 7 == 7                   # the tile max -> 6
+        assert sf[0, 0, t * 128 + r, c // 16] == 0x7E                 # with scale 448
+        assert g[0, 0, t] == np.float32(np.float32(np.abs(blk).max()) / np.float32(2688))
+        den = (enc.ue4m3_decode(sf[0, 0, t * 128:(t + 1) * 128]).astype(np.float32)
+               * g[0, 0, t]).astype(np.float32).astype(np.float64)
+        den = np.repeat(den, 16, axis=1)
+        deq = enc.e2m1_decode(codes[0, 0, t * 128:(t + 1) * 128]) * den
+        sat = np.maximum(np.abs(blk) - 6 * den, 0)
+        assert np.all(np.abs(deq - blk) <= den * (1 + 1e-6) + sat)
+
+
+def test_fp4_v_layout_and_zero_channel():
+    v = rnd((1, 1, 256, 32), 22)
+    v[0, 0, :, 3] = 0.0
+    codes, sf, g = pp.quant_v_fp4(v)
+    assert codes.shape == (1, 1, 32, 256) and sf.shape == (1, 1, 32, 16)
+    assert np.all(codes[0, 0, 3] == 0) and np.all(sf[0, 0, 3] == 0)
+    # encoding V^T with the token routine on the transposed tile gives the same
+    c2, s2, g2 = pp.quant_fp4_tokens(np.ascontiguousarray(v.transpose(0, 1, 3, 2))[:, :, :, :128]
+                                     .transpose(0, 1, 3, 2).copy())
+    assert g2[0, 0, 0] == g[0, 0, 0]
+
+
+def test_integer_qk_is_exact():
+    q = np.random.default_rng(3).integers(-127, 128, (128, 128))
+    k = np.random.default_rng(4).integers(-127, 128, (128, 128))
+    assert np.array_equal((q.astype(np.float64) @ k.T.astype(np.float64)).astype(np.int64),
+                          q.astype(np.int64) @ k.T.astype(np.int64))
+
+
+# ------------------------------------------------------------- emulated ----
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [128, 300, 384])
+def test_emulated_identity_equals_exact(causal, N):
+    q, k, v = rnd((1, 2, N, 16), 30, 2.0), rnd((1, 2, N, 16), 31, 2.0), rnd((1, 2, N, 16), 32)
+    a = att.emulated_sage_attention(q, k, v, causal, 0.3, quantizers="identity")
+    b = att.exact_attention(q, k, v, causal, 0.3)
+    assert np.max(np.abs(a - b)) <= 1e-12
+
+
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp4"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulated_constant_k_gives_visible_mean(mode, causal):
+    # K rows all equal -> smoothed K = 0 -> all scores 0 -> P~ = 1 exactly;
+    # V on the format grid with an exact scale -> O is the visible mean of V.
+    N, d = 256, 32
+    rng = np.random.default_rng(5)
+    q = rnd((1, 1, N, d), 33)
+    k = np.broadcast_to(rnd((1, 1, 1, d), 34), (1, 1, N, d)).copy()
+    if mode == "int8_fp8":
+        grid = enc.e4m3_decode(np.arange(0x7F))
+        v = rng.choice(grid, (1, 1, N, d)) * rng.choice([-1, 1], (1, 1, N, d))
+        v[0, 0, 0, :] = 448.0                        # channel max 448 -> s_V = 1
+        tol = 1e-12
+    else:
+        grid = enc.E2M1_VALUES
+        v = rng.choice(grid, (1, 1, N, d)) * rng.choice([-1, 1], (1, 1, N, d))
+        v[0, 0, ::16, :] = 6.0                        # every 16-block holds 6
+        tol = 1e-6                                    # g = 6/2688 is inexact in fp32
+    v = v.astype(np.float32)
+    o = att.emulated_sage_attention(q, k, v, causal, 0.2, mode=mode)
+    v64 = v[0, 0].astype(np.float64)
+    want = (np.cumsum(v64, axis=0) / np.arange(1, N + 1)[:, None]) if causal \
+        else np.broadcast_to(v64.mean(axis=0), (N, d))
+    assert np.max(np.abs(o[0, 0] - want)) <= tol * max(1.0, np.abs(want).max())
+
+
+def test_emulated_two_key_closed_form():
+    # One query direction, keys arranged so that exactly two keys matter with
+    # P~ = 1 and 1/1.1; every quantizer step except P~ is exact, and P~ = 1/1.1
+    # encodes as 448/1.1 = 407.27 -> 416.  l sums the unquantized P~.
+    N, d = 128, 16
+    q = np.zeros((1, 1, N, d), np.float32)
+    q[..., 0] = 127.0                                   # s_Q = 1, codes 127
+    k = np.zeros((1, 1, N, d), np.float32)
+    kc = np.full(N, -2.0)
+    kc[0], kc[1], kc[2] = 127.0, 126.0, -3.0            # channel sum 0 -> mean 0
+    k[0, 0, :, 0] = kc
+    sm_scale = math.log(1.1) / 127.0                    # S0 - S1 = ln 1.1
+    rng = np.random.default_rng(6)
+    grid = enc.e4m3_decode(np.arange(0x7F))
+    v = (rng.choice(grid, (1, 1, N, d)) * rng.choice([-1, 1], (1, 1, N, d))).astype(np.float32)
+    v[0, 0, 5, :] = 448.0                               # s_V = 1
+    o = att.emulated_sage_attention(q, k, v, False, sm_scale)
+    v0, v1 = v[0, 0, 0].astype(np.float64), v[0, 0, 1].astype(np.float64)
+    p1 = math.exp(-math.log(1.1))
+    others = sum(math.exp(127 * (x - 127.0) * sm_scale) for x in kc[2:])
+    assert enc.e4m3_decode(enc.e4m3_encode(448 * p1)) == 416.0
+    want = (v0 + (416.0 / 448.0) * v1) / (1.0 + p1 + others)
+    # the other keys' P~ (< 1e-4) quantize to small nonzero codes; bound them
+    rest = (np.abs(v[0, 0, 2:]).max() * others * 1.1)
+    assert np.max(np.abs(o[0, 0] - want[None, :])) <= rest + 1e-12
+
+
+def test_emulated_v_scaling_is_exact():
+    q, k, v = rnd((1, 1, 256, 32), 40), rnd((1, 1, 256, 32), 41), rnd((1, 1, 256, 32), 42)
+    for mode in ["int8_fp8", "fp4"]:
+        a = att.emulated_sage_attention(q, k, v, False, 0.2, mode=mode)
+        b = att.emulated_sage_attention(q, k, v * np.float32(8), False, 0.2, mode=mode)
+        assert np.array_equal(8 * a, b)
+
+
+def test_emulated_k_and_sm_scale_trade_exactly():
+    q, k, v = rnd((1, 1, 256, 32), 43), rnd((1, 1, 256, 32), 44), rnd((1, 1, 256, 32), 45)
+    for mode in ["int8_fp8", "fp4"]:
+        a = att.emulated_sage_attention(q, k, v, True, 0.25, mode=mode)
+        b = att.emulated_sage_attention(q, k * np.float32(4), v, True, 0.0625, mode=mode)
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("mode,tol", [("int8_fp8", 0.999), ("fp4", 0.97)])
+def test_emulated_close_to_exact(mode, tol):
+    q, k = rnd((1, 2, 512, 64), 50), rnd((1, 2, 512, 64), 51) + np.float32(2.0)
+    v = rnd((1, 2, 512, 64), 52)
+    a = att.emulated_sage_attention(q, k, v, False, 0.125, mode=mode)
+    b = att.exact_attention(q, k, v, False, 0.125)
+    cos = np.sum(a * b) / np.sqrt(np.sum(a * a) * np.sum(b * b))
+    assert cos >= tol
+
+
+def test_output_rounding_matches_dtype():
+    o = np.random.default_rng(7).standard_normal((4, 4))
+    r = enc.round_to_dtype(o, "bf16")
+    assert np.array_equal(r, enc.bf16_round(r))
+    assert np.max(np.abs(r - o)) <= np.abs(o).max() * 2.0 ** -8
