@@ -1,0 +1,156 @@
+/*
+ * sage.h -- C ABI of the B200 (sm_100a) quantized attention forward pass.
+ *
+ * The library computes O = softmax(Q K^T * sm_scale) V the SageAttention
+ * way:
+ *   - K is smoothed by subtracting its per-channel mean over tokens
+ *     (SageAttention abstract, dblp author page on taxoreview.com: accurate
+ *     8-bit attention; softmax is unchanged by a per-row shift);
+ *   - Q and K are quantized per 128-token block to INT8
+ *     ("Flash Attention vs Sage Attention: Kernel Comparison", section "How
+ *     SageAttention uses quantization for more throughput"), or to FP4 with
+ *     one UE4M3 scale per 16 elements (SageAttention3 abstract: FP4 tensor
+ *     cores of Blackwell GPUs);
+ *   - Q K^T runs on the tensor cores and is dequantized by the product of
+ *     the scales;
+ *   - an online (flash-style) softmax follows (kernel-comparison blog,
+ *     section "How FlashAttention reduces memory traffic");
+ *   - the unnormalised P~ and V are quantized to FP8 (SageAttention2
+ *     abstract) or FP4, and P~V accumulates in two levels: a fresh FP32
+ *     partial per 128-key tile folded into an FP32 running accumulator
+ *     (SageAttention2 abstract: "two-level accumulation strategy").
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are row-major and contiguous.  Q, K, V, O are [B, H, N, d] in
+ *     the input dtype (fp16 or bf16).
+ *   - All pointers are DEVICE pointers of the current CUDA device, owned by
+ *     the caller, and must be 16-byte aligned.  `stream` is a cudaStream_t
+ *     (NULL = legacy default stream).  Every call is asynchronous on
+ *     `stream`; the library never synchronises it.
+ *   - Supported shapes: d in {64, 128}; N % 128 == 0 (FP4 mode: d == 128).
+ *     A call with B, H or N equal to zero does nothing and returns SAGE_OK.
+ *   - Return value: SAGE_OK (0) or a negative sage_status_t.  No exception
+ *     or process exit crosses the ABI.  sage_status_string() describes the
+ *     most recent error of the calling thread.
+ *   - Quantized buffers (sizes from sage_buffer_bytes):
+ *       INT8/FP8 mode
+ *         q_codes, k_codes  int8  [B, H, N, d]
+ *         q_scales, k_scales float [B, H, N/128]    one scale per 128 tokens
+ *         k_mean            float [B, H, d]
+ *         v_codes           e4m3  [B, H, d, N]      V transposed
+ *         v_scales          float [B, H, d]         one scale per channel
+ *       FP4 mode
+ *         q_codes, k_codes  e2m1x2 [B, H, N, d/2]   low nibble = even channel
+ *         q_scales, k_scales float [B, H, N/128]    tile scale g
+ *         q_sf, k_sf        ue4m3 per 16 channels, tensor-core layout (below)
+ *         v_codes           e2m1x2 [B, H, d, N/2]   V transposed, low nibble =
+ *                                                    even token
+ *         v_scales          float [B, H, N/128]     tile scale g
+ *         v_sf              ue4m3 per 16 tokens, tensor-core layout (below)
+ *       Tensor-core scale layout: for each (b, h, 128-token tile t, 64-wide
+ *       chunk c of the contraction axis) one 512-byte block; inside it byte
+ *       16*l + 4*j + s holds the scale of row 32*j + l (row = token for
+ *       Q/K, channel for V; rows >= d are zero) and 16-element group
+ *       4*c + s.  Blocks are ordered (b, h, t, c).
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                         /* == cudaStream_t */
+typedef struct CUstream_st* sage_stream_t;
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = -1,     /* null pointer, negative size, bad enum   */
+  SAGE_ERR_UNSUPPORTED = -2,     /* shape/alignment/device not supported    */
+  SAGE_ERR_CUDA = -3,            /* a CUDA runtime/driver call failed       */
+  SAGE_ERR_DEVICE_TIMEOUT = -4   /* a bounded wait inside a kernel expired  */
+} sage_status_t;
+
+typedef enum { SAGE_MODE_INT8_FP8 = 0, SAGE_MODE_FP4 = 1 } sage_mode_t;
+typedef enum { SAGE_DTYPE_F16 = 0, SAGE_DTYPE_BF16 = 1 } sage_dtype_t;
+
+typedef enum {
+  SAGE_BUF_Q_CODES = 0, SAGE_BUF_Q_SCALES, SAGE_BUF_Q_SF,
+  SAGE_BUF_K_CODES, SAGE_BUF_K_SCALES, SAGE_BUF_K_SF, SAGE_BUF_K_MEAN,
+  SAGE_BUF_V_CODES, SAGE_BUF_V_SCALES, SAGE_BUF_V_SF
+} sage_buffer_t;
+
+/* Bytes of one quantized buffer for the given mode and shape (0 for a
+ * buffer the mode does not use, e.g. *_SF in INT8/FP8 mode). */
+size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, int64_t d);
+
+/* Q/K pre-pass: K channel mean (FP64 accumulation: per 128-token chunk in
+ * token order, then over chunks; mean = fp32(sum / N)), K smoothing
+ * (one FP32 subtraction), then per-128-token-block quantization of Q and
+ * of smoothed K.
+ *   INT8 mode: s = fp32(amax / 127); code = clamp(rne(fp32(x / s)), +-127);
+ *              q_sf, k_sf must be NULL.
+ *   FP4 mode:  g = fp32(amax_tile / 2688); per 16 channels
+ *              s16 = ue4m3(fp32(amax16 / fp32(6 g))),
+ *              code = e2m1(fp32(x / fp32(s16 * g))); q_scales/k_scales
+ *              receive g.
+ * All divisions are IEEE FP32 divisions; all casts round to nearest-even
+ * and saturate.  Codes and scales are bit-identical to the CPU oracle.
+ * Uses a stream-ordered library workspace for the mean partial sums. */
+int sage_quant_qk(const void* q, const void* k, int dtype,
+                  int64_t B, int64_t H, int64_t N, int64_t d, int mode,
+                  void* q_codes, float* q_scales, void* q_sf,
+                  void* k_codes, float* k_scales, void* k_sf,
+                  float* k_mean, sage_stream_t stream);
+
+/* V pre-pass.
+ *   FP8 mode: s_V[c] = fp32(amax_c / 448) over all N tokens of the (b, h);
+ *             code = e4m3(fp32(V / s_V)); written transposed; v_sf NULL.
+ *   FP4 mode: per 128-token tile g = fp32(amax_tile / 2688); per channel
+ *             and 16 tokens s16 = ue4m3(fp32(amax16 / fp32(6 g))),
+ *             code = e2m1(fp32(V / fp32(s16 * g))); v_scales receive g.
+ * (SageAttention2 abstract: V to FP8; SageAttention3 abstract: FP4.) */
+int sage_quant_v(const void* v, int dtype,
+                 int64_t B, int64_t H, int64_t N, int64_t d, int mode,
+                 void* v_codes, float* v_scales, void* v_sf, sage_stream_t stream);
+
+/* Attention on already-quantized operands (the buffers written by the two
+ * pre-pass calls); writes O [B, H, N, d] in `dtype`.  causal != 0 applies
+ * the top-left-aligned causal mask (query t sees keys 0..t).  sm_scale is
+ * applied at dequantization, not folded into the stored scales.
+ * P~ is quantized inside the kernel: FP8 mode e4m3(448 P~); FP4 mode per
+ * 16 keys s16 = ue4m3(448 amax16), code = e2m1(2688 P~ / s16). */
+int sage_attn_fwd_quantized(int mode,
+                            const void* q_codes, const float* q_scales, const void* q_sf,
+                            const void* k_codes, const float* k_scales, const void* k_sf,
+                            const void* v_codes, const float* v_scales, const void* v_sf,
+                            void* o, int dtype,
+                            int64_t B, int64_t H, int64_t N, int64_t d,
+                            int causal, float sm_scale, sage_stream_t stream);
+
+/* The whole forward pass: pre-pass into a library-owned workspace (grown
+ * on demand with stream-ordered allocation, one per device, freed at
+ * unload), then the attention kernel.  sm_scale <= 0 means 1/sqrt(d). */
+int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype,
+                  int64_t B, int64_t H, int64_t N, int64_t d,
+                  int causal, float sm_scale, int mode, sage_stream_t stream);
+
+/* Reads and clears the device status word written by the kernels' bounded
+ * waits (0 = none expired).  Synchronises the current device. */
+int sage_get_last_device_status(void);
+
+/* Human-readable text of a status, with the detail of the calling thread's
+ * most recent error when `status` is that error. */
+const char* sage_status_string(int status);
+
+/* Library version string. */
+const char* sage_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H */

@@ -44,27 +44,29 @@ P_FP8_SCALE = 448.0
 P_FP4_G = 1.0 / 2688.0
 
 
-def exact_attention(q, k, v, causal=False, sm_scale=None, row_chunk=1024):
-    """softmax(Q K^T sm_scale + mask) V in FP64, rows in chunks of row_chunk."""
+def exact_attention(q, k, v, causal=False, sm_scale=None, row_chunk=1024, rows=None):
+    """softmax(Q K^T sm_scale + mask) V in FP64, rows in chunks of row_chunk.
+
+    rows: optional query-row indices; then O is [B, H, len(rows), d].
+    """
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
     B, H, N, d = q.shape
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(d)
-    out = np.zeros((B, H, N, d), np.float64)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.zeros((B, H, len(rows), d), np.float64)
     for b in range(B):
         for h in range(H):
-            for r0 in range(0, N, row_chunk):
-                r1 = min(r0 + row_chunk, N)
-                s = (q[b, h, r0:r1] @ k[b, h].T) * sm_scale
+            for r0 in range(0, len(rows), row_chunk):
+                rr = rows[r0:r0 + row_chunk]
+                s = (q[b, h, rr] @ k[b, h].T) * sm_scale
                 if causal:
-                    rows = np.arange(r0, r1)[:, None]
-                    cols = np.arange(N)[None, :]
-                    s = np.where(cols <= rows, s, -np.inf)
+                    s = np.where(np.arange(N)[None, :] <= rr[:, None], s, -np.inf)
                 m = s.max(axis=1, keepdims=True)
                 p = np.exp(s - m)
-                out[b, h, r0:r1] = (p @ v[b, h]) / p.sum(axis=1, keepdims=True)
+                out[b, h, r0:r0 + len(rr)] = (p @ v[b, h]) / p.sum(axis=1, keepdims=True)
     return out
 
 
@@ -79,6 +81,25 @@ def quant_p_fp8(pt):
     the caller multiplies by 1/448 at the fold.
     """
     return e4m3_decode(e4m3_encode(pt * P_FP8_SCALE))
+
+
+def fp8_p_ambiguity(pt, eps):
+    """Size of the possible e4m3 code change of 448 P~ under a relative
+    perturbation of at most eps (0 where the code is unambiguous).
+
+    A kernel that evaluates P~ in FP32 can land on the other side of a
+    rounding midpoint when 448 P~ lies within eps of it; both codes are then
+    correct.  Returns |neighbour - code| for such elements.
+    """
+    x = pt * P_FP8_SCALE
+    code = e4m3_encode(x).astype(np.int64) & 0x7F
+    r = e4m3_decode(code)
+    up = e4m3_decode(np.minimum(code + 1, 0x7E))
+    dn = e4m3_decode(np.maximum(code - 1, 0))
+    tol = eps * np.maximum(x, 2.0 ** -10)
+    near_up = (code < 0x7E) & (np.abs(x - 0.5 * (r + up)) <= tol)
+    near_dn = (code > 0) & (np.abs(x - 0.5 * (r + dn)) <= tol)
+    return np.where(near_up, up - r, 0.0) + np.where(near_dn, r - dn, 0.0)
 
 
 def quant_p_fp4(pt):
@@ -103,7 +124,8 @@ def quant_p_fp4(pt):
 # The tile loop
 # --------------------------------------------------------------------------
 
-def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale):
+def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows=None,
+               p_ambiguity=None):
     """Online softmax + two-level P~V accumulation for one (b, h).
 
     qd [N, d], kd [N, d]: decoded code values (exact FP64).
@@ -112,27 +134,43 @@ def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale):
     s_key [N]: per-key dequant factor of A (s_K of the key's block).
     v_fold [ntiles, d]: factor applied to a tile's level-1 partial at the fold.
     p_quant: P~ -> quantized P~ values (scaled as the partial expects).
-    Returns O [N, d] in FP64 (before the output rounding).
+    rows: query rows to compute (default all); each row's arithmetic does not
+    depend on which other rows are computed.
+    p_ambiguity: optional P~ -> size of a possible code change (see
+    fp8_p_ambiguity); then a second array bounds, per output element, how far
+    O can move when every ambiguous code takes its other valid value.
+    Returns O [len(rows), d] in FP64 (before the output rounding), and the
+    bound when p_ambiguity is given.
     """
     N, d = qd.shape
-    O = np.zeros((N, d))
-    m = np.full(N, -np.inf)
-    l = np.zeros(N)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    R = len(rows)
+    O = np.zeros((R, d))
+    Bd = np.zeros((R, d)) if p_ambiguity is not None else None
+    m = np.full(R, -np.inf)
+    l = np.zeros(R)
     for j, (ks, ke) in enumerate(pp._blocks(N)):
-        r0 = ks if causal else 0                  # rows before ks see no key of tile j
-        rows = np.arange(r0, N)
-        A = qd[r0:] @ kd[ks:ke].T                 # exact
-        S = A * s_row[r0:, None] * s_key[None, ks:ke] * sm_scale
+        act = np.nonzero(rows >= ks)[0] if causal else np.arange(R)   # rows that see tile j
+        if act.size == 0:
+            continue
+        r_act = rows[act]
+        A = qd[r_act] @ kd[ks:ke].T               # exact
+        S = A * s_row[r_act, None] * s_key[None, ks:ke] * sm_scale
         if causal:
-            S = np.where(np.arange(ks, ke)[None, :] <= rows[:, None], S, -np.inf)
-        m_new = np.maximum(m[r0:], S.max(axis=1))
-        alpha = np.exp(m[r0:] - m_new)            # exp(-inf) = 0 on the first tile
+            S = np.where(np.arange(ks, ke)[None, :] <= r_act[:, None], S, -np.inf)
+        m_new = np.maximum(m[act], S.max(axis=1))
+        alpha = np.exp(m[act] - m_new)            # exp(-inf) = 0 on the first tile
         Pt = np.exp(S - m_new[:, None])
         p = p_quant(Pt)
         partial = p @ vd[ks:ke]                   # level 1: exact
-        O[r0:] = alpha[:, None] * O[r0:] + partial * v_fold[j][None, :]
-        l[r0:] = alpha * l[r0:] + Pt.sum(axis=1)
-        m[r0:] = m_new
+        O[act] = alpha[:, None] * O[act] + partial * v_fold[j][None, :]
+        if Bd is not None:
+            Bd[act] = alpha[:, None] * Bd[act] + \
+                (p_ambiguity(Pt) @ np.abs(vd[ks:ke])) * np.abs(v_fold[j])[None, :]
+        l[act] = alpha * l[act] + Pt.sum(axis=1)
+        m[act] = m_new
+    if Bd is not None:
+        return O / l[:, None], Bd / l[:, None]
     return O / l[:, None]
 
 
@@ -141,13 +179,18 @@ def _identity(x):
 
 
 def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8",
-                            quantizers="faithful"):
+                            quantizers="faithful", rows=None, ambiguity_eps=None):
     """Step-by-step emulation of the quantized forward pass, FP64 O [B,H,N,d].
 
     mode: "int8_fp8" (INT8 Q/K, FP8 P~ and V) or "fp4" (FP4 Q/K/P~/V).
     quantizers="identity" replaces every quantizer by the identity (codes =
     the values, scales = 1, P~ unrounded); the result must then equal
     ``exact_attention`` up to FP64 rounding.
+    rows: optional query-row indices; then O is [B, H, len(rows), d] and only
+    those rows are computed (the pre-pass still sees every token).
+    ambiguity_eps: (INT8/FP8 mode) when given, also return a per-element bound
+    on how far O moves if every P~ code lying within this relative distance of
+    an e4m3 rounding midpoint takes its other (equally valid) value.
     """
     q = np.asarray(q, np.float32)
     k = np.asarray(k, np.float32)
@@ -155,7 +198,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     B, H, N, d = q.shape
     if sm_scale is None:
         sm_scale = 1.0 / np.sqrt(d)
-    out = np.zeros((B, H, N, d))
+    nrows = N if rows is None else len(rows)
+    out = np.zeros((B, H, nrows, d))
     ntiles = -(-N // BLOCK)
     tile_of = np.arange(N) // BLOCK
 
@@ -165,12 +209,14 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                 ones_n = np.ones(N)
                 out[b, h] = _tile_loop(q[b, h].astype(np.float64), k[b, h].astype(np.float64),
                                        v[b, h].astype(np.float64), ones_n, ones_n,
-                                       np.ones((ntiles, d)), _identity, causal, sm_scale)
+                                       np.ones((ntiles, d)), _identity, causal, sm_scale, rows)
         return out
     if quantizers != "faithful":
         raise ValueError(quantizers)
 
     if mode == "int8_fp8":
+        bound = np.zeros_like(out) if ambiguity_eps is not None else None
+        amb = (lambda pt: fp8_p_ambiguity(pt, ambiguity_eps)) if bound is not None else None
         qk = pp.quant_qk_int8(q, k)
         vc, vs = pp.quant_v_fp8(v)
         for b in range(B):
@@ -181,9 +227,13 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                 s_row = qk["q_scales"][b, h].astype(np.float64)[tile_of]
                 s_key = qk["k_scales"][b, h].astype(np.float64)[tile_of]
                 v_fold = np.broadcast_to(vs[b, h].astype(np.float64) / P_FP8_SCALE, (ntiles, d))
-                out[b, h] = _tile_loop(qd, kd, vd, s_row, s_key, v_fold, quant_p_fp8,
-                                       causal, sm_scale)
-        return out
+                res = _tile_loop(qd, kd, vd, s_row, s_key, v_fold, quant_p_fp8,
+                                 causal, sm_scale, rows, amb)
+                if bound is None:
+                    out[b, h] = res
+                else:
+                    out[b, h], bound[b, h] = res
+        return out if bound is None else (out, bound)
 
     if mode == "fp4":
         qk = pp.quant_qk_fp4(q, k)
@@ -199,7 +249,7 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                 s_key = qk["k_g"][b, h].astype(np.float64)[tile_of]
                 v_fold = (vg[b, h].astype(np.float64) * P_FP4_G)[:, None] * np.ones((1, d))
                 out[b, h] = _tile_loop(qd, kd, vdt.T, s_row, s_key, v_fold, quant_p_fp4,
-                                       causal, sm_scale)
+                                       causal, sm_scale, rows)
         return out
     raise ValueError(mode)
 

@@ -1,0 +1,418 @@
+// api.cu -- the C ABI (include/sage.h): argument checks, buffer sizing, the
+// per-(device, stream) workspace, tensor-map encoding and the device status
+// word.  No exception crosses the ABI.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include "../../include/sage.h"
+#include "sage_internal.h"
+
+namespace sage {
+
+__device__ uint32_t g_device_status;  // bits from sage_ptx.cuh, per device
+
+namespace {
+
+thread_local int t_last_status = 0;
+thread_local std::string t_last_detail;
+
+int fail(int status, const std::string& detail) {
+  t_last_status = status;
+  t_last_detail = detail;
+  return status;
+}
+
+int fail_cuda(cudaError_t e, const char* where) {
+  std::string d = std::string(where) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) +
+                  ")";
+  return fail(SAGE_ERR_CUDA, d);
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device facts, looked up once.
+struct DeviceInfo {
+  bool checked = false;
+  bool sm100 = false;
+  uint32_t* status = nullptr;
+};
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_dev;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.checked) {
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute");
+    di.sm100 = (major == 10 && minor == 0);
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_status);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(status)");
+    di.status = static_cast<uint32_t*>(p);
+    di.checked = true;
+  }
+  if (!di.sm100)
+    return fail(SAGE_ERR_UNSUPPORTED, "the current device is not compute capability 10.0 (sm_100)");
+  *out = &di;
+  return SAGE_OK;
+}
+
+// Stream-ordered workspace, one per (device, stream): a call on stream S
+// only ever touches the workspace of S, so calls on different streams
+// never share scratch memory.
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+int workspace(cudaStream_t st, size_t need, void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, st}];
+  if (w.bytes < need) {
+    if (w.ptr) {
+      e = cudaFreeAsync(w.ptr, st);
+      if (e != cudaSuccess) return fail_cuda(e, "cudaFreeAsync(workspace)");
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    const size_t grow = need + need / 4;
+    e = cudaMallocAsync(&w.ptr, grow, st);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMallocAsync(workspace)");
+    w.bytes = grow;
+  }
+  *out = w.ptr;
+  return SAGE_OK;
+}
+
+struct WorkspaceReleaser {
+  ~WorkspaceReleaser() {
+    // Best effort at unload; during process teardown the runtime may already
+    // be gone, in which case the calls fail harmlessly.
+    for (auto& kv : g_ws)
+      if (kv.second.ptr) cudaFree(kv.second.ptr);
+  }
+} g_ws_releaser;
+
+// ---------------------------------------------------------------- checks
+
+int check_common(int dtype, int mode, int64_t B, int64_t H, int64_t N, int64_t d, bool* empty) {
+  if (dtype != SAGE_DTYPE_F16 && dtype != SAGE_DTYPE_BF16)
+    return fail(SAGE_ERR_INVALID_ARG, "dtype must be SAGE_DTYPE_F16 or SAGE_DTYPE_BF16");
+  if (mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_FP4)
+    return fail(SAGE_ERR_INVALID_ARG, "mode must be SAGE_MODE_INT8_FP8 or SAGE_MODE_FP4");
+  if (B < 0 || H < 0 || N < 0 || d < 0) return fail(SAGE_ERR_INVALID_ARG, "negative size");
+  *empty = (B == 0 || H == 0 || N == 0);
+  if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d must be 64 or 128");
+  if (mode == SAGE_MODE_FP4 && d != 128)
+    return fail(SAGE_ERR_UNSUPPORTED, "FP4 mode supports d == 128 only");
+  if (N % 128 != 0) return fail(SAGE_ERR_UNSUPPORTED, "N must be a multiple of 128");
+  if (!*empty) {
+    if (B * H > 65535) return fail(SAGE_ERR_UNSUPPORTED, "B*H must be <= 65535");
+    if (B * H * N > 2147483647LL) return fail(SAGE_ERR_UNSUPPORTED, "B*H*N must be < 2^31");
+  }
+  return SAGE_OK;
+}
+
+int check_ptr(const void* p, const char* name, bool required) {
+  if (!p) {
+    if (required) return fail(SAGE_ERR_INVALID_ARG, std::string(name) + " is NULL");
+    return SAGE_OK;
+  }
+  if (!aligned16(p)) return fail(SAGE_ERR_UNSUPPORTED, std::string(name) + " is not 16-byte aligned");
+  return SAGE_OK;
+}
+
+int check_unused(const void* p, const char* name) {
+  if (p) return fail(SAGE_ERR_INVALID_ARG, std::string(name) + " must be NULL in INT8/FP8 mode");
+  return SAGE_OK;
+}
+
+#define SAGE_TRY(x)           \
+  do {                        \
+    int _s = (x);             \
+    if (_s != SAGE_OK) return _s; \
+  } while (0)
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn(const char** detail) {
+  static std::once_flag once;
+  static EncodeFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  if (!fn && detail) *detail = "cuTensorMapEncodeTiled is not available from the driver";
+  return fn;
+}
+
+size_t ws_ksum_bytes(int64_t BH, int64_t N, int64_t d) { return (size_t)(BH * (N / 128) * d * 8); }
+size_t ws_vmax_bytes(int64_t BH, int64_t N, int64_t d) { return (size_t)(BH * (N / 128) * d * 4); }
+
+}  // namespace
+
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t dim0,
+                    uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                    CUtensorMapSwizzle swz, const char** detail) {
+  EncodeFn fn = encode_fn(detail);
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {dim0, dim1};
+  const cuuint64_t strides[1] = {stride1_bytes};
+  const cuuint32_t box[2] = {box0, box1};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (detail) *detail = "cuTensorMapEncodeTiled rejected a tensor map";
+    return false;
+  }
+  return true;
+}
+
+}  // namespace sage
+
+using namespace sage;
+
+extern "C" {
+
+size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, int64_t d) {
+  if (B < 0 || H < 0 || N < 0 || d < 0) return 0;
+  const int64_t BH = B * H;
+  const int64_t nt = (N + 127) / 128;
+  const bool fp4 = mode == SAGE_MODE_FP4;
+  switch (which) {
+    case SAGE_BUF_Q_CODES:
+    case SAGE_BUF_K_CODES:
+    case SAGE_BUF_V_CODES:
+      return (size_t)(fp4 ? BH * N * d / 2 : BH * N * d);
+    case SAGE_BUF_Q_SCALES:
+    case SAGE_BUF_K_SCALES:
+      return (size_t)(BH * nt * 4);
+    case SAGE_BUF_Q_SF:
+    case SAGE_BUF_K_SF:
+      return fp4 ? (size_t)(BH * nt * ((d + 63) / 64) * 512) : 0;
+    case SAGE_BUF_K_MEAN:
+      return (size_t)(BH * d * 4);
+    case SAGE_BUF_V_SCALES:
+      return (size_t)(fp4 ? BH * nt * 4 : BH * d * 4);
+    case SAGE_BUF_V_SF:
+      return fp4 ? (size_t)(BH * nt * 2 * 512) : 0;
+    default:
+      return 0;
+  }
+}
+
+int sage_quant_qk(const void* q, const void* k, int dtype, int64_t B, int64_t H, int64_t N,
+                  int64_t d, int mode, void* q_codes, float* q_scales, void* q_sf, void* k_codes,
+                  float* k_scales, void* k_sf, float* k_mean, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_ptr(q, "q", true));
+  SAGE_TRY(check_ptr(k, "k", true));
+  SAGE_TRY(check_ptr(q_codes, "q_codes", true));
+  SAGE_TRY(check_ptr(q_scales, "q_scales", true));
+  SAGE_TRY(check_ptr(k_codes, "k_codes", true));
+  SAGE_TRY(check_ptr(k_scales, "k_scales", true));
+  SAGE_TRY(check_ptr(k_mean, "k_mean", true));
+  if (mode == SAGE_MODE_FP4) {
+    SAGE_TRY(check_ptr(q_sf, "q_sf", true));
+    SAGE_TRY(check_ptr(k_sf, "k_sf", true));
+  } else {
+    SAGE_TRY(check_unused(q_sf, "q_sf"));
+    SAGE_TRY(check_unused(k_sf, "k_sf"));
+  }
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  SAGE_TRY(workspace(st, ws_ksum_bytes(B * H, N, d), &ws));
+  QuantQKArgs a{q, k, dtype, mode, B, H, N, d, q_codes, q_scales, q_sf,
+                k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws)};
+  cudaError_t e = launch_quant_qk(a, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
+  return SAGE_OK;
+}
+
+int sage_quant_v(const void* v, int dtype, int64_t B, int64_t H, int64_t N, int64_t d, int mode,
+                 void* v_codes, float* v_scales, void* v_sf, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_ptr(v, "v", true));
+  SAGE_TRY(check_ptr(v_codes, "v_codes", true));
+  SAGE_TRY(check_ptr(v_scales, "v_scales", true));
+  if (mode == SAGE_MODE_FP4) SAGE_TRY(check_ptr(v_sf, "v_sf", true));
+  else SAGE_TRY(check_unused(v_sf, "v_sf"));
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  const size_t ks = align_up(ws_ksum_bytes(B * H, N, d));
+  if (mode == SAGE_MODE_INT8_FP8) SAGE_TRY(workspace(st, ks + ws_vmax_bytes(B * H, N, d), &ws));
+  QuantVArgs a{v, dtype, mode, B, H, N, d, v_codes, v_scales, v_sf,
+               static_cast<double*>(ws),
+               ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + ks) : nullptr};
+  cudaError_t e = launch_quant_v(a, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
+  return SAGE_OK;
+}
+
+int sage_attn_fwd_quantized(int mode, const void* q_codes, const float* q_scales, const void* q_sf,
+                            const void* k_codes, const float* k_scales, const void* k_sf,
+                            const void* v_codes, const float* v_scales, const void* v_sf, void* o,
+                            int dtype, int64_t B, int64_t H, int64_t N, int64_t d, int causal,
+                            float sm_scale, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_ptr(q_codes, "q_codes", true));
+  SAGE_TRY(check_ptr(q_scales, "q_scales", true));
+  SAGE_TRY(check_ptr(k_codes, "k_codes", true));
+  SAGE_TRY(check_ptr(k_scales, "k_scales", true));
+  SAGE_TRY(check_ptr(v_codes, "v_codes", true));
+  SAGE_TRY(check_ptr(v_scales, "v_scales", true));
+  SAGE_TRY(check_ptr(o, "o", true));
+  if (mode == SAGE_MODE_FP4) {
+    SAGE_TRY(check_ptr(q_sf, "q_sf", true));
+    SAGE_TRY(check_ptr(k_sf, "k_sf", true));
+    SAGE_TRY(check_ptr(v_sf, "v_sf", true));
+  } else {
+    SAGE_TRY(check_unused(q_sf, "q_sf"));
+    SAGE_TRY(check_unused(k_sf, "k_sf"));
+    SAGE_TRY(check_unused(v_sf, "v_sf"));
+  }
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
+    return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be positive and finite");
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a{mode, q_codes, q_scales, q_sf, k_codes, k_scales, k_sf, v_codes, v_scales, v_sf,
+             o, dtype, B, H, N, d, causal != 0, sm_scale, di->status};
+  const char* detail = nullptr;
+  cudaError_t e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(a, st, &detail)
+                                        : launch_attn_i8f8(a, st, &detail);
+  if (detail) return fail(SAGE_ERR_CUDA, detail);
+  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  return SAGE_OK;
+}
+
+int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,
+                  int64_t H, int64_t N, int64_t d, int causal, float sm_scale, int mode,
+                  sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_ptr(q, "q", true));
+  SAGE_TRY(check_ptr(k, "k", true));
+  SAGE_TRY(check_ptr(v, "v", true));
+  SAGE_TRY(check_ptr(o, "o", true));
+  if (!(sm_scale > 0.f)) sm_scale = 1.0f / std::sqrt((float)d);
+  if (!std::isfinite(sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be finite");
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  size_t off[SAGE_BUF_V_SF + 1];
+  size_t total = 0;
+  for (int w = 0; w <= SAGE_BUF_V_SF; ++w) {
+    off[w] = total;
+    total += align_up(sage_buffer_bytes(mode, w, B, H, N, d));
+  }
+  const size_t off_ksum = total;
+  total += align_up(ws_ksum_bytes(B * H, N, d));
+  const size_t off_vmax = total;
+  total += align_up(ws_vmax_bytes(B * H, N, d));
+  void* ws = nullptr;
+  SAGE_TRY(workspace(st, total, &ws));
+  char* base = static_cast<char*>(ws);
+  auto at = [&](int w) -> void* {
+    return sage_buffer_bytes(mode, w, B, H, N, d) ? base + off[w] : nullptr;
+  };
+  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d,
+                 at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+                 at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum)};
+  cudaError_t e = launch_quant_qk(qa, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
+  QuantVArgs va{v, dtype, mode, B, H, N, d,
+                at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+                reinterpret_cast<double*>(base + off_ksum),
+                reinterpret_cast<float*>(base + off_vmax)};
+  e = launch_quant_v(va, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
+  AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+              at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+              at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+              o, dtype, B, H, N, d, causal != 0, sm_scale, di->status};
+  const char* detail = nullptr;
+  e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
+  if (detail) return fail(SAGE_ERR_CUDA, detail);
+  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  return SAGE_OK;
+}
+
+int sage_get_last_device_status(void) {
+  DeviceInfo* di = nullptr;
+  int s = device_info(&di);
+  if (s != SAGE_OK) return s;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceSynchronize");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, di->status, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e, "read status");
+  const uint32_t zero = 0;
+  e = cudaMemcpy(di->status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return fail_cuda(e, "clear status");
+  return (int)v;
+}
+
+const char* sage_status_string(int status) {
+  static thread_local std::string s;
+  const char* base = "unknown status";
+  switch (status) {
+    case SAGE_OK: base = "ok"; break;
+    case SAGE_ERR_INVALID_ARG: base = "invalid argument"; break;
+    case SAGE_ERR_UNSUPPORTED: base = "unsupported"; break;
+    case SAGE_ERR_CUDA: base = "CUDA error"; break;
+    case SAGE_ERR_DEVICE_TIMEOUT: base = "device wait timed out"; break;
+    default: break;
+  }
+  s = base;
+  if (status != SAGE_OK && status == t_last_status && !t_last_detail.empty())
+    s += ": " + t_last_detail;
+  return s.c_str();
+}
+
+const char* sage_version(void) { return "sage-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// sage_internal.h -- launcher argument blocks shared by the C-ABI layer and
+// the kernels (host side only).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace sage {
+
+struct QuantQKArgs {
+  const void* q;
+  const void* k;
+  int dtype;  // 0 = f16, 1 = bf16
+  int mode;   // 0 = INT8, 1 = FP4
+  int64_t B, H, N, d;
+  void* q_codes;
+  float* q_scales;
+  void* q_sf;
+  void* k_codes;
+  float* k_scales;
+  void* k_sf;
+  float* k_mean;
+  double* ws_ksum;  // [B*H, N/128, d] FP64 chunk partial sums (workspace)
+};
+
+struct QuantVArgs {
+  const void* v;
+  int dtype;
+  int mode;  // 0 = FP8, 1 = FP4
+  int64_t B, H, N, d;
+  void* v_codes;
+  float* v_scales;
+  void* v_sf;
+  double* ws_ksum;  // scratch the V statistics pass may write (same size as above)
+  float* ws_vmax;   // [B*H, N/128, d] per-chunk |V| maxima (workspace)
+};
+
+struct AttnArgs {
+  int mode;
+  const void* q_codes;
+  const float* q_scales;
+  const void* q_sf;
+  const void* k_codes;
+  const float* k_scales;
+  const void* k_sf;
+  const void* v_codes;
+  const float* v_scales;
+  const void* v_sf;
+  void* o;
+  int dtype;
+  int64_t B, H, N, d;
+  int causal;
+  float sm_scale;
+  uint32_t* status;  // device status word
+};
+
+cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st);
+cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st);
+
+// Returns cudaSuccess, or an error; `detail` receives a message on failure
+// of something other than a CUDA call (e.g. tensor-map encoding).
+cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** detail);
+cudaError_t launch_attn_fp4(const AttnArgs& a, cudaStream_t st, const char** detail);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library does not link libcuda).  Returns false with a message on failure.
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t dim0,
+                    uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                    CUtensorMapSwizzle swz, const char** detail);
+
+}  // namespace sage

@@ -1,0 +1,103 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports every
+symbol include/sage.h declares, and rejects bad arguments before touching a
+device (CPU only: no compute call is made)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_attention_quant_b200 import build as qb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qb.build()
+    import quantized_attention_quant_b200 as q
+    return q.library()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "sage.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_match_header(lib):
+    import quantized_attention_quant_b200 as q
+    names = header_functions()
+    assert names == sorted(q.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.sage_version().decode().startswith("sage-b200")
+
+
+def test_buffer_bytes(lib):
+    import quantized_attention_quant_b200 as q
+    B, H, N, d = 2, 3, 256, 128
+    assert q.buffer_bytes("int8_fp8", "q_codes", B, H, N, d) == B * H * N * d
+    assert q.buffer_bytes("int8_fp8", "q_scales", B, H, N, d) == B * H * 2 * 4
+    assert q.buffer_bytes("int8_fp8", "q_sf", B, H, N, d) == 0
+    assert q.buffer_bytes("int8_fp8", "v_scales", B, H, N, d) == B * H * d * 4
+    assert q.buffer_bytes("fp4", "q_codes", B, H, N, d) == B * H * N * d // 2
+    assert q.buffer_bytes("fp4", "q_sf", B, H, N, d) == B * H * 2 * 2 * 512
+    assert q.buffer_bytes("fp4", "v_sf", B, H, N, d) == B * H * 2 * 2 * 512
+    assert q.buffer_bytes("fp4", "v_scales", B, H, N, d) == B * H * 2 * 4
+    assert lib.sage_buffer_bytes(0, 0, -1, 1, 1, 1) == 0
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def call_attn(lib, **kw):
+    a = dict(mode=0, qc=FAKE, qs=FAKE, qsf=None, kc=FAKE, ks=FAKE, ksf=None, vc=FAKE, vs=FAKE,
+             vsf=None, o=FAKE, dtype=1, B=1, H=1, N=128, d=64, causal=0, sm=0.125)
+    a.update(kw)
+    return lib.sage_attn_fwd_quantized(a["mode"], a["qc"], a["qs"], a["qsf"], a["kc"], a["ks"],
+                                       a["ksf"], a["vc"], a["vs"], a["vsf"], a["o"], a["dtype"],
+                                       a["B"], a["H"], a["N"], a["d"], a["causal"],
+                                       ctypes.c_float(a["sm"]), None)
+
+
+@pytest.mark.parametrize("kw,status,text", [
+    (dict(dtype=7), -1, "dtype"),
+    (dict(mode=3), -1, "mode"),
+    (dict(B=-1), -1, "negative"),
+    (dict(d=96), -2, "head dim"),
+    (dict(mode=1, d=64, qsf=FAKE, ksf=FAKE, vsf=FAKE), -2, "FP4"),
+    (dict(N=200), -2, "multiple of 128"),
+    (dict(qc=None), -1, "q_codes is NULL"),
+    (dict(o=FAKE + 4), -2, "aligned"),
+    (dict(qsf=FAKE), -1, "must be NULL"),
+    (dict(mode=1, d=128), -1, "q_sf is NULL"),
+    (dict(sm=-1.0), -1, "sm_scale"),
+    (dict(B=70000, H=1), -2, "65535"),
+])
+def test_attn_argument_errors(lib, kw, status, text):
+    s = call_attn(lib, **kw)
+    assert s == status
+    assert text in lib.sage_status_string(s).decode()
+
+
+def test_empty_is_a_noop(lib):
+    for B, H, N in [(0, 4, 128), (2, 0, 128), (2, 4, 0)]:
+        assert call_attn(lib, B=B, H=H, N=N) == 0
+        assert lib.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, B, H, N, 128, 0,
+                                 ctypes.c_float(0.0), 0, None) == 0
+
+
+def test_quant_argument_errors(lib):
+    s = lib.sage_quant_qk(FAKE, FAKE, 1, 1, 1, 128, 64, 0, FAKE, FAKE, None, FAKE, FAKE, None,
+                          None, None)
+    assert s == -1 and "k_mean" in lib.sage_status_string(s).decode()
+    s = lib.sage_quant_v(FAKE, 1, 1, 1, 128, 128, 1, FAKE, FAKE, None, None)
+    assert s == -1 and "v_sf" in lib.sage_status_string(s).decode()
+    assert lib.sage_quant_v(FAKE, 1, 0, 1, 128, 128, 0, FAKE, FAKE, None, None) == 0
+
+
+def test_status_strings(lib):
+    for s, t in [(0, "ok"), (-1, "invalid"), (-2, "unsupported"), (-3, "CUDA"), (-4, "timed out")]:
+        assert t in lib.sage_status_string(s).decode()

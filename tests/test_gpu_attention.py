@@ -1,0 +1,171 @@
+"""GPU attention parity against the oracle (through the C ABI).
+
+Bars (floating point):
+  * |O_gpu - O_emulated| <= 2e-3 + half an ulp of the output dtype at
+    |O_emulated| (the kernel's result is rounded to bf16/fp16 on output,
+    which by itself moves a value by up to half an ulp) + the oracle's bound
+    for P~ codes that lie within a relative 2^-15 of an e4m3 rounding
+    midpoint (the kernel evaluates P~ in FP32, so either neighbouring code is
+    a correct result there; see oracle.attention.fp8_p_ambiguity);
+  * cosine(O_gpu, O_exact) >= 0.999 where the quantization scheme itself
+    reaches it on the workload, and never more than 2e-4 below the
+    emulated oracle's own cosine.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import quantized_attention_quant_b200 as sage
+from oracle import attention as att
+from oracle import encoders as enc
+from quantized_attention_quant_b200.workloads import WORKLOADS, make_qkv, to_numpy32
+from tests.test_gpu_prepass import rand_qkv
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-3
+AMBIGUITY_EPS = 2.0 ** -15
+
+
+def half_ulp(x, dtype):
+    bits = 8 if dtype == "bf16" else 11
+    a = np.maximum(np.abs(x), 2.0 ** -14)
+    return np.ldexp(1.0, np.floor(np.log2(a)).astype(int) - bits)
+
+
+def cosine(a, b):
+    a = a.astype(np.float64).ravel()
+    b = b.astype(np.float64).ravel()
+    return float(a @ b / math.sqrt((a @ a) * (b @ b)))
+
+
+def check_against_oracle(o_gpu, q, k, v, causal, sm_scale, mode, dtype, rows=None, cos_floor=None):
+    qs, ks, vs = (to_numpy32(t) for t in (q, k, v))
+    if mode == "int8_fp8":
+        emu, amb = att.emulated_sage_attention(qs, ks, vs, causal, sm_scale, mode=mode, rows=rows,
+                                               ambiguity_eps=AMBIGUITY_EPS)
+    else:
+        emu = att.emulated_sage_attention(qs, ks, vs, causal, sm_scale, mode=mode, rows=rows)
+        amb = 0.0
+    ex = att.exact_attention(qs, ks, vs, causal, sm_scale, rows=rows)
+    g = o_gpu.astype(np.float64)
+    err = np.abs(g - emu)
+    tol = MAX_ABS + half_ulp(emu, dtype) + amb
+    bad = err > tol
+    assert not bad.any(), (
+        f"{bad.sum()} of {bad.size} outside tolerance; worst excess "
+        f"{(err - tol).max():.3e} at {np.unravel_index((err - tol).argmax(), err.shape)}")
+    c_gpu, c_emu = cosine(g, ex), cosine(emu, ex)
+    assert c_gpu >= c_emu - 2e-4, (c_gpu, c_emu)
+    if cos_floor is not None:
+        assert c_gpu >= cos_floor, (c_gpu, c_emu)
+    return err.max(), c_gpu, c_emu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("N", [128, 512])
+def test_int8_fp8_random(cuda_device, N, dtype, d, causal):
+    q, k, v = rand_qkv(2, 2, N, d, dtype, seed=100 + N + d + causal)
+    o = sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, mode="int8_fp8")
+    torch.cuda.synchronize()
+    check_against_oracle(to_numpy32(o), q, k, v, causal, 1 / math.sqrt(d), "int8_fp8", dtype)
+    assert sage.device_status() == 0
+
+
+def test_int8_fp8_zero_q_gives_mean_v(cuda_device):
+    # Q = 0 -> every score 0 -> P~ = 1 (code 448) -> O = mean of dequantized V.
+    B, H, N, d = 1, 2, 512, 128
+    _, k, v = rand_qkv(B, H, N, d, "bf16", seed=5)
+    q = torch.zeros_like(k)
+    for causal in (False, True):
+        o = to_numpy32(sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal))
+        vs = to_numpy32(v)
+        from oracle import prepass as pp
+        vc, s = pp.quant_v_fp8(vs)
+        vd = enc.e4m3_decode(vc).transpose(0, 1, 3, 2) * s[:, :, None, :]
+        if causal:
+            want = np.cumsum(vd, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+        else:
+            want = np.broadcast_to(vd.mean(axis=2, keepdims=True), vd.shape)
+        assert np.max(np.abs(o - want) - half_ulp(want, "bf16") - 1e-5) <= 0
+
+
+def test_int8_fp8_onehot_selects_rows(cuda_device):
+    # Query r points at key pi(r) only; the logit gap makes P~ one-hot, so
+    # O[r] = dequantized V[pi(r)].  Exercises the Q K^T row/column mapping.
+    B, H, N, d = 1, 1, 128, 128
+    dev = torch.device("cuda")
+    perm = np.random.default_rng(3).permutation(N)
+    qc = np.zeros((N, d), np.int8)
+    qc[np.arange(N), perm] = 127
+    kc = np.zeros((N, d), np.int8)
+    kc[np.arange(N), np.arange(N)] = 127
+    v = torch.from_numpy(np.random.default_rng(4).standard_normal((B, H, N, d)).astype(np.float32)
+                         ).to(torch.bfloat16)
+    vq = sage.sage_quant_v(v.to(dev))
+    qk = {"q_codes": torch.from_numpy(qc.view(np.uint8).ravel()).to(dev),
+          "q_scales": torch.ones(1, dtype=torch.float32, device=dev).view(torch.uint8),
+          "q_sf": None,
+          "k_codes": torch.from_numpy(kc.view(np.uint8).ravel()).to(dev),
+          "k_scales": torch.ones(1, dtype=torch.float32, device=dev).view(torch.uint8),
+          "k_sf": None}
+    o = to_numpy32(sage.sage_attn_fwd_quantized(qk, vq, (B, H, N, d), sm_scale=0.05))
+    from oracle import prepass as pp
+    vc, s = pp.quant_v_fp8(to_numpy32(v))
+    vd = enc.e4m3_decode(vc).transpose(0, 1, 3, 2) * s[:, :, None, :]
+    want = vd[0, 0, perm]
+    assert np.max(np.abs(o[0, 0] - want) - half_ulp(want, "bf16")) <= 1e-6
+
+
+def test_fwd_equals_prepass_plus_attention(cuda_device):
+    q, k, v = rand_qkv(1, 4, 384, 128, "bf16", seed=9)
+    dev = torch.device("cuda")
+    qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
+    for mode in ["int8_fp8"]:
+        a = sage.sage_attn_fwd(qg, kg, vg, causal=True, mode=mode)
+        qk = sage.sage_quant_qk(qg, kg, mode)
+        vq = sage.sage_quant_v(vg, mode)
+        b = sage.sage_attn_fwd_quantized(qk, vq, tuple(q.shape), mode, causal=True,
+                                         out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b)
+
+
+def test_side_stream(cuda_device):
+    q, k, v = rand_qkv(1, 2, 256, 64, "bf16", seed=10)
+    dev = torch.device("cuda")
+    ref = sage.sage_attn_fwd(q.to(dev), k.to(dev), v.to(dev))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = sage.sage_attn_fwd(q.to(dev), k.to(dev), v.to(dev))
+    s.synchronize()
+    assert torch.equal(ref, out)
+
+
+FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", None), ("long_causal", None)]
+
+
+@pytest.mark.parametrize("name,cos_floor", FULL)
+def test_int8_fp8_full_workloads(cuda_device, name, cos_floor):
+    """Full-size launch (as timed by bench.py); sampled heads and rows."""
+    w = WORKLOADS[name]
+    q, k, v = make_qkv(w)
+    dev = torch.device("cuda")
+    o = sage.sage_attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=w.causal, mode=w.mode)
+    torch.cuda.synchronize()
+    assert sage.device_status() == 0
+    rng = np.random.default_rng(0)
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    n_rows = w.N if w.N <= 512 else 256
+    rows = np.sort(rng.choice(w.N, n_rows, replace=False))
+    rows[-1] = w.N - 1                                   # always include the last row
+    og = to_numpy32(o)
+    for (b, h) in heads:
+        sel = (slice(b, b + 1), slice(h, h + 1))
+        check_against_oracle(og[sel][:, :, rows], q[sel], k[sel], v[sel], w.causal, w.sm_scale,
+                             w.mode, w.dtype, rows=rows, cos_floor=cos_floor)

@@ -309,3 +309,48 @@ def test_output_rounding_matches_dtype():
     r = enc.round_to_dtype(o, "bf16")
     assert np.array_equal(r, enc.bf16_round(r))
     assert np.max(np.abs(r - o)) <= np.abs(o).max() * 2.0 ** -8
+
+
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp4"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_subset_matches_full(mode, causal):
+    # computing a subset of query rows gives exactly those rows of the full run
+    q, k, v = rnd((1, 2, 384, 32), 60), rnd((1, 2, 384, 32), 61), rnd((1, 2, 384, 32), 62)
+    rows = np.array([0, 5, 127, 128, 200, 383])
+    full = att.emulated_sage_attention(q, k, v, causal, 0.2, mode=mode)
+    sub = att.emulated_sage_attention(q, k, v, causal, 0.2, mode=mode, rows=rows)
+    assert np.array_equal(full[:, :, rows], sub)
+    fe = att.exact_attention(q, k, v, causal, 0.2)
+    se = att.exact_attention(q, k, v, causal, 0.2, rows=rows)
+    assert np.max(np.abs(fe[:, :, rows] - se)) <= 1e-15
+
+
+def test_fp8_p_ambiguity_marks_midpoints():
+    # 448 P~ exactly at / near the midpoint of two e4m3 values is ambiguous;
+    # far from any midpoint it is not
+    mids = np.array([432.0, 17.0, 1.0625, 2.0 ** -9 * 1.5]) / 448.0     # 416|448, 16|18, 1|1.125
+    amb = att.fp8_p_ambiguity(mids, 1e-6)
+    assert np.array_equal(amb, np.array([32.0, 2.0, 0.125, 2.0 ** -9]))
+    far = np.array([440.0, 16.1, 1.01]) / 448.0
+    assert np.all(att.fp8_p_ambiguity(far, 1e-6) == 0)
+
+
+def test_ambiguity_bound_covers_flipped_codes():
+    # Perturbing P~ by a relative 1e-4 before quantization (a stand-in for a
+    # kernel's FP32 evaluation) moves O by no more than the bound for 1e-4,
+    # and does move it (some codes flip).
+    q, k, v = rnd((1, 1, 256, 32), 70, 2.0), rnd((1, 1, 256, 32), 71, 2.0), rnd((1, 1, 256, 32), 72)
+    o, bnd = att.emulated_sage_attention(q, k, v, True, 0.3, ambiguity_eps=1e-4)
+    base = att.quant_p_fp8
+    moved = 0
+    try:
+        for sgn in (+1, -1):
+            att.quant_p_fp8 = lambda pt, s=sgn: base(pt * (1 + s * 1e-4))
+            # the tile loop receives the perturbed quantizer through the module
+            o2 = att.emulated_sage_attention(q, k, v, True, 0.3)
+            assert np.all(np.abs(o2 - o) <= bnd + 1e-12)
+            moved += int(np.any(o2 != o))
+    finally:
+        att.quant_p_fp8 = base
+    assert moved == 2
+    assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.3), o)
