@@ -104,6 +104,62 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   return r;
 }
 
+constexpr uint32_t kBiasBits = 0x4B400000u;  // bit pattern of 1.5 * 2^23
+constexpr float kBias = 12582912.0f;
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Max of 128 non-negative floats given as bits: 8 independent 3-input max
+// chains, then a short tree.
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(__uint_as_float(s[k]), __uint_as_float(s[k + 8]));
+#pragma unroll
+  for (int i = 16; i < 128; i += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      a[k] = fmax3(a[k], __uint_as_float(s[i + k]), __uint_as_float(s[i + 8 + k]));
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// 448 P~ = 2^((x - bias) c + neg) for the 128 biased scores of a row,
+// quantized to e4m3 (four codes per 32-bit word, key i in byte i % 4), and
+// the sum of the unquantized values.  MASKED: keys i > r contribute 0.
+template <bool MASKED>
+__device__ __forceinline__ float exp_quant128(const uint32_t (&s)[128], float c, float neg, int r,
+                                              uint32_t (&p)[32]) {
+  const float2 c2 = make_float2(c, c);
+  const float2 n2 = make_float2(neg, neg);
+  const float2 mb = make_float2(-kBias, -kBias);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int i = 0; i < 128; i += 4) {
+    const float2 x01 = __fadd2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), mb);
+    const float2 x23 =
+        __fadd2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), mb);
+    const float2 t01 = __ffma2_rn(x01, c2, n2);
+    const float2 t23 = __ffma2_rn(x23, c2, n2);
+    float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
+    if (MASKED) {
+      f0 = (i + 0 <= r) ? f0 : 0.f;
+      f1 = (i + 1 <= r) ? f1 : 0.f;
+      f2 = (i + 2 <= r) ? f2 : 0.f;
+      f3 = (i + 3 <= r) ? f3 : 0.f;
+    }
+    acc[(i >> 2) & 3] = __fadd2_rn(acc[(i >> 2) & 3], make_float2(f0, f1));
+    acc[(i >> 2) & 3] = __fadd2_rn(acc[(i >> 2) & 3], make_float2(f2, f3));
+    p[i >> 2] = cvt_e4m3x2(f0, f1) | (cvt_e4m3x2(f2, f3) << 16);
+  }
+  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return t.x + t.y;
+}
+
 template <typename OutT>
 __device__ __forceinline__ uint32_t pack2(float a, float b);
 template <>
@@ -280,28 +336,24 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       tmem_wait_ld();
       const bool diag = CAUSAL && (j == qt);
       const float c = qs * ks * scale_log2;
-      int mx = INT_MIN;
+      // Integer scores -> floats without a conversion instruction: with the
+      // bias 1.5 * 2^23 added, the bit pattern is the float 1.5 * 2^23 + A
+      // exactly (|A| <= 127^2 * 128 < 2^22); subtracting the bias back is
+      // exact too.  The biased floats are ordered like A, so the row max is
+      // taken on them directly.
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        const int v = (int)s[i];
-        if (!diag || i <= r) mx = max(mx, v);
+      for (int i = 0; i < 128; ++i) s[i] += kBiasBits;
+      if (diag) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i > r) s[i] = 0u;  // masked keys: +0.0, below every biased score
       }
-      const float m_new = fmaxf(m, (float)mx * c);
+      const float m_new = fmaxf(m, (row_max128(s) - kBias) * c);
       const float alpha = ex2(m - m_new);
-      const float neg = kLog2_448 - m_new;
-      float sum = 0.f;
+      const float neg = kLog2_448 - m_new;  // yields 448 P~ directly
       uint32_t p[32];
-#pragma unroll
-      for (int i = 0; i < 128; i += 4) {
-        float f[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x = ex2(fmaf((float)(int)s[i + e], c, neg));
-          f[e] = (!diag || (i + e) <= r) ? x : 0.f;
-          sum += f[e];
-        }
-        p[i / 4] = cvt_e4m3x2(f[0], f[1]) | (cvt_e4m3x2(f[2], f[3]) << 16);
-      }
+      const float sum = diag ? exp_quant128<true>(s, c, neg, r, p)
+                             : exp_quant128<false>(s, c, neg, r, p);
       l = fmaf(alpha, l, sum);
       m = m_new;
       alpha_s[(j & 3) * 128 + r] = alpha;
@@ -318,9 +370,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    float o[D];
+    float2 o2[D / 2];
 #pragma unroll
-    for (int c = 0; c < D; ++c) o[c] = 0.f;
+    for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.f, 0.f);
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const int b = j & 1;
@@ -336,13 +388,16 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         break;
       }
       tc_fence_after();
+      const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t t[32];
         tmem_ld32(lane_base + tPV(b) + cc * 32, t);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[cc * 32 + i] = fmaf(alpha, o[cc * 32 + i], __uint_as_float(t[i]));
+        for (int i = 0; i < 16; ++i)
+          o2[cc * 16 + i] = __ffma2_rn(
+              a2, o2[cc * 16 + i], make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])));
       }
       tc_fence_before();
       mbar_arrive(&bar.pv_empty[b]);
@@ -353,12 +408,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 8) {
-        uint4 w;
-        w.x = pack2<OutT>(o[c + 0] * __ldg(vs + c + 0) * inv_l, o[c + 1] * __ldg(vs + c + 1) * inv_l);
-        w.y = pack2<OutT>(o[c + 2] * __ldg(vs + c + 2) * inv_l, o[c + 3] * __ldg(vs + c + 3) * inv_l);
-        w.z = pack2<OutT>(o[c + 4] * __ldg(vs + c + 4) * inv_l, o[c + 5] * __ldg(vs + c + 5) * inv_l);
-        w.w = pack2<OutT>(o[c + 6] * __ldg(vs + c + 6) * inv_l, o[c + 7] * __ldg(vs + c + 7) * inv_l);
-        *reinterpret_cast<uint4*>(dst + c) = w;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 v = o2[c / 2 + e];
+          w[e] = pack2<OutT>(v.x * __ldg(vs + c + 2 * e) * inv_l,
+                             v.y * __ldg(vs + c + 2 * e + 1) * inv_l);
+        }
+        *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
