@@ -9,26 +9,34 @@
 //   per query row, over 128-key tiles j (causal: j <= query tile):
 //     A      = q_codes . k_codes_j^T                 (tcgen05 kind::i8, exact)
 //     t      = A * (s_Q s_Kj sm_scale log2 e)        (log2 domain)
-//     m_new  = max(m, rowmax t); alpha = 2^(m - m_new)
-//     p      = e4m3(448 * 2^(t - m_new))             (448 P~, quantized)
-//     l      = alpha l + sum 448 P~                  (unquantized P~)
+//     m_j    = max(m_{j-1}, rowmax t); alpha_j = 2^(m_{j-1} - m_j)
+//     p      = e4m3(448 * 2^(t - m_j))               (448 P~, quantized)
+//     l      = alpha_j l + sum 448 P~                (unquantized P~)
 //     part_j = p . v_codes_j                         (kind::f8f6f4, fresh FP32)
-//     O      = alpha O + part_j                      (FP32, registers)
+//     O      = alpha_j O + part_j                    (FP32, registers)
 //   O_out = O * s_V[c] / l
 //
-// One CTA owns one 128-row query tile of one (b, h) and walks all key tiles.
-// Warp roles (320 threads):
-//   warp 0      TMA producer: Q once, then K_j and V_j^T into 4/6-deep rings
-//   warp 1      TMEM allocator and the single-thread tcgen05 issuer
-//   warps 2..5  softmax: thread = one query row (TMEM lane); reads S_j from
-//               TMEM, writes the e4m3 P~ tile back into TMEM (aliasing the
-//               first 32 columns of S_j) as the A operand of the P~V MMA
-//   warps 6..9  correction: reads each per-tile FP32 partial from TMEM and
-//               folds it into the row's running FP32 accumulator (level 2),
-//               then normalises and writes O
-// TMEM columns: S[0] 0..127, S[1] 128..255, PV[0] 256.., PV[1] 256+D.. .
-// Every barrier wait is bounded; an expired wait sets the device status
-// word and makes every role leave its loop.
+// One CTA owns one 128-row query tile of one (b, h).  The exponentials are
+// the throughput limit (the tensor core finishes a 128x128 tile in far fewer
+// cycles than the SFU needs for its 16K exponentials, and one warp per SM
+// sub-partition keeps the SFU only about half busy), so two warpgroups share
+// every tile.  Warp roles (512 threads):
+//   warpgroup 0: warp 0 TMA producer (Q once, K_j and V_j^T rings),
+//                warp 1 TMEM allocator and single-thread tcgen05 issuer
+//   warpgroups 1, 2 ("exp"): key columns 0..63 / 64..127 of every tile.
+//                Thread = query row = TMEM lane.  448 P~, e4m3 codes into a
+//                swizzled shared-memory tile (the A operand of the P~V MMA),
+//                the row sum, and the bias written back into S.
+//   warpgroup 3 ("stats"): per key tile the row max, the running max m_j and
+//                alpha_j (published for both exp warpgroups), then the level-2
+//                fold of the tile's FP32 partial into the running FP32
+//                accumulator (registers); finally normalise and store O.
+// TMEM columns: S[0] 0..127, S[1] 128..255 (key tile j uses S[j % 2]),
+// PV[0] 256.., PV[1] 256+D.. .  Before each Q K^T the S columns hold the bit
+// pattern of 1.5 * 2^23; the INT8 MMA accumulates onto it, so a score reads
+// back as the float 1.5*2^23 + A exactly (|A| <= 127^2*128 < 2^22) with no
+// conversion instruction.  Every barrier wait is bounded; an expired wait
+// sets the device status word and makes every role leave its loop.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -37,34 +45,59 @@
 #include "sage_ptx.cuh"
 
 namespace sage {
+
+// Optional timeline trace (builds with -DSAGE_TRACE only): %clock64 of
+// selected events of one steady-state CTA, read back by sage_trace_read.
+#ifdef SAGE_TRACE
+__device__ long long g_sage_trace[16][512];
+#define SAGE_TR(ev, j)                                                                  \
+  do {                                                                                  \
+    if (blockIdx.x == 7 && blockIdx.y == 1 && (j) < 512) {                              \
+      long long t_;                                                                     \
+      asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                \
+      g_sage_trace[ev][j] = t_;                                                         \
+    }                                                                                   \
+  } while (0)
+#else
+#define SAGE_TR(ev, j) \
+  do {                 \
+  } while (0)
+#endif
+
 namespace {
 
-constexpr int kThreadsAttn = 320;
+constexpr int kThreadsAttn = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448)
+constexpr uint32_t kBiasBits = 0x4B400000u;       // bit pattern of 1.5 * 2^23
+constexpr float kBias = 12582912.0f;
+// Register split (launch: 512 threads x 128 = 65536):
+//   producer/MMA 32, two exp warpgroups keep 128, stats/fold 216
+//   -> 128 x (32 + 128 + 128 + 216) = 64512 <= 65536.
+constexpr uint32_t kRegsProducer = 32;
+constexpr uint32_t kRegsStats = 216;
 
 template <int D>
-struct I8F8Layout {
-  static constexpr int KS = D == 128 ? 4 : 6;  // K ring depth
-  static constexpr int VS = D == 128 ? 4 : 6;  // V ring depth
+struct Layout {
+  static constexpr int KS = D == 128 ? 3 : 5;  // K ring depth
+  static constexpr int VS = D == 128 ? 3 : 5;  // V ring depth
   static constexpr int Q_BYTES = 128 * D;
   static constexpr int K_BYTES = 128 * D;
   static constexpr int V_BYTES = D * 128;
+  static constexpr int P_BYTES = 128 * 128;  // e4m3 P~ tile, 128-byte swizzled rows
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KS * K_BYTES;
-  static constexpr int OFF_MISC = OFF_V + VS * V_BYTES;
-  // misc: barriers (64 x 8 B), tmem slot, abort flag, alpha ring [4][128],
-  // l [128]
-  static constexpr int OFF_BAR = OFF_MISC;
+  static constexpr int OFF_P = OFF_V + VS * V_BYTES;
+  static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_MISC;           // barriers (<= 64 x 8 B)
   static constexpr int OFF_TMEM = OFF_MISC + 512;
   static constexpr int OFF_ABORT = OFF_MISC + 528;
-  static constexpr int OFF_ALPHA = OFF_MISC + 1024;
-  static constexpr int OFF_L = OFF_ALPHA + 4 * 128 * 4;
-  static constexpr int END = OFF_L + 128 * 4;
+  static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
+  static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
+  static constexpr int END = OFF_L + 2 * 128 * 4;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
-  // shared-memory descriptor strides
   static constexpr uint32_t QK_SBO = 8 * D;  // 8 rows of D bytes
   static constexpr Swz QK_SWZ = D == 128 ? Swz::k128 : Swz::k64;
 };
@@ -75,18 +108,20 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;
   uint64_t* v_empty;
-  uint64_t* s_full;    // [2] MMA -> softmax
-  uint64_t* p_full;    // [2] softmax -> MMA
-  uint64_t* pv_full;   // [2] MMA -> correction
-  uint64_t* pv_empty;  // [2] correction -> MMA
-  uint64_t* a_full;    // [4] softmax -> correction (alpha ring)
-  uint64_t* l_ready;   // [1] softmax -> correction (final l)
-  uint64_t* drain;     // [1] MMA drain on abort
+  uint64_t* s_full;    // [2] MMA -> stats, exp: S[b] holds Q K_j^T
+  uint64_t* m_full;    // [2] stats -> exp: m_j, alpha_j of tile j (slot j % 2)
+  uint64_t* s_ready;   // [2] exp -> MMA: S[b] read and re-biased (both halves)
+  uint64_t* p_full;    // [2] exp -> MMA: P~ tile b written (both halves)
+  uint64_t* p_empty;   // [2] MMA -> exp: P~ tile b read by the P~V MMA
+  uint64_t* pv_full;   // [2] MMA -> stats: PV[b] holds tile j's partial
+  uint64_t* pv_empty;  // [2] stats -> MMA: PV[b] read
+  uint64_t* l_ready;   // [1] exp -> stats: final row sums
+  uint64_t* drain;     // MMA drain on abort
 };
 
 template <int D>
 __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
-  using L = I8F8Layout<D>;
+  using L = Layout<D>;
   uint64_t* b = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   Bars r;
   r.q_full = b;
@@ -95,17 +130,25 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.v_full = r.k_empty + L::KS;
   r.v_empty = r.v_full + L::VS;
   r.s_full = r.v_empty + L::VS;
-  r.p_full = r.s_full + 2;
-  r.pv_full = r.p_full + 2;
+  r.m_full = r.s_full + 2;
+  r.s_ready = r.m_full + 2;
+  r.p_full = r.s_ready + 2;
+  r.p_empty = r.p_full + 2;
+  r.pv_full = r.p_empty + 2;
   r.pv_empty = r.pv_full + 2;
-  r.a_full = r.pv_empty + 2;
-  r.l_ready = r.a_full + 4;
+  r.l_ready = r.pv_empty + 2;
   r.drain = r.l_ready + 1;
   return r;
 }
 
-constexpr uint32_t kBiasBits = 0x4B400000u;  // bit pattern of 1.5 * 2^23
-constexpr float kBias = 12582912.0f;
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -113,33 +156,63 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Max of 128 non-negative floats given as bits: 8 independent 3-input max
-// chains, then a short tree.
-__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
-  float a[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) a[k] = fmaxf(__uint_as_float(s[k]), __uint_as_float(s[k + 8]));
-#pragma unroll
-  for (int i = 16; i < 128; i += 16)
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      a[k] = fmax3(a[k], __uint_as_float(s[i + k]), __uint_as_float(s[i + 8 + k]));
-  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+
+// 32 columns of the same 32-bit value.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
 }
 
-// 448 P~ = 2^((x - bias) c + neg) for the 128 biased scores of a row,
-// quantized to e4m3 (four codes per 32-bit word, key i in byte i % 4), and
-// the sum of the unquantized values.  MASKED: keys i > r contribute 0.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Max of 64 biased scores (as float bits) and a running value.  MASKED:
+// columns col0 + i > r are ignored (causal diagonal tile).
 template <bool MASKED>
-__device__ __forceinline__ float exp_quant128(const uint32_t (&s)[128], float c, float neg, int r,
-                                              uint32_t (&p)[32]) {
+__device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float acc) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float x = __uint_as_float(s[k]), y = __uint_as_float(s[k + 8]);
+    if (MASKED) {
+      x = (col0 + k <= r) ? x : 0.f;
+      y = (col0 + k + 8 <= r) ? y : 0.f;
+    }
+    a[k] = fmaxf(x, y);
+  }
+#pragma unroll
+  for (int i = 16; i < 64; i += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float x = __uint_as_float(s[i + k]), y = __uint_as_float(s[i + 8 + k]);
+      if (MASKED) {
+        x = (col0 + i + k <= r) ? x : 0.f;
+        y = (col0 + i + 8 + k <= r) ? y : 0.f;
+      }
+      a[k] = fmax3(a[k], x, y);
+    }
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], acc));
+}
+
+// 448 P~ for 32 biased scores of a row -> 8 words of e4m3 codes (key i in
+// byte i % 4) and the sum of the unquantized values.
+template <bool MASKED>
+__device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
+                                             int r, uint32_t (&p)[8]) {
   const float2 c2 = make_float2(c, c);
   const float2 n2 = make_float2(neg, neg);
   const float2 mb = make_float2(-kBias, -kBias);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int i = 0; i < 128; i += 4) {
+  for (int i = 0; i < 32; i += 4) {
     const float2 x01 = __fadd2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), mb);
     const float2 x23 =
         __fadd2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), mb);
@@ -147,16 +220,16 @@ __device__ __forceinline__ float exp_quant128(const uint32_t (&s)[128], float c,
     const float2 t23 = __ffma2_rn(x23, c2, n2);
     float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
     if (MASKED) {
-      f0 = (i + 0 <= r) ? f0 : 0.f;
-      f1 = (i + 1 <= r) ? f1 : 0.f;
-      f2 = (i + 2 <= r) ? f2 : 0.f;
-      f3 = (i + 3 <= r) ? f3 : 0.f;
+      f0 = (col0 + i + 0 <= r) ? f0 : 0.f;
+      f1 = (col0 + i + 1 <= r) ? f1 : 0.f;
+      f2 = (col0 + i + 2 <= r) ? f2 : 0.f;
+      f3 = (col0 + i + 3 <= r) ? f3 : 0.f;
     }
-    acc[(i >> 2) & 3] = __fadd2_rn(acc[(i >> 2) & 3], make_float2(f0, f1));
-    acc[(i >> 2) & 3] = __fadd2_rn(acc[(i >> 2) & 3], make_float2(f2, f3));
+    acc0 = __fadd2_rn(acc0, make_float2(f0, f1));
+    acc1 = __fadd2_rn(acc1, make_float2(f2, f3));
     p[i >> 2] = cvt_e4m3x2(f0, f1) | (cvt_e4m3x2(f2, f3) << 16);
   }
-  const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  const float2 t = __fadd2_rn(acc0, acc1);
   return t.x + t.y;
 }
 
@@ -173,6 +246,200 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// One 32-column chunk of the exp pass: quantized P~ to shared memory, bias
+// back into the chunk's S columns, returns the chunk's row sum.
+template <bool MASKED>
+__device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int cc, float c, float neg,
+                                           int r, uint32_t S, uint32_t prow) {
+  uint32_t p[8];
+  const float sum = exp_quant32<MASKED>(s, c, neg, 32 * cc, r, p);
+  // row r of the 128-byte-swizzled P~ tile: 16-byte chunk q lands at q ^ (r & 7)
+  const uint32_t q0 = (uint32_t)(2 * cc), sw = (uint32_t)(r & 7);
+  st_shared_v4(prow + (((q0) ^ sw) << 4), p[0], p[1], p[2], p[3]);
+  st_shared_v4(prow + (((q0 + 1) ^ sw) << 4), p[4], p[5], p[6], p[7]);
+  tmem_fill32(S + 32 * cc, kBiasBits);
+  return sum;
+}
+
+// Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
+template <int D, bool CAUSAL>
+__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int bh,
+                                         const int ntiles, const uint32_t tmem, const Bars& bar,
+                                         uint8_t* smem, volatile int* abort_flag,
+                                         uint32_t* status, const float* __restrict__ q_scales,
+                                         const float* __restrict__ k_scales,
+                                         const float scale_log2) {
+  using L = Layout<D>;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+  const float* m_s = reinterpret_cast<const float*>(smem + L::OFF_M);
+  float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
+
+  // the first Q K^T into each S buffer accumulates onto the bias
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    tmem_fill32(tmem + lanes + 128u * b + 64u * h, kBiasBits);
+    tmem_fill32(tmem + lanes + 128u * b + 64u * h + 32u, kBiasBits);
+  }
+  tmem_wait_st();
+  tc_fence_before();
+  mbar_arrive(&bar.s_ready[0]);
+  mbar_arrive(&bar.s_ready[1]);
+
+  const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
+  const float* ksp = k_scales + (int64_t)bh * ntiles;
+  float l = 0.f;
+  float ks_next = __ldg(ksp);
+  for (int j = 0; j < nkv; ++j) {
+    const int b = j & 1;
+    const uint32_t ph = (j >> 1) & 1;
+    const float c = qs * ks_next * scale_log2;
+    if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&bar.s_full[b], ph, abort_flag, status, kDevTimeoutMma) &&
+                        mbar_wait(&bar.m_full[b], ph, abort_flag, status, kDevTimeoutEpi)))
+      return;
+    tc_fence_after();
+    if (r == 0) SAGE_TR(h, j);
+    const float m_j = m_s[(2 * b) * 128 + r];
+    const float alpha = m_s[(2 * b + 1) * 128 + r];
+    const float neg = kLog2_448 - m_j;  // yields 448 P~ directly
+    const bool diag = CAUSAL && (j == qt);
+    const uint32_t S = tmem + lanes + 128u * b + 64u * h;
+    uint32_t sa[32], sb[32];
+    tmem_ld32(S, sa);
+    tmem_ld32(S + 32, sb);
+    // P~ tile b is free once the P~V MMA of tile j - 2 has read it
+    if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
+                                                     kDevTimeoutMma)))
+      return;
+    const uint32_t prow = smem_u32(smem + L::OFF_P + b * L::P_BYTES + r * 128);
+    tmem_wait_ld_regs(sa);
+    reg_fence(sb);
+    float sum = diag ? exp_chunk<true>(sa, 2 * h, c, neg, r, S - 32u * (2 * h), prow)
+                     : exp_chunk<false>(sa, 2 * h, c, neg, r, S - 32u * (2 * h), prow);
+    sum += diag ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, S - 32u * (2 * h), prow)
+                : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, S - 32u * (2 * h), prow);
+    l = fmaf(alpha, l, sum);
+    tmem_wait_st();
+    tc_fence_before();
+    if (r == 0) SAGE_TR(2 + h, j);
+    mbar_arrive(&bar.s_ready[b]);   // S[b] free for Q K_{j+2}^T
+    fence_proxy_async_smem();       // P~ stores visible to the tensor core
+    mbar_arrive(&bar.p_full[b]);
+  }
+  l_s[h * 128 + r] = l;
+  mbar_arrive(bar.l_ready);
+}
+
+// Stats warpgroup: row max / running max per key tile, level-2 fold,
+// epilogue.
+template <int D, bool CAUSAL, typename OutT>
+__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh, const int N,
+                                           const int ntiles, const uint32_t tmem, const Bars& bar,
+                                           uint8_t* smem, volatile int* abort_flag,
+                                           uint32_t* status, const float* __restrict__ q_scales,
+                                           const float* __restrict__ k_scales,
+                                           const float* __restrict__ v_scales,
+                                           OutT* __restrict__ out, const float scale_log2) {
+  using L = Layout<D>;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+  float* m_s = reinterpret_cast<float*>(smem + L::OFF_M);
+  const float* l_s = reinterpret_cast<const float*>(smem + L::OFF_L);
+  const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
+  const float* ksp = k_scales + (int64_t)bh * ntiles;
+
+  float2 o2[D / 2];
+#pragma unroll
+  for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.f, 0.f);
+  float m = -INFINITY;
+  auto fold = [&](int i, float alpha) -> bool {
+    const int b = i & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.pv_full[b], (i >> 1) & 1, abort_flag, status,
+                                           kDevTimeoutMma)))
+      return false;
+    tc_fence_after();
+    if (r == 0) SAGE_TR(6, i);
+    const uint32_t PV = tmem + lanes + 256u + (uint32_t)b * (uint32_t)D;
+    const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t pv[32];
+      tmem_ld32(PV + 32 * cc, pv);
+      tmem_wait_ld_regs(pv);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        o2[cc * 16 + k] = __ffma2_rn(
+            a2, o2[cc * 16 + k], make_float2(__uint_as_float(pv[2 * k]), __uint_as_float(pv[2 * k + 1])));
+    }
+    if (r == 0) SAGE_TR(7, i);
+    tc_fence_before();
+    mbar_arrive(&bar.pv_empty[b]);
+    return true;
+  };
+
+  // The fold lags the max by two tiles, so the max of tile j + 1 (which the
+  // exp warpgroups wait for) never queues behind the P~V product of tile j.
+  float alpha_hist[2] = {0.f, 0.f};
+  float ks_next = __ldg(ksp);
+  for (int j = 0; j < nkv; ++j) {
+    const int b = j & 1;
+    const float c = qs * ks_next * scale_log2;
+    if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], (j >> 1) & 1, abort_flag, status,
+                                           kDevTimeoutMma)))
+      return;
+    tc_fence_after();
+    if (r == 0) SAGE_TR(4, j);
+    const bool diag = CAUSAL && (j == qt);
+    const uint32_t S = tmem + lanes + (uint32_t)b * 128u;
+    float mx = 0.f;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t s[2][32];
+      tmem_ld32(S + 64 * hh, s[0]);
+      tmem_ld32(S + 64 * hh + 32, s[1]);
+      tmem_wait_ld_regs(s[0]);
+      reg_fence(s[1]);
+      mx = diag ? max64<true>(&s[0][0], 64 * hh, r, mx) : max64<false>(&s[0][0], 64 * hh, r, mx);
+    }
+    const float m_j = fmaxf(m, (mx - kBias) * c);
+    const float alpha = ex2(m - m_j);
+    m = m_j;
+    m_s[(2 * b) * 128 + r] = m_j;
+    m_s[(2 * b + 1) * 128 + r] = alpha;
+    if (r == 0) SAGE_TR(5, j);
+    mbar_arrive(&bar.m_full[b]);
+    if (j > 1 && !fold(j - 2, alpha_hist[b])) return;
+    alpha_hist[b] = alpha;
+  }
+  for (int i = nkv > 2 ? nkv - 2 : 0; i < nkv; ++i)
+    if (!fold(i, alpha_hist[i & 1])) return;
+  if (!__all_sync(0xffffffffu,
+                  mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)))
+    return;
+  const float inv_l = 1.f / (l_s[r] + l_s[128 + r]);
+  const float* vs = v_scales + (int64_t)bh * D;
+  OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
+#pragma unroll
+  for (int cv = 0; cv < D; cv += 8) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v = o2[cv / 2 + e];
+      w4[e] = pack2<OutT>(v.x * __ldg(vs + cv + 2 * e) * inv_l, v.y * __ldg(vs + cv + 2 * e + 1) * inv_l);
+    }
+    *reinterpret_cast<uint4*>(dst + cv) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+}
+
 template <int D, bool CAUSAL, typename OutT>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -180,7 +447,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scales,
                      const float* __restrict__ k_scales, const float* __restrict__ v_scales,
                      OutT* __restrict__ out, int N, float scale_log2, uint32_t* status) {
-  using L = I8F8Layout<D>;
+  using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -188,14 +455,12 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const int lane = threadIdx.x & 31;
   const int ntiles = N / 128;
   const int bh = blockIdx.y;
-  const int qt = CAUSAL ? (ntiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int qt = CAUSAL ? (ntiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy first
   const int nkv = CAUSAL ? qt + 1 : ntiles;
 
   Bars bar = carve_bars<D>(smem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
-  float* alpha_s = reinterpret_cast<float*>(smem + L::OFF_ALPHA);
-  float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full, 1);
@@ -209,12 +474,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.p_full[i], 128);
+      mbar_init(&bar.m_full[i], 128);
+      mbar_init(&bar.s_ready[i], 256);
+      mbar_init(&bar.p_full[i], 256);
+      mbar_init(&bar.p_empty[i], 1);
       mbar_init(&bar.pv_full[i], 1);
       mbar_init(&bar.pv_empty[i], 128);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&bar.a_full[i], 128);
-    mbar_init(bar.l_ready, 128);
+    mbar_init(bar.l_ready, 256);
     mbar_init(bar.drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -232,192 +499,110 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM column bases of the double-buffered S/P~ and P~V tiles
-  auto tS = [tmem](int b) -> uint32_t { return tmem + (uint32_t)b * 128u; };
-  auto tPV = [tmem](int b) -> uint32_t { return tmem + 256u + (uint32_t)b * (uint32_t)D; };
 
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sP = smem + L::OFF_P;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (elect_one()) {
-      mbar_arrive_expect_tx(bar.q_full, L::Q_BYTES);
-      tma_load_2d(sQ, &tm_q, 0, bh * N + qt * 128, bar.q_full);
-      for (int j = 0; j < nkv; ++j) {
-        const int sk = j % L::KS;
-        if (!mbar_wait(&bar.k_empty[sk], ((j / L::KS) & 1) ^ 1, abort_flag, status, kDevTimeoutMma))
-          break;
-        mbar_arrive_expect_tx(&bar.k_full[sk], L::K_BYTES);
-        tma_load_2d(sK + sk * L::K_BYTES, &tm_k, 0, bh * N + j * 128, &bar.k_full[sk]);
-        const int sv = j % L::VS;
-        if (!mbar_wait(&bar.v_empty[sv], ((j / L::VS) & 1) ^ 1, abort_flag, status, kDevTimeoutMma))
-          break;
-        mbar_arrive_expect_tx(&bar.v_full[sv], L::V_BYTES);
-        tma_load_2d(sV + sv * L::V_BYTES, &tm_v, j * 128, bh * D, &bar.v_full[sv]);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------- tcgen05 issuer
-    if (elect_one()) {
-      constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*s8*/, 1 /*s8*/, 128, 128);
-      constexpr uint32_t idesc_pv = make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, D);
-      const uint64_t q_desc = make_sdesc(smem_u32(sQ), L::QK_SBO, 16, L::QK_SWZ);
-      bool ok = mbar_wait(bar.q_full, 0, abort_flag, status, kDevTimeoutTma);
-      auto issue_pv = [&](int jj) -> bool {
-        const int b = jj & 1;
-        const int sv = jj % L::VS;
-        if (!mbar_wait(&bar.p_full[b], (jj >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax))
-          return false;
-        if (!mbar_wait(&bar.v_full[sv], (jj / L::VS) & 1, abort_flag, status, kDevTimeoutTma))
-          return false;
-        if (!mbar_wait(&bar.pv_empty[b], ((jj >> 1) & 1) ^ 1, abort_flag, status, kDevTimeoutEpi))
-          return false;
-        tc_fence_after();
-        const uint64_t v_desc = make_sdesc(smem_u32(sV + sv * L::V_BYTES), 1024, 16, Swz::k128);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ts(tPV(b), tS(b) + kk * 8, v_desc + 2 * kk, idesc_pv, kk > 0);
-        mma_commit(&bar.pv_full[b]);
-        mma_commit(&bar.v_empty[sv]);
-        return true;
-      };
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int sk = j % L::KS;
-        if (!mbar_wait(&bar.k_full[sk], (j / L::KS) & 1, abort_flag, status, kDevTimeoutTma)) {
-          ok = false;
-          break;
+  const int wg = warp >> 2;
+  if (wg == 0) {
+    setmaxnreg_dec<kRegsProducer>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar.q_full, L::Q_BYTES);
+        tma_load_2d(sQ, &tm_q, 0, bh * N + qt * 128, bar.q_full);
+        for (int j = 0; j < nkv; ++j) {
+          const int sk = j % L::KS;
+          if (!mbar_wait<true>(&bar.k_empty[sk], ((j / L::KS) & 1) ^ 1, abort_flag, status,
+                               kDevTimeoutMma))
+            break;
+          mbar_arrive_expect_tx(&bar.k_full[sk], L::K_BYTES);
+          tma_load_2d(sK + sk * L::K_BYTES, &tm_k, 0, bh * N + j * 128, &bar.k_full[sk]);
+          const int sv = j % L::VS;
+          if (!mbar_wait<true>(&bar.v_empty[sv], ((j / L::VS) & 1) ^ 1, abort_flag, status,
+                               kDevTimeoutMma))
+            break;
+          mbar_arrive_expect_tx(&bar.v_full[sv], L::V_BYTES);
+          tma_load_2d(sV + sv * L::V_BYTES, &tm_v, j * 128, bh * D, &bar.v_full[sv]);
         }
-        tc_fence_after();
-        const int b = j & 1;
-        const uint64_t k_desc = make_sdesc(smem_u32(sK + sk * L::K_BYTES), L::QK_SBO, 16, L::QK_SWZ);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ---------------------------------------------------- tcgen05 issuer
+      if (elect_one()) {
+        constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*s8*/, 1 /*s8*/, 128, 128);
+        constexpr uint32_t idesc_pv = make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, D);
+        const uint64_t qdesc = make_sdesc(smem_u32(sQ), L::QK_SBO, 16, L::QK_SWZ);
+        bool ok = mbar_wait(bar.q_full, 0, abort_flag, status, kDevTimeoutTma);
+        // S[j % 2] = Q K_j^T (onto the bias)
+        auto qk = [&](int j) -> bool {
+          const int sk = j % L::KS;
+          const int b = j & 1;
+          if (!mbar_wait(&bar.k_full[sk], (j / L::KS) & 1, abort_flag, status, kDevTimeoutTma) ||
+              !mbar_wait(&bar.s_ready[b], (j >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax))
+            return false;
+          tc_fence_after();
+          SAGE_TR(8, j);
+          const uint64_t kdesc = make_sdesc(smem_u32(sK + sk * L::K_BYTES), L::QK_SBO, 16, L::QK_SWZ);
 #pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8_ss(tS(b), q_desc + 2 * kk, k_desc + 2 * kk, idesc_qk, kk > 0);
-        mma_commit(&bar.s_full[b]);
-        mma_commit(&bar.k_empty[sk]);
-        if (j > 0 && !issue_pv(j - 1)) ok = false;
+          for (int kk = 0; kk < D / 32; ++kk)
+            mma_i8_ss(tmem + (uint32_t)b * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
+          mma_commit(&bar.s_full[b]);
+          mma_commit(&bar.k_empty[sk]);
+          return true;
+        };
+        if (ok) ok = qk(0);
+        if (ok && nkv > 1) ok = qk(1);
+        for (int i = 0; ok && i < nkv; ++i) {
+          // the exp warpgroups are done with tile i: first the next Q K^T into
+          // the freed S buffer, then P~_i V_i into PV[i % 2] (level 1)
+          const int b = i & 1;
+          if (!mbar_wait(&bar.p_full[b], (i >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax)) {
+            ok = false;
+            break;
+          }
+          SAGE_TR(10, i);
+          if (i + 2 < nkv && !qk(i + 2)) {
+            ok = false;
+            break;
+          }
+          const int sv = i % L::VS;
+          if (!mbar_wait(&bar.v_full[sv], (i / L::VS) & 1, abort_flag, status, kDevTimeoutTma) ||
+              !mbar_wait(&bar.pv_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, status,
+                         kDevTimeoutEpi)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          SAGE_TR(9, i);
+          const uint64_t pdesc = make_sdesc(smem_u32(sP + b * L::P_BYTES), 1024, 16, Swz::k128);
+          const uint64_t vdesc = make_sdesc(smem_u32(sV + sv * L::V_BYTES), 1024, 16, Swz::k128);
+          const uint32_t d = tmem + 256u + (uint32_t)b * (uint32_t)D;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, pdesc + 2 * kk, vdesc + 2 * kk, idesc_pv, kk > 0);
+          mma_commit(&bar.pv_full[b]);
+          mma_commit(&bar.p_empty[b]);
+          mma_commit(&bar.v_empty[sv]);
+        }
+        if (!ok) {
+          // let every MMA already issued finish before TMEM is released
+          mma_commit(bar.drain);
+          volatile int no_abort = 0;
+          mbar_wait(bar.drain, 0, &no_abort, status, kDevTimeoutMma);
+        }
       }
-      if (ok) ok = issue_pv(nkv - 1);
-      if (!ok) {
-        // let every MMA already issued finish before TMEM is released
-        mma_commit(bar.drain);
-        volatile int no_abort = 0;
-        mbar_wait(bar.drain, 0, &no_abort, status, kDevTimeoutMma);
-      }
+      __syncwarp();
     }
-    __syncwarp();
-  } else if (warp < 6) {
-    // ------------------------------------------------------------- softmax
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
-    const float* ksp = k_scales + (int64_t)bh * ntiles;
-    float m = -INFINITY;
-    float l = 0.f;
-    float ks_next = __ldg(ksp);
-    for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      const float ks = ks_next;
-      if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
-      // warp-uniform decision: the tcgen05.ld/st below are .sync.aligned
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(&bar.s_full[b], (j >> 1) & 1, abort_flag, status, kDevTimeoutMma)))
-        break;
-      tc_fence_after();
-      uint32_t s[128];
-      tmem_ld32(lane_base + tS(b) + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(lane_base + tS(b) + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(lane_base + tS(b) + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld32(lane_base + tS(b) + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-      tmem_wait_ld();
-      const bool diag = CAUSAL && (j == qt);
-      const float c = qs * ks * scale_log2;
-      // Integer scores -> floats without a conversion instruction: with the
-      // bias 1.5 * 2^23 added, the bit pattern is the float 1.5 * 2^23 + A
-      // exactly (|A| <= 127^2 * 128 < 2^22); subtracting the bias back is
-      // exact too.  The biased floats are ordered like A, so the row max is
-      // taken on them directly.
-#pragma unroll
-      for (int i = 0; i < 128; ++i) s[i] += kBiasBits;
-      if (diag) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > r) s[i] = 0u;  // masked keys: +0.0, below every biased score
-      }
-      const float m_new = fmaxf(m, (row_max128(s) - kBias) * c);
-      const float alpha = ex2(m - m_new);
-      const float neg = kLog2_448 - m_new;  // yields 448 P~ directly
-      uint32_t p[32];
-      const float sum = diag ? exp_quant128<true>(s, c, neg, r, p)
-                             : exp_quant128<false>(s, c, neg, r, p);
-      l = fmaf(alpha, l, sum);
-      m = m_new;
-      alpha_s[(j & 3) * 128 + r] = alpha;
-      mbar_arrive(&bar.a_full[j & 3]);
-      tmem_st32(lane_base + tS(b), p);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar.p_full[b]);
-    }
-    l_s[r] = l;
-    mbar_arrive(bar.l_ready);
+  } else if (wg < 3) {
+    // the exp warpgroups keep the 128 registers they were launched with
+    exp_loop<D, CAUSAL>(wg - 1, qt, nkv, bh, ntiles, tmem, bar, smem, abort_flag, status,
+                        q_scales, k_scales, scale_log2);
   } else {
-    // ---------------------------------------------------------- correction
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    float2 o2[D / 2];
-#pragma unroll
-    for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.f, 0.f);
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.a_full[j & 3], (j >> 2) & 1, abort_flag,
-                                             status, kDevTimeoutSoftmax))) {
-        ok = false;
-        break;
-      }
-      const float alpha = alpha_s[(j & 3) * 128 + r];
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.pv_full[b], (j >> 1) & 1, abort_flag, status,
-                                             kDevTimeoutMma))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t t[32];
-        tmem_ld32(lane_base + tPV(b) + cc * 32, t);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          o2[cc * 16 + i] = __ffma2_rn(
-              a2, o2[cc * 16 + i], make_float2(__uint_as_float(t[2 * i]), __uint_as_float(t[2 * i + 1])));
-      }
-      tc_fence_before();
-      mbar_arrive(&bar.pv_empty[b]);
-    }
-    if (ok && mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)) {
-      const float inv_l = 1.f / l_s[r];
-      const float* vs = v_scales + (int64_t)bh * D;
-      OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
-#pragma unroll
-      for (int c = 0; c < D; c += 8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 v = o2[c / 2 + e];
-          w[e] = pack2<OutT>(v.x * __ldg(vs + c + 2 * e) * inv_l,
-                             v.y * __ldg(vs + c + 2 * e + 1) * inv_l);
-        }
-        *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
+    setmaxnreg_inc<kRegsStats>();
+    stats_loop<D, CAUSAL, OutT>(qt, nkv, bh, N, ntiles, tmem, bar, smem, abort_flag, status,
+                                q_scales, k_scales, v_scales, out, scale_log2);
   }
 
   tc_fence_before();
@@ -431,7 +616,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 template <int D, bool CAUSAL, typename OutT>
 cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, cudaStream_t st) {
-  using L = I8F8Layout<D>;
+  using L = Layout<D>;
   auto kern = attn_i8f8_kernel<D, CAUSAL, OutT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
@@ -474,3 +659,9 @@ cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** de
 }
 
 }  // namespace sage
+
+#ifdef SAGE_TRACE
+extern "C" int sage_trace_read(long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, sage::g_sage_trace, sizeof(long long) * 16 * 512);
+}
+#endif
