@@ -138,6 +138,30 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
                   int64_t B, int64_t H, int64_t N, int64_t d,
                   int causal, float sm_scale, int mode, sage_stream_t stream);
 
+/* The same forward pass for callers that cannot allocate device memory
+ * while they run (a memory pool that admits no new allocations, an
+ * allocator that owns the whole device, a caller that may not take the
+ * driver's allocation locks).  The paper has no counterpart: this is a
+ * deployment variant of sage_attn_fwd.
+ *
+ * All scratch (codes, scales, statistics partials) lives in one fixed
+ * array of SAGE_NOALLOC_SCRATCH_BYTES inside the library's device image,
+ * reserved on every GPU that loads the library and held until the process
+ * exits; the call itself allocates and frees nothing.  The caller still
+ * passes Q, K, V and O as with sage_attn_fwd (same arguments, same result).
+ *   - A shape whose scratch exceeds the array is rejected with
+ *     SAGE_ERR_UNSUPPORTED and a message giving both sizes (about 3.1 bytes
+ *     per element of Q in INT8/FP8 mode: B*H*N*d up to about 21 million).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind: calls whose GPU work overlaps (different streams, or threads)
+ *     race on it and must be serialised by the caller. */
+#define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int dtype,
+                          int64_t B, int64_t H, int64_t N, int64_t d,
+                          int causal, float sm_scale, int mode, sage_stream_t stream);
+
 /* Reads and clears the device status word written by the kernels' bounded
  * waits (0 = none expired).  Synchronises the current device. */
 int sage_get_last_device_status(void);

@@ -18,7 +18,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_quantized",
+__all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
            "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,7 +32,8 @@ BUF = {name: i for i, name in enumerate(
 
 # every symbol include/sage.h declares
 EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd_quantized",
-           "sage_attn_fwd", "sage_get_last_device_status", "sage_status_string", "sage_version"]
+           "sage_attn_fwd", "sage_attn_fwd_noalloc", "sage_get_last_device_status",
+           "sage_status_string", "sage_version"]
 
 _lib = None
 
@@ -67,6 +68,9 @@ def library():
     lib.sage_attn_fwd.restype = i32
     lib.sage_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i32,
                                   ctypes.c_float, i32, vp]
+    lib.sage_attn_fwd_noalloc.restype = i32
+    lib.sage_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i32,
+                                          ctypes.c_float, i32, vp]
     lib.sage_get_last_device_status.restype = i32
     lib.sage_get_last_device_status.argtypes = []
     lib.sage_status_string.restype = ctypes.c_char_p
@@ -178,6 +182,25 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=Non
     if out is None:
         out = torch.empty_like(q)
     _check(library().sage_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, N, d,
+        int(bool(causal)), float(sm_scale or 0.0), MODES[mode], _stream()))
+    return out
+
+
+def sage_attn_fwd_noalloc(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None):
+    """sage_attn_fwd for callers that cannot allocate device memory while they
+    run: all scratch lives in the library's fixed per-device array (see
+    include/sage.h).  `out` should be passed (pre-allocated) by such callers;
+    calls that overlap on the GPU share the array and must be serialised."""
+    import torch
+    B, H, N, d = _shape(q)
+    if _shape(k) != (B, H, N, d) or _shape(v) != (B, H, N, d):
+        raise ValueError("q, k, v must have the same shape")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must have the same dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(library().sage_attn_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, N, d,
         int(bool(causal)), float(sm_scale or 0.0), MODES[mode], _stream()))
     return out

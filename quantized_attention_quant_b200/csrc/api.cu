@@ -416,3 +416,118 @@ const char* sage_status_string(int status) {
 const char* sage_version(void) { return "sage-b200 0.1 (sm_100a)"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of sage_attn_fwd.
+//
+// Some callers cannot allocate device memory at call time: code running
+// under a memory-pool policy that forbids new allocations, allocators that
+// own every byte of the device, or real-time callers that may not take the
+// driver's allocation locks.  For them the whole forward pass can run out of
+// one fixed scratch area that is part of the library's device image: a
+// file-scope array of kNoAllocScratchBytes, reserved on every GPU that loads
+// the library and held until the process exits.
+// ---------------------------------------------------------------------------
+
+namespace sage {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB per device
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device with that
+// device current (in host code the array's name is only a host-side stand-in,
+// never a device address).
+std::map<int, void*> g_noalloc_addr;
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_noalloc_addr.find(dev);
+  if (it != g_noalloc_addr.end()) {
+    *out = it->second;
+    return SAGE_OK;
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(no-allocation scratch)");
+  g_noalloc_addr[dev] = p;
+  *out = p;
+  return SAGE_OK;
+}
+
+}  // namespace
+}  // namespace sage
+
+static_assert(sage::kNoAllocScratchBytes == SAGE_NOALLOC_SCRATCH_BYTES,
+              "the header states the scratch size");
+
+extern "C" {
+
+int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int dtype,
+                          int64_t B, int64_t H, int64_t N, int64_t d, int causal, float sm_scale,
+                          int mode, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_ptr(q, "q", true));
+  SAGE_TRY(check_ptr(k, "k", true));
+  SAGE_TRY(check_ptr(v, "v", true));
+  SAGE_TRY(check_ptr(o, "o", true));
+  if (!(sm_scale > 0.f)) sm_scale = 1.0f / std::sqrt((float)d);
+  if (!std::isfinite(sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be finite");
+  if (empty) return SAGE_OK;
+  // scratch layout: every quantized buffer, then the statistics partials
+  size_t off[SAGE_BUF_V_SF + 1];
+  size_t total = 0;
+  for (int w = 0; w <= SAGE_BUF_V_SF; ++w) {
+    off[w] = total;
+    total += align_up(sage_buffer_bytes(mode, w, B, H, N, d));
+  }
+  const size_t off_ksum = total;
+  total += align_up(ws_ksum_bytes(B * H, N, d));
+  const size_t off_vmax = total;
+  total += align_up(ws_vmax_bytes(B * H, N, d));
+  if (total > kNoAllocScratchBytes) {
+    return fail(SAGE_ERR_UNSUPPORTED,
+                "this shape needs " + std::to_string(total) +
+                    " bytes of scratch; the no-allocation entry point has " +
+                    std::to_string(kNoAllocScratchBytes) + " (use sage_attn_fwd)");
+  }
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  void* ws = nullptr;
+  SAGE_TRY(noalloc_scratch(&ws));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(ws);
+  auto at = [&](int w) -> void* {
+    return sage_buffer_bytes(mode, w, B, H, N, d) ? base + off[w] : nullptr;
+  };
+  // Every scratch byte the kernels read is written earlier in the same call
+  // (codes, scales, statistics partials), so nothing needs clearing.
+  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d,
+                 at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+                 at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum)};
+  cudaError_t e = launch_quant_qk(qa, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
+  QuantVArgs va{v, dtype, mode, B, H, N, d,
+                at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+                reinterpret_cast<double*>(base + off_ksum),
+                reinterpret_cast<float*>(base + off_vmax)};
+  e = launch_quant_v(va, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
+  AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+              at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+              at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+              o, dtype, B, H, N, d, causal != 0, sm_scale, di->status};
+  const char* detail = nullptr;
+  e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
+  if (detail) return fail(SAGE_ERR_CUDA, detail);
+  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  return SAGE_OK;
+}
+
+}  // extern "C"
