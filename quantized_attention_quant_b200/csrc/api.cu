@@ -362,14 +362,12 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
                  at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
                  at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
                  (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum)};
-  cudaError_t e = launch_quant_qk(qa, st);
-  if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
   QuantVArgs va{v, dtype, mode, B, H, N, d,
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax)};
-  e = launch_quant_v(va, st);
-  if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
+  cudaError_t e = launch_prepass(qa, va, st);
+  if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
@@ -511,14 +509,12 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                  at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
                  at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
                  (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum)};
-  cudaError_t e = launch_quant_qk(qa, st);
-  if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
   QuantVArgs va{v, dtype, mode, B, H, N, d,
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax)};
-  e = launch_quant_v(va, st);
-  if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
+  cudaError_t e = launch_prepass(qa, va, st);
+  if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
