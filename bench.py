@@ -2,9 +2,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl sage|reference]
 
-One step = the whole hot path over one batch: the Q/K pre-pass, the V
-pre-pass and the fused attention kernel (the launches sage_attn_fwd makes),
-inputs resident in HBM.  L2 is flushed (a 256 MiB device write) between
+One step = the whole hot path over one batch: the Q/K pre-pass
+(sage_quant_qk), the V pre-pass (sage_quant_v) and the fused attention
+kernel (sage_attn_fwd_quantized), inputs resident in HBM.  L2 is flushed (a 256 MiB device write) between
 timed steps; each step is bracketed by CUDA events on the launching stream.
 Metric: effective TOPS = 4*B*H*N^2*d / t (summed over ranks; weak scaling,
 each rank processes its own batch of heads with no collective on the data
@@ -15,6 +15,7 @@ the host cores, on a bounded sample of the same workload per step.
 """
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -299,9 +300,13 @@ def read_traffic(workload):
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            t = json.load(f)
-        return t.get(workload)
-    except (OSError, ValueError):
+            entry = json.load(f).get(workload)
+        if not entry:
+            return None
+        with open(os.path.join(ROOT, entry["kernel_source"]), "rb") as f:
+            current = hashlib.sha256(f.read()).hexdigest()
+        return entry["bytes"] if current == entry["kernel_source_sha256"] else None
+    except (OSError, ValueError, KeyError):
         return None
 
 

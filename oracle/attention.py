@@ -120,6 +120,54 @@ def quant_p_fp4(pt):
     return (codes * s16[..., None]).reshape(R, C)
 
 
+def _e2m1_flip(t, eps):
+    """|neighbour - value| for the e2m1 code of t >= 0 where t lies within a
+    relative eps of a rounding midpoint (either code is then correct); 0
+    elsewhere."""
+    code = e2m1_encode(t).astype(np.int64) & 0x7
+    r = e2m1_decode(code)
+    up = e2m1_decode(np.minimum(code + 1, 7))
+    dn = e2m1_decode(np.maximum(code - 1, 0))
+    tol = eps * np.maximum(t, 2.0 ** -30)
+    near_up = (code < 7) & (np.abs(t - 0.5 * (r + up)) <= tol)
+    near_dn = (code > 0) & (np.abs(t - 0.5 * (r + dn)) <= tol)
+    return np.where(near_up, up - r, 0.0) + np.where(near_dn, r - dn, 0.0)
+
+
+def fp4_p_ambiguity(pt, eps):
+    """Bound on the change of the FP4 P~ values (in the units quant_p_fp4
+    returns: code * s16) when P~ is perturbed by a relative eps at most.
+
+    Two decisions can go either way near a midpoint: the UE4M3 group scale
+    s16 = ue4m3(448 amax16), which moves every value of the 16-key group,
+    and each e2m1 code.  Where the scale is ambiguous the bound covers the
+    whole group re-quantized with the neighbouring scale.
+    """
+    R, C = pt.shape
+    blk = pt.reshape(R, C // 16, 16)
+    x = blk.max(axis=-1) * P_FP8_SCALE
+    code = ue4m3_encode(x).astype(np.int64)
+    s = ue4m3_decode(code)
+    up = ue4m3_decode(np.minimum(code + 1, 0x7E))
+    dn = ue4m3_decode(np.maximum(code - 1, 0))
+    tol = eps * np.maximum(x, 2.0 ** -30)
+    near_up = (code < 0x7E) & (np.abs(x - 0.5 * (s + up)) <= tol)
+    near_dn = (code > 0) & (np.abs(x - 0.5 * (s + dn)) <= tol)
+
+    def values(scale):
+        den = scale * P_FP4_G
+        with np.errstate(divide="ignore", invalid="ignore"):
+            t = np.where(den[..., None] > 0, blk / np.where(den > 0, den, 1.0)[..., None], 0.0)
+        return e2m1_decode(e2m1_encode(t)) * scale[..., None], _e2m1_flip(t, eps) * scale[..., None]
+
+    base, bound = values(s)
+    for near, alt in ((near_up, up), (near_dn, dn)):
+        if np.any(near):
+            v_alt, b_alt = values(np.where(near, alt, s))
+            bound = bound + np.where(near[..., None], np.abs(v_alt - base) + b_alt, 0.0)
+    return bound.reshape(R, C)
+
+
 # --------------------------------------------------------------------------
 # The tile loop
 # --------------------------------------------------------------------------
@@ -188,9 +236,10 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     ``exact_attention`` up to FP64 rounding.
     rows: optional query-row indices; then O is [B, H, len(rows), d] and only
     those rows are computed (the pre-pass still sees every token).
-    ambiguity_eps: (INT8/FP8 mode) when given, also return a per-element bound
-    on how far O moves if every P~ code lying within this relative distance of
-    an e4m3 rounding midpoint takes its other (equally valid) value.
+    ambiguity_eps: when given, also return a per-element bound on how far O
+    moves if every P~ decision lying within this relative distance of a
+    rounding midpoint takes its other (equally valid) value: the e4m3 codes in
+    INT8/FP8 mode; the UE4M3 group scales and e2m1 codes in FP4 mode.
     """
     q = np.asarray(q, np.float32)
     k = np.asarray(k, np.float32)
@@ -236,6 +285,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
         return out if bound is None else (out, bound)
 
     if mode == "fp4":
+        bound = np.zeros_like(out) if ambiguity_eps is not None else None
+        amb = (lambda pt: fp4_p_ambiguity(pt, ambiguity_eps)) if bound is not None else None
         qk = pp.quant_qk_fp4(q, k)
         vc, vsf, vg = pp.quant_v_fp4(v)
         for b in range(B):
@@ -248,9 +299,13 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                 s_row = qk["q_g"][b, h].astype(np.float64)[tile_of]
                 s_key = qk["k_g"][b, h].astype(np.float64)[tile_of]
                 v_fold = (vg[b, h].astype(np.float64) * P_FP4_G)[:, None] * np.ones((1, d))
-                out[b, h] = _tile_loop(qd, kd, vdt.T, s_row, s_key, v_fold, quant_p_fp4,
-                                       causal, sm_scale, rows)
-        return out
+                res = _tile_loop(qd, kd, vdt.T, s_row, s_key, v_fold, quant_p_fp4,
+                                 causal, sm_scale, rows, amb)
+                if bound is None:
+                    out[b, h] = res
+                else:
+                    out[b, h], bound[b, h] = res
+        return out if bound is None else (out, bound)
     raise ValueError(mode)
 
 

@@ -6,7 +6,9 @@ Bars (floating point):
     which by itself moves a value by up to half an ulp) + the oracle's bound
     for P~ codes that lie within a relative 2^-15 of an e4m3 rounding
     midpoint (the kernel evaluates P~ in FP32, so either neighbouring code is
-    a correct result there; see oracle.attention.fp8_p_ambiguity);
+    a correct result there; see oracle.attention.fp8_p_ambiguity), and in
+    FP4 mode of an e2m1 midpoint or of a UE4M3 group-scale midpoint
+    (oracle.attention.fp4_p_ambiguity);
   * cosine(O_gpu, O_exact) >= 0.999 where the quantization scheme itself
     reaches it on the workload, and never more than 2e-4 below the
     emulated oracle's own cosine.
@@ -44,12 +46,8 @@ def cosine(a, b):
 
 def check_against_oracle(o_gpu, q, k, v, causal, sm_scale, mode, dtype, rows=None, cos_floor=None):
     qs, ks, vs = (to_numpy32(t) for t in (q, k, v))
-    if mode == "int8_fp8":
-        emu, amb = att.emulated_sage_attention(qs, ks, vs, causal, sm_scale, mode=mode, rows=rows,
-                                               ambiguity_eps=AMBIGUITY_EPS)
-    else:
-        emu = att.emulated_sage_attention(qs, ks, vs, causal, sm_scale, mode=mode, rows=rows)
-        amb = 0.0
+    emu, amb = att.emulated_sage_attention(qs, ks, vs, causal, sm_scale, mode=mode, rows=rows,
+                                           ambiguity_eps=AMBIGUITY_EPS)
     ex = att.exact_attention(qs, ks, vs, causal, sm_scale, rows=rows)
     g = o_gpu.astype(np.float64)
     err = np.abs(g - emu)
@@ -74,6 +72,41 @@ def test_int8_fp8_random(cuda_device, N, dtype, d, causal):
     o = sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, mode="int8_fp8")
     torch.cuda.synchronize()
     check_against_oracle(to_numpy32(o), q, k, v, causal, 1 / math.sqrt(d), "int8_fp8", dtype)
+    assert sage.device_status() == 0
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("N", [128, 512])
+def test_fp4_random(cuda_device, N, dtype, causal):
+    q, k, v = rand_qkv(2, 2, N, 128, dtype, seed=300 + N + causal)
+    o = sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, mode="fp4")
+    torch.cuda.synchronize()
+    check_against_oracle(to_numpy32(o), q, k, v, causal, 1 / math.sqrt(128), "fp4", dtype)
+    assert sage.device_status() == 0
+
+
+def test_fp4_zero_q_gives_mean_v(cuda_device):
+    # Q = 0 -> every score 0 -> P~ = 1 -> s16 = 448, code e2m1(6) = 6, whose
+    # value 6 * 448 / 2688 is exactly 1 -> O = mean of the FP4-dequantized V
+    # (prefix means when causal).  Exercises the FP4 P~V path and its
+    # scale factors in closed form.
+    B, H, N, d = 1, 2, 512, 128
+    _, k, v = rand_qkv(B, H, N, d, "bf16", seed=6)
+    q = torch.zeros_like(k)
+    from oracle import prepass as pp
+    vc, vsf, vg = pp.quant_v_fp4(to_numpy32(v))
+    # [B, H, d, N] values -> [B, H, N, d]
+    tile_of = np.arange(N) // 128
+    vd = (enc.e2m1_decode(vc) * np.repeat(enc.ue4m3_decode(vsf), 16, axis=-1)
+          * vg[:, :, None, tile_of]).transpose(0, 1, 3, 2)
+    for causal in (False, True):
+        o = to_numpy32(sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, mode="fp4"))
+        if causal:
+            want = np.cumsum(vd, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+        else:
+            want = np.broadcast_to(vd.mean(axis=2, keepdims=True), vd.shape)
+        assert np.max(np.abs(o - want) - half_ulp(want, "bf16") - 1e-5) <= 0
     assert sage.device_status() == 0
 
 
@@ -126,7 +159,7 @@ def test_fwd_equals_prepass_plus_attention(cuda_device):
     q, k, v = rand_qkv(1, 4, 384, 128, "bf16", seed=9)
     dev = torch.device("cuda")
     qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
-    for mode in ["int8_fp8"]:
+    for mode in ["int8_fp8", "fp4"]:
         a = sage.sage_attn_fwd(qg, kg, vg, causal=True, mode=mode)
         qk = sage.sage_quant_qk(qg, kg, mode)
         vq = sage.sage_quant_v(vg, mode)
@@ -147,11 +180,12 @@ def test_side_stream(cuda_device):
     assert torch.equal(ref, out)
 
 
-FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", None), ("long_causal", None)]
+FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", None), ("long_causal", None),
+        ("fp4", None)]
 
 
 @pytest.mark.parametrize("name,cos_floor", FULL)
-def test_int8_fp8_full_workloads(cuda_device, name, cos_floor):
+def test_full_workloads(cuda_device, name, cos_floor):
     """Full-size launch (as timed by bench.py); sampled heads and rows."""
     w = WORKLOADS[name]
     q, k, v = make_qkv(w)

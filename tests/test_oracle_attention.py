@@ -354,3 +354,43 @@ def test_ambiguity_bound_covers_flipped_codes():
         att.quant_p_fp8 = base
     assert moved == 2
     assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.3), o)
+
+
+def test_fp4_p_ambiguity_marks_midpoints():
+    # one row of two 16-key groups:
+    #   group 0: amax = 1 (s16 = 448, a grid value, unambiguous); 6 P~ = 2.5 is
+    #            an e2m1 midpoint (2|3), so that value may move by 1 * s16;
+    #            6 P~ = 0.6 and 6 P~ = 4.2 are far from any midpoint
+    #   group 1: 448 amax = 17 lies between e4m3 16 and 18: the scale itself is
+    #            ambiguous, and the bound covers the group re-quantized
+    row = np.zeros((1, 32))
+    row[0, 0], row[0, 1], row[0, 2], row[0, 3] = 1.0, 2.5 / 6, 0.1, 0.7
+    row[0, 16], row[0, 17] = 17.0 / 448, 5.0 / 448
+    b = att.fp4_p_ambiguity(row, 1e-6)
+    assert b[0, 1] == 448.0
+    assert np.all(b[0, [0, 2, 3]] == 0) and np.all(b[0, 4:16] == 0)
+    # group 1 with s16 = 16 or 18 (g = 1/2688): the element at 17/448 codes to
+    # 6 * 17/16 -> 6 (sat) * 16 = 96 or 6 * 17/18 -> 6 * 18 = 108
+    base = att.quant_p_fp4(row)
+    assert base[0, 16] in (96.0, 108.0)
+    assert b[0, 16] >= 12.0
+    assert np.all(b[0, 18:] == 0)
+
+
+def test_fp4_ambiguity_bound_covers_flipped_codes():
+    # FP4 mode: a relative 1e-4 perturbation of P~ before quantization moves O
+    # by no more than the bound, and does move it.
+    q, k, v = rnd((1, 1, 256, 32), 80, 2.0), rnd((1, 1, 256, 32), 81, 2.0), rnd((1, 1, 256, 32), 82)
+    o, bnd = att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp4", ambiguity_eps=1e-4)
+    base = att.quant_p_fp4
+    moved = 0
+    try:
+        for sgn in (+1, -1):
+            att.quant_p_fp4 = lambda pt, s=sgn: base(pt * (1 + s * 1e-4))
+            o2 = att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp4")
+            assert np.all(np.abs(o2 - o) <= bnd + 1e-12)
+            moved += int(np.any(o2 != o))
+    finally:
+        att.quant_p_fp4 = base
+    assert moved == 2
+    assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp4"), o)
