@@ -121,6 +121,34 @@ def rank_workload(w, rank):
     return w.with_(seed=w.seed + 1000 * rank)
 
 
+def config_of(w, world):
+    """The JSON `config` of a run: the workload one rank processes, and the
+    job-wide head count (weak scaling: every rank its own batch of heads)."""
+    return {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} "
+                        f"{'causal' if w.causal else 'non-causal'} {w.dtype} {w.mode}",
+            "global_batch_heads": w.B * w.H * world, "seq_len": w.N, "head_dim": w.d,
+            "causal": w.causal, "input_dtype": w.dtype, "mode": w.mode,
+            "l2": "flushed between timed steps (256 MiB device write)",
+            "parallelism": f"dp{world} (heads sharded by batch, no collective)"}
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of a list of floats over all ranks (identity at
+    world 1).  Every rank must call it, in the same order."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(ops_per_rank, world, t_ms):
+    """Whole-job TOPS: the work of all ranks over the slowest rank's time."""
+    return ops_per_rank * world / (t_ms * 1e-3) / 1e12
+
+
 def run_sage(args):
     import ctypes
 
@@ -239,15 +267,11 @@ def run_sage(args):
     t_step = sum(step_ms) / len(step_ms)
     t_attn = sum(attn_ms) / len(attn_ms)
     t_e2e = sum(e2e_ms) / len(e2e_ms)
-    if world > 1:
-        tt = torch.tensor([t_step, t_attn, t_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, t_attn, t_e2e = tt.tolist()
+    t_step, t_attn, t_e2e = max_over_ranks([t_step, t_attn, t_e2e], world, dev)
 
     heads = B * H
-    eff_ops = w.ops * world                             # 4 B H N^2 d, all ranks
-    value = eff_ops / (t_step * 1e-3) / 1e12
-    e2e_val = eff_ops / (t_e2e * 1e-3) / 1e12
+    value = job_throughput(w.ops, world, t_step)        # 4 B H N^2 d, all ranks
+    e2e_val = job_throughput(w.ops, world, t_e2e)
     peaks, src = measured_peaks()
     ratio = 4.0 if w.mode == "fp4" else 2.0             # vs bf16, nominal dense ratios
     peak = peaks["bf16_tflops"] * ratio
@@ -267,12 +291,7 @@ def run_sage(args):
         "vs_baseline": None,
         "dtype": "fp4e2m1" if w.mode == "fp4" else "int8+fp8e4m3",
         "data": "synthetic",
-        "config": {"workload": f"{w0.name}: B={B} H={H} N={N} d={d} "
-                               f"{'causal' if w.causal else 'non-causal'} {w.dtype} {w.mode}",
-                   "global_batch_heads": heads * world, "seq_len": N, "head_dim": d,
-                   "causal": w.causal, "input_dtype": w.dtype, "mode": w.mode,
-                   "l2": "flushed between timed steps (256 MiB device write)",
-                   "parallelism": f"dp{world} (heads sharded by batch, no collective)"},
+        "config": config_of(w0, world),
         "attn_kernel_ms": round(t_attn, 4),
         "prepass_ms": round(t_step - t_attn, 4),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
@@ -381,8 +400,7 @@ def run_reference(args):
         "value": round(value, 6), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} "
-                               f"{'causal' if w.causal else 'non-causal'} {w.dtype} {w.mode}"},
+        "config": config_of(w, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,

@@ -18,25 +18,34 @@
 //
 // One CTA owns one 128-row query tile of one (b, h).  The exponentials are
 // the throughput limit (the tensor core finishes a 128x128 tile in far fewer
-// cycles than the SFU needs for its 16K exponentials, and one warp per SM
-// sub-partition keeps the SFU only about half busy), so two warpgroups share
-// every tile.  Warp roles (512 threads):
+// cycles than the SFU needs for its 16K exponentials; one warp per SM
+// sub-partition keeps the SFU only about half busy, two about 80 %), so two
+// warpgroups share every tile.  The scores stay biased floats end to end:
+// an integer add or an int-to-float conversion per score costs the exp
+// pass about a third of its SFU rate.  Warp roles (512 threads):
 //   warpgroup 0: warp 0 TMA producer (Q once, K_j and V_j^T rings),
 //                warp 1 TMEM allocator and single-thread tcgen05 issuer
 //   warpgroups 1, 2 ("exp"): key columns 0..63 / 64..127 of every tile.
-//                Thread = query row = TMEM lane.  448 P~, e4m3 codes into a
-//                swizzled shared-memory tile (the A operand of the P~V MMA),
+//                Thread = query row = TMEM lane.  448 P~ as e4m3 codes into
+//                a TMEM tile (the A operand of the P~V MMA, read from TMEM),
 //                the row sum, and the bias written back into S.
 //   warpgroup 3 ("stats"): per key tile the row max, the running max m_j and
 //                alpha_j (published for both exp warpgroups), then the level-2
 //                fold of the tile's FP32 partial into the running FP32
 //                accumulator (registers); finally normalise and store O.
-// TMEM columns: S[0] 0..127, S[1] 128..255 (key tile j uses S[j % 2]),
-// PV[0] 256.., PV[1] 256+D.. .  Before each Q K^T the S columns hold the bit
-// pattern of 1.5 * 2^23; the INT8 MMA accumulates onto it, so a score reads
-// back as the float 1.5*2^23 + A exactly (|A| <= 127^2*128 < 2^22) with no
-// conversion instruction.  Every barrier wait is bounded; an expired wait
-// sets the device status word and makes every role leave its loop.
+// TMEM columns: d = 128: S 0..127 (one buffer), PV[0] 128.., PV[1] 256..;
+// d = 64: S[0] 0..127, S[1] 128..255, PV[0] 256.., PV[1] 320..; both:
+// P~[0] 384..415, P~[1] 416..447 (four e4m3 codes per column, keys
+// 64h .. 64h+63 in columns 16h .. 16h+15).  Key tile j uses S[j % SB],
+// PV[j % 2] (folded two tiles behind) and P~[j % 2].  The exp warpgroups
+// read their S columns first, write the bias back and release S at once,
+// so the next Q K^T runs while they work on the exponentials; the MMA
+// thread issues it ahead of the P~V of the previous tile.  Before each
+// Q K^T the S columns hold the bit pattern of 1.5 * 2^23; the INT8 MMA
+// accumulates onto it, so a score reads back as the float
+// 1.5*2^23 + A exactly (|A| <= 127^2*128 < 2^22) with no conversion
+// instruction.  Every barrier wait is bounded; an expired wait sets the
+// device status word and makes every role leave its loop.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -49,13 +58,17 @@ namespace sage {
 // Optional timeline trace (builds with -DSAGE_TRACE only): %clock64 of
 // selected events of one steady-state CTA, read back by sage_trace_read.
 #ifdef SAGE_TRACE
+// Timestamps go to shared memory while the kernel runs (a global store would
+// make the next release-arrive wait for it) and are copied out at the end.
 __device__ long long g_sage_trace[16][512];
+__shared__ long long s_sage_trace[16][64];
+#define SAGE_TRACED_CTA (blockIdx.x == 7 && blockIdx.y == 1)
 #define SAGE_TR(ev, j)                                                                  \
   do {                                                                                  \
-    if (blockIdx.x == 7 && blockIdx.y == 1 && (j) < 512) {                              \
+    if (SAGE_TRACED_CTA && (j) < 64) {                                                  \
       long long t_;                                                                     \
       asm volatile("mov.u64 %0, %%clock64;" : "=l"(t_));                                \
-      g_sage_trace[ev][j] = t_;                                                         \
+      s_sage_trace[ev][j] = t_;                                                         \
     }                                                                                   \
   } while (0)
 #else
@@ -79,26 +92,29 @@ constexpr uint32_t kRegsStats = 216;
 
 template <int D>
 struct Layout {
-  static constexpr int KS = D == 128 ? 3 : 5;  // K ring depth
-  static constexpr int VS = D == 128 ? 3 : 5;  // V ring depth
+  static constexpr int KS = D == 128 ? 4 : 6;  // K ring depth
+  static constexpr int VS = D == 128 ? 4 : 6;  // V ring depth
   static constexpr int Q_BYTES = 128 * D;
   static constexpr int K_BYTES = 128 * D;
   static constexpr int V_BYTES = D * 128;
-  static constexpr int P_BYTES = 128 * 128;  // e4m3 P~ tile, 128-byte swizzled rows
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KS * K_BYTES;
-  static constexpr int OFF_P = OFF_V + VS * V_BYTES;
-  static constexpr int OFF_MISC = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_MISC = OFF_V + VS * V_BYTES;
   static constexpr int OFF_BAR = OFF_MISC;           // barriers (<= 64 x 8 B)
   static constexpr int OFF_TMEM = OFF_MISC + 512;
   static constexpr int OFF_ABORT = OFF_MISC + 528;
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
-  static constexpr int END = OFF_L + 2 * 128 * 4;
+  static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots] dequant factor of the tile
+  static constexpr int END = OFF_C + 16;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t QK_SBO = 8 * D;  // 8 rows of D bytes
+  static constexpr int SB = D == 128 ? 1 : 2;    // S buffers
+  static constexpr int PVB = 2;                  // level-1 partial buffers
+  static constexpr uint32_t COL_PV = 128 * SB;   // PV[b] at COL_PV + D b
+  static constexpr uint32_t COL_P = 384;         // P~[b] at COL_P + 32 b
   static constexpr Swz QK_SWZ = D == 128 ? Swz::k128 : Swz::k64;
 };
 
@@ -108,13 +124,14 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;
   uint64_t* v_empty;
-  uint64_t* s_full;    // [2] MMA -> stats, exp: S[b] holds Q K_j^T
+  uint64_t* s_init;    // [1] exp -> MMA: the S buffers hold the bias
+  uint64_t* s_full;    // [SB] MMA -> stats: S[b] holds bias + Q K_j^T
+  uint64_t* s_ready;   // [SB] exp -> MMA: S[b] read and re-biased
   uint64_t* m_full;    // [2] stats -> exp: m_j, alpha_j of tile j (slot j % 2)
-  uint64_t* s_ready;   // [2] exp -> MMA: S[b] read and re-biased (both halves)
-  uint64_t* p_full;    // [2] exp -> MMA: P~ tile b written (both halves)
-  uint64_t* p_empty;   // [2] MMA -> exp: P~ tile b read by the P~V MMA
-  uint64_t* pv_full;   // [2] MMA -> stats: PV[b] holds tile j's partial
-  uint64_t* pv_empty;  // [2] stats -> MMA: PV[b] read
+  uint64_t* p_full;    // [2] exp -> MMA: P~[b] written
+  uint64_t* p_empty;   // [2] MMA -> exp: P~[b] read by the P~V MMA
+  uint64_t* pv_full;   // [PVB] MMA -> stats: PV[b] holds a tile's partial
+  uint64_t* pv_empty;  // [PVB] stats -> MMA: PV[b] read
   uint64_t* l_ready;   // [1] exp -> stats: final row sums
   uint64_t* drain;     // MMA drain on abort
 };
@@ -129,14 +146,15 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.k_empty = r.k_full + L::KS;
   r.v_full = r.k_empty + L::KS;
   r.v_empty = r.v_full + L::VS;
-  r.s_full = r.v_empty + L::VS;
-  r.m_full = r.s_full + 2;
-  r.s_ready = r.m_full + 2;
-  r.p_full = r.s_ready + 2;
+  r.s_init = r.v_empty + L::VS;
+  r.s_full = r.s_init + 1;
+  r.s_ready = r.s_full + L::SB;
+  r.m_full = r.s_ready + L::SB;
+  r.p_full = r.m_full + 2;
   r.p_empty = r.p_full + 2;
   r.pv_full = r.p_empty + 2;
-  r.pv_empty = r.pv_full + 2;
-  r.l_ready = r.pv_empty + 2;
+  r.pv_empty = r.pv_full + L::PVB;
+  r.l_ready = r.pv_empty + L::PVB;
   r.drain = r.l_ready + 1;
   return r;
 }
@@ -167,21 +185,26 @@ __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
       : "memory");
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
+// Global load the compiler keeps where it is written (a plain load of a
+// value needed only in the next loop iteration may be sunk to the end of
+// the current one, exposing its latency at the top of the next).
+__device__ __forceinline__ float ldg_early(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
 }
 
-// Max of 64 biased scores (as float bits) and a running value.  MASKED:
-// columns col0 + i > r are ignored (causal diagonal tile).
+// A score as read from TMEM: the float 1.5 * 2^23 + A (exact).
+__device__ __forceinline__ float biased(uint32_t a) { return __uint_as_float(a); }
+
+// Max of 64 biased scores and a running value.  MASKED: columns col0 + i > r
+// are ignored (causal diagonal tile).
 template <bool MASKED>
 __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float acc) {
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    float x = __uint_as_float(s[k]), y = __uint_as_float(s[k + 8]);
+    float x = biased(s[k]), y = biased(s[k + 8]);
     if (MASKED) {
       x = (col0 + k <= r) ? x : 0.f;
       y = (col0 + k + 8 <= r) ? y : 0.f;
@@ -192,7 +215,7 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
   for (int i = 16; i < 64; i += 16)
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      float x = __uint_as_float(s[i + k]), y = __uint_as_float(s[i + 8 + k]);
+      float x = biased(s[i + k]), y = biased(s[i + 8 + k]);
       if (MASKED) {
         x = (col0 + i + k <= r) ? x : 0.f;
         y = (col0 + i + 8 + k <= r) ? y : 0.f;
@@ -202,8 +225,8 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
   return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], acc));
 }
 
-// 448 P~ for 32 biased scores of a row -> 8 words of e4m3 codes (key i in
-// byte i % 4) and the sum of the unquantized values.
+// 448 P~ for 32 scores of a row -> 8 words of e4m3 codes (key i in byte
+// i % 4 of word i / 4) and the sum of the unquantized values.
 template <bool MASKED>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
                                              int r, uint32_t (&p)[8]) {
@@ -213,9 +236,9 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
-    const float2 x01 = __fadd2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), mb);
-    const float2 x23 =
-        __fadd2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), mb);
+    // (1.5*2^23 + A) - 1.5*2^23 = A exactly
+    const float2 x01 = __fadd2_rn(make_float2(biased(s[i]), biased(s[i + 1])), mb);
+    const float2 x23 = __fadd2_rn(make_float2(biased(s[i + 2]), biased(s[i + 3])), mb);
     const float2 t01 = __ffma2_rn(x01, c2, n2);
     const float2 t23 = __ffma2_rn(x23, c2, n2);
     float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
@@ -246,29 +269,23 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// One 32-column chunk of the exp pass: quantized P~ to shared memory, bias
-// back into the chunk's S columns, returns the chunk's row sum.
+// One 32-key chunk cc (0..3) of the exp pass: its e4m3 codes go to the 8
+// TMEM columns pcol (four keys per column, the A-operand layout of the
+// P~V MMA); returns the chunk's row sum.
 template <bool MASKED>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int cc, float c, float neg,
-                                           int r, uint32_t S, uint32_t prow) {
+                                           int r, uint32_t pcol) {
   uint32_t p[8];
   const float sum = exp_quant32<MASKED>(s, c, neg, 32 * cc, r, p);
-  // row r of the 128-byte-swizzled P~ tile: 16-byte chunk q lands at q ^ (r & 7)
-  const uint32_t q0 = (uint32_t)(2 * cc), sw = (uint32_t)(r & 7);
-  st_shared_v4(prow + (((q0) ^ sw) << 4), p[0], p[1], p[2], p[3]);
-  st_shared_v4(prow + (((q0 + 1) ^ sw) << 4), p[4], p[5], p[6], p[7]);
-  tmem_fill32(S + 32 * cc, kBiasBits);
+  tmem_st8(pcol, p);
   return sum;
 }
 
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
 template <int D, bool CAUSAL>
-__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int bh,
-                                         const int ntiles, const uint32_t tmem, const Bars& bar,
-                                         uint8_t* smem, volatile int* abort_flag,
-                                         uint32_t* status, const float* __restrict__ q_scales,
-                                         const float* __restrict__ k_scales,
-                                         const float scale_log2) {
+__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv,
+                                         const uint32_t tmem, const Bars& bar, uint8_t* smem,
+                                         volatile int* abort_flag, uint32_t* status) {
   using L = Layout<D>;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -276,60 +293,67 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
   const int r = quarter * 32 + lane;
   const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
   const float* m_s = reinterpret_cast<const float*>(smem + L::OFF_M);
+  const float* c_s = reinterpret_cast<const float*>(smem + L::OFF_C);
   float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
 
   // the first Q K^T into each S buffer accumulates onto the bias
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
+  for (int b = 0; b < L::SB; ++b) {
     tmem_fill32(tmem + lanes + 128u * b + 64u * h, kBiasBits);
     tmem_fill32(tmem + lanes + 128u * b + 64u * h + 32u, kBiasBits);
   }
   tmem_wait_st();
   tc_fence_before();
-  mbar_arrive(&bar.s_ready[0]);
-  mbar_arrive(&bar.s_ready[1]);
+  mbar_arrive(bar.s_init);
 
-  const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
-  const float* ksp = k_scales + (int64_t)bh * ntiles;
   float l = 0.f;
-  float ks_next = __ldg(ksp);
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
     const uint32_t ph = (j >> 1) & 1;
-    const float c = qs * ks_next * scale_log2;
-    if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
+    if (r == 0 && h == 0) SAGE_TR(12, j);
+    // m_full(j) is published by the stats warpgroup after it waited for
+    // s_full(j) and read S[b]: it orders this warpgroup after the Q K^T too
     if (!__all_sync(0xffffffffu,
-                    mbar_wait(&bar.s_full[b], ph, abort_flag, status, kDevTimeoutMma) &&
-                        mbar_wait(&bar.m_full[b], ph, abort_flag, status, kDevTimeoutEpi)))
+                    mbar_wait(&bar.m_full[b], ph, abort_flag, status, kDevTimeoutEpi)))
       return;
     tc_fence_after();
     if (r == 0) SAGE_TR(h, j);
+    const float c = c_s[b];
     const float m_j = m_s[(2 * b) * 128 + r];
     const float alpha = m_s[(2 * b + 1) * 128 + r];
     const float neg = kLog2_448 - m_j;  // yields 448 P~ directly
     const bool diag = CAUSAL && (j == qt);
-    const uint32_t S = tmem + lanes + 128u * b + 64u * h;
+    const int sbuf = j % L::SB;
+    const uint32_t S = tmem + lanes + 128u * sbuf + 64u * h;
+    const uint32_t P = tmem + lanes + L::COL_P + 32u * b + 16u * h;
     uint32_t sa[32], sb[32];
     tmem_ld32(S, sa);
     tmem_ld32(S + 32, sb);
-    // P~ tile b is free once the P~V MMA of tile j - 2 has read it
+    tmem_wait_ld_regs(sa);
+    reg_fence(sb);
+    if (r == 0 && h == 0) SAGE_TR(13, j);
+    // S read: the bias back, and S free for the next Q K^T into it
+    tmem_fill32(S, kBiasBits);
+    tmem_fill32(S + 32, kBiasBits);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&bar.s_ready[sbuf]);
+    // P~[b] is free once the P~V MMA of tile j - 2 has read it
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    const uint32_t prow = smem_u32(smem + L::OFF_P + b * L::P_BYTES + r * 128);
-    tmem_wait_ld_regs(sa);
-    reg_fence(sb);
-    float sum = diag ? exp_chunk<true>(sa, 2 * h, c, neg, r, S - 32u * (2 * h), prow)
-                     : exp_chunk<false>(sa, 2 * h, c, neg, r, S - 32u * (2 * h), prow);
-    sum += diag ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, S - 32u * (2 * h), prow)
-                : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, S - 32u * (2 * h), prow);
+    float sum = diag ? exp_chunk<true>(sa, 2 * h, c, neg, r, P)
+                     : exp_chunk<false>(sa, 2 * h, c, neg, r, P);
+    if (r == 0 && h == 0) SAGE_TR(14, j);
+    sum += diag ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, P + 8)
+                : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, P + 8);
     l = fmaf(alpha, l, sum);
+    if (r == 0 && h == 0) SAGE_TR(10, j);
     tmem_wait_st();
     tc_fence_before();
     if (r == 0) SAGE_TR(2 + h, j);
-    mbar_arrive(&bar.s_ready[b]);   // S[b] free for Q K_{j+2}^T
-    fence_proxy_async_smem();       // P~ stores visible to the tensor core
     mbar_arrive(&bar.p_full[b]);
+    if (r == 0 && h == 0) SAGE_TR(11, j);
   }
   l_s[h * 128 + r] = l;
   mbar_arrive(bar.l_ready);
@@ -361,13 +385,13 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   for (int c = 0; c < D / 2; ++c) o2[c] = make_float2(0.f, 0.f);
   float m = -INFINITY;
   auto fold = [&](int i, float alpha) -> bool {
-    const int b = i & 1;
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.pv_full[b], (i >> 1) & 1, abort_flag, status,
+    const int b = i % L::PVB;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.pv_full[b], (i / L::PVB) & 1, abort_flag, status,
                                            kDevTimeoutMma)))
       return false;
     tc_fence_after();
     if (r == 0) SAGE_TR(6, i);
-    const uint32_t PV = tmem + lanes + 256u + (uint32_t)b * (uint32_t)D;
+    const uint32_t PV = tmem + lanes + L::COL_PV + (uint32_t)b * (uint32_t)D;
     const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -385,21 +409,23 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     return true;
   };
 
-  // The fold lags the max by two tiles, so the max of tile j + 1 (which the
+  // The fold lags the max by PVB tiles, so the max of tile j + 1 (which the
   // exp warpgroups wait for) never queues behind the P~V product of tile j.
   float alpha_hist[2] = {0.f, 0.f};
-  float ks_next = __ldg(ksp);
+  float* c_s = reinterpret_cast<float*>(smem + L::OFF_C);
+  float ks_cur = ldg_early(ksp);
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
-    const float c = qs * ks_next * scale_log2;
-    if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], (j >> 1) & 1, abort_flag, status,
-                                           kDevTimeoutMma)))
+    const float c = qs * ks_cur * scale_log2;
+    const float ks_nxt = j + 1 < nkv ? ldg_early(ksp + j + 1) : 0.f;
+    const int sbuf = j % L::SB;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[sbuf], (j / L::SB) & 1, abort_flag,
+                                           status, kDevTimeoutMma)))
       return;
     tc_fence_after();
     if (r == 0) SAGE_TR(4, j);
     const bool diag = CAUSAL && (j == qt);
-    const uint32_t S = tmem + lanes + (uint32_t)b * 128u;
+    const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
     float mx = 0.f;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -415,13 +441,17 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     m = m_j;
     m_s[(2 * b) * 128 + r] = m_j;
     m_s[(2 * b + 1) * 128 + r] = alpha;
+    if (r == 0) c_s[b] = c;
     if (r == 0) SAGE_TR(5, j);
+    // S[b] has been read: the exp warpgroups may overwrite it with P~ codes
+    tc_fence_before();
     mbar_arrive(&bar.m_full[b]);
-    if (j > 1 && !fold(j - 2, alpha_hist[b])) return;
-    alpha_hist[b] = alpha;
+    if (j >= L::PVB && !fold(j - L::PVB, alpha_hist[j % L::PVB])) return;
+    alpha_hist[j % L::PVB] = alpha;
+    ks_cur = ks_nxt;
   }
-  for (int i = nkv > 2 ? nkv - 2 : 0; i < nkv; ++i)
-    if (!fold(i, alpha_hist[i & 1])) return;
+  for (int i = nkv > L::PVB ? nkv - L::PVB : 0; i < nkv; ++i)
+    if (!fold(i, alpha_hist[i % L::PVB])) return;
   if (!__all_sync(0xffffffffu,
                   mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)))
     return;
@@ -472,15 +502,20 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       mbar_init(&bar.v_full[i], 1);
       mbar_init(&bar.v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < L::SB; ++i) {
       mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.m_full[i], 128);
       mbar_init(&bar.s_ready[i], 256);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.m_full[i], 128);
       mbar_init(&bar.p_full[i], 256);
       mbar_init(&bar.p_empty[i], 1);
+    }
+    for (int i = 0; i < L::PVB; ++i) {
       mbar_init(&bar.pv_full[i], 1);
       mbar_init(&bar.pv_empty[i], 128);
     }
+    mbar_init(bar.s_init, 256);
     mbar_init(bar.l_ready, 256);
     mbar_init(bar.drain, 1);
     *abort_flag = 0;
@@ -503,7 +538,6 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
-  uint8_t* sP = smem + L::OFF_P;
 
   const int wg = warp >> 2;
   if (wg == 0) {
@@ -536,56 +570,71 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         constexpr uint32_t idesc_pv = make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, D);
         const uint64_t qdesc = make_sdesc(smem_u32(sQ), L::QK_SBO, 16, L::QK_SWZ);
         bool ok = mbar_wait(bar.q_full, 0, abort_flag, status, kDevTimeoutTma);
-        // S[j % 2] = Q K_j^T (onto the bias)
+        // S[j % SB] = bias + Q K_j^T
         auto qk = [&](int j) -> bool {
           const int sk = j % L::KS;
-          const int b = j & 1;
-          if (!mbar_wait(&bar.k_full[sk], (j / L::KS) & 1, abort_flag, status, kDevTimeoutTma) ||
-              !mbar_wait(&bar.s_ready[b], (j >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax))
+          const int sbuf = j % L::SB;
+          if (!mbar_wait(&bar.k_full[sk], (j / L::KS) & 1, abort_flag, status, kDevTimeoutTma))
             return false;
           tc_fence_after();
           SAGE_TR(8, j);
-          const uint64_t kdesc = make_sdesc(smem_u32(sK + sk * L::K_BYTES), L::QK_SBO, 16, L::QK_SWZ);
+          const uint64_t kdesc =
+              make_sdesc(smem_u32(sK + sk * L::K_BYTES), L::QK_SBO, 16, L::QK_SWZ);
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(tmem + (uint32_t)b * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
-          mma_commit(&bar.s_full[b]);
+            mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
+          mma_commit(&bar.s_full[sbuf]);
           mma_commit(&bar.k_empty[sk]);
           return true;
         };
-        if (ok) ok = qk(0);
-        if (ok && nkv > 1) ok = qk(1);
-        for (int i = 0; ok && i < nkv; ++i) {
-          // the exp warpgroups are done with tile i: first the next Q K^T into
-          // the freed S buffer, then P~_i V_i into PV[i % 2] (level 1)
+        // P~_i V_i into PV[i % 2] (level 1)
+        auto pv = [&](int i) -> bool {
           const int b = i & 1;
-          if (!mbar_wait(&bar.p_full[b], (i >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax)) {
-            ok = false;
-            break;
-          }
-          SAGE_TR(10, i);
-          if (i + 2 < nkv && !qk(i + 2)) {
-            ok = false;
-            break;
-          }
           const int sv = i % L::VS;
-          if (!mbar_wait(&bar.v_full[sv], (i / L::VS) & 1, abort_flag, status, kDevTimeoutTma) ||
-              !mbar_wait(&bar.pv_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, status,
-                         kDevTimeoutEpi)) {
-            ok = false;
-            break;
-          }
+          const int pb = i % L::PVB;
+          if (!mbar_wait(&bar.p_full[b], (i >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax) ||
+              !mbar_wait(&bar.v_full[sv], (i / L::VS) & 1, abort_flag, status, kDevTimeoutTma) ||
+              !mbar_wait(&bar.pv_empty[pb], ((i / L::PVB) & 1) ^ 1, abort_flag, status,
+                         kDevTimeoutEpi))
+            return false;
           tc_fence_after();
           SAGE_TR(9, i);
-          const uint64_t pdesc = make_sdesc(smem_u32(sP + b * L::P_BYTES), 1024, 16, Swz::k128);
           const uint64_t vdesc = make_sdesc(smem_u32(sV + sv * L::V_BYTES), 1024, 16, Swz::k128);
-          const uint32_t d = tmem + 256u + (uint32_t)b * (uint32_t)D;
+          const uint32_t d = tmem + L::COL_PV + (uint32_t)pb * (uint32_t)D;
+          const uint32_t pa = tmem + L::COL_P + 32u * (uint32_t)b;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) mma_f8_ss(d, pdesc + 2 * kk, vdesc + 2 * kk, idesc_pv, kk > 0);
-          mma_commit(&bar.pv_full[b]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ts(d, pa + 8u * kk, vdesc + 2 * kk, idesc_pv, kk > 0);
+          mma_commit(&bar.pv_full[pb]);
           mma_commit(&bar.p_empty[b]);
           mma_commit(&bar.v_empty[sv]);
+          return true;
+        };
+        if (ok) ok = mbar_wait(bar.s_init, 0, abort_flag, status, kDevTimeoutSoftmax);
+        for (int j = 0; ok && j < L::SB && j < nkv; ++j) ok = qk(j);
+        // The exp warpgroups release S for tile i early in their pass over
+        // it: the Q K^T of tile i + SB goes first (the scores the stats
+        // warpgroup needs next), the P~V of tile i - 1 (the fold runs two
+        // tiles behind) second, so the scores never queue behind it.
+        for (int i = 0; ok && i < nkv; ++i) {
+          if (i + L::SB < nkv) {
+            if (!mbar_wait(&bar.s_ready[i % L::SB], (i / L::SB) & 1, abort_flag, status,
+                           kDevTimeoutSoftmax)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (!qk(i + L::SB)) {
+              ok = false;
+              break;
+            }
+          }
+          if (i >= 1 && !pv(i - 1)) {
+            ok = false;
+            break;
+          }
         }
+        if (ok && nkv > 0) ok = pv(nkv - 1);
         if (!ok) {
           // let every MMA already issued finish before TMEM is released
           mma_commit(bar.drain);
@@ -597,8 +646,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL>(wg - 1, qt, nkv, bh, ntiles, tmem, bar, smem, abort_flag, status,
-                        q_scales, k_scales, scale_log2);
+    exp_loop<D, CAUSAL>(wg - 1, qt, nkv, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
     stats_loop<D, CAUSAL, OutT>(qt, nkv, bh, N, ntiles, tmem, bar, smem, abort_flag, status,
@@ -611,6 +659,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+#ifdef SAGE_TRACE
+  if (SAGE_TRACED_CTA && threadIdx.x < 64)
+    for (int e = 0; e < 16; ++e) g_sage_trace[e][threadIdx.x] = s_sage_trace[e][threadIdx.x];
+#endif
 }
 
 template <int D, bool CAUSAL, typename OutT>
