@@ -29,11 +29,12 @@
 //     thread moves them into TMEM with tcgen05.cp (32x128b, replicated to
 //     the four lane quadrants) just before the MMA that reads them;
 //   - the exp warpgroups also write the P~ scale factors of their rows;
-//   - S is a plain FP32 accumulator (no bias trick), and the level-1
-//     partial is single-buffered: the scale factors take the TMEM columns a
-//     second partial would need.  The fold therefore lags the max by one
-//     tile instead of two.
-// TMEM columns: S[0] 0..127, S[1] 128..255, PV 256..383, scale factors
+//   - S is a plain FP32 accumulator (no bias trick), single-buffered: the
+//     exp warpgroups release it as soon as they hold their 64 scores, and
+//     the MMA thread issues the next Q K^T ahead of the previous tile's
+//     P~V, so the scores the stats warpgroup needs next never queue behind
+//     a partial that is folded two tiles later.
+// TMEM columns: S 0..127, PV[0] 128..255, PV[1] 256..383, scale factors
 // SFA_Q 384, SFB_K 392, SFA_P 400, SFB_V 408 (8 columns each: two 64-wide
 // K blocks of 4 columns).  Every barrier wait is bounded; an expired wait
 // sets the device status word and makes every role leave its loop.
@@ -59,7 +60,7 @@ constexpr uint32_t kRegsProducer = 32;
 constexpr uint32_t kRegsStats = 216;
 
 // TMEM column offsets.
-constexpr uint32_t kColPV = 256;
+constexpr uint32_t kColPV = 128;  // PV[b] at 128 + 128 b
 constexpr uint32_t kColSfaQ = 384;
 constexpr uint32_t kColSfbK = 392;
 constexpr uint32_t kColSfaP = 400;
@@ -84,7 +85,8 @@ struct Layout {
   static constexpr int OFF_ABORT = OFF_MISC + 528;
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
-  static constexpr int END = OFF_L + 2 * 128 * 4;
+  static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots] dequant factor of the tile
+  static constexpr int END = OFF_C + 16;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t SBO = 8 * 64;  // 8 rows of 64 bytes (64-byte swizzle atom)
@@ -97,13 +99,13 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;
   uint64_t* v_empty;
-  uint64_t* s_full;    // [2] MMA -> stats, exp: S[b] holds Q K_j^T
+  uint64_t* s_full;    // [1] MMA -> stats: S holds Q K_j^T
   uint64_t* m_full;    // [2] stats -> exp: m_j, alpha_j of tile j (slot j % 2)
-  uint64_t* s_ready;   // [2] exp -> MMA: S[b] read (both halves)
+  uint64_t* s_ready;   // [1] exp -> MMA: S read (both halves)
   uint64_t* p_full;    // [2] exp -> MMA: P~ tile b and its scales written
   uint64_t* p_empty;   // [2] MMA -> exp: P~ tile b read by the P~V MMA
-  uint64_t* pv_full;   // [1] MMA -> stats: PV holds a tile's partial
-  uint64_t* pv_empty;  // [1] stats -> MMA: PV read
+  uint64_t* pv_full;   // [2] MMA -> stats: PV[b] holds a tile's partial
+  uint64_t* pv_empty;  // [2] stats -> MMA: PV[b] read
   uint64_t* l_ready;   // [1] exp -> stats: final row sums
   uint64_t* drain;     // MMA drain on abort
 };
@@ -118,13 +120,13 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.v_full = r.k_empty + L::KS;
   r.v_empty = r.v_full + L::VS;
   r.s_full = r.v_empty + L::VS;
-  r.m_full = r.s_full + 2;
+  r.m_full = r.s_full + 1;
   r.s_ready = r.m_full + 2;
-  r.p_full = r.s_ready + 2;
+  r.p_full = r.s_ready + 1;
   r.p_empty = r.p_full + 2;
   r.pv_full = r.p_empty + 2;
-  r.pv_empty = r.pv_full + 1;
-  r.l_ready = r.pv_empty + 1;
+  r.pv_empty = r.pv_full + 2;
+  r.l_ready = r.pv_empty + 2;
   r.drain = r.l_ready + 1;
   return r;
 }
@@ -153,6 +155,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 
 __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Global load the compiler keeps where it is written (a plain load of a
+// value needed only in the next loop iteration may be sunk to the end of
+// the current one, exposing its latency at the top of the next).
+__device__ __forceinline__ float ldg_early(const float* p) {
+  float v;
+  asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
 }
 
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -296,40 +307,34 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
   const int r = quarter * 32 + lane;
   const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
   const float* m_s = reinterpret_cast<const float*>(smem + L::OFF_M);
+  const float* c_s = reinterpret_cast<const float*>(smem + L::OFF_C);
   float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
 
-  // both S buffers start free
-  mbar_arrive(&bar.s_ready[0]);
-  mbar_arrive(&bar.s_ready[1]);
-
-  const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
-  const float* ksp = k_scales + (int64_t)bh * ntiles;
   float l = 0.f;
-  float ks_next = __ldg(ksp);
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
     const uint32_t ph = (j >> 1) & 1;
-    const float c = qs * ks_next * scale_log2;
-    if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
+    // m_full(j) is published by the stats warpgroup after it waited for
+    // s_full(j) and read S: it orders this warpgroup after the Q K^T too
     if (!__all_sync(0xffffffffu,
-                    mbar_wait(&bar.s_full[b], ph, abort_flag, status, kDevTimeoutMma) &&
-                        mbar_wait(&bar.m_full[b], ph, abort_flag, status, kDevTimeoutEpi)))
+                    mbar_wait(&bar.m_full[b], ph, abort_flag, status, kDevTimeoutEpi)))
       return;
     tc_fence_after();
+    const float c = c_s[b];
     const float m_j = m_s[(2 * b) * 128 + r];
     const float alpha = m_s[(2 * b + 1) * 128 + r];
     const float neg = -m_j;
     const bool diag = CAUSAL && (j == qt);
-    const uint32_t S = tmem + lanes + 128u * b + 64u * h;
+    const uint32_t S = tmem + lanes + 64u * h;
     uint32_t sa[32], sb[32];
     tmem_ld32(S, sa);
     tmem_ld32(S + 32, sb);
     tmem_wait_ld_regs(sa);
     reg_fence(sb);
-    // S[b] is in registers (and the stats warpgroup took its max before
-    // publishing m_j): free for Q K_{j+2}^T
+    // S is in registers (and the stats warpgroup took its max before
+    // publishing m_j): free for Q K_{j+1}^T
     tc_fence_before();
-    mbar_arrive(&bar.s_ready[b]);
+    mbar_arrive(bar.s_ready);
     // P~ tile b is free once the P~V MMA of tile j - 2 has read it
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
@@ -380,13 +385,14 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float m = -INFINITY;
   // O = alpha_i O + part_i * g_V,i / 2688
   auto fold = [&](int i, float alpha) -> bool {
+    const int pb = i & 1;
     if (!__all_sync(0xffffffffu,
-                    mbar_wait(bar.pv_full, i & 1, abort_flag, status, kDevTimeoutMma)))
+                    mbar_wait(&bar.pv_full[pb], (i >> 1) & 1, abort_flag, status, kDevTimeoutMma)))
       return false;
     tc_fence_after();
-    const uint32_t PV = tmem + lanes + kColPV;
+    const uint32_t PV = tmem + lanes + kColPV + 128u * (uint32_t)pb;
     const float2 a2 = make_float2(alpha, alpha);
-    const float cv = __ldg(vgp + i) * kPG;
+    const float cv = ldg_early(vgp + i) * kPG;
     const float2 cv2 = make_float2(cv, cv);
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -401,22 +407,23 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
                        cv2));
     }
     tc_fence_before();
-    mbar_arrive(bar.pv_empty);
+    mbar_arrive(&bar.pv_empty[pb]);
     return true;
   };
 
-  float alpha_prev = 0.f;
-  float ks_next = __ldg(ksp);
+  float alpha_hist[2] = {0.f, 0.f};
+  float* c_s = reinterpret_cast<float*>(smem + L::OFF_C);
+  float ks_cur = ldg_early(ksp);
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
-    const float c = qs * ks_next * scale_log2;
-    if (j + 1 < nkv) ks_next = __ldg(ksp + j + 1);
-    if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[b], (j >> 1) & 1, abort_flag, status,
-                                           kDevTimeoutMma)))
+    const float c = qs * ks_cur * scale_log2;
+    const float ks_nxt = j + 1 < nkv ? ldg_early(ksp + j + 1) : 0.f;
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(bar.s_full, j & 1, abort_flag, status, kDevTimeoutMma)))
       return;
     tc_fence_after();
     const bool diag = CAUSAL && (j == qt);
-    const uint32_t S = tmem + lanes + (uint32_t)b * 128u;
+    const uint32_t S = tmem + lanes;
     float mx = -INFINITY;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -432,12 +439,16 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     m = m_j;
     m_s[(2 * b) * 128 + r] = m_j;
     m_s[(2 * b + 1) * 128 + r] = alpha;
+    if (r == 0) c_s[b] = c;
     tc_fence_before();
     mbar_arrive(&bar.m_full[b]);
-    if (j > 0 && !fold(j - 1, alpha_prev)) return;
-    alpha_prev = alpha;
+    // the fold runs two tiles behind the max
+    if (j > 1 && !fold(j - 2, alpha_hist[b])) return;
+    alpha_hist[b] = alpha;
+    ks_cur = ks_nxt;
   }
-  if (nkv > 0 && !fold(nkv - 1, alpha_prev)) return;
+  for (int i = nkv > 2 ? nkv - 2 : 0; i < nkv; ++i)
+    if (!fold(i, alpha_hist[i & 1])) return;
   if (!__all_sync(0xffffffffu,
                   mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)))
     return;
@@ -489,15 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.v_full[i], 1);
       mbar_init(&bar.v_empty[i], 1);
     }
+    mbar_init(bar.s_full, 1);
+    mbar_init(bar.s_ready, 256);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar.s_full[i], 1);
       mbar_init(&bar.m_full[i], 128);
-      mbar_init(&bar.s_ready[i], 256);
       mbar_init(&bar.p_full[i], 256);
       mbar_init(&bar.p_empty[i], 1);
+      mbar_init(&bar.pv_full[i], 1);
+      mbar_init(&bar.pv_empty[i], 128);
     }
-    mbar_init(bar.pv_full, 1);
-    mbar_init(bar.pv_empty, 128);
     mbar_init(bar.l_ready, 256);
     mbar_init(bar.drain, 1);
     *abort_flag = 0;
@@ -565,12 +576,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_cp_32x128b_x4(tmem + kColSfaQ, sf_desc(sSFQ));
           tmem_cp_32x128b_x4(tmem + kColSfaQ + 4, sf_desc(sSFQ + 512));
         }
-        // S[j % 2] = Q K_j^T, two K blocks of 64 channels
+        // S = Q K_j^T, two K blocks of 64 channels (S free: for j >= 1 the
+        // caller waited for s_ready of tile j - 1)
         auto qk = [&](int j) -> bool {
           const int sk = j % L::KS;
-          const int b = j & 1;
-          if (!mbar_wait(&bar.k_full[sk], (j / L::KS) & 1, abort_flag, status, kDevTimeoutTma) ||
-              !mbar_wait(&bar.s_ready[b], (j >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax))
+          if (!mbar_wait(&bar.k_full[sk], (j / L::KS) & 1, abort_flag, status, kDevTimeoutTma))
             return false;
           tc_fence_after();
           tmem_cp_32x128b_x4(tmem + kColSfbK, sf_desc(sSFK + sk * L::SF));
@@ -578,30 +588,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t kdesc = make_sdesc(smem_u32(sK + sk * L::TILE), L::SBO, 16, Swz::k64);
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_nvf4_ss(tmem + (uint32_t)b * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc,
-                        tmem + kColSfaQ + 4 * kk, tmem + kColSfbK + 4 * kk, kk > 0);
-          mma_commit(&bar.s_full[b]);
+            mma_nvf4_ss(tmem, qdesc + 2 * kk, kdesc + 2 * kk, idesc, tmem + kColSfaQ + 4 * kk,
+                        tmem + kColSfbK + 4 * kk, kk > 0);
+          mma_commit(bar.s_full);
           mma_commit(&bar.k_empty[sk]);
           return true;
         };
-        if (ok) ok = qk(0);
-        if (ok && nkv > 1) ok = qk(1);
-        for (int i = 0; ok && i < nkv; ++i) {
+        // P~_i V_i into PV[i % 2] (level 1)
+        auto pv = [&](int i) -> bool {
           const int b = i & 1;
-          if (!mbar_wait(&bar.p_full[b], (i >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax)) {
-            ok = false;
-            break;
-          }
-          if (i + 2 < nkv && !qk(i + 2)) {
-            ok = false;
-            break;
-          }
           const int sv = i % L::VS;
-          if (!mbar_wait(&bar.v_full[sv], (i / L::VS) & 1, abort_flag, status, kDevTimeoutTma) ||
-              !mbar_wait(bar.pv_empty, (i & 1) ^ 1, abort_flag, status, kDevTimeoutEpi)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(&bar.p_full[b], (i >> 1) & 1, abort_flag, status, kDevTimeoutSoftmax) ||
+              !mbar_wait(&bar.v_full[sv], (i / L::VS) & 1, abort_flag, status, kDevTimeoutTma) ||
+              !mbar_wait(&bar.pv_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, status,
+                         kDevTimeoutEpi))
+            return false;
           tc_fence_after();
           tmem_cp_32x128b_x4(tmem + kColSfaP, sf_desc(sSFP + b * L::SF));
           tmem_cp_32x128b_x4(tmem + kColSfaP + 4, sf_desc(sSFP + b * L::SF + 512));
@@ -611,12 +612,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t vdesc = make_sdesc(smem_u32(sV + sv * L::TILE), L::SBO, 16, Swz::k64);
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_nvf4_ss(tmem + kColPV, pdesc + 2 * kk, vdesc + 2 * kk, idesc,
+            mma_nvf4_ss(tmem + kColPV + 128u * (uint32_t)b, pdesc + 2 * kk, vdesc + 2 * kk, idesc,
                         tmem + kColSfaP + 4 * kk, tmem + kColSfbV + 4 * kk, kk > 0);
-          mma_commit(bar.pv_full);
+          mma_commit(&bar.pv_full[b]);
           mma_commit(&bar.p_empty[b]);
           mma_commit(&bar.v_empty[sv]);
+          return true;
+        };
+        if (ok) ok = qk(0);
+        // The exp warpgroups release S early in their pass over tile i: the
+        // Q K^T of tile i + 1 goes first (the scores the stats warpgroup
+        // needs next), the P~V of tile i - 1 (folded two tiles behind)
+        // second, so the scores never queue behind it.
+        for (int i = 0; ok && i < nkv; ++i) {
+          if (i + 1 < nkv) {
+            if (!mbar_wait(bar.s_ready, i & 1, abort_flag, status, kDevTimeoutSoftmax)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (!qk(i + 1)) {
+              ok = false;
+              break;
+            }
+          }
+          if (i >= 1 && !pv(i - 1)) {
+            ok = false;
+            break;
+          }
         }
+        if (ok && nkv > 0) ok = pv(nkv - 1);
         if (!ok) {
           // let every MMA already issued finish before TMEM is released
           mma_commit(bar.drain);
