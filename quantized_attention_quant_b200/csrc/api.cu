@@ -77,14 +77,17 @@ int device_info(DeviceInfo** out) {
 
 // Stream-ordered workspace, one per (device, stream): a call on stream S
 // only ever touches the workspace of S, so calls on different streams
-// never share scratch memory.
+// never share scratch memory.  Its first kStatsCounterBytes hold the
+// per-head statistics counters of the pre-pass: zeroed when the workspace
+// is (re)allocated, and left at zero by every pre-pass.
 struct Workspace {
   void* ptr = nullptr;
   size_t bytes = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-int workspace(cudaStream_t st, size_t need, void** out) {
+int workspace(cudaStream_t st, size_t need, void** out, uint32_t** counters) {
+  need += kStatsCounterBytes;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
@@ -101,8 +104,11 @@ int workspace(cudaStream_t st, size_t need, void** out) {
     e = cudaMallocAsync(&w.ptr, grow, st);
     if (e != cudaSuccess) return fail_cuda(e, "cudaMallocAsync(workspace)");
     w.bytes = grow;
+    e = cudaMemsetAsync(w.ptr, 0, kStatsCounterBytes, st);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(workspace counters)");
   }
-  *out = w.ptr;
+  *counters = static_cast<uint32_t*>(w.ptr);
+  *out = static_cast<char*>(w.ptr) + kStatsCounterBytes;
   return SAGE_OK;
 }
 
@@ -256,9 +262,10 @@ int sage_quant_qk(const void* q, const void* k, int dtype, int64_t B, int64_t H,
   SAGE_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void* ws = nullptr;
-  SAGE_TRY(workspace(st, ws_ksum_bytes(B * H, N, d), &ws));
+  uint32_t* cnt = nullptr;
+  SAGE_TRY(workspace(st, ws_ksum_bytes(B * H, N, d), &ws, &cnt));
   QuantQKArgs a{q, k, dtype, mode, B, H, N, d, q_codes, q_scales, q_sf,
-                k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws)};
+                k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws), cnt};
   cudaError_t e = launch_quant_qk(a, st);
   if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
   return SAGE_OK;
@@ -278,11 +285,13 @@ int sage_quant_v(const void* v, int dtype, int64_t B, int64_t H, int64_t N, int6
   SAGE_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void* ws = nullptr;
+  uint32_t* cnt = nullptr;
   const size_t ks = align_up(ws_ksum_bytes(B * H, N, d));
-  if (mode == SAGE_MODE_INT8_FP8) SAGE_TRY(workspace(st, ks + ws_vmax_bytes(B * H, N, d), &ws));
+  if (mode == SAGE_MODE_INT8_FP8)
+    SAGE_TRY(workspace(st, ks + ws_vmax_bytes(B * H, N, d), &ws, &cnt));
   QuantVArgs a{v, dtype, mode, B, H, N, d, v_codes, v_scales, v_sf,
                static_cast<double*>(ws),
-               ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + ks) : nullptr};
+               ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + ks) : nullptr, cnt};
   cudaError_t e = launch_quant_v(a, st);
   if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
   return SAGE_OK;
@@ -353,7 +362,8 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
   const size_t off_vmax = total;
   total += align_up(ws_vmax_bytes(B * H, N, d));
   void* ws = nullptr;
-  SAGE_TRY(workspace(st, total, &ws));
+  uint32_t* cnt = nullptr;
+  SAGE_TRY(workspace(st, total, &ws, &cnt));
   char* base = static_cast<char*>(ws);
   auto at = [&](int w) -> void* {
     return sage_buffer_bytes(mode, w, B, H, N, d) ? base + off[w] : nullptr;
@@ -361,11 +371,11 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
   QuantQKArgs qa{q, k, dtype, mode, B, H, N, d,
                  at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
                  at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
-                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum)};
+                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum), cnt};
   QuantVArgs va{v, dtype, mode, B, H, N, d,
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
-                reinterpret_cast<float*>(base + off_vmax)};
+                reinterpret_cast<float*>(base + off_vmax), cnt};
   cudaError_t e = launch_prepass(qa, va, st);
   if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
@@ -488,6 +498,7 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
   total += align_up(ws_ksum_bytes(B * H, N, d));
   const size_t off_vmax = total;
   total += align_up(ws_vmax_bytes(B * H, N, d));
+  total += kStatsCounterBytes;  // the per-head statistics counters, first
   if (total > kNoAllocScratchBytes) {
     return fail(SAGE_ERR_UNSUPPORTED,
                 "this shape needs " + std::to_string(total) +
@@ -499,20 +510,22 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
   void* ws = nullptr;
   SAGE_TRY(noalloc_scratch(&ws));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  char* base = static_cast<char*>(ws);
+  uint32_t* cnt = static_cast<uint32_t*>(ws);
+  char* base = static_cast<char*>(ws) + kStatsCounterBytes;
   auto at = [&](int w) -> void* {
     return sage_buffer_bytes(mode, w, B, H, N, d) ? base + off[w] : nullptr;
   };
   // Every scratch byte the kernels read is written earlier in the same call
-  // (codes, scales, statistics partials), so nothing needs clearing.
+  // (codes, scales, statistics partials), except the per-head counters:
+  // zero in the loaded image, and returned to zero by every pre-pass.
   QuantQKArgs qa{q, k, dtype, mode, B, H, N, d,
                  at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
                  at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
-                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum)};
+                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum), cnt};
   QuantVArgs va{v, dtype, mode, B, H, N, d,
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
-                reinterpret_cast<float*>(base + off_vmax)};
+                reinterpret_cast<float*>(base + off_vmax), cnt};
   cudaError_t e = launch_prepass(qa, va, st);
   if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),

@@ -13,11 +13,12 @@
 //
 // Launch structure (one 256-thread CTA per 128-token tile and role):
 //   kernel A  roles that need no head-wide statistic: Q codes, FP4 V codes,
-//             and the per-chunk K sums / V maxima;
-//   finalize  per (b, h): fold the chunk partials in chunk order into the
-//             K mean and the per-channel V scale;
+//             and the per-chunk K sums / V maxima.  The last statistics CTA
+//             of each (b, h) (a per-head counter tells it) folds the chunk
+//             partials in chunk order into the K mean and the per-channel V
+//             scale, then resets the counter;
 //   kernel B  roles that need them: smoothed K codes, FP8 V codes.
-// sage_attn_fwd runs all roles of Q, K and V in these three launches.
+// sage_attn_fwd runs all roles of Q, K and V in these two launches.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -67,7 +68,10 @@ struct PrepassPtrs {
   uint8_t* v_sf;
   double* ksum;  // [B*H, N/128, d] FP64 chunk sums of K
   float* vmax;   // [B*H, N/128, d] chunk maxima of |V|
+  uint32_t* cnt;  // [2][kMaxHeads] statistics CTAs done per head (K, V); 0 between passes
 };
+
+constexpr int kMaxHeads = 65536;
 
 template <typename T>
 __device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
@@ -103,29 +107,44 @@ __device__ __forceinline__ float load1(const T* p) {
 constexpr float kBracketLo = 1.0f - 0x1p-20f;
 constexpr float kBracketHi = 1.0f + 0x1p-20f;
 
-// INT8 code clamp(rne(fp32(x / s)), +-127), s != 0.  Rounding to an integer
-// is an FP32 add of 1.5 * 2^23 (exact round-half-even for |v| < 2^22; here
-// |x / s| < 128), read back from the bits, so no conversion instruction is
-// needed; the bracket test compares the two rounded ends bit for bit.
+// INT8 rounding to an integer is an FP32 add of 1.5 * 2^23 (exact
+// round-half-even for |v| < 2^22; here |x / s| < 128), read back from the
+// bits, so no conversion instruction is needed.
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-constexpr int kRoundMagicBits = 0x4B400000;
 
-__device__ __forceinline__ int int8_code(float x, float s, float rs) {
-  const float q = x * rs;
-  const float2 ends = __fadd2_rn(__fmul2_rn(make_float2(q, q), make_float2(kBracketLo, kBracketHi)),
-                                 make_float2(kRoundMagic, kRoundMagic));
-  const float rounded = (rs != 0.f && __float_as_uint(ends.x) == __float_as_uint(ends.y))
-                            ? ends.y
-                            : __fdiv_rn(x, s) + kRoundMagic;
-  const int c = __float_as_int(rounded) - kRoundMagicBits;
-  return max(-127, min(127, c));
-}
-
-__device__ __forceinline__ float quot_e4m3(float x, float s, float rs) {
-  const float q = x * rs;
-  const uint32_t pk = cvt_e4m3x2(q * kBracketLo, q * kBracketHi);
-  if (rs != 0.f && (pk & 0xFFu) == (pk >> 8)) return q;
-  return __fdiv_rn(x, s);
+// Eight INT8 codes clamp(rne(fp32(v / s)), +-127) for one block scale
+// s != 0, packed little-endian (code of v[i] in byte i).  The bracket test
+// runs on the whole vector without a branch: for each value the
+// two ends are rounded to integers by one FFMA2 each (q * bound + 1.5 * 2^23,
+// a single rounding of the exact product, as monotonic as the quotient),
+// and their bit patterns are XOR-accumulated; only when some end pair
+// differs (or 1/s is unusable) is the vector redone on IEEE quotients.  The
+// low byte of the float 1.5*2^23 + c is c mod 256, so the codes are packed
+// straight from the rounded bits (|c| <= 127 here since |v| <= 127 s).
+__device__ __forceinline__ uint2 int8_codes8(const float (&v)[8], float s, float rs) {
+  const float2 rs2 = make_float2(rs, rs);
+  const float2 lo2 = make_float2(kBracketLo, kBracketLo);
+  const float2 hi2 = make_float2(kBracketHi, kBracketHi);
+  const float2 m2 = make_float2(kRoundMagic, kRoundMagic);
+  uint32_t hb[8];
+  uint32_t diff = rs == 0.f ? 1u : 0u;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 q = __fmul2_rn(make_float2(v[e], v[e + 1]), rs2);
+    const float2 a = __ffma2_rn(q, lo2, m2);
+    const float2 b = __ffma2_rn(q, hi2, m2);
+    diff |= (__float_as_uint(a.x) ^ __float_as_uint(b.x)) |
+            (__float_as_uint(a.y) ^ __float_as_uint(b.y));
+    hb[e] = __float_as_uint(b.x);
+    hb[e + 1] = __float_as_uint(b.y);
+  }
+  if (diff != 0u) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hb[e] = __float_as_uint(__fdiv_rn(v[e], s) + kRoundMagic);
+  }
+  const uint32_t w0 = __byte_perm(__byte_perm(hb[0], hb[1], 0x0040), __byte_perm(hb[2], hb[3], 0x0040), 0x5410);
+  const uint32_t w1 = __byte_perm(__byte_perm(hb[4], hb[5], 0x0040), __byte_perm(hb[6], hb[7], 0x0040), 0x5410);
+  return make_uint2(w0, w1);
 }
 
 __device__ __forceinline__ float quot_e2m1(float x, float s, float rs) {
@@ -161,32 +180,92 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
+// Copies one 128-token tile [128][D] of T into shared memory with 16-byte
+// loads (consecutive threads, consecutive vectors).
+template <typename T, int D>
+__device__ __forceinline__ void stage_tile(const T* __restrict__ src, T* tile) {
+  constexpr int VPT = 128 * D / 8 / kThreads;
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint4* d = reinterpret_cast<uint4*>(tile);
+  uint4 v[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) v[i] = __ldg(s + threadIdx.x + i * kThreads);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) d[threadIdx.x + i * kThreads] = v[i];
+}
+
 // ------------------------------------------------------------------ stats
-// One CTA per (128-token chunk, b*h).  Thread c < D walks K's channel c over
-// the chunk's tokens in order with an FP64 sum; thread D + c keeps the max
-// of |V| of channel c.  Consecutive threads read consecutive channels.
+// One CTA per (128-token chunk, b*h).  K: the tile is staged in shared
+// memory, then thread c < D walks channel c over the chunk's tokens in
+// order with an FP64 sum.  V: each thread keeps the max of |V| over its
+// vectors (8 channels each) and merges it into a shared per-channel max
+// (non-negative floats order like their bit patterns).
 template <typename T, int D>
 __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int chunk,
-                                           bool do_k, bool do_v) {
+                                           bool do_k, bool do_v, T* tile, uint32_t* vmax_s) {
+  constexpr int VPT = 128 * D / 8 / kThreads;
   const int nchunks = p.N / 128;
   const int t = threadIdx.x;
   const int64_t row0 = bh * p.N + (int64_t)chunk * 128;
   const int64_t out = (bh * nchunks + chunk) * D;
+  if (do_v && t < D) vmax_s[t] = 0u;
+  if (do_k) stage_tile<T, D>(reinterpret_cast<const T*>(p.k) + row0 * D, tile);
+  __syncthreads();
+  if (do_v) {
+    const T* src = reinterpret_cast<const T*>(p.v) + row0 * D;
+    const int c0 = (t % (D / 8)) * 8;
+    float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      float x[8];
+      load8(src + (t + i * kThreads) * 8, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(x[e]));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) atomicMax(vmax_s + c0 + e, __float_as_uint(m[e]));
+  }
+  __syncthreads();
   if (t < D) {
-    if (!do_k) return;
-    const T* src = reinterpret_cast<const T*>(p.k) + row0 * D + t;
-    double s = 0.0;
+    if (do_k) {
+      double acc = 0.0;
 #pragma unroll 16
-    for (int i = 0; i < 128; ++i) s += (double)load1(src + (int64_t)i * D);
-    p.ksum[out + t] = s;
-  } else if (t < 2 * D) {
-    if (!do_v) return;
-    const int c = t - D;
-    const T* src = reinterpret_cast<const T*>(p.v) + row0 * D + c;
-    float m = 0.f;
-#pragma unroll 16
-    for (int i = 0; i < 128; ++i) m = fmaxf(m, fabsf(load1(src + (int64_t)i * D)));
-    p.vmax[out + c] = m;
+      for (int i = 0; i < 128; ++i) acc += (double)static_cast<float>(tile[i * D + t]);
+      p.ksum[out + t] = acc;
+    }
+    if (do_v) p.vmax[out + t] = __uint_as_float(vmax_s[t]);
+  }
+  // The last chunk of this head to finish folds all partials (threadfence
+  // reduction: each CTA publishes its partials before taking a ticket, the
+  // CTA with the last ticket sees every partial).
+  __shared__ int last[2];
+  __threadfence();
+  __syncthreads();
+  if (t == 0) {
+    last[0] = do_k && atomicAdd(p.cnt + bh, 1u) == (uint32_t)(nchunks - 1);
+    last[1] = do_v && atomicAdd(p.cnt + kMaxHeads + bh, 1u) == (uint32_t)(nchunks - 1);
+  }
+  __syncthreads();
+  if (!last[0] && !last[1]) return;
+  __threadfence();
+  if (t < D) {
+    const int64_t base = bh * nchunks * D + t;
+    if (last[0]) {
+      // sum of the chunk partials in chunk order; mean = fp32(sum / N)
+      double acc = 0.0;
+      for (int i = 0; i < nchunks; ++i) acc += __ldcg(p.ksum + base + (int64_t)i * D);
+      p.k_mean[bh * D + t] = __double2float_rn(__ddiv_rn(acc, (double)p.N));
+    }
+    if (last[1]) {
+      // s_V = fp32(amax / 448)
+      float m = 0.f;
+      for (int i = 0; i < nchunks; ++i) m = fmaxf(m, __ldcg(p.vmax + base + (int64_t)i * D));
+      p.v_scales[bh * D + t] = __fdiv_rn(m, 448.f);
+    }
+  }
+  if (t == 0) {
+    if (last[0]) p.cnt[bh] = 0u;
+    if (last[1]) p.cnt[kMaxHeads + bh] = 0u;
   }
 }
 
@@ -201,23 +280,32 @@ __device__ __forceinline__ void role_quant_int8(const T* __restrict__ src, const
                                                 float* red) {
   constexpr int VPT = 128 * D / 8 / kThreads;  // 16-byte vectors per thread
   const int c0 = (threadIdx.x % (D / 8)) * 8;
-  float mu[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  // x - mu as x + (-mu): the same single rounding
+  float nmu[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (mean) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(mean + c0));
     const float4 b = __ldg(reinterpret_cast<const float4*>(mean + c0 + 4));
-    mu[0] = a.x; mu[1] = a.y; mu[2] = a.z; mu[3] = a.w;
-    mu[4] = b.x; mu[5] = b.y; mu[6] = b.z; mu[7] = b.w;
+    nmu[0] = -a.x; nmu[1] = -a.y; nmu[2] = -a.z; nmu[3] = -a.w;
+    nmu[4] = -b.x; nmu[5] = -b.y; nmu[6] = -b.z; nmu[7] = -b.w;
   }
+  auto smooth = [&](float (&x)[8]) {
+    if (mean) {
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float2 t = __fadd2_rn(make_float2(x[e], x[e + 1]), make_float2(nmu[e], nmu[e + 1]));
+        x[e] = t.x;
+        x[e + 1] = t.y;
+      }
+    }
+  };
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     float x[8];
     load8(src + (threadIdx.x + i * kThreads) * 8, x);
+    smooth(x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float v = mean ? __fsub_rn(x[e], mu[e]) : x[e];
-      amax = fmaxf(amax, fabsf(v));
-    }
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
   }
   amax = block_max(amax, red);
   const float s = __fdiv_rn(amax, 127.f);
@@ -225,62 +313,100 @@ __device__ __forceinline__ void role_quant_int8(const T* __restrict__ src, const
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vec = threadIdx.x + i * kThreads;
-    uint32_t w[2] = {0u, 0u};
+    uint2 w = make_uint2(0u, 0u);
     if (s != 0.f) {
       float x[8];
       load8(src + vec * 8, x);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float v = mean ? __fsub_rn(x[e], mu[e]) : x[e];
-        const int c = int8_code(v, s, rs);
-        w[e >> 2] |= (uint32_t)(c & 0xFF) << (8 * (e & 3));
-      }
+      smooth(x);
+      w = int8_codes8(x, s, rs);
     }
-    *reinterpret_cast<uint2*>(dst + vec * 8) = make_uint2(w[0], w[1]);
+    *reinterpret_cast<uint2*>(dst + vec * 8) = w;
   }
   if (threadIdx.x == 0) *scale_out = s;
 }
 
 // ---------------------------------------------------------------- FP8 V
-// codes = e4m3(V / s_V[c]) written transposed into V^T.  A thread owns a
-// channel pair and 32 consecutive tokens: it reads the pair at each token
-// (consecutive threads -> consecutive pairs, so a warp reads 128 contiguous
-// bytes per token) and writes each channel's 32 codes as a whole 32-byte
-// sector (two 16-byte stores).
+// codes = e4m3(V / s_V[c]) written transposed into V^T.  The tile is staged
+// in shared memory; a thread then owns a channel pair and 32 consecutive
+// tokens (reads conflict-free: consecutive threads, consecutive pairs) and
+// writes each channel's 32 codes as one 32-byte sector (two 16-byte stores).  The bracket
+// test of the INT8 path runs per pair of tokens: both ends of two tokens go
+// through one e4m3x2 conversion each, and the two 16-bit results must match
+// (else the unit is redone on IEEE quotients); the matching result is the
+// two codes, already packed.
 template <typename T, int D>
 __device__ __forceinline__ void role_quant_v_fp8(const T* __restrict__ src,
                                                  const float* __restrict__ vs,
-                                                 uint8_t* __restrict__ dst, int N) {
-  constexpr int UNITS = (D / 2) * 8;  // channel pairs x 16-token groups
+                                                 uint8_t* __restrict__ dst, int N, T* tile) {
+  stage_tile<T, D>(src, tile);
+  __syncthreads();
+  constexpr int UNITS = (D / 2) * 4;  // channel pairs x 32-token groups
+  const float2 lo2 = make_float2(kBracketLo, kBracketLo);
+  const float2 hi2 = make_float2(kBracketHi, kBracketHi);
   for (int u = threadIdx.x; u < UNITS; u += kThreads) {
     const int cp = u % (D / 2), grp = u / (D / 2);
     const float s0 = __ldg(vs + 2 * cp), s1 = __ldg(vs + 2 * cp + 1);
     const float r0 = recip_or_zero(s0), r1 = recip_or_zero(s1);
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(src + (int64_t)(grp * 16) * D + 2 * cp);
-    uint32_t w0[4] = {0u, 0u, 0u, 0u}, w1[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      const uint32_t pair = __ldg(p + t * (D / 2));
-      float x0, x1;
+    const uint32_t* col = reinterpret_cast<const uint32_t*>(tile) + (grp * 32) * (D / 2) + cp;
+    auto pair_of = [&](int tok, float& x0, float& x1) {
+      const uint32_t w = col[tok * (D / 2)];
       if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-        x0 = __uint_as_float(pair << 16);
-        x1 = __uint_as_float(pair & 0xFFFF0000u);
+        x0 = __uint_as_float(w << 16);
+        x1 = __uint_as_float(w & 0xFFFF0000u);
       } else {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pair));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
         x0 = f.x;
         x1 = f.y;
       }
-      const float a = s0 != 0.f ? quot_e4m3(x0, s0, r0) : 0.f;
-      const float b = s1 != 0.f ? quot_e4m3(x1, s1, r1) : 0.f;
-      const uint32_t pk = cvt_e4m3x2(a, b);  // a in bits 0..7, b in 8..15
-      w0[t >> 2] |= (pk & 0xFFu) << (8 * (t & 3));
-      w1[t >> 2] |= (pk >> 8) << (8 * (t & 3));
-    }
+    };
+    // 1/s unusable for a nonzero scale: decide on quotients throughout
+    const uint32_t bad = ((s0 != 0.f && r0 == 0.f) || (s1 != 0.f && r1 == 0.f)) ? 1u : 0u;
     // dst points at V^T[c = 0][tile start]
-    *reinterpret_cast<uint4*>(dst + (int64_t)(2 * cp) * N + grp * 16) =
-        make_uint4(w0[0], w0[1], w0[2], w0[3]);
-    *reinterpret_cast<uint4*>(dst + (int64_t)(2 * cp + 1) * N + grp * 16) =
-        make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    uint8_t* d0 = dst + (int64_t)(2 * cp) * N + grp * 32;
+    uint8_t* d1 = dst + (int64_t)(2 * cp + 1) * N + grp * 32;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t diff = bad;
+      uint32_t w0[4], w1[4];
+#pragma unroll
+      for (int k = 0; k < 16; k += 4) {
+        float a[4], b[4];  // channel 2cp / 2cp+1 at 4 consecutive tokens
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pair_of(16 * half + k + i, a[i], b[i]);
+        uint32_t ca[2], cb[2];
+#pragma unroll
+        for (int i = 0; i < 4; i += 2) {
+          const float2 qa = __fmul2_rn(make_float2(a[i], a[i + 1]), make_float2(r0, r0));
+          const float2 qb = __fmul2_rn(make_float2(b[i], b[i + 1]), make_float2(r1, r1));
+          const float2 qal = __fmul2_rn(qa, lo2), qah = __fmul2_rn(qa, hi2);
+          const float2 qbl = __fmul2_rn(qb, lo2), qbh = __fmul2_rn(qb, hi2);
+          const uint32_t al = cvt_e4m3x2(qal.x, qal.y), ah = cvt_e4m3x2(qah.x, qah.y);
+          const uint32_t bl = cvt_e4m3x2(qbl.x, qbl.y), bhh = cvt_e4m3x2(qbh.x, qbh.y);
+          diff |= (al ^ ah) | (bl ^ bhh);
+          ca[i >> 1] = ah;
+          cb[i >> 1] = bhh;
+        }
+        w0[k >> 2] = ca[0] | (ca[1] << 16);
+        w1[k >> 2] = cb[0] | (cb[1] << 16);
+      }
+      if (diff != 0u) {
+#pragma unroll 1
+        for (int k = 0; k < 16; k += 4) {
+          float a[4], b[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) pair_of(16 * half + k + i, a[i], b[i]);
+          w0[k >> 2] = cvt_e4m3x2(__fdiv_rn(a[0], s0), __fdiv_rn(a[1], s0)) |
+                       (cvt_e4m3x2(__fdiv_rn(a[2], s0), __fdiv_rn(a[3], s0)) << 16);
+          w1[k >> 2] = cvt_e4m3x2(__fdiv_rn(b[0], s1), __fdiv_rn(b[1], s1)) |
+                       (cvt_e4m3x2(__fdiv_rn(b[2], s1), __fdiv_rn(b[3], s1)) << 16);
+        }
+      }
+      // a zero scale (an all-zero channel) gives +0 codes
+      const uint4 v0 = s0 != 0.f ? make_uint4(w0[0], w0[1], w0[2], w0[3]) : make_uint4(0, 0, 0, 0);
+      const uint4 v1 = s1 != 0.f ? make_uint4(w1[0], w1[1], w1[2], w1[3]) : make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(d0 + 16 * half) = v0;
+      *reinterpret_cast<uint4*>(d1 + 16 * half) = v1;
+    }
   }
 }
 
@@ -427,8 +553,16 @@ __device__ __forceinline__ void role_quant_fp4_v(const T* __restrict__ src, int 
 #define SAGE_ROLE(r) if constexpr (((MASK >> (r)) & 1) != 0)
 template <typename T, int D, int MASK>
 __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles roles) {
-  constexpr int V4_BYTES = ((MASK >> kQuantV4) & 1) ? 128 * (D + 2) * (int)sizeof(T) : 16;
-  __shared__ __align__(16) uint8_t smem_raw[V4_BYTES];
+  // one staging buffer, sized for the largest role of the mask (a CTA runs
+  // one role)
+  constexpr bool kV4 = ((MASK >> kQuantV4) & 1) != 0;
+  constexpr bool kTile = ((MASK >> kQuantV8) & 1) || ((MASK >> kStatsK) & 1) ||
+                         ((MASK >> kStatsKV) & 1);
+  constexpr int V4_BYTES = kV4 ? 128 * (D + 2) * (int)sizeof(T) : 16;
+  constexpr int TILE_BYTES = kTile ? 128 * D * (int)sizeof(T) : 16;
+  constexpr int SMEM_BYTES = V4_BYTES > TILE_BYTES ? V4_BYTES : TILE_BYTES;
+  __shared__ __align__(16) uint8_t smem_raw[SMEM_BYTES];
+  __shared__ uint32_t vmax_s[D];
   __shared__ float red[kThreads / 32];
   const int role = roles.r[blockIdx.z];
   const int64_t bh = blockIdx.y;
@@ -453,7 +587,7 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
       role_quant_v_fp8<T, D>(reinterpret_cast<const T*>(p.v) + row0 * D, p.v_scales + bh * D,
                              reinterpret_cast<uint8_t*>(p.v_codes) + bh * D * (int64_t)p.N +
                                  (int64_t)tile * 128,
-                             p.N);
+                             p.N, reinterpret_cast<T*>(smem_raw));
       break;
     case kQuantQ4:
       SAGE_ROLE(kQuantQ4)
@@ -474,13 +608,16 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
                              p.v_sf, bh, ntiles, tile, reinterpret_cast<T(*)[D + 2]>(smem_raw), red);
       break;
     case kStatsK:
-      SAGE_ROLE(kStatsK) role_stats<T, D>(p, bh, tile, true, false);
+      SAGE_ROLE(kStatsK)
+      role_stats<T, D>(p, bh, tile, true, false, reinterpret_cast<T*>(smem_raw), vmax_s);
       break;
     case kStatsKV:
-      SAGE_ROLE(kStatsKV) role_stats<T, D>(p, bh, tile, true, true);
+      SAGE_ROLE(kStatsKV)
+      role_stats<T, D>(p, bh, tile, true, true, reinterpret_cast<T*>(smem_raw), vmax_s);
       break;
     case kStatsV:
-      SAGE_ROLE(kStatsV) role_stats<T, D>(p, bh, tile, false, true);
+      SAGE_ROLE(kStatsV)
+      role_stats<T, D>(p, bh, tile, false, true, reinterpret_cast<T*>(smem_raw), vmax_s);
       break;
     default:
       break;
@@ -490,48 +627,25 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
 
 constexpr int bit(int r) { return 1 << r; }
 
-// Fold the chunk partials in chunk order: mean = fp32(sum / N); and, for
-// FP8 V, s_V = fp32(amax / 448).
-__global__ void finalize_kernel(const double* __restrict__ ksum, const float* __restrict__ vmax,
-                                int D, int N, int nchunks, float* __restrict__ k_mean,
-                                float* __restrict__ v_scales) {
-  const int64_t bh = blockIdx.x;
-  for (int c = threadIdx.x; c < D; c += blockDim.x) {
-    if (ksum) {
-      double s = 0.0;
-      for (int i = 0; i < nchunks; ++i) s += ksum[(bh * nchunks + i) * D + c];
-      k_mean[bh * D + c] = __double2float_rn(__ddiv_rn(s, (double)N));
-    }
-    if (vmax) {
-      float m = 0.f;
-      for (int i = 0; i < nchunks; ++i) m = fmaxf(m, vmax[(bh * nchunks + i) * D + c]);
-      v_scales[bh * D + c] = __fdiv_rn(m, 448.f);
-    }
-  }
-}
-
-// kernel A (roles a), finalize (K mean and/or V scales), kernel B (roles b)
+// kernel A (roles a; its statistics CTAs also fold the head statistics),
+// then kernel B (roles b)
 template <typename T, int D, int MA, int MB>
-cudaError_t run_plan(const PrepassPtrs& p, int64_t BH, Roles a, bool fin_k, bool fin_v, Roles b,
-                     cudaStream_t st) {
+cudaError_t run_plan(const PrepassPtrs& p, int64_t BH, Roles a, Roles b, cudaStream_t st) {
   const int ntiles = p.N / 128;
   if (a.n) prepass_kernel<T, D, MA><<<dim3(ntiles, (unsigned)BH, a.n), kThreads, 0, st>>>(p, a);
-  if (fin_k || fin_v)
-    finalize_kernel<<<(unsigned)BH, 128, 0, st>>>(fin_k ? p.ksum : nullptr, fin_v ? p.vmax : nullptr,
-                                                  D, p.N, ntiles, p.k_mean, p.v_scales);
   if (b.n) prepass_kernel<T, D, MB><<<dim3(ntiles, (unsigned)BH, b.n), kThreads, 0, st>>>(p, b);
   return cudaGetLastError();
 }
 
 // MA / MB: the role masks of kernels A and B (they must cover a.r / b.r).
 template <int MA, int MB>
-cudaError_t dispatch(const PrepassPtrs& p, int dtype, int64_t d, int64_t BH, Roles a, bool fin_k,
-                     bool fin_v, Roles b, cudaStream_t st) {
+cudaError_t dispatch(const PrepassPtrs& p, int dtype, int64_t d, int64_t BH, Roles a, Roles b,
+                     cudaStream_t st) {
   if (dtype == 1)
-    return d == 128 ? run_plan<__nv_bfloat16, 128, MA, MB>(p, BH, a, fin_k, fin_v, b, st)
-                    : run_plan<__nv_bfloat16, 64, MA, MB>(p, BH, a, fin_k, fin_v, b, st);
-  return d == 128 ? run_plan<__half, 128, MA, MB>(p, BH, a, fin_k, fin_v, b, st)
-                  : run_plan<__half, 64, MA, MB>(p, BH, a, fin_k, fin_v, b, st);
+    return d == 128 ? run_plan<__nv_bfloat16, 128, MA, MB>(p, BH, a, b, st)
+                    : run_plan<__nv_bfloat16, 64, MA, MB>(p, BH, a, b, st);
+  return d == 128 ? run_plan<__half, 128, MA, MB>(p, BH, a, b, st)
+                  : run_plan<__half, 64, MA, MB>(p, BH, a, b, st);
 }
 
 PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
@@ -547,6 +661,7 @@ PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
   p.k_sf = static_cast<uint8_t*>(a.k_sf);
   p.k_mean = a.k_mean;
   p.ksum = a.ws_ksum;
+  p.cnt = a.ws_cnt;
   return p;
 }
 
@@ -557,6 +672,7 @@ void add_v(PrepassPtrs& p, const QuantVArgs& a) {
   p.v_scales = a.v_scales;
   p.v_sf = static_cast<uint8_t*>(a.v_sf);
   p.vmax = a.ws_vmax;
+  p.cnt = a.ws_cnt;
 }
 
 }  // namespace
@@ -565,11 +681,9 @@ cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
   const PrepassPtrs p = ptrs_qk(a);
   if (a.mode == 0)
     return dispatch<bit(kQuantQ8) | bit(kStatsK), bit(kQuantK8)>(
-        p, a.dtype, a.d, a.B * a.H, Roles{2, {kQuantQ8, kStatsK}}, true, false,
-        Roles{1, {kQuantK8}}, st);
+        p, a.dtype, a.d, a.B * a.H, Roles{2, {kQuantQ8, kStatsK}}, Roles{1, {kQuantK8}}, st);
   return dispatch<bit(kQuantQ4) | bit(kStatsK), bit(kQuantK4)>(
-      p, a.dtype, a.d, a.B * a.H, Roles{2, {kQuantQ4, kStatsK}}, true, false,
-      Roles{1, {kQuantK4}}, st);
+      p, a.dtype, a.d, a.B * a.H, Roles{2, {kQuantQ4, kStatsK}}, Roles{1, {kQuantK4}}, st);
 }
 
 cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st) {
@@ -577,9 +691,9 @@ cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st) {
   add_v(p, a);
   if (a.mode == 0)
     return dispatch<bit(kStatsV), bit(kQuantV8)>(p, a.dtype, a.d, a.B * a.H, Roles{1, {kStatsV}},
-                                                 false, true, Roles{1, {kQuantV8}}, st);
-  return dispatch<bit(kQuantV4), 0>(p, a.dtype, a.d, a.B * a.H, Roles{1, {kQuantV4}}, false,
-                                    false, Roles{0, {}}, st);
+                                                 Roles{1, {kQuantV8}}, st);
+  return dispatch<bit(kQuantV4), 0>(p, a.dtype, a.d, a.B * a.H, Roles{1, {kQuantV4}},
+                                    Roles{0, {}}, st);
 }
 
 cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st) {
@@ -587,10 +701,10 @@ cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStre
   add_v(p, va);
   if (qa.mode == 0)
     return dispatch<bit(kQuantQ8) | bit(kStatsKV), bit(kQuantK8) | bit(kQuantV8)>(
-        p, qa.dtype, qa.d, qa.B * qa.H, Roles{2, {kQuantQ8, kStatsKV}}, true, true,
+        p, qa.dtype, qa.d, qa.B * qa.H, Roles{2, {kQuantQ8, kStatsKV}},
         Roles{2, {kQuantK8, kQuantV8}}, st);
   return dispatch<bit(kQuantQ4) | bit(kQuantV4) | bit(kStatsK), bit(kQuantK4)>(
-      p, qa.dtype, qa.d, qa.B * qa.H, Roles{3, {kQuantQ4, kQuantV4, kStatsK}}, true, false,
+      p, qa.dtype, qa.d, qa.B * qa.H, Roles{3, {kQuantQ4, kQuantV4, kStatsK}},
       Roles{1, {kQuantK4}}, st);
 }
 

@@ -22,6 +22,8 @@ struct QuantQKArgs {
   void* k_sf;
   float* k_mean;
   double* ws_ksum;  // [B*H, N/128, d] FP64 chunk partial sums (workspace)
+  uint32_t* ws_cnt;  // [2][65536] per-head statistics counters: zero before the
+                     // call, zero again after it (workspace)
 };
 
 struct QuantVArgs {
@@ -34,7 +36,11 @@ struct QuantVArgs {
   void* v_sf;
   double* ws_ksum;  // scratch the V statistics pass may write (same size as above)
   float* ws_vmax;   // [B*H, N/128, d] per-chunk |V| maxima (workspace)
+  uint32_t* ws_cnt;  // as in QuantQKArgs
 };
+
+// Bytes of the per-head counters at the start of every workspace.
+constexpr size_t kStatsCounterBytes = size_t(2) * 65536 * 4;
 
 struct AttnArgs {
   int mode;
