@@ -206,7 +206,8 @@ def run_sage(args):
         if ev_attn:
             ev_attn[1].record(stream)
 
-    launches_per_step = 3 + (3 if w.mode == "int8_fp8" else 1) + 1
+    # sage_quant_qk: 2 launches; sage_quant_v: 2 (FP8) or 1 (FP4); attention: 1
+    launches_per_step = 2 + (2 if w.mode == "int8_fp8" else 1) + 1
 
     uuid = None
     try:
