@@ -163,8 +163,17 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                           int causal, float sm_scale, int mode, sage_stream_t stream);
 
 /* Reads and clears the device status word written by the kernels' bounded
- * waits (0 = none expired).  Synchronises the current device. */
+ * waits: SAGE_OK when no wait expired since the last call, else
+ * SAGE_ERR_DEVICE_TIMEOUT (sage_status_string then gives the status bits).
+ * Synchronises the current device. */
 int sage_get_last_device_status(void);
+
+/* Self-test of the kernels' bounded waits: launches a kernel whose
+ * mbarrier wait can never complete.  The wait gives up after about one
+ * second and records a timeout in the device status word (read it with
+ * sage_get_last_device_status); the kernel exits normally and the context
+ * stays usable.  No counterpart on the pages: a failure-detection check. */
+int sage_selftest_bounded_wait(sage_stream_t stream);
 
 /* Human-readable text of a status, with the detail of the calling thread's
  * most recent error when `status` is that error. */

@@ -19,7 +19,8 @@ import math
 import os
 
 __all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
-           "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS"]
+           "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS",
+           "selftest_bounded_wait"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libsage_b200.so")
@@ -33,7 +34,7 @@ BUF = {name: i for i, name in enumerate(
 # every symbol include/sage.h declares
 EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd_quantized",
            "sage_attn_fwd", "sage_attn_fwd_noalloc", "sage_get_last_device_status",
-           "sage_status_string", "sage_version"]
+           "sage_selftest_bounded_wait", "sage_status_string", "sage_version"]
 
 _lib = None
 
@@ -73,6 +74,8 @@ def library():
                                           ctypes.c_float, i32, vp]
     lib.sage_get_last_device_status.restype = i32
     lib.sage_get_last_device_status.argtypes = []
+    lib.sage_selftest_bounded_wait.restype = i32
+    lib.sage_selftest_bounded_wait.argtypes = [vp]
     lib.sage_status_string.restype = ctypes.c_char_p
     lib.sage_status_string.argtypes = [i32]
     lib.sage_version.restype = ctypes.c_char_p
@@ -207,8 +210,17 @@ def sage_attn_fwd_noalloc(q, k, v, causal=False, sm_scale=None, mode="int8_fp8",
 
 
 def device_status():
-    """Reads and clears the kernels' bounded-wait status bits (0 = none)."""
+    """Reads and clears the kernels' bounded-wait status: 0 when no wait
+    expired, else raises SageError (SAGE_ERR_DEVICE_TIMEOUT)."""
     s = library().sage_get_last_device_status()
     if s < 0:
         _check(s)
     return s
+
+
+def selftest_bounded_wait():
+    """Launches the bounded-wait self-test kernel on the current stream (its
+    wait expires after about a second; device_status() then reports it)."""
+    import torch
+    _check(library().sage_selftest_bounded_wait(
+        torch.cuda.current_stream().cuda_stream))

@@ -15,10 +15,27 @@
 
 #include "../../include/sage.h"
 #include "sage_internal.h"
+#include "sage_ptx.cuh"
 
 namespace sage {
 
 __device__ uint32_t g_device_status;  // bits from sage_ptx.cuh, per device
+
+// Self-test of the bounded waits: an mbarrier that nothing arrives on, so
+// the wait runs out (after kWaitLimitNs), records its bit in the status word
+// and returns; the kernel then exits normally.
+__global__ void wait_selftest_kernel(uint32_t* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, kDevTimeoutSoftmax);
+  __syncthreads();
+}
 
 namespace {
 
@@ -401,7 +418,20 @@ int sage_get_last_device_status(void) {
   const uint32_t zero = 0;
   e = cudaMemcpy(di->status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return fail_cuda(e, "clear status");
-  return (int)v;
+  if (v == 0) return SAGE_OK;
+  char bits[96];
+  std::snprintf(bits, sizeof bits, "a bounded wait expired in a kernel (status bits 0x%x)", v);
+  return fail(SAGE_ERR_DEVICE_TIMEOUT, bits);
+}
+
+int sage_selftest_bounded_wait(sage_stream_t stream) {
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  sage::wait_selftest_kernel<<<1, 32, 0, st>>>(di->status);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail_cuda(e, "self-test launch");
+  return SAGE_OK;
 }
 
 const char* sage_status_string(int status) {

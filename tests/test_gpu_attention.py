@@ -203,3 +203,18 @@ def test_full_workloads(cuda_device, name, cos_floor):
         sel = (slice(b, b + 1), slice(h, h + 1))
         check_against_oracle(og[sel][:, :, rows], q[sel], k[sel], v[sel], w.causal, w.sm_scale,
                              w.mode, w.dtype, rows=rows, cos_floor=cos_floor)
+
+
+def test_bounded_wait_expires_and_context_survives(cuda_device):
+    # a wait that nothing completes gives up after about a second, records
+    # the timeout in the device status word, and leaves the context usable
+    assert sage.device_status() == 0
+    sage.selftest_bounded_wait()
+    with pytest.raises(sage.SageError, match="timed out|bounded wait expired"):
+        sage.device_status()
+    assert sage.device_status() == 0          # read-and-clear
+    q, k, v = rand_qkv(1, 2, 256, 128, "bf16", seed=77)
+    o = sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    torch.cuda.synchronize()
+    check_against_oracle(to_numpy32(o), q, k, v, True, 1 / math.sqrt(128), "int8_fp8", "bf16")
+    assert sage.device_status() == 0
