@@ -138,6 +138,21 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
                   int64_t B, int64_t H, int64_t N, int64_t d,
                   int causal, float sm_scale, int mode, sage_stream_t stream);
 
+/* Grouped-query (and multi-query) attention: the kernel-comparison blog
+ * ("Attention kernel benchmarks: speed and memory use") notes that
+ * grouped-query attention changes the shape of the K/V tensors being
+ * quantized.  Here Q and O are [B, H, N, d] while K and V are
+ * [B, Hkv, N, d]; query head h reads key/value head h / (H / Hkv).
+ * Hkv must divide H (Hkv == 1 is multi-query attention; Hkv == H is
+ * exactly sage_attn_fwd).  K is smoothed and K and V are quantized once
+ * per key/value head, so the result equals sage_attn_fwd on K and V
+ * repeated across each group of H / Hkv query heads, bit for bit.  Other
+ * arguments, the workspace and the errors are those of sage_attn_fwd; a
+ * bad Hkv is SAGE_ERR_INVALID_ARG. */
+int sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, int dtype,
+                      int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t d,
+                      int causal, float sm_scale, int mode, sage_stream_t stream);
+
 /* The same forward pass for callers that cannot allocate device memory
  * while they run (a memory pool that admits no new allocations, an
  * allocator that owns the whole device, a caller that may not take the

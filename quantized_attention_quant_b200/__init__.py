@@ -12,13 +12,15 @@ Entry points (same names as the C ABI in include/sage.h):
     sage_quant_v(v, mode="int8_fp8")          -> dict of code/scale tensors
     sage_attn_fwd_quantized(qk, vq, mode, causal, sm_scale, out_dtype) -> O
     sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8") -> O
+    sage_attn_fwd_gqa(q, k, v, ...)           -> O  (K/V with fewer heads than Q)
 """
 
 import ctypes
 import math
 import os
 
-__all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
+__all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_gqa",
+           "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
            "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS",
            "selftest_bounded_wait"]
 
@@ -33,7 +35,8 @@ BUF = {name: i for i, name in enumerate(
 
 # every symbol include/sage.h declares
 EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd_quantized",
-           "sage_attn_fwd", "sage_attn_fwd_noalloc", "sage_get_last_device_status",
+           "sage_attn_fwd", "sage_attn_fwd_gqa", "sage_attn_fwd_noalloc",
+           "sage_get_last_device_status",
            "sage_selftest_bounded_wait", "sage_status_string", "sage_version"]
 
 _lib = None
@@ -69,6 +72,9 @@ def library():
     lib.sage_attn_fwd.restype = i32
     lib.sage_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i32,
                                   ctypes.c_float, i32, vp]
+    lib.sage_attn_fwd_gqa.restype = i32
+    lib.sage_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, i32,
+                                      ctypes.c_float, i32, vp]
     lib.sage_attn_fwd_noalloc.restype = i32
     lib.sage_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i32,
                                           ctypes.c_float, i32, vp]
@@ -175,9 +181,13 @@ def sage_attn_fwd_quantized(qk, vq, shape, mode="int8_fp8", causal=False, sm_sca
 
 
 def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None):
-    """O = softmax(Q K^T sm_scale) V through the quantized path; O has q's dtype."""
+    """O = softmax(Q K^T sm_scale) V through the quantized path; O has q's dtype.
+    K and V with fewer heads than Q (grouped-query attention) go to
+    sage_attn_fwd_gqa."""
     import torch
     B, H, N, d = _shape(q)
+    if _shape(k)[1] != H:
+        return sage_attn_fwd_gqa(q, k, v, causal=causal, sm_scale=sm_scale, mode=mode, out=out)
     if _shape(k) != (B, H, N, d) or _shape(v) != (B, H, N, d):
         raise ValueError("q, k, v must have the same shape")
     if not (q.dtype == k.dtype == v.dtype):
@@ -186,6 +196,24 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=Non
         out = torch.empty_like(q)
     _check(library().sage_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, N, d,
+        int(bool(causal)), float(sm_scale or 0.0), MODES[mode], _stream()))
+    return out
+
+
+def sage_attn_fwd_gqa(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None):
+    """Grouped-query attention: q is [B, H, N, d], k and v are [B, Hkv, N, d]
+    with Hkv dividing H; query head h reads key/value head h // (H // Hkv)."""
+    import torch
+    B, H, N, d = _shape(q)
+    Hkv = _shape(k)[1]
+    if _shape(k) != (B, Hkv, N, d) or _shape(v) != (B, Hkv, N, d):
+        raise ValueError("k and v must be [B, Hkv, N, d] with q's B, N and d")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must have the same dtype")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(library().sage_attn_fwd_gqa(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, Hkv, N, d,
         int(bool(causal)), float(sm_scale or 0.0), MODES[mode], _stream()))
     return out
 

@@ -226,6 +226,83 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
 
 using namespace sage;
 
+extern "C" size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N,
+                                    int64_t d);
+
+namespace {
+
+// H >= 0 is already checked; no query heads means no key/value heads
+int check_kv_heads(int64_t H, int64_t Hkv) {
+  if (H == 0 ? Hkv != 0 : (Hkv < 1 || Hkv > H || H % Hkv != 0))
+    return fail(SAGE_ERR_INVALID_ARG, "Hkv must be >= 1 and divide H");
+  return SAGE_OK;
+}
+
+// Q-side buffers are per query head, K/V-side ones per key/value head
+int64_t heads_of(int which, int64_t H, int64_t Hkv) {
+  return which == SAGE_BUF_Q_CODES || which == SAGE_BUF_Q_SCALES || which == SAGE_BUF_Q_SF ? H
+                                                                                          : Hkv;
+}
+
+// The whole pipeline (pre-pass, then attention) with every buffer carved
+// from the per-stream workspace. Q and O have H heads, K and V have Hkv heads
+// (Hkv divides H; Hkv == H is plain multi-head attention).
+int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,
+                  int64_t H, int64_t Hkv, int64_t N, int64_t d, int causal, float sm_scale,
+                  int mode, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_kv_heads(H, Hkv));
+  SAGE_TRY(check_ptr(q, "q", true));
+  SAGE_TRY(check_ptr(k, "k", true));
+  SAGE_TRY(check_ptr(v, "v", true));
+  SAGE_TRY(check_ptr(o, "o", true));
+  if (!(sm_scale > 0.f)) sm_scale = 1.0f / std::sqrt((float)d);
+  if (!std::isfinite(sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be finite");
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  size_t off[SAGE_BUF_V_SF + 1];
+  size_t total = 0;
+  for (int w = 0; w <= SAGE_BUF_V_SF; ++w) {
+    off[w] = total;
+    total += align_up(sage_buffer_bytes(mode, w, B, heads_of(w, H, Hkv), N, d));
+  }
+  const size_t off_ksum = total;
+  total += align_up(ws_ksum_bytes(B * Hkv, N, d));
+  const size_t off_vmax = total;
+  total += align_up(ws_vmax_bytes(B * Hkv, N, d));
+  void* ws = nullptr;
+  uint32_t* cnt = nullptr;
+  SAGE_TRY(workspace(st, total, &ws, &cnt));
+  char* base = static_cast<char*>(ws);
+  auto at = [&](int w) -> void* {
+    return sage_buffer_bytes(mode, w, B, heads_of(w, H, Hkv), N, d) ? base + off[w] : nullptr;
+  };
+  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d, Hkv,
+                 at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+                 at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum), cnt};
+  QuantVArgs va{v, dtype, mode, B, Hkv, N, d,
+                at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+                reinterpret_cast<double*>(base + off_ksum),
+                reinterpret_cast<float*>(base + off_vmax), cnt};
+  cudaError_t e = launch_prepass(qa, va, st);
+  if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
+  AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+              at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+              at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+              o, dtype, B, H, N, d, Hkv, causal != 0, sm_scale, di->status};
+  const char* detail = nullptr;
+  e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
+  if (detail) return fail(SAGE_ERR_CUDA, detail);
+  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  return SAGE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, int64_t d) {
@@ -281,7 +358,7 @@ int sage_quant_qk(const void* q, const void* k, int dtype, int64_t B, int64_t H,
   void* ws = nullptr;
   uint32_t* cnt = nullptr;
   SAGE_TRY(workspace(st, ws_ksum_bytes(B * H, N, d), &ws, &cnt));
-  QuantQKArgs a{q, k, dtype, mode, B, H, N, d, q_codes, q_scales, q_sf,
+  QuantQKArgs a{q, k, dtype, mode, B, H, N, d, H, q_codes, q_scales, q_sf,
                 k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws), cnt};
   cudaError_t e = launch_quant_qk(a, st);
   if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
@@ -344,7 +421,7 @@ int sage_attn_fwd_quantized(int mode, const void* q_codes, const float* q_scales
   SAGE_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   AttnArgs a{mode, q_codes, q_scales, q_sf, k_codes, k_scales, k_sf, v_codes, v_scales, v_sf,
-             o, dtype, B, H, N, d, causal != 0, sm_scale, di->status};
+             o, dtype, B, H, N, d, H, causal != 0, sm_scale, di->status};
   const char* detail = nullptr;
   cudaError_t e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(a, st, &detail)
                                         : launch_attn_i8f8(a, st, &detail);
@@ -356,54 +433,13 @@ int sage_attn_fwd_quantized(int mode, const void* q_codes, const float* q_scales
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,
                   int64_t H, int64_t N, int64_t d, int causal, float sm_scale, int mode,
                   sage_stream_t stream) {
-  bool empty = false;
-  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
-  SAGE_TRY(check_ptr(q, "q", true));
-  SAGE_TRY(check_ptr(k, "k", true));
-  SAGE_TRY(check_ptr(v, "v", true));
-  SAGE_TRY(check_ptr(o, "o", true));
-  if (!(sm_scale > 0.f)) sm_scale = 1.0f / std::sqrt((float)d);
-  if (!std::isfinite(sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be finite");
-  if (empty) return SAGE_OK;
-  DeviceInfo* di = nullptr;
-  SAGE_TRY(device_info(&di));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  size_t off[SAGE_BUF_V_SF + 1];
-  size_t total = 0;
-  for (int w = 0; w <= SAGE_BUF_V_SF; ++w) {
-    off[w] = total;
-    total += align_up(sage_buffer_bytes(mode, w, B, H, N, d));
-  }
-  const size_t off_ksum = total;
-  total += align_up(ws_ksum_bytes(B * H, N, d));
-  const size_t off_vmax = total;
-  total += align_up(ws_vmax_bytes(B * H, N, d));
-  void* ws = nullptr;
-  uint32_t* cnt = nullptr;
-  SAGE_TRY(workspace(st, total, &ws, &cnt));
-  char* base = static_cast<char*>(ws);
-  auto at = [&](int w) -> void* {
-    return sage_buffer_bytes(mode, w, B, H, N, d) ? base + off[w] : nullptr;
-  };
-  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d,
-                 at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
-                 at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
-                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum), cnt};
-  QuantVArgs va{v, dtype, mode, B, H, N, d,
-                at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
-                reinterpret_cast<double*>(base + off_ksum),
-                reinterpret_cast<float*>(base + off_vmax), cnt};
-  cudaError_t e = launch_prepass(qa, va, st);
-  if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
-  AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
-              at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
-              at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
-              o, dtype, B, H, N, d, causal != 0, sm_scale, di->status};
-  const char* detail = nullptr;
-  e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
-  if (detail) return fail(SAGE_ERR_CUDA, detail);
-  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
-  return SAGE_OK;
+  return attn_fwd_full(q, k, v, o, dtype, B, H, H, N, d, causal, sm_scale, mode, stream);
+}
+
+int sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,
+                      int64_t H, int64_t Hkv, int64_t N, int64_t d, int causal, float sm_scale,
+                      int mode, sage_stream_t stream) {
+  return attn_fwd_full(q, k, v, o, dtype, B, H, Hkv, N, d, causal, sm_scale, mode, stream);
 }
 
 int sage_get_last_device_status(void) {
@@ -548,7 +584,7 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
   // Every scratch byte the kernels read is written earlier in the same call
   // (codes, scales, statistics partials), except the per-head counters:
   // zero in the loaded image, and returned to zero by every pre-pass.
-  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d,
+  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d, H,
                  at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
                  at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
                  (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum), cnt};
@@ -561,7 +597,7 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
-              o, dtype, B, H, N, d, causal != 0, sm_scale, di->status};
+              o, dtype, B, H, N, d, H, causal != 0, sm_scale, di->status};
   const char* detail = nullptr;
   e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
   if (detail) return fail(SAGE_ERR_CUDA, detail);

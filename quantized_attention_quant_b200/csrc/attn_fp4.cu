@@ -360,7 +360,8 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 // Stats warpgroup: row max / running max per key tile, level-2 fold (one
 // tile behind), epilogue.
 template <bool CAUSAL, typename OutT>
-__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh, const int N,
+__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh,
+                                           const int H, const int G, const int N,
                                            const int ntiles, const uint32_t tmem, const Bars& bar,
                                            uint8_t* smem, volatile int* abort_flag,
                                            uint32_t* status, const float* __restrict__ q_scales,
@@ -376,8 +377,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float* m_s = reinterpret_cast<float*>(smem + L::OFF_M);
   const float* l_s = reinterpret_cast<const float*>(smem + L::OFF_L);
   const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
-  const float* ksp = k_scales + (int64_t)bh * ntiles;
-  const float* vgp = v_scales + (int64_t)bh * ntiles;
+  const float* ksp = k_scales + (int64_t)kv_head(bh, H, G) * ntiles;
+  const float* vgp = v_scales + (int64_t)kv_head(bh, H, G) * ntiles;
 
   float2 o2[D / 2];
 #pragma unroll
@@ -473,8 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scales,
                     const float* __restrict__ k_scales, const float* __restrict__ v_scales,
                     const uint8_t* __restrict__ q_sf, const uint8_t* __restrict__ k_sf,
-                    const uint8_t* __restrict__ v_sf, OutT* __restrict__ out, int N,
-                    float scale_log2, uint32_t* status) {
+                    const uint8_t* __restrict__ v_sf, OutT* __restrict__ out, int N, int H,
+                    int G, float scale_log2, uint32_t* status) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -483,6 +484,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int ntiles = N / 128;
   const int bh = blockIdx.y;
+  // K/V head of this query head (grouped-query attention: G query heads per
+  // K/V head; G = 1 is plain multi-head attention)
+  const int bhk = kv_head(bh, H, G);
   const int qt = CAUSAL ? (ntiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy first
   const int nkv = CAUSAL ? qt + 1 : ntiles;
 
@@ -543,24 +547,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (elect_one()) {
-        const int64_t tile0 = (int64_t)bh * ntiles;
+        const int64_t tile0 = (int64_t)bhk * ntiles;
         mbar_arrive_expect_tx(bar.q_full, L::TILE + L::SF);
         tma_load_2d(sQ, &tm_q, 0, bh * N + qt * 128, bar.q_full);
-        bulk_load(sSFQ, q_sf + (tile0 + qt) * L::SF, L::SF, bar.q_full);
+        bulk_load(sSFQ, q_sf + ((int64_t)bh * ntiles + qt) * L::SF, L::SF, bar.q_full);
         for (int j = 0; j < nkv; ++j) {
           const int sk = j % L::KS;
           if (!mbar_wait<true>(&bar.k_empty[sk], ((j / L::KS) & 1) ^ 1, abort_flag, status,
                                kDevTimeoutMma))
             break;
           mbar_arrive_expect_tx(&bar.k_full[sk], L::TILE + L::SF);
-          tma_load_2d(sK + sk * L::TILE, &tm_k, 0, bh * N + j * 128, &bar.k_full[sk]);
+          tma_load_2d(sK + sk * L::TILE, &tm_k, 0, bhk * N + j * 128, &bar.k_full[sk]);
           bulk_load(sSFK + sk * L::SF, k_sf + (tile0 + j) * L::SF, L::SF, &bar.k_full[sk]);
           const int sv = j % L::VS;
           if (!mbar_wait<true>(&bar.v_empty[sv], ((j / L::VS) & 1) ^ 1, abort_flag, status,
                                kDevTimeoutMma))
             break;
           mbar_arrive_expect_tx(&bar.v_full[sv], L::TILE + L::SF);
-          tma_load_2d(sV + sv * L::TILE, &tm_v, j * 64, bh * D, &bar.v_full[sv]);
+          tma_load_2d(sV + sv * L::TILE, &tm_v, j * 64, bhk * D, &bar.v_full[sv]);
           bulk_load(sSFV + sv * L::SF, v_sf + (tile0 + j) * L::SF, L::SF, &bar.v_full[sv]);
         }
       }
@@ -657,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      k_scales, scale_log2);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<CAUSAL, OutT>(qt, nkv, bh, N, ntiles, tmem, bar, smem, abort_flag, status,
+    stats_loop<CAUSAL, OutT>(qt, nkv, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
                              q_scales, k_scales, v_scales, out, scale_log2);
   }
 
@@ -681,7 +685,8 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtenso
   kern<<<grid, kThreads, L::SMEM, st>>>(
       tq, tk, tv, a.q_scales, a.k_scales, a.v_scales, static_cast<const uint8_t*>(a.q_sf),
       static_cast<const uint8_t*>(a.k_sf), static_cast<const uint8_t*>(a.v_sf),
-      reinterpret_cast<OutT*>(a.o), (int)a.N, a.sm_scale * kLog2e, a.status);
+      reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H, (int)(a.H / a.Hkv), a.sm_scale * kLog2e,
+      a.status);
   return cudaGetLastError();
 }
 
@@ -693,14 +698,15 @@ cudaError_t launch_attn_fp4(const AttnArgs& a, cudaStream_t st, const char** det
     return cudaErrorInvalidValue;
   }
   const uint64_t BH = (uint64_t)(a.B * a.H);
+  const uint64_t BHK = (uint64_t)(a.B * a.Hkv);
   const uint64_t N = (uint64_t)a.N;
   CUtensorMap tq, tk, tv;
   // Q, K: [B*H*N rows, 64 bytes]; V^T: [B*H*128 rows (channels), N/2 bytes]
   if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q_codes, 64, BH * N, 64, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_64B, detail) ||
-      !encode_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.k_codes, 64, BH * N, 64, 64, 128,
+      !encode_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.k_codes, 64, BHK * N, 64, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_64B, detail) ||
-      !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.v_codes, N / 2, BH * D, N / 2, 64, 128,
+      !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.v_codes, N / 2, BHK * D, N / 2, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_64B, detail))
     return cudaErrorInvalidValue;
   if (a.causal)

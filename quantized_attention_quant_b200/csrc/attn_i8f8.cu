@@ -362,7 +362,8 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 // Stats warpgroup: row max / running max per key tile, level-2 fold,
 // epilogue.
 template <int D, bool CAUSAL, typename OutT>
-__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh, const int N,
+__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh,
+                                           const int H, const int G, const int N,
                                            const int ntiles, const uint32_t tmem, const Bars& bar,
                                            uint8_t* smem, volatile int* abort_flag,
                                            uint32_t* status, const float* __restrict__ q_scales,
@@ -378,7 +379,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float* m_s = reinterpret_cast<float*>(smem + L::OFF_M);
   const float* l_s = reinterpret_cast<const float*>(smem + L::OFF_L);
   const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
-  const float* ksp = k_scales + (int64_t)bh * ntiles;
+  const float* ksp = k_scales + (int64_t)kv_head(bh, H, G) * ntiles;
 
   float2 o2[D / 2];
 #pragma unroll
@@ -456,7 +457,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
                   mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)))
     return;
   const float inv_l = 1.f / (l_s[r] + l_s[128 + r]);
-  const float* vs = v_scales + (int64_t)bh * D;
+  const float* vs = v_scales + (int64_t)kv_head(bh, H, G) * D;
   OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
 #pragma unroll
   for (int cv = 0; cv < D; cv += 8) {
@@ -476,7 +477,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scales,
                      const float* __restrict__ k_scales, const float* __restrict__ v_scales,
-                     OutT* __restrict__ out, int N, float scale_log2, uint32_t* status) {
+                     OutT* __restrict__ out, int N, int H, int G, float scale_log2,
+                     uint32_t* status) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -485,6 +487,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const int lane = threadIdx.x & 31;
   const int ntiles = N / 128;
   const int bh = blockIdx.y;
+  // K/V head of this query head (grouped-query attention: G query heads per
+  // K/V head; G = 1 is plain multi-head attention)
+  const int bhk = kv_head(bh, H, G);
   const int qt = CAUSAL ? (ntiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy first
   const int nkv = CAUSAL ? qt + 1 : ntiles;
 
@@ -553,13 +558,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                kDevTimeoutMma))
             break;
           mbar_arrive_expect_tx(&bar.k_full[sk], L::K_BYTES);
-          tma_load_2d(sK + sk * L::K_BYTES, &tm_k, 0, bh * N + j * 128, &bar.k_full[sk]);
+          tma_load_2d(sK + sk * L::K_BYTES, &tm_k, 0, bhk * N + j * 128, &bar.k_full[sk]);
           const int sv = j % L::VS;
           if (!mbar_wait<true>(&bar.v_empty[sv], ((j / L::VS) & 1) ^ 1, abort_flag, status,
                                kDevTimeoutMma))
             break;
           mbar_arrive_expect_tx(&bar.v_full[sv], L::V_BYTES);
-          tma_load_2d(sV + sv * L::V_BYTES, &tm_v, j * 128, bh * D, &bar.v_full[sv]);
+          tma_load_2d(sV + sv * L::V_BYTES, &tm_v, j * 128, bhk * D, &bar.v_full[sv]);
         }
       }
       __syncwarp();
@@ -649,7 +654,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     exp_loop<D, CAUSAL>(wg - 1, qt, nkv, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<D, CAUSAL, OutT>(qt, nkv, bh, N, ntiles, tmem, bar, smem, abort_flag, status,
+    stats_loop<D, CAUSAL, OutT>(qt, nkv, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
                                 q_scales, k_scales, v_scales, out, scale_log2);
   }
 
@@ -675,8 +680,8 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtenso
   const int ntiles = (int)(a.N / 128);
   dim3 grid((unsigned)ntiles, (unsigned)(a.B * a.H));
   kern<<<grid, kThreadsAttn, L::SMEM, st>>>(tq, tk, tv, a.q_scales, a.k_scales, a.v_scales,
-                                           reinterpret_cast<OutT*>(a.o), (int)a.N,
-                                           a.sm_scale * kLog2e, a.status);
+                                           reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H,
+                                           (int)(a.H / a.Hkv), a.sm_scale * kLog2e, a.status);
   return cudaGetLastError();
 }
 
@@ -695,6 +700,7 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap
 
 cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** detail) {
   const uint64_t BH = (uint64_t)(a.B * a.H);
+  const uint64_t BHK = (uint64_t)(a.B * a.Hkv);
   const uint64_t N = (uint64_t)a.N;
   const uint64_t D = (uint64_t)a.d;
   CUtensorMap tq, tk, tv;
@@ -702,9 +708,9 @@ cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** de
       D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q_codes, D, BH * N, D, (uint32_t)D, 128,
                       qk_swz, detail) ||
-      !encode_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.k_codes, D, BH * N, D, (uint32_t)D, 128,
-                      qk_swz, detail) ||
-      !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.v_codes, N, BH * D, N, 128, (uint32_t)D,
+      !encode_tmap_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.k_codes, D, BHK * N, D, (uint32_t)D,
+                      128, qk_swz, detail) ||
+      !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.v_codes, N, BHK * D, N, 128, (uint32_t)D,
                       CU_TENSOR_MAP_SWIZZLE_128B, detail))
     return cudaErrorInvalidValue;
   return D == 128 ? launch_d<128>(a, tq, tk, tv, st) : launch_d<64>(a, tq, tk, tv, st);

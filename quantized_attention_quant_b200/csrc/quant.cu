@@ -69,6 +69,8 @@ struct PrepassPtrs {
   double* ksum;  // [B*H, N/128, d] FP64 chunk sums of K
   float* vmax;   // [B*H, N/128, d] chunk maxima of |V|
   uint32_t* cnt;  // [2][kMaxHeads] statistics CTAs done per head (K, V); 0 between passes
+  int64_t bh_q;   // Q heads (B * H)
+  int64_t bh_kv;  // K/V heads (B * Hkv; fewer than bh_q under grouped-query attention)
 };
 
 constexpr int kMaxHeads = 65536;
@@ -567,6 +569,10 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   const int role = roles.r[blockIdx.z];
   const int64_t bh = blockIdx.y;
   const int tile = blockIdx.x;
+  // the grid spans the larger head count: Q roles cover bh_q heads, K/V
+  // roles bh_kv (a CTA leaves as a whole, before any barrier)
+  const bool q_role = role == kQuantQ8 || role == kQuantQ4;
+  if (bh >= (q_role ? p.bh_q : p.bh_kv)) return;
   const int ntiles = p.N / 128;
   const int64_t row0 = bh * p.N + (int64_t)tile * 128;
   switch (role) {
@@ -628,10 +634,12 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
 constexpr int bit(int r) { return 1 << r; }
 
 // kernel A (roles a; its statistics CTAs also fold the head statistics),
-// then kernel B (roles b)
+// then kernel B (roles b); the grids span the larger of the Q and K/V head
+// counts
 template <typename T, int D, int MA, int MB>
-cudaError_t run_plan(const PrepassPtrs& p, int64_t BH, Roles a, Roles b, cudaStream_t st) {
+cudaError_t run_plan(const PrepassPtrs& p, Roles a, Roles b, cudaStream_t st) {
   const int ntiles = p.N / 128;
+  const int64_t BH = p.bh_q > p.bh_kv ? p.bh_q : p.bh_kv;
   if (a.n) prepass_kernel<T, D, MA><<<dim3(ntiles, (unsigned)BH, a.n), kThreads, 0, st>>>(p, a);
   if (b.n) prepass_kernel<T, D, MB><<<dim3(ntiles, (unsigned)BH, b.n), kThreads, 0, st>>>(p, b);
   return cudaGetLastError();
@@ -639,13 +647,13 @@ cudaError_t run_plan(const PrepassPtrs& p, int64_t BH, Roles a, Roles b, cudaStr
 
 // MA / MB: the role masks of kernels A and B (they must cover a.r / b.r).
 template <int MA, int MB>
-cudaError_t dispatch(const PrepassPtrs& p, int dtype, int64_t d, int64_t BH, Roles a, Roles b,
+cudaError_t dispatch(const PrepassPtrs& p, int dtype, int64_t d, Roles a, Roles b,
                      cudaStream_t st) {
   if (dtype == 1)
-    return d == 128 ? run_plan<__nv_bfloat16, 128, MA, MB>(p, BH, a, b, st)
-                    : run_plan<__nv_bfloat16, 64, MA, MB>(p, BH, a, b, st);
-  return d == 128 ? run_plan<__half, 128, MA, MB>(p, BH, a, b, st)
-                  : run_plan<__half, 64, MA, MB>(p, BH, a, b, st);
+    return d == 128 ? run_plan<__nv_bfloat16, 128, MA, MB>(p, a, b, st)
+                    : run_plan<__nv_bfloat16, 64, MA, MB>(p, a, b, st);
+  return d == 128 ? run_plan<__half, 128, MA, MB>(p, a, b, st)
+                  : run_plan<__half, 64, MA, MB>(p, a, b, st);
 }
 
 PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
@@ -662,6 +670,8 @@ PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
   p.k_mean = a.k_mean;
   p.ksum = a.ws_ksum;
   p.cnt = a.ws_cnt;
+  p.bh_q = a.B * a.H;
+  p.bh_kv = a.B * a.Hkv;
   return p;
 }
 
@@ -673,6 +683,7 @@ void add_v(PrepassPtrs& p, const QuantVArgs& a) {
   p.v_sf = static_cast<uint8_t*>(a.v_sf);
   p.vmax = a.ws_vmax;
   p.cnt = a.ws_cnt;
+  p.bh_kv = a.B * a.H;  // QuantVArgs counts K/V heads in H
 }
 
 }  // namespace
@@ -681,18 +692,18 @@ cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
   const PrepassPtrs p = ptrs_qk(a);
   if (a.mode == 0)
     return dispatch<bit(kQuantQ8) | bit(kStatsK), bit(kQuantK8)>(
-        p, a.dtype, a.d, a.B * a.H, Roles{2, {kQuantQ8, kStatsK}}, Roles{1, {kQuantK8}}, st);
+        p, a.dtype, a.d, Roles{2, {kQuantQ8, kStatsK}}, Roles{1, {kQuantK8}}, st);
   return dispatch<bit(kQuantQ4) | bit(kStatsK), bit(kQuantK4)>(
-      p, a.dtype, a.d, a.B * a.H, Roles{2, {kQuantQ4, kStatsK}}, Roles{1, {kQuantK4}}, st);
+      p, a.dtype, a.d, Roles{2, {kQuantQ4, kStatsK}}, Roles{1, {kQuantK4}}, st);
 }
 
 cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st) {
   PrepassPtrs p{};
   add_v(p, a);
   if (a.mode == 0)
-    return dispatch<bit(kStatsV), bit(kQuantV8)>(p, a.dtype, a.d, a.B * a.H, Roles{1, {kStatsV}},
+    return dispatch<bit(kStatsV), bit(kQuantV8)>(p, a.dtype, a.d, Roles{1, {kStatsV}},
                                                  Roles{1, {kQuantV8}}, st);
-  return dispatch<bit(kQuantV4), 0>(p, a.dtype, a.d, a.B * a.H, Roles{1, {kQuantV4}},
+  return dispatch<bit(kQuantV4), 0>(p, a.dtype, a.d, Roles{1, {kQuantV4}},
                                     Roles{0, {}}, st);
 }
 
@@ -701,10 +712,10 @@ cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStre
   add_v(p, va);
   if (qa.mode == 0)
     return dispatch<bit(kQuantQ8) | bit(kStatsKV), bit(kQuantK8) | bit(kQuantV8)>(
-        p, qa.dtype, qa.d, qa.B * qa.H, Roles{2, {kQuantQ8, kStatsKV}},
+        p, qa.dtype, qa.d, Roles{2, {kQuantQ8, kStatsKV}},
         Roles{2, {kQuantK8, kQuantV8}}, st);
   return dispatch<bit(kQuantQ4) | bit(kQuantV4) | bit(kStatsK), bit(kQuantK4)>(
-      p, qa.dtype, qa.d, qa.B * qa.H, Roles{3, {kQuantQ4, kQuantV4, kStatsK}},
+      p, qa.dtype, qa.d, Roles{3, {kQuantQ4, kQuantV4, kStatsK}},
       Roles{1, {kQuantK4}}, st);
 }
 

@@ -14,6 +14,7 @@ struct QuantQKArgs {
   int dtype;  // 0 = f16, 1 = bf16
   int mode;   // 0 = INT8, 1 = FP4
   int64_t B, H, N, d;
+  int64_t Hkv;  // K heads (H % Hkv == 0; Hkv == H without grouped-query attention)
   void* q_codes;
   float* q_scales;
   void* q_sf;
@@ -56,6 +57,7 @@ struct AttnArgs {
   void* o;
   int dtype;
   int64_t B, H, N, d;
+  int64_t Hkv;  // K/V heads: query head h reads K/V head h / (H / Hkv)
   int causal;
   float sm_scale;
   uint32_t* status;  // device status word
@@ -70,6 +72,12 @@ cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStre
 // of something other than a CUDA call (e.g. tensor-map encoding).
 cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** detail);
 cudaError_t launch_attn_fp4(const AttnArgs& a, cudaStream_t st, const char** detail);
+
+// Grouped-query attention: the key/value head read by flattened query head
+// bh = b * H + h, with G query heads per key/value head (G = 1: multi-head).
+__host__ __device__ __forceinline__ int kv_head(int bh, int H, int G) {
+  return (bh / H) * (H / G) + (bh % H) / G;
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (the
 // library does not link libcuda).  Returns false with a message on failure.

@@ -101,3 +101,24 @@ def test_quant_argument_errors(lib):
 def test_status_strings(lib):
     for s, t in [(0, "ok"), (-1, "invalid"), (-2, "unsupported"), (-3, "CUDA"), (-4, "timed out")]:
         assert t in lib.sage_status_string(s).decode()
+
+
+def gqa(lib, B=2, H=8, Hkv=2, N=128, d=128, mode=0):
+    lib.sage_attn_fwd_gqa.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] + \
+        [ctypes.c_int64] * 5 + [ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
+    return lib.sage_attn_fwd_gqa(FAKE, FAKE, FAKE, FAKE, 1, B, H, Hkv, N, d, 0,
+                                 ctypes.c_float(0.0), mode, None)
+
+
+@pytest.mark.parametrize("H,Hkv", [(8, 0), (8, 3), (8, 16), (8, -1), (0, 1)])
+def test_gqa_head_count_errors(lib, H, Hkv):
+    s = gqa(lib, H=H, Hkv=Hkv)
+    assert s == -1 and "Hkv" in lib.sage_status_string(s).decode()
+
+
+def test_gqa_empty_and_shape_errors(lib):
+    assert gqa(lib, B=0) == 0
+    assert gqa(lib, N=0) == 0
+    assert gqa(lib, H=0, Hkv=0) == 0
+    s = gqa(lib, N=200)
+    assert s == -2 and "multiple of 128" in lib.sage_status_string(s).decode()
