@@ -12,7 +12,8 @@ traffic" for the tiled online softmax):
 
   for each query row, over key tiles j = 0, 1, ... of 128 keys, in order
   (causal: only keys t_k <= t_q):
-    A      = q_codes . k_codes^T                (exact integer / exact FP64)
+    A      = q_codes . k_codes^T                (exact integer / exact FP64;
+                                                 FP8 Q/K mode: e4m3 codes)
     S      = A * s_Q * s_K * sm_scale           (FP4: A * g_Q * g_K * sm_scale,
                                                  block scales inside A)
     m_new  = max(m, rowmax S)
@@ -42,6 +43,11 @@ from .encoders import (e4m3_encode, e4m3_decode, e2m1_encode, e2m1_decode,
 BLOCK = pp.BLOCK
 P_FP8_SCALE = 448.0
 P_FP4_G = 1.0 / 2688.0
+# FP8 Q/K mode: a product of two e4m3 values is exact in FP32, but their sum
+# over the d channels is accumulated in FP32 by the tensor core, in an order
+# the oracle does not know.  Any order of n FP32 additions errs by at most
+# (n - 1) u sum|terms| (u = 2^-24, first order); n <= 128 gives this bound.
+FP8_QK_ACC_REL = 2.0 ** -17
 
 
 def exact_attention(q, k, v, causal=False, sm_scale=None, row_chunk=1024, rows=None):
@@ -173,7 +179,7 @@ def fp4_p_ambiguity(pt, eps):
 # --------------------------------------------------------------------------
 
 def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows=None,
-               p_ambiguity=None):
+               p_ambiguity=None, qk_acc_rel=0.0):
     """Online softmax + two-level P~V accumulation for one (b, h).
 
     qd [N, d], kd [N, d]: decoded code values (exact FP64).
@@ -184,9 +190,16 @@ def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows
     p_quant: P~ -> quantized P~ values (scaled as the partial expects).
     rows: query rows to compute (default all); each row's arithmetic does not
     depend on which other rows are computed.
-    p_ambiguity: optional P~ -> size of a possible code change (see
-    fp8_p_ambiguity); then a second array bounds, per output element, how far
-    O can move when every ambiguous code takes its other valid value.
+    p_ambiguity: optional (P~, extra relative perturbation) -> size of a
+    possible code change (see fp8_p_ambiguity); then a second array bounds,
+    per output element, how far O can move when every ambiguous code takes
+    its other valid value.
+    qk_acc_rel: relative accumulation error of the kernel's Q K^T (0 when it
+    is exact, as in INT8 mode).  With the bound requested, each score may
+    then be off by dS = qk_acc_rel |q| . |k| (dequantized), the running max by
+    the largest dS so far (Dm), so each P~ by a factor within exp(+-(dS +
+    Dm)): the code decisions get that much extra room, and the row sum (thus
+    O / l) a relative deviation of at most expm1(2 Dm).
     Returns O [len(rows), d] in FP64 (before the output rounding), and the
     bound when p_ambiguity is given.
     """
@@ -197,12 +210,13 @@ def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows
     Bd = np.zeros((R, d)) if p_ambiguity is not None else None
     m = np.full(R, -np.inf)
     l = np.zeros(R)
+    Dm = np.zeros(R)
     for j, (ks, ke) in enumerate(pp._blocks(N)):
         act = np.nonzero(rows >= ks)[0] if causal else np.arange(R)   # rows that see tile j
         if act.size == 0:
             continue
         r_act = rows[act]
-        A = qd[r_act] @ kd[ks:ke].T               # exact
+        A = qk_product(qd[r_act], kd[ks:ke])       # exact
         S = A * s_row[r_act, None] * s_key[None, ks:ke] * sm_scale
         if causal:
             S = np.where(np.arange(ks, ke)[None, :] <= r_act[:, None], S, -np.inf)
@@ -213,13 +227,31 @@ def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows
         partial = p @ vd[ks:ke]                   # level 1: exact
         O[act] = alpha[:, None] * O[act] + partial * v_fold[j][None, :]
         if Bd is not None:
+            extra = 0.0
+            if qk_acc_rel:
+                dS = qk_acc_rel * (np.abs(qd[r_act]) @ np.abs(kd[ks:ke]).T) * \
+                    s_row[r_act, None] * s_key[None, ks:ke] * sm_scale
+                if causal:
+                    dS = np.where(np.arange(ks, ke)[None, :] <= r_act[:, None], dS, 0.0)
+                Dm[act] = np.maximum(Dm[act], dS.max(axis=1))
+                extra = np.expm1(dS + Dm[act][:, None])
             Bd[act] = alpha[:, None] * Bd[act] + \
-                (p_ambiguity(Pt) @ np.abs(vd[ks:ke])) * np.abs(v_fold[j])[None, :]
+                (p_ambiguity(Pt, extra) @ np.abs(vd[ks:ke])) * np.abs(v_fold[j])[None, :]
         l[act] = alpha * l[act] + Pt.sum(axis=1)
         m[act] = m_new
     if Bd is not None:
-        return O / l[:, None], Bd / l[:, None]
+        grow = np.exp(2.0 * Dm)[:, None]
+        return O / l[:, None], Bd / l[:, None] * grow + np.abs(O / l[:, None]) * (grow - 1.0)
     return O / l[:, None]
+
+
+def qk_product(qd, kd):
+    """A = qd . kd^T for decoded code values in FP64.  Exact for INT8 codes
+    (integer sums below 2^53) and for e4m3 codes (products of 8 significant
+    bits spanning 2^-18 .. 2^17.6: 8 + 36 + 7 bits for 128 terms < 53).  FP4
+    values times their UE4M3 group scales can span a wider range, where FP64
+    errs by at most 128 * 2^-53 of sum|terms| (far below any tolerance)."""
+    return qd @ kd.T
 
 
 def _identity(x):
@@ -230,7 +262,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                             quantizers="faithful", rows=None, ambiguity_eps=None):
     """Step-by-step emulation of the quantized forward pass, FP64 O [B,H,N,d].
 
-    mode: "int8_fp8" (INT8 Q/K, FP8 P~ and V) or "fp4" (FP4 Q/K/P~/V).
+    mode: "int8_fp8" (INT8 Q/K, FP8 P~ and V), "fp8" (FP8 Q/K, P~ and V) or
+    "fp4" (FP4 Q/K/P~/V).
     quantizers="identity" replaces every quantizer by the identity (codes =
     the values, scales = 1, P~ unrounded); the result must then equal
     ``exact_attention`` up to FP64 rounding.
@@ -239,7 +272,9 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     ambiguity_eps: when given, also return a per-element bound on how far O
     moves if every P~ decision lying within this relative distance of a
     rounding midpoint takes its other (equally valid) value: the e4m3 codes in
-    INT8/FP8 mode; the UE4M3 group scales and e2m1 codes in FP4 mode.
+    INT8/FP8 and FP8 mode; the UE4M3 group scales and e2m1 codes in FP4 mode.
+    In FP8 mode the bound also covers the FP32 accumulation of Q K^T
+    (FP8_QK_ACC_REL).
     """
     q = np.asarray(q, np.float32)
     k = np.asarray(k, np.float32)
@@ -263,21 +298,28 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     if quantizers != "faithful":
         raise ValueError(quantizers)
 
-    if mode == "int8_fp8":
+    if mode in ("int8_fp8", "fp8"):
+        fp8_qk = mode == "fp8"
         bound = np.zeros_like(out) if ambiguity_eps is not None else None
-        amb = (lambda pt: fp8_p_ambiguity(pt, ambiguity_eps)) if bound is not None else None
-        qk = pp.quant_qk_int8(q, k)
+        amb = ((lambda pt, extra: fp8_p_ambiguity(pt, ambiguity_eps + extra))
+               if bound is not None else None)
+        qk = pp.quant_qk_fp8(q, k) if fp8_qk else pp.quant_qk_int8(q, k)
         vc, vs = pp.quant_v_fp8(v)
         for b in range(B):
             for h in range(H):
-                qd = qk["q_codes"][b, h].astype(np.float64)
-                kd = qk["k_codes"][b, h].astype(np.float64)
+                if fp8_qk:
+                    qd = e4m3_decode(qk["q_codes"][b, h])
+                    kd = e4m3_decode(qk["k_codes"][b, h])
+                else:
+                    qd = qk["q_codes"][b, h].astype(np.float64)
+                    kd = qk["k_codes"][b, h].astype(np.float64)
                 vd = e4m3_decode(vc[b, h]).T                      # [N, d]
                 s_row = qk["q_scales"][b, h].astype(np.float64)[tile_of]
                 s_key = qk["k_scales"][b, h].astype(np.float64)[tile_of]
                 v_fold = np.broadcast_to(vs[b, h].astype(np.float64) / P_FP8_SCALE, (ntiles, d))
                 res = _tile_loop(qd, kd, vd, s_row, s_key, v_fold, quant_p_fp8,
-                                 causal, sm_scale, rows, amb)
+                                 causal, sm_scale, rows, amb,
+                                 FP8_QK_ACC_REL if fp8_qk else 0.0)
                 if bound is None:
                     out[b, h] = res
                 else:
@@ -286,7 +328,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
 
     if mode == "fp4":
         bound = np.zeros_like(out) if ambiguity_eps is not None else None
-        amb = (lambda pt: fp4_p_ambiguity(pt, ambiguity_eps)) if bound is not None else None
+        amb = ((lambda pt, extra: fp4_p_ambiguity(pt, ambiguity_eps + extra))
+               if bound is not None else None)
         qk = pp.quant_qk_fp4(q, k)
         vc, vsf, vg = pp.quant_v_fp4(v)
         for b in range(B):

@@ -28,6 +28,12 @@ Readings of the pages (they give the method only at abstract level):
    s16 = ue4m3(fp32(amax16 / fp32(6 * g))); code = e2m1(fp32(x / fp32(s16 *
    g))); a zero g or s16 gives code 0.  V: the same, with the 16-element
    blocks running over tokens (per channel) inside each 128-token tile.
+6. FP8 Q/K (the kernel-comparison blog, "How SageAttention uses
+   quantization for more throughput": queries and keys go to INT8 or FP8):
+   the INT8 scheme of reading 3 with the e4m3 grid in place of the
+   integers: per 128-token block s = fp32(amax / 448); code =
+   e4m3(fp32(x / s)) (round to nearest even, saturating); an all-zero
+   block gets s = 0 and codes 0.  K is smoothed first, as in reading 1.
 """
 
 import numpy as np
@@ -87,6 +93,39 @@ def quant_int8_blocks(x):
         scales[:, :, i] = sc
         codes[:, :, s:e, :] = int8_quantize(blk, sc[:, :, None, None])
     return codes, scales
+
+
+def quant_fp8_blocks(x):
+    """Per-128-token-block FP8 e4m3 (reading 6).
+
+    x: float32 [B, H, N, d].  Returns (codes uint8 e4m3 [B,H,N,d],
+    scales float32 [B,H,ceil(N/128)]).
+    """
+    x = np.asarray(x, np.float32)
+    B, H, N, d = x.shape
+    nb = -(-N // BLOCK)
+    codes = np.zeros((B, H, N, d), np.uint8)
+    scales = np.zeros((B, H, nb), np.float32)
+    for i, (s, e) in enumerate(_blocks(N)):
+        blk = x[:, :, s:e, :]
+        amax = np.abs(blk).max(axis=(2, 3)).astype(np.float32)
+        sc = (amax / FP8_DIV).astype(np.float32)
+        scales[:, :, i] = sc
+        den = np.where(sc != 0, sc, np.float32(1))[:, :, None, None]
+        t = np.where(sc[:, :, None, None] != 0, blk / den, np.float32(0)).astype(np.float32)
+        codes[:, :, s:e, :] = e4m3_encode(t)
+    return codes, scales
+
+
+def quant_qk_fp8(q, k):
+    """FP8 Q/K mode pre-pass (reading 6; K smoothed as in reading 1).
+
+    Returns dict with q_codes, q_scales, k_codes, k_scales, k_mean.
+    """
+    mean = k_channel_mean(k)
+    qc, qs = quant_fp8_blocks(np.asarray(q, np.float32))
+    kc, ks = quant_fp8_blocks(smooth_k(k, mean))
+    return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean)
 
 
 def quant_qk_int8(q, k):

@@ -394,3 +394,170 @@ def test_fp4_ambiguity_bound_covers_flipped_codes():
         att.quant_p_fp4 = base
     assert moved == 2
     assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp4"), o)
+
+
+# ------------------------------------------------------------ FP8 Q/K ----
+
+def test_fp8_blocks_properties():
+    x = rnd((1, 2, 300, 64), 90, 3.0)
+    x[0, 1, 128:256] = 0.0                               # an all-zero block
+    codes, scales = pp.quant_fp8_blocks(x)
+    assert codes.dtype == np.uint8 and scales.shape == (1, 2, 3)
+    assert scales[0, 1, 1] == 0 and np.all(codes[0, 1, 128:256] == 0)
+    for h in range(2):
+        for i, (s, e) in enumerate([(0, 128), (128, 256), (256, 300)]):
+            blk = x[0, h, s:e].astype(np.float64)
+            sc = float(scales[0, h, i])
+            if sc == 0:
+                continue
+            assert scales[0, h, i] == np.float32(np.float32(np.abs(blk).max()) / np.float32(448))
+            dec = enc.e4m3_decode(codes[0, h, s:e]) * sc
+            # the block maximum lands on the top of the grid
+            assert np.abs(enc.e4m3_decode(codes[0, h, s:e])).max() == 448.0
+            # e4m3 relative error 2^-4 in the normal range, half the
+            # subnormal step (2^-10 s) below it
+            err = np.abs(dec - blk)
+            assert np.all(err <= np.maximum(np.abs(blk) * 2.0 ** -4, sc * 2.0 ** -10) * (1 + 1e-6))
+            # codes: the independent brute-force nearest-grid encoder on the
+            # FP32 quotients
+            t = (x[0, h, s:e] / np.float32(sc)).astype(np.float32)
+            assert np.array_equal(codes[0, h, s:e], enc.e4m3_encode_bruteforce(t))
+
+
+def test_quant_qk_fp8_smooths_k_only():
+    q, k = rnd((1, 1, 256, 32), 91), rnd((1, 1, 256, 32), 92) + np.float32(10)
+    r = pp.quant_qk_fp8(q, k)
+    c2, s2 = pp.quant_fp8_blocks(q)
+    assert np.array_equal(r["q_codes"], c2) and np.array_equal(r["q_scales"], s2)
+    kc, ks = pp.quant_fp8_blocks(k.astype(np.float32) - r["k_mean"][:, :, None, :])
+    assert np.array_equal(r["k_codes"], kc) and np.array_equal(r["k_scales"], ks)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_constant_k_gives_visible_mean(causal):
+    # K rows all equal -> smoothed K = 0 -> s_K = 0, codes 0 -> P~ = 1 -> O is
+    # the visible mean of V (V on the e4m3 grid with s_V = 1: exact)
+    N, d = 256, 32
+    rng = np.random.default_rng(93)
+    q = rnd((1, 1, N, d), 94)
+    k = np.broadcast_to(rnd((1, 1, 1, d), 95), (1, 1, N, d)).copy()
+    grid = enc.e4m3_decode(np.arange(0x7F))
+    v = (rng.choice(grid, (1, 1, N, d)) * rng.choice([-1, 1], (1, 1, N, d))).astype(np.float32)
+    v[0, 0, 0, :] = 448.0
+    o = att.emulated_sage_attention(q, k, v, causal, 0.2, mode="fp8")
+    v64 = v[0, 0].astype(np.float64)
+    want = (np.cumsum(v64, axis=0) / np.arange(1, N + 1)[:, None]) if causal \
+        else np.broadcast_to(v64.mean(axis=0), (N, d))
+    assert np.max(np.abs(o[0, 0] - want)) <= 1e-12 * max(1.0, np.abs(want).max())
+
+
+def test_fp8_two_key_closed_form():
+    # Q and K on the e4m3 grid with block maxima 448 (scales exactly 1): the
+    # emulated scores are the exact q . k; the top two keys have P~ = 1 and
+    # 1/1.1, the latter encoding as 448/1.1 -> 416 (as in INT8 mode).
+    N, d = 128, 16
+    q = np.zeros((1, 1, N, d), np.float32)
+    q[..., 0] = 448.0
+    k = np.zeros((1, 1, N, d), np.float32)
+    kc = np.full(N, -7.0)
+    kc[0], kc[1], kc[2] = 448.0, 416.0, 0.0
+    kc[3] = -(kc[:3].sum() + kc[4:].sum())               # = 4: channel sum 0 -> mean 0
+    assert enc.e4m3_decode(enc.e4m3_encode(np.float32(kc[3]))) == kc[3]
+    k[0, 0, :, 0] = kc
+    sm_scale = math.log(1.1) / (448.0 * 32.0)            # S0 - S1 = ln 1.1
+    rng = np.random.default_rng(96)
+    grid = enc.e4m3_decode(np.arange(0x7F))
+    v = (rng.choice(grid, (1, 1, N, d)) * rng.choice([-1, 1], (1, 1, N, d))).astype(np.float32)
+    v[0, 0, 5, :] = 448.0
+    o = att.emulated_sage_attention(q, k, v, False, sm_scale, mode="fp8")
+    S = 448.0 * kc * sm_scale
+    p = np.exp(S - S.max())
+    codes = enc.e4m3_decode(enc.e4m3_encode(448.0 * p)) / 448.0
+    assert codes[1] == 416.0 / 448.0
+    want = (codes[:, None] * v[0, 0].astype(np.float64)).sum(axis=0) / p.sum()
+    assert np.max(np.abs(o[0, 0] - want[None, :])) <= 1e-12
+
+
+def test_fp8_scaling_laws_and_subsets():
+    q, k, v = rnd((1, 1, 256, 32), 97), rnd((1, 1, 256, 32), 98), rnd((1, 1, 256, 32), 99)
+    a = att.emulated_sage_attention(q, k, v, True, 0.25, mode="fp8")
+    assert np.array_equal(att.emulated_sage_attention(q, k * np.float32(4), v, True, 0.0625,
+                                                      mode="fp8"), a)
+    assert np.array_equal(att.emulated_sage_attention(q, k, v * np.float32(8), True, 0.25,
+                                                      mode="fp8"), 8 * a)
+    rows = np.array([0, 77, 128, 255])
+    assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.25, mode="fp8",
+                                                      rows=rows), a[:, :, rows])
+
+
+def test_fp8_close_to_exact():
+    q, k = rnd((1, 2, 512, 64), 100), rnd((1, 2, 512, 64), 101) + np.float32(2.0)
+    v = rnd((1, 2, 512, 64), 102)
+    a = att.emulated_sage_attention(q, k, v, False, 0.125, mode="fp8")
+    b = att.exact_attention(q, k, v, False, 0.125)
+    assert np.sum(a * b) / np.sqrt(np.sum(a * a) * np.sum(b * b)) >= 0.998
+
+
+def _fp32_dot_orders(a, b):
+    """Sums of the (exact FP32) products a_c b_c in FP32 in several orders."""
+    t = (a.astype(np.float32) * b.astype(np.float32)).astype(np.float32)
+    outs = []
+    for order in (t, t[::-1], np.random.default_rng(0).permutation(t)):
+        acc = np.float32(0)
+        for x in order:
+            acc = np.float32(acc + x)
+        outs.append(float(acc))
+    w = t.copy()                                   # pairwise (tree) order
+    while len(w) > 1:
+        w = (w[0::2] + w[1::2]).astype(np.float32)
+    outs.append(float(w[0]))
+    return outs
+
+
+def test_fp8_accumulation_bound_covers_fp32_sums():
+    # the bound the FP8 mode grants the kernel's Q K^T holds for FP32
+    # accumulation in any of several orders, including adversarial terms
+    rng = np.random.default_rng(103)
+    grid = enc.e4m3_decode(np.arange(0x7F))
+    cases = [(rng.choice(grid, 128) * rng.choice([-1, 1], 128),
+              rng.choice(grid, 128) * rng.choice([-1, 1], 128)) for _ in range(200)]
+    big = np.full(128, 2.0 ** -9)
+    big[0] = 448.0
+    cases.append((big, big.copy()))                # one huge product, 127 tiny ones
+    alt = np.where(np.arange(128) % 2 == 0, 448.0, -448.0) * 1.0
+    alt[-1] = 2.0 ** -9
+    cases.append((alt, np.abs(alt)))               # cancellation down to a tiny remainder
+    for a, b in cases:
+        exact = float(np.dot(a, b))                # exact in FP64 (e4m3 products)
+        bound = att.FP8_QK_ACC_REL * float(np.dot(np.abs(a), np.abs(b)))
+        for s in _fp32_dot_orders(a, b):
+            assert abs(s - exact) <= bound
+
+
+def test_fp8_ambiguity_bound_covers_fp32_accumulation():
+    # The kernel's Q K^T in FP32 (here: sequential FP32 sums, forward or
+    # backward over the channels) moves O by no more than the bound the FP8
+    # mode returns, and does move it.
+    q, k, v = rnd((1, 1, 256, 64), 104, 2.0), rnd((1, 1, 256, 64), 105, 2.0), rnd((1, 1, 256, 64), 106)
+    o, bnd = att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp8", ambiguity_eps=2.0 ** -15)
+    base = att.qk_product
+
+    def fp32_seq(qd, kd, rev):
+        qf, kf = qd.astype(np.float32), kd.astype(np.float32)
+        acc = np.zeros((len(qd), len(kd)), np.float32)
+        chans = range(qd.shape[1] - 1, -1, -1) if rev else range(qd.shape[1])
+        for c in chans:
+            acc = (acc + (qf[:, c, None] * kf[None, :, c]).astype(np.float32)).astype(np.float32)
+        return acc.astype(np.float64)
+
+    moved = 0
+    try:
+        for rev in (False, True):
+            att.qk_product = lambda qd, kd, r=rev: fp32_seq(qd, kd, r)
+            o2 = att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp8")
+            assert np.all(np.abs(o2 - o) <= bnd + 1e-12)
+            moved += int(np.any(o2 != o))
+    finally:
+        att.qk_product = base
+    assert moved >= 1
+    assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp8"), o)
