@@ -207,7 +207,7 @@ def run_sage(args):
             ev_attn[1].record(stream)
 
     # sage_quant_qk: 2 launches; sage_quant_v: 2 (FP8) or 1 (FP4); attention: 1
-    launches_per_step = 2 + (2 if w.mode == "int8_fp8" else 1) + 1
+    launches_per_step = 2 + (1 if w.mode == "fp4" else 2) + 1
 
     uuid = None
     try:
@@ -290,7 +290,7 @@ def run_sage(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp4e2m1" if w.mode == "fp4" else "int8+fp8e4m3",
+        "dtype": {"fp4": "fp4e2m1", "fp8": "fp8e4m3"}.get(w.mode, "int8+fp8e4m3"),
         "data": "synthetic",
         "config": config_of(w0, world),
         "attn_kernel_ms": round(t_attn, 4),
@@ -355,7 +355,7 @@ def sample_rows(w):
     """Query rows of one head that fill about a second of oracle time, and the
     effective (metric) pair count they stand for: N keys per query row, as
     in 4*B*H*N^2*d."""
-    target_pairs = 2.5e7 if w.mode == "int8_fp8" else 6e6
+    target_pairs = 6e6 if w.mode == "fp4" else 2.5e7
     if w.N * w.N <= target_pairs:
         return None, w.N * w.N
     n = max(128, int(target_pairs / w.N))

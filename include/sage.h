@@ -6,7 +6,7 @@
  *   - K is smoothed by subtracting its per-channel mean over tokens
  *     (SageAttention abstract, dblp author page on taxoreview.com: accurate
  *     8-bit attention; softmax is unchanged by a per-row shift);
- *   - Q and K are quantized per 128-token block to INT8
+ *   - Q and K are quantized per 128-token block to INT8 or FP8
  *     ("Flash Attention vs Sage Attention: Kernel Comparison", section "How
  *     SageAttention uses quantization for more throughput"), or to FP4 with
  *     one UE4M3 scale per 16 elements (SageAttention3 abstract: FP4 tensor
@@ -33,8 +33,8 @@
  *     or process exit crosses the ABI.  sage_status_string() describes the
  *     most recent error of the calling thread.
  *   - Quantized buffers (sizes from sage_buffer_bytes):
- *       INT8/FP8 mode
- *         q_codes, k_codes  int8  [B, H, N, d]
+ *       INT8/FP8 and FP8 modes
+ *         q_codes, k_codes  int8 (FP8 mode: e4m3) [B, H, N, d]
  *         q_scales, k_scales float [B, H, N/128]    one scale per 128 tokens
  *         k_mean            float [B, H, d]
  *         v_codes           e4m3  [B, H, d, N]      V transposed
@@ -74,7 +74,10 @@ typedef enum {
   SAGE_ERR_DEVICE_TIMEOUT = -4   /* a bounded wait inside a kernel expired  */
 } sage_status_t;
 
-typedef enum { SAGE_MODE_INT8_FP8 = 0, SAGE_MODE_FP4 = 1 } sage_mode_t;
+/* INT8_FP8: INT8 Q/K, FP8 P~ and V.  FP4: FP4 Q/K/P~/V.  FP8: FP8 Q/K
+ * (e4m3, per-block scale amax/448), FP8 P~ and V; its Q K^T accumulates in
+ * FP32 on the tensor cores instead of exactly in INT32. */
+typedef enum { SAGE_MODE_INT8_FP8 = 0, SAGE_MODE_FP4 = 1, SAGE_MODE_FP8 = 2 } sage_mode_t;
 typedef enum { SAGE_DTYPE_F16 = 0, SAGE_DTYPE_BF16 = 1 } sage_dtype_t;
 
 typedef enum {
@@ -84,7 +87,7 @@ typedef enum {
 } sage_buffer_t;
 
 /* Bytes of one quantized buffer for the given mode and shape (0 for a
- * buffer the mode does not use, e.g. *_SF in INT8/FP8 mode). */
+ * buffer the mode does not use, e.g. *_SF outside FP4 mode). */
 size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, int64_t d);
 
 /* Q/K pre-pass: K channel mean (FP64 accumulation: per 128-token chunk in
@@ -93,6 +96,8 @@ size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, i
  * of smoothed K.
  *   INT8 mode: s = fp32(amax / 127); code = clamp(rne(fp32(x / s)), +-127);
  *              q_sf, k_sf must be NULL.
+ *   FP8 mode:  s = fp32(amax / 448); code = e4m3(fp32(x / s)); q_sf, k_sf
+ *              must be NULL.
  *   FP4 mode:  g = fp32(amax_tile / 2688); per 16 channels
  *              s16 = ue4m3(fp32(amax16 / fp32(6 g))),
  *              code = e2m1(fp32(x / fp32(s16 * g))); q_scales/k_scales
@@ -107,7 +112,8 @@ int sage_quant_qk(const void* q, const void* k, int dtype,
                   float* k_mean, sage_stream_t stream);
 
 /* V pre-pass.
- *   FP8 mode: s_V[c] = fp32(amax_c / 448) over all N tokens of the (b, h);
+ *   INT8_FP8 and FP8 modes: s_V[c] = fp32(amax_c / 448) over all N tokens
+ *             of the (b, h);
  *             code = e4m3(fp32(V / s_V)); written transposed; v_sf NULL.
  *   FP4 mode: per 128-token tile g = fp32(amax_tile / 2688); per channel
  *             and 16 tokens s16 = ue4m3(fp32(amax16 / fp32(6 g))),
@@ -121,8 +127,8 @@ int sage_quant_v(const void* v, int dtype,
  * pre-pass calls); writes O [B, H, N, d] in `dtype`.  causal != 0 applies
  * the top-left-aligned causal mask (query t sees keys 0..t).  sm_scale is
  * applied at dequantization, not folded into the stored scales.
- * P~ is quantized inside the kernel: FP8 mode e4m3(448 P~); FP4 mode per
- * 16 keys s16 = ue4m3(448 amax16), code = e2m1(2688 P~ / s16). */
+ * P~ is quantized inside the kernel: INT8_FP8 and FP8 modes e4m3(448 P~);
+ * FP4 mode per 16 keys s16 = ue4m3(448 amax16), code = e2m1(2688 P~ / s16). */
 int sage_attn_fwd_quantized(int mode,
                             const void* q_codes, const float* q_scales, const void* q_sf,
                             const void* k_codes, const float* k_scales, const void* k_sf,

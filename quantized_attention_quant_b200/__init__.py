@@ -27,7 +27,7 @@ __all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_gqa"
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libsage_b200.so")
 
-MODES = {"int8_fp8": 0, "fp4": 1}
+MODES = {"int8_fp8": 0, "fp4": 1, "fp8": 2}
 DTYPES = {"f16": 0, "bf16": 1}
 BUF = {name: i for i, name in enumerate(
     ["q_codes", "q_scales", "q_sf", "k_codes", "k_scales", "k_sf", "k_mean",

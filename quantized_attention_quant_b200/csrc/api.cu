@@ -143,8 +143,9 @@ struct WorkspaceReleaser {
 int check_common(int dtype, int mode, int64_t B, int64_t H, int64_t N, int64_t d, bool* empty) {
   if (dtype != SAGE_DTYPE_F16 && dtype != SAGE_DTYPE_BF16)
     return fail(SAGE_ERR_INVALID_ARG, "dtype must be SAGE_DTYPE_F16 or SAGE_DTYPE_BF16");
-  if (mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_FP4)
-    return fail(SAGE_ERR_INVALID_ARG, "mode must be SAGE_MODE_INT8_FP8 or SAGE_MODE_FP4");
+  if (mode != SAGE_MODE_INT8_FP8 && mode != SAGE_MODE_FP4 && mode != SAGE_MODE_FP8)
+    return fail(SAGE_ERR_INVALID_ARG,
+                "mode must be SAGE_MODE_INT8_FP8, SAGE_MODE_FP4 or SAGE_MODE_FP8");
   if (B < 0 || H < 0 || N < 0 || d < 0) return fail(SAGE_ERR_INVALID_ARG, "negative size");
   *empty = (B == 0 || H == 0 || N == 0);
   if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d must be 64 or 128");
@@ -168,7 +169,7 @@ int check_ptr(const void* p, const char* name, bool required) {
 }
 
 int check_unused(const void* p, const char* name) {
-  if (p) return fail(SAGE_ERR_INVALID_ARG, std::string(name) + " must be NULL in INT8/FP8 mode");
+  if (p) return fail(SAGE_ERR_INVALID_ARG, std::string(name) + " must be NULL outside FP4 mode");
   return SAGE_OK;
 }
 
@@ -381,7 +382,7 @@ int sage_quant_v(const void* v, int dtype, int64_t B, int64_t H, int64_t N, int6
   void* ws = nullptr;
   uint32_t* cnt = nullptr;
   const size_t ks = align_up(ws_ksum_bytes(B * H, N, d));
-  if (mode == SAGE_MODE_INT8_FP8)
+  if (mode != SAGE_MODE_FP4)
     SAGE_TRY(workspace(st, ks + ws_vmax_bytes(B * H, N, d), &ws, &cnt));
   QuantVArgs a{v, dtype, mode, B, H, N, d, v_codes, v_scales, v_sf,
                static_cast<double*>(ws),

@@ -1,5 +1,5 @@
-// attn_i8f8.cu -- fused quantized attention forward, INT8 Q K^T + FP8 P~V,
-// for sm_100a (tcgen05 tensor cores, TMEM accumulators, TMA).
+// attn_i8f8.cu -- fused quantized attention forward, INT8 (or FP8) Q K^T +
+// FP8 P~V, for sm_100a (tcgen05 tensor cores, TMEM accumulators, TMA).
 //
 // What it computes (SageAttention abstract: INT8 Q K^T; SageAttention2
 // abstract: FP8 P~ and V with two-level accumulation of P~V; the online
@@ -7,7 +7,8 @@
 // section "How FlashAttention reduces memory traffic"):
 //
 //   per query row, over 128-key tiles j (causal: j <= query tile):
-//     A      = q_codes . k_codes_j^T                 (tcgen05 kind::i8, exact)
+//     A      = q_codes . k_codes_j^T                 (tcgen05 kind::i8, exact;
+//                                                     FP8 Q/K: kind::f8f6f4, FP32)
 //     t      = A * (s_Q s_Kj sm_scale log2 e)        (log2 domain)
 //     m_j    = max(m_{j-1}, rowmax t); alpha_j = 2^(m_{j-1} - m_j)
 //     p      = e4m3(448 * 2^(t - m_j))               (448 P~, quantized)
@@ -44,8 +45,11 @@
 // Q K^T the S columns hold the bit pattern of 1.5 * 2^23; the INT8 MMA
 // accumulates onto it, so a score reads back as the float
 // 1.5*2^23 + A exactly (|A| <= 127^2*128 < 2^22) with no conversion
-// instruction.  Every barrier wait is bounded; an expired wait sets the
-// device status word and makes every role leave its loop.
+// instruction.  The FP8 Q/K variant (QF8; the kernel-comparison blog's
+// "INT8 or FP8" queries and keys) runs the same pipeline with an FP32
+// Q K^T that overwrites S, so it has no bias to write back or remove.
+// Every barrier wait is bounded; an expired wait sets the device status
+// word and makes every role leave its loop.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -197,17 +201,19 @@ __device__ __forceinline__ float ldg_early(const float* p) {
 // A score as read from TMEM: the float 1.5 * 2^23 + A (exact).
 __device__ __forceinline__ float biased(uint32_t a) { return __uint_as_float(a); }
 
-// Max of 64 biased scores and a running value.  MASKED: columns col0 + i > r
-// are ignored (causal diagonal tile).
-template <bool MASKED>
+// Max of 64 scores and a running value.  MASKED: columns col0 + i > r are
+// ignored (causal diagonal tile): they read as 0, below every biased INT8
+// score, or -inf for the plain FP32 scores of the FP8 Q K^T.
+template <bool MASKED, bool QF8>
 __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float acc) {
+  constexpr float kLow = QF8 ? -INFINITY : 0.f;
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     float x = biased(s[k]), y = biased(s[k + 8]);
     if (MASKED) {
-      x = (col0 + k <= r) ? x : 0.f;
-      y = (col0 + k + 8 <= r) ? y : 0.f;
+      x = (col0 + k <= r) ? x : kLow;
+      y = (col0 + k + 8 <= r) ? y : kLow;
     }
     a[k] = fmaxf(x, y);
   }
@@ -217,8 +223,8 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
     for (int k = 0; k < 8; ++k) {
       float x = biased(s[i + k]), y = biased(s[i + 8 + k]);
       if (MASKED) {
-        x = (col0 + i + k <= r) ? x : 0.f;
-        y = (col0 + i + 8 + k <= r) ? y : 0.f;
+        x = (col0 + i + k <= r) ? x : kLow;
+        y = (col0 + i + 8 + k <= r) ? y : kLow;
       }
       a[k] = fmax3(a[k], x, y);
     }
@@ -226,8 +232,9 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
 }
 
 // 448 P~ for 32 scores of a row -> 8 words of e4m3 codes (key i in byte
-// i % 4 of word i / 4) and the sum of the unquantized values.
-template <bool MASKED>
+// i % 4 of word i / 4) and the sum of the unquantized values.  QF8: the
+// scores are plain FP32 (no bias to remove).
+template <bool MASKED, bool QF8>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
                                              int r, uint32_t (&p)[8]) {
   const float2 c2 = make_float2(c, c);
@@ -237,8 +244,12 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
     // (1.5*2^23 + A) - 1.5*2^23 = A exactly
-    const float2 x01 = __fadd2_rn(make_float2(biased(s[i]), biased(s[i + 1])), mb);
-    const float2 x23 = __fadd2_rn(make_float2(biased(s[i + 2]), biased(s[i + 3])), mb);
+    float2 x01 = make_float2(biased(s[i]), biased(s[i + 1]));
+    float2 x23 = make_float2(biased(s[i + 2]), biased(s[i + 3]));
+    if (!QF8) {
+      x01 = __fadd2_rn(x01, mb);
+      x23 = __fadd2_rn(x23, mb);
+    }
     const float2 t01 = __ffma2_rn(x01, c2, n2);
     const float2 t23 = __ffma2_rn(x23, c2, n2);
     float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
@@ -272,17 +283,17 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
 // One 32-key chunk cc (0..3) of the exp pass: its e4m3 codes go to the 8
 // TMEM columns pcol (four keys per column, the A-operand layout of the
 // P~V MMA); returns the chunk's row sum.
-template <bool MASKED>
+template <bool MASKED, bool QF8>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int cc, float c, float neg,
                                            int r, uint32_t pcol) {
   uint32_t p[8];
-  const float sum = exp_quant32<MASKED>(s, c, neg, 32 * cc, r, p);
+  const float sum = exp_quant32<MASKED, QF8>(s, c, neg, 32 * cc, r, p);
   tmem_st8(pcol, p);
   return sum;
 }
 
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool QF8>
 __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv,
                                          const uint32_t tmem, const Bars& bar, uint8_t* smem,
                                          volatile int* abort_flag, uint32_t* status) {
@@ -296,13 +307,16 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
   const float* c_s = reinterpret_cast<const float*>(smem + L::OFF_C);
   float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
 
-  // the first Q K^T into each S buffer accumulates onto the bias
+  // the first Q K^T into each S buffer accumulates onto the bias (the FP8
+  // Q K^T overwrites S instead)
+  if (!QF8) {
 #pragma unroll
-  for (int b = 0; b < L::SB; ++b) {
-    tmem_fill32(tmem + lanes + 128u * b + 64u * h, kBiasBits);
-    tmem_fill32(tmem + lanes + 128u * b + 64u * h + 32u, kBiasBits);
+    for (int b = 0; b < L::SB; ++b) {
+      tmem_fill32(tmem + lanes + 128u * b + 64u * h, kBiasBits);
+      tmem_fill32(tmem + lanes + 128u * b + 64u * h + 32u, kBiasBits);
+    }
+    tmem_wait_st();
   }
-  tmem_wait_st();
   tc_fence_before();
   mbar_arrive(bar.s_init);
 
@@ -333,20 +347,22 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     reg_fence(sb);
     if (r == 0 && h == 0) SAGE_TR(13, j);
     // S read: the bias back, and S free for the next Q K^T into it
-    tmem_fill32(S, kBiasBits);
-    tmem_fill32(S + 32, kBiasBits);
-    tmem_wait_st();
+    if (!QF8) {
+      tmem_fill32(S, kBiasBits);
+      tmem_fill32(S + 32, kBiasBits);
+      tmem_wait_st();
+    }
     tc_fence_before();
     mbar_arrive(&bar.s_ready[sbuf]);
     // P~[b] is free once the P~V MMA of tile j - 2 has read it
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    float sum = diag ? exp_chunk<true>(sa, 2 * h, c, neg, r, P)
-                     : exp_chunk<false>(sa, 2 * h, c, neg, r, P);
+    float sum = diag ? exp_chunk<true, QF8>(sa, 2 * h, c, neg, r, P)
+                     : exp_chunk<false, QF8>(sa, 2 * h, c, neg, r, P);
     if (r == 0 && h == 0) SAGE_TR(14, j);
-    sum += diag ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, P + 8)
-                : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, P + 8);
+    sum += diag ? exp_chunk<true, QF8>(sb, 2 * h + 1, c, neg, r, P + 8)
+                : exp_chunk<false, QF8>(sb, 2 * h + 1, c, neg, r, P + 8);
     l = fmaf(alpha, l, sum);
     if (r == 0 && h == 0) SAGE_TR(10, j);
     tmem_wait_st();
@@ -361,7 +377,7 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 
 // Stats warpgroup: row max / running max per key tile, level-2 fold,
 // epilogue.
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool QF8>
 __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh,
                                            const int H, const int G, const int N,
                                            const int ntiles, const uint32_t tmem, const Bars& bar,
@@ -427,7 +443,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     if (r == 0) SAGE_TR(4, j);
     const bool diag = CAUSAL && (j == qt);
     const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
-    float mx = 0.f;
+    float mx = QF8 ? -INFINITY : 0.f;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       uint32_t s[2][32];
@@ -435,9 +451,11 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      mx = diag ? max64<true>(&s[0][0], 64 * hh, r, mx) : max64<false>(&s[0][0], 64 * hh, r, mx);
+      mx = diag ? max64<true, QF8>(&s[0][0], 64 * hh, r, mx)
+                : max64<false, QF8>(&s[0][0], 64 * hh, r, mx);
     }
-    const float m_j = fmaxf(m, (mx - kBias) * c);
+    // c >= 0, so the max of the scaled scores is the scaled max
+    const float m_j = fmaxf(m, (QF8 ? mx : mx - kBias) * c);
     const float alpha = ex2(m - m_j);
     m = m_j;
     m_s[(2 * b) * 128 + r] = m_j;
@@ -471,7 +489,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   }
 }
 
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool QF8>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -571,7 +589,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     } else if (warp == 1) {
       // ---------------------------------------------------- tcgen05 issuer
       if (elect_one()) {
-        constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*s8*/, 1 /*s8*/, 128, 128);
+        constexpr uint32_t idesc_qk = QF8 ? make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, 128)
+                                          : make_idesc(2 /*S32*/, 1 /*s8*/, 1 /*s8*/, 128, 128);
         constexpr uint32_t idesc_pv = make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, D);
         const uint64_t qdesc = make_sdesc(smem_u32(sQ), L::QK_SBO, 16, L::QK_SWZ);
         bool ok = mbar_wait(bar.q_full, 0, abort_flag, status, kDevTimeoutTma);
@@ -586,8 +605,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
           const uint64_t kdesc =
               make_sdesc(smem_u32(sK + sk * L::K_BYTES), L::QK_SBO, 16, L::QK_SWZ);
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            if (QF8)
+              mma_f8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk,
+                        kk > 0);
+            else
+              mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
+          }
           mma_commit(&bar.s_full[sbuf]);
           mma_commit(&bar.k_empty[sk]);
           return true;
@@ -651,10 +675,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL>(wg - 1, qt, nkv, tmem, bar, smem, abort_flag, status);
+    exp_loop<D, CAUSAL, QF8>(wg - 1, qt, nkv, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<D, CAUSAL, OutT>(qt, nkv, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
+    stats_loop<D, CAUSAL, OutT, QF8>(qt, nkv, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
                                 q_scales, k_scales, v_scales, out, scale_log2);
   }
 
@@ -670,11 +694,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #endif
 }
 
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool QF8>
 cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, cudaStream_t st) {
   using L = Layout<D>;
-  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT>;
+  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, QF8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)(a.N / 128);
@@ -685,15 +709,15 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtenso
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool QF8>
 cudaError_t launch_d(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                      const CUtensorMap& tv, cudaStream_t st) {
   if (a.causal) {
-    return a.dtype == 1 ? launch_typed<D, true, __nv_bfloat16>(a, tq, tk, tv, st)
-                        : launch_typed<D, true, __half>(a, tq, tk, tv, st);
+    return a.dtype == 1 ? launch_typed<D, true, __nv_bfloat16, QF8>(a, tq, tk, tv, st)
+                        : launch_typed<D, true, __half, QF8>(a, tq, tk, tv, st);
   }
-  return a.dtype == 1 ? launch_typed<D, false, __nv_bfloat16>(a, tq, tk, tv, st)
-                      : launch_typed<D, false, __half>(a, tq, tk, tv, st);
+  return a.dtype == 1 ? launch_typed<D, false, __nv_bfloat16, QF8>(a, tq, tk, tv, st)
+                      : launch_typed<D, false, __half, QF8>(a, tq, tk, tv, st);
 }
 
 }  // namespace
@@ -713,7 +737,9 @@ cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** de
       !encode_tmap_2d(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.v_codes, N, BHK * D, N, 128, (uint32_t)D,
                       CU_TENSOR_MAP_SWIZZLE_128B, detail))
     return cudaErrorInvalidValue;
-  return D == 128 ? launch_d<128>(a, tq, tk, tv, st) : launch_d<64>(a, tq, tk, tv, st);
+  if (a.mode == kModeFp8)
+    return D == 128 ? launch_d<128, true>(a, tq, tk, tv, st) : launch_d<64, true>(a, tq, tk, tv, st);
+  return D == 128 ? launch_d<128, false>(a, tq, tk, tv, st) : launch_d<64, false>(a, tq, tk, tv, st);
 }
 
 }  // namespace sage

@@ -43,6 +43,8 @@ enum Role : int {
   kStatsK = 6,    // K chunk sums
   kStatsKV = 7,   // K chunk sums and V chunk maxima
   kStatsV = 8,    // V chunk maxima
+  kQuantQF8 = 9,  // FP8 (e4m3) Q codes + block scales
+  kQuantKF8 = 10, // FP8 (e4m3) smoothed-K codes + block scales (needs the K mean)
 };
 
 struct Roles {
@@ -147,6 +149,33 @@ __device__ __forceinline__ uint2 int8_codes8(const float (&v)[8], float s, float
   const uint32_t w0 = __byte_perm(__byte_perm(hb[0], hb[1], 0x0040), __byte_perm(hb[2], hb[3], 0x0040), 0x5410);
   const uint32_t w1 = __byte_perm(__byte_perm(hb[4], hb[5], 0x0040), __byte_perm(hb[6], hb[7], 0x0040), 0x5410);
   return make_uint2(w0, w1);
+}
+
+// Eight e4m3 codes e4m3(fp32(v / s)) for one block scale s != 0, packed
+// little-endian.  The same bracket test: both ends of each pair of
+// quotients go through one e4m3x2 conversion each (rounding to e4m3 is
+// monotonic, saturation included); any mismatch (or an unusable 1/s) redoes
+// the vector on IEEE quotients.
+__device__ __forceinline__ uint2 fp8_codes8(const float (&v)[8], float s, float rs) {
+  const float2 rs2 = make_float2(rs, rs);
+  const float2 lo2 = make_float2(kBracketLo, kBracketLo);
+  const float2 hi2 = make_float2(kBracketHi, kBracketHi);
+  uint32_t c[4];
+  uint32_t diff = rs == 0.f ? 1u : 0u;
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 q = __fmul2_rn(make_float2(v[e], v[e + 1]), rs2);
+    const float2 a = __fmul2_rn(q, lo2);
+    const float2 b = __fmul2_rn(q, hi2);
+    const uint32_t ca = cvt_e4m3x2(a.x, a.y), cb = cvt_e4m3x2(b.x, b.y);
+    diff |= ca ^ cb;
+    c[e / 2] = cb;
+  }
+  if (diff != 0u) {
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) c[e / 2] = cvt_e4m3x2(__fdiv_rn(v[e], s), __fdiv_rn(v[e + 1], s));
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 __device__ __forceinline__ float quot_e2m1(float x, float s, float rs) {
@@ -271,14 +300,15 @@ __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int
   }
 }
 
-// ------------------------------------------------------------- INT8 Q / K
-// Load, (smooth), block amax, s = amax / 127, codes = clamp(rne(x / s)).
+// ------------------------------------------------------- INT8 / FP8 Q / K
+// Load, (smooth), block amax, s = amax / 127, codes = clamp(rne(x / s))
+// (FP8: s = amax / 448, codes = e4m3(x / s)).
 // Two passes over the 128-token tile: the amax pass keeps nothing, the code
 // pass reads the tile again (from L1/L2), so the role needs few registers and
 // many CTAs fit on an SM.  A thread's vectors all cover the same 8 channels.
-template <typename T, int D>
-__device__ __forceinline__ void role_quant_int8(const T* __restrict__ src, const float* mean,
-                                                int8_t* __restrict__ dst, float* scale_out,
+template <typename T, int D, bool FP8>
+__device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const float* mean,
+                                                uint8_t* __restrict__ dst, float* scale_out,
                                                 float* red) {
   constexpr int VPT = 128 * D / 8 / kThreads;  // 16-byte vectors per thread
   const int c0 = (threadIdx.x % (D / 8)) * 8;
@@ -310,7 +340,7 @@ __device__ __forceinline__ void role_quant_int8(const T* __restrict__ src, const
     for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
   }
   amax = block_max(amax, red);
-  const float s = __fdiv_rn(amax, 127.f);
+  const float s = __fdiv_rn(amax, FP8 ? 448.f : 127.f);
   const float rs = recip_or_zero(s);
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -320,7 +350,7 @@ __device__ __forceinline__ void role_quant_int8(const T* __restrict__ src, const
       float x[8];
       load8(src + vec * 8, x);
       smooth(x);
-      w = int8_codes8(x, s, rs);
+      w = FP8 ? fp8_codes8(x, s, rs) : int8_codes8(x, s, rs);
     }
     *reinterpret_cast<uint2*>(dst + vec * 8) = w;
   }
@@ -571,22 +601,34 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   const int tile = blockIdx.x;
   // the grid spans the larger head count: Q roles cover bh_q heads, K/V
   // roles bh_kv (a CTA leaves as a whole, before any barrier)
-  const bool q_role = role == kQuantQ8 || role == kQuantQ4;
+  const bool q_role = role == kQuantQ8 || role == kQuantQ4 || role == kQuantQF8;
   if (bh >= (q_role ? p.bh_q : p.bh_kv)) return;
   const int ntiles = p.N / 128;
   const int64_t row0 = bh * p.N + (int64_t)tile * 128;
   switch (role) {
     case kQuantQ8:
       SAGE_ROLE(kQuantQ8)
-      role_quant_int8<T, D>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
-                            reinterpret_cast<int8_t*>(p.q_codes) + row0 * D,
-                            p.q_scales + bh * ntiles + tile, red);
+      role_quant_8bit<T, D, false>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+                                   reinterpret_cast<uint8_t*>(p.q_codes) + row0 * D,
+                                   p.q_scales + bh * ntiles + tile, red);
       break;
     case kQuantK8:
       SAGE_ROLE(kQuantK8)
-      role_quant_int8<T, D>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
-                            reinterpret_cast<int8_t*>(p.k_codes) + row0 * D,
-                            p.k_scales + bh * ntiles + tile, red);
+      role_quant_8bit<T, D, false>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+                                   reinterpret_cast<uint8_t*>(p.k_codes) + row0 * D,
+                                   p.k_scales + bh * ntiles + tile, red);
+      break;
+    case kQuantQF8:
+      SAGE_ROLE(kQuantQF8)
+      role_quant_8bit<T, D, true>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+                                  reinterpret_cast<uint8_t*>(p.q_codes) + row0 * D,
+                                  p.q_scales + bh * ntiles + tile, red);
+      break;
+    case kQuantKF8:
+      SAGE_ROLE(kQuantKF8)
+      role_quant_8bit<T, D, true>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+                                  reinterpret_cast<uint8_t*>(p.k_codes) + row0 * D,
+                                  p.k_scales + bh * ntiles + tile, red);
       break;
     case kQuantV8:
       SAGE_ROLE(kQuantV8)
@@ -690,9 +732,12 @@ void add_v(PrepassPtrs& p, const QuantVArgs& a) {
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
   const PrepassPtrs p = ptrs_qk(a);
-  if (a.mode == 0)
+  if (a.mode == kModeInt8Fp8)
     return dispatch<bit(kQuantQ8) | bit(kStatsK), bit(kQuantK8)>(
         p, a.dtype, a.d, Roles{2, {kQuantQ8, kStatsK}}, Roles{1, {kQuantK8}}, st);
+  if (a.mode == kModeFp8)
+    return dispatch<bit(kQuantQF8) | bit(kStatsK), bit(kQuantKF8)>(
+        p, a.dtype, a.d, Roles{2, {kQuantQF8, kStatsK}}, Roles{1, {kQuantKF8}}, st);
   return dispatch<bit(kQuantQ4) | bit(kStatsK), bit(kQuantK4)>(
       p, a.dtype, a.d, Roles{2, {kQuantQ4, kStatsK}}, Roles{1, {kQuantK4}}, st);
 }
@@ -700,7 +745,7 @@ cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
 cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st) {
   PrepassPtrs p{};
   add_v(p, a);
-  if (a.mode == 0)
+  if (a.mode != kModeFp4)
     return dispatch<bit(kStatsV), bit(kQuantV8)>(p, a.dtype, a.d, Roles{1, {kStatsV}},
                                                  Roles{1, {kQuantV8}}, st);
   return dispatch<bit(kQuantV4), 0>(p, a.dtype, a.d, Roles{1, {kQuantV4}},
@@ -710,10 +755,14 @@ cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st) {
 cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st) {
   PrepassPtrs p = ptrs_qk(qa);
   add_v(p, va);
-  if (qa.mode == 0)
+  if (qa.mode == kModeInt8Fp8)
     return dispatch<bit(kQuantQ8) | bit(kStatsKV), bit(kQuantK8) | bit(kQuantV8)>(
         p, qa.dtype, qa.d, Roles{2, {kQuantQ8, kStatsKV}},
         Roles{2, {kQuantK8, kQuantV8}}, st);
+  if (qa.mode == kModeFp8)
+    return dispatch<bit(kQuantQF8) | bit(kStatsKV), bit(kQuantKF8) | bit(kQuantV8)>(
+        p, qa.dtype, qa.d, Roles{2, {kQuantQF8, kStatsKV}},
+        Roles{2, {kQuantKF8, kQuantV8}}, st);
   return dispatch<bit(kQuantQ4) | bit(kQuantV4) | bit(kStatsK), bit(kQuantK4)>(
       p, qa.dtype, qa.d, Roles{3, {kQuantQ4, kQuantV4, kStatsK}},
       Roles{1, {kQuantK4}}, st);

@@ -8,11 +8,16 @@
 
 namespace sage {
 
+// sage_mode_t values (include/sage.h)
+constexpr int kModeInt8Fp8 = 0;  // INT8 Q/K, FP8 P~ and V
+constexpr int kModeFp4 = 1;      // FP4 Q/K/P~/V
+constexpr int kModeFp8 = 2;      // FP8 Q/K, FP8 P~ and V
+
 struct QuantQKArgs {
   const void* q;
   const void* k;
   int dtype;  // 0 = f16, 1 = bf16
-  int mode;   // 0 = INT8, 1 = FP4
+  int mode;   // kModeInt8Fp8 / kModeFp4 / kModeFp8 (sage_mode_t values)
   int64_t B, H, N, d;
   int64_t Hkv;  // K heads (H % Hkv == 0; Hkv == H without grouped-query attention)
   void* q_codes;
@@ -30,7 +35,7 @@ struct QuantQKArgs {
 struct QuantVArgs {
   const void* v;
   int dtype;
-  int mode;  // 0 = FP8, 1 = FP4
+  int mode;  // as above; V is FP8 in both 8-bit modes
   int64_t B, H, N, d;
   void* v_codes;
   float* v_scales;

@@ -60,6 +60,10 @@ WORKLOADS = {
     "long_causal": Workload("long_causal", 1, 16, 32768, 128, True, "bf16", "int8_fp8", 3,
                             "student_t", 2.0),
     "fp4": Workload("fp4", 2, 32, 16384, 128, False, "bf16", "fp4", 4, "normal", 3.0),
+    # the long-context inputs through the FP8 Q/K mode
+    "long_fp8": Workload("long_fp8", 1, 16, 32768, 128, False, "bf16", "fp8", 3, "student_t",
+                         2.0),
+    "llm_fp8": Workload("llm_fp8", 1, 32, 4096, 128, True, "bf16", "fp8", 1, "llm_outliers", 2.0),
 }
 
 

@@ -86,6 +86,18 @@ def test_fp4_random(cuda_device, N, dtype, causal):
     assert sage.device_status() == 0
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("N", [128, 512])
+def test_fp8_qk_random(cuda_device, N, dtype, d, causal):
+    q, k, v = rand_qkv(2, 2, N, d, dtype, seed=500 + N + d + causal)
+    o = sage.sage_attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, mode="fp8")
+    torch.cuda.synchronize()
+    check_against_oracle(to_numpy32(o), q, k, v, causal, 1 / math.sqrt(d), "fp8", dtype)
+    assert sage.device_status() == 0
+
+
 def test_fp4_zero_q_gives_mean_v(cuda_device):
     # Q = 0 -> every score 0 -> P~ = 1 -> s16 = 448, code e2m1(6) = 6, whose
     # value 6 * 448 / 2688 is exactly 1 -> O = mean of the FP4-dequantized V
@@ -159,7 +171,7 @@ def test_fwd_equals_prepass_plus_attention(cuda_device):
     q, k, v = rand_qkv(1, 4, 384, 128, "bf16", seed=9)
     dev = torch.device("cuda")
     qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
-    for mode in ["int8_fp8", "fp4"]:
+    for mode in ["int8_fp8", "fp4", "fp8"]:
         a = sage.sage_attn_fwd(qg, kg, vg, causal=True, mode=mode)
         qk = sage.sage_quant_qk(qg, kg, mode)
         vq = sage.sage_quant_v(vg, mode)
@@ -181,7 +193,7 @@ def test_side_stream(cuda_device):
 
 
 FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", None), ("long_causal", None),
-        ("fp4", None)]
+        ("fp4", None), ("long_fp8", None), ("llm_fp8", None)]
 
 
 @pytest.mark.parametrize("name,cos_floor", FULL)

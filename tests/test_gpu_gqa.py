@@ -39,7 +39,7 @@ CASES = [  # (B, H, Hkv, N, d)
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("mode", ["int8_fp8", "fp4"])
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp4", "fp8"])
 @pytest.mark.parametrize("B,H,Hkv,N,d", CASES)
 def test_gqa_matches_repeated_kv(cuda_device, B, H, Hkv, N, d, mode, causal):
     if mode == "fp4" and d != 128:

@@ -28,17 +28,19 @@ def rand_qkv(B, H, N, d, dtype, seed, k_bias=3.0):
     return [torch.from_numpy(x).to(TDT[dtype]) for x in (q, k, v)]
 
 
-def check_int8(q, k, v, heads=None):
-    """Run the INT8/FP8 pre-pass on the GPU; compare (sampled) heads."""
+def check_int8(q, k, v, heads=None, mode="int8_fp8"):
+    """Run the INT8/FP8 (or FP8 Q/K) pre-pass on the GPU; compare (sampled)
+    heads."""
     B, H, N, d = q.shape
     dev = torch.device("cuda")
-    qk = sage.sage_quant_qk(q.to(dev), k.to(dev), "int8_fp8")
-    vq = sage.sage_quant_v(v.to(dev), "int8_fp8")
+    qk = sage.sage_quant_qk(q.to(dev), k.to(dev), mode)
+    vq = sage.sage_quant_v(v.to(dev), mode)
     torch.cuda.synchronize()
     nt = N // 128
-    g = dict(q_codes=L.int8_codes(qk["q_codes"], B, H, N, d),
+    codes = L.u8 if mode == "fp8" else L.int8_codes
+    g = dict(q_codes=codes(qk["q_codes"], B, H, N, d),
              q_scales=L.f32(qk["q_scales"], B, H, nt),
-             k_codes=L.int8_codes(qk["k_codes"], B, H, N, d),
+             k_codes=codes(qk["k_codes"], B, H, N, d),
              k_scales=L.f32(qk["k_scales"], B, H, nt),
              k_mean=L.f32(qk["k_mean"], B, H, d),
              v_codes=L.u8(vq["v_codes"], B, H, d, N),
@@ -46,7 +48,7 @@ def check_int8(q, k, v, heads=None):
     heads = heads or [(b, h) for b in range(B) for h in range(H)]
     for (b, h) in heads:
         qs, ks, vs = (to_numpy32(t[b:b + 1, h:h + 1]) for t in (q, k, v))
-        want = pp.quant_qk_int8(qs, ks)
+        want = pp.quant_qk_fp8(qs, ks) if mode == "fp8" else pp.quant_qk_int8(qs, ks)
         vc, vsc = pp.quant_v_fp8(vs)
         want.update(v_codes=vc, v_scales=vsc)
         for name, arr in want.items():
@@ -104,6 +106,44 @@ def test_int8_prepass_edge_values(cuda_device):
     q[0, 2, 5, 7] = 3.0e38                    # near the bf16 max
     v[0, 0, 9, 1] = -1.0e-38                  # bf16 subnormal range
     check_int8(q, k, v)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp8_qk_prepass_random(cuda_device, dtype, d):
+    q, k, v = rand_qkv(2, 2, 384, d, dtype, seed=3 * d + 1)
+    check_int8(q, k, v, mode="fp8")
+
+
+def test_fp8_qk_prepass_edge_values(cuda_device):
+    B, H, N, d = 1, 3, 384, 128
+    q, k, v = rand_qkv(B, H, N, d, "bf16", seed=8)
+    q[0, 0, 128:256] = 0                      # an all-zero Q block -> s = 0, codes 0
+    k[0, 1] = -7.0                            # constant K -> smoothed K = 0
+    q[0, 2, 5, 7] = 3.0e38                    # near the bf16 max: the rest of its block
+                                              # lands in the e4m3 subnormals or at 0
+    q[0, 1, 300, 0] = 1.0e-37                 # tiny values next to normal ones
+    check_int8(q, k, v, mode="fp8")
+
+
+def test_fp8_qk_encoder_exhaustive(cuda_device):
+    # every finite fp16 value of magnitude <= 448 as Q, with a 448 in each
+    # 128-token block (so s = 1 and the code is exactly e4m3(x))
+    x = np.arange(1 << 16, dtype=np.uint16).view(np.float16).astype(np.float32)
+    x = x[np.isfinite(x) & (np.abs(x) <= 448)]
+    per = 127 * 64                            # values per block (one row keeps the 448)
+    nblk = -(-x.size // per)
+    blocks = np.zeros((nblk, 128, 64), np.float32)
+    flat = np.zeros(nblk * per, np.float32)
+    flat[:x.size] = x
+    blocks[:, 1:, :] = flat.reshape(nblk, 127, 64)
+    blocks[:, 0, 0] = 448.0
+    q = torch.from_numpy(blocks.reshape(1, 1, nblk * 128, 64)).to(torch.float16)
+    qk = sage.sage_quant_qk(q.cuda(), q.cuda(), "fp8")
+    torch.cuda.synchronize()
+    assert np.all(L.f32(qk["q_scales"], 1, 1, nblk) == 1.0)
+    codes = L.u8(qk["q_codes"], 1, 1, nblk * 128, 64)[0, 0].reshape(nblk, 128, 64)
+    assert np.array_equal(codes[:, 1:, :].reshape(-1)[:x.size], enc.e4m3_encode(x))
 
 
 def test_fp8_v_encoder_exhaustive(cuda_device):
