@@ -108,22 +108,35 @@ def fp8_p_ambiguity(pt, eps):
     return np.where(near_up, up - r, 0.0) + np.where(near_dn, r - dn, 0.0)
 
 
+def _pad16(pt):
+    """P~ with the key axis padded by zeros to a multiple of 16: the last tile
+    of a ragged sequence has a partial 16-key group, whose missing keys have
+    P~ = 0 (they change neither the group max nor any code)."""
+    R, C = pt.shape
+    Cp = -(-C // 16) * 16
+    if Cp == C:
+        return pt
+    return np.concatenate([pt, np.zeros((R, Cp - C))], axis=1)
+
+
 def quant_p_fp4(pt):
     """FP4 P~ with the static tile scale g = 1/2688 and per-16-key UE4M3 scales.
 
     s16 = ue4m3(amax16 * 448); code = e2m1(P~ / (s16 * g)).  Returns the
-    value code * s16 (the caller multiplies by g at the fold).  Requires the
-    key axis to be a multiple of 16.
+    value code * s16 (the caller multiplies by g at the fold).  A partial
+    16-key group (ragged last tile) counts its missing keys as P~ = 0.
     """
-    R, C = pt.shape
-    blk = pt.reshape(R, C // 16, 16)
+    C = pt.shape[1]
+    pt = _pad16(pt)
+    R, Cp = pt.shape
+    blk = pt.reshape(R, Cp // 16, 16)
     a16 = blk.max(axis=-1)
     s16 = ue4m3_decode(ue4m3_encode(a16 * P_FP8_SCALE))
     den = s16 * P_FP4_G
     with np.errstate(divide="ignore", invalid="ignore"):
         t = np.where(den[..., None] > 0, blk / np.where(den > 0, den, 1.0)[..., None], 0.0)
     codes = e2m1_decode(e2m1_encode(t))
-    return (codes * s16[..., None]).reshape(R, C)
+    return (codes * s16[..., None]).reshape(R, Cp)[:, :C]
 
 
 def _e2m1_flip(t, eps):
@@ -147,10 +160,13 @@ def fp4_p_ambiguity(pt, eps):
     Two decisions can go either way near a midpoint: the UE4M3 group scale
     s16 = ue4m3(448 amax16), which moves every value of the 16-key group,
     and each e2m1 code.  Where the scale is ambiguous the bound covers the
-    whole group re-quantized with the neighbouring scale.
+    whole group re-quantized with the neighbouring scale.  eps is a scalar;
+    a partial 16-key group is padded as in quant_p_fp4.
     """
-    R, C = pt.shape
-    blk = pt.reshape(R, C // 16, 16)
+    C = pt.shape[1]
+    pt = _pad16(pt)
+    R, Cp = pt.shape
+    blk = pt.reshape(R, Cp // 16, 16)
     x = blk.max(axis=-1) * P_FP8_SCALE
     code = ue4m3_encode(x).astype(np.int64)
     s = ue4m3_decode(code)
@@ -171,7 +187,7 @@ def fp4_p_ambiguity(pt, eps):
         if np.any(near):
             v_alt, b_alt = values(np.where(near, alt, s))
             bound = bound + np.where(near[..., None], np.abs(v_alt - base) + b_alt, 0.0)
-    return bound.reshape(R, C)
+    return bound.reshape(R, Cp)[:, :C]
 
 
 # --------------------------------------------------------------------------
@@ -338,7 +354,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                     ue4m3_decode(qk["q_sf"][b, h]), 16, axis=1)
                 kd = e2m1_decode(qk["k_codes"][b, h]) * np.repeat(
                     ue4m3_decode(qk["k_sf"][b, h]), 16, axis=1)
-                vdt = e2m1_decode(vc[b, h]) * np.repeat(ue4m3_decode(vsf[b, h]), 16, axis=1)
+                vdt = e2m1_decode(vc[b, h]) * np.repeat(ue4m3_decode(vsf[b, h]), 16,
+                                                         axis=1)[:, :N]
                 s_row = qk["q_g"][b, h].astype(np.float64)[tile_of]
                 s_key = qk["k_g"][b, h].astype(np.float64)[tile_of]
                 v_fold = (vg[b, h].astype(np.float64) * P_FP4_G)[:, None] * np.ones((1, d))

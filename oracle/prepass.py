@@ -34,6 +34,11 @@ Readings of the pages (they give the method only at abstract level):
    integers: per 128-token block s = fp32(amax / 448); code =
    e4m3(fp32(x / s)) (round to nearest even, saturating); an all-zero
    block gets s = 0 and codes 0.  K is smoothed first, as in reading 1.
+7. Ragged sequences (N not a multiple of 128): the last 128-token block is
+   shorter and its scale covers its tokens only; the K mean and the V
+   scales divide by / range over the N real tokens; in FP4 mode a partial
+   16-element group (V over tokens, P~ over keys) counts its missing
+   elements as zeros, which change neither its maximum nor any code.
 """
 
 import numpy as np
@@ -214,19 +219,20 @@ def quant_qk_fp4(q, k):
 def quant_v_fp4(v):
     """FP4 V (reading 5): transposed [B,H,d,N], 16-blocks over tokens.
 
-    Requires N % 16 == 0.  Returns (codes uint8 [B,H,d,N], sf [B,H,d,N/16],
-    g float32 [B,H,ceil(N/128)]).
+    A ragged sequence (N % 16 != 0) ends in a partial 16-token group whose
+    missing tokens count as zeros (reading 7).  Returns (codes uint8
+    [B,H,d,N], sf [B,H,d,ceil(N/16)], g float32 [B,H,ceil(N/128)]).
     """
     v = np.asarray(v, np.float32)
     B, H, N, d = v.shape
-    if N % FP4_VEC:
-        raise ValueError("FP4 V needs N % 16 == 0")
-    vt = np.ascontiguousarray(v.transpose(0, 1, 3, 2))                # [B,H,d,N]
+    N16 = -(-N // FP4_VEC) * FP4_VEC
+    vt = np.zeros((B, H, d, N16), np.float32)                          # [B,H,d,N16]
+    vt[..., :N] = v.transpose(0, 1, 3, 2)
     nb = -(-N // BLOCK)
-    codes = np.zeros((B, H, d, N), np.uint8)
-    sf = np.zeros((B, H, d, N // FP4_VEC), np.uint8)
+    codes = np.zeros((B, H, d, N16), np.uint8)
+    sf = np.zeros((B, H, d, N16 // FP4_VEC), np.uint8)
     g = np.zeros((B, H, nb), np.float32)
-    for i, (s, e) in enumerate(_blocks(N)):
+    for i, (s, e) in enumerate(_blocks(N16)):
         blk = vt[:, :, :, s:e]
         amax = np.abs(blk).max(axis=(2, 3)).astype(np.float32)
         gi = (amax / FP4_G_DIV).astype(np.float32)
@@ -234,4 +240,4 @@ def quant_v_fp4(v):
         c, f = _fp4_encode_tile(blk, gi)
         codes[:, :, :, s:e] = c
         sf[:, :, :, s // FP4_VEC:e // FP4_VEC] = f
-    return codes, sf, g
+    return np.ascontiguousarray(codes[..., :N]), sf, g

@@ -224,12 +224,14 @@ def test_emulated_identity_equals_exact(causal, N):
     assert np.max(np.abs(a - b)) <= 1e-12
 
 
+@pytest.mark.parametrize("N", [256, 200])
 @pytest.mark.parametrize("mode", ["int8_fp8", "fp4"])
 @pytest.mark.parametrize("causal", [False, True])
-def test_emulated_constant_k_gives_visible_mean(mode, causal):
+def test_emulated_constant_k_gives_visible_mean(mode, causal, N):
     # K rows all equal -> smoothed K = 0 -> all scores 0 -> P~ = 1 exactly;
     # V on the format grid with an exact scale -> O is the visible mean of V.
-    N, d = 256, 32
+    # N = 200 ends in a partial tile (and, in FP4 mode, a partial 16-group).
+    d = 32
     rng = np.random.default_rng(5)
     q = rnd((1, 1, N, d), 33)
     k = np.broadcast_to(rnd((1, 1, 1, d), 34), (1, 1, N, d)).copy()
@@ -311,12 +313,13 @@ def test_output_rounding_matches_dtype():
     assert np.max(np.abs(r - o)) <= np.abs(o).max() * 2.0 ** -8
 
 
-@pytest.mark.parametrize("mode", ["int8_fp8", "fp4"])
+@pytest.mark.parametrize("N", [384, 300])
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp4", "fp8"])
 @pytest.mark.parametrize("causal", [False, True])
-def test_row_subset_matches_full(mode, causal):
+def test_row_subset_matches_full(mode, causal, N):
     # computing a subset of query rows gives exactly those rows of the full run
-    q, k, v = rnd((1, 2, 384, 32), 60), rnd((1, 2, 384, 32), 61), rnd((1, 2, 384, 32), 62)
-    rows = np.array([0, 5, 127, 128, 200, 383])
+    q, k, v = rnd((1, 2, N, 32), 60), rnd((1, 2, N, 32), 61), rnd((1, 2, N, 32), 62)
+    rows = np.array([0, 5, 127, 128, 200, N - 1])
     full = att.emulated_sage_attention(q, k, v, causal, 0.2, mode=mode)
     sub = att.emulated_sage_attention(q, k, v, causal, 0.2, mode=mode, rows=rows)
     assert np.array_equal(full[:, :, rows], sub)
@@ -433,11 +436,12 @@ def test_quant_qk_fp8_smooths_k_only():
     assert np.array_equal(r["k_codes"], kc) and np.array_equal(r["k_scales"], ks)
 
 
+@pytest.mark.parametrize("N", [256, 139])
 @pytest.mark.parametrize("causal", [False, True])
-def test_fp8_constant_k_gives_visible_mean(causal):
+def test_fp8_constant_k_gives_visible_mean(causal, N):
     # K rows all equal -> smoothed K = 0 -> s_K = 0, codes 0 -> P~ = 1 -> O is
     # the visible mean of V (V on the e4m3 grid with s_V = 1: exact)
-    N, d = 256, 32
+    d = 32
     rng = np.random.default_rng(93)
     q = rnd((1, 1, N, d), 94)
     k = np.broadcast_to(rnd((1, 1, 1, d), 95), (1, 1, N, d)).copy()
@@ -561,3 +565,39 @@ def test_fp8_ambiguity_bound_covers_fp32_accumulation():
         att.qk_product = base
     assert moved >= 1
     assert np.array_equal(att.emulated_sage_attention(q, k, v, True, 0.3, mode="fp8"), o)
+
+
+# ----------------------------------------------------------- ragged N ----
+
+def test_fp4_v_ragged_counts_missing_tokens_as_zeros():
+    # N = 200: the last 16-token group (tokens 192..199) is partial; its scale
+    # and codes equal those of V padded with zero tokens to 208
+    v = rnd((1, 2, 200, 32), 110, 2.0)
+    c, f, g = pp.quant_v_fp4(v)
+    assert c.shape == (1, 2, 32, 200) and f.shape == (1, 2, 32, 13) and g.shape == (1, 2, 2)
+    vp = np.concatenate([v, np.zeros((1, 2, 8, 32), np.float32)], axis=2)
+    cp, fp_, gp = pp.quant_v_fp4(vp)
+    assert np.array_equal(c, cp[..., :200]) and np.array_equal(f, fp_) and np.array_equal(g, gp)
+    assert np.all(cp[..., 200:] == 0)
+
+
+def test_fp4_p_partial_group():
+    # a 40-key row: groups 0..15, 16..31 and the partial 32..39
+    pt = np.random.default_rng(111).random((3, 40))
+    full = att.quant_p_fp4(np.concatenate([pt, np.zeros((3, 8))], axis=1))
+    assert np.array_equal(att.quant_p_fp4(pt), full[:, :40])
+    assert att.fp4_p_ambiguity(pt, 1e-6).shape == (3, 40)
+
+
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp8", "fp4"])
+def test_ragged_identity_and_close_to_exact(mode):
+    # a ragged length through every mode stays as close to exact attention as
+    # the same data at a full-tile length does
+    d = 64 if mode != "fp4" else 32
+    q, k, v = rnd((1, 1, 300, d), 112), rnd((1, 1, 300, d), 113) + np.float32(1.0), \
+        rnd((1, 1, 300, d), 114)
+    for causal in (False, True):
+        a = att.emulated_sage_attention(q, k, v, causal, 0.125, mode=mode)
+        b = att.exact_attention(q, k, v, causal, 0.125)
+        cos = np.sum(a * b) / np.sqrt(np.sum(a * a) * np.sum(b * b))
+        assert cos >= (0.97 if mode == "fp4" else 0.995)
