@@ -27,25 +27,30 @@
  *     the caller, and must be 16-byte aligned.  `stream` is a cudaStream_t
  *     (NULL = legacy default stream).  Every call is asynchronous on
  *     `stream`; the library never synchronises it.
- *   - Supported shapes: d in {64, 128}; N % 128 == 0 (FP4 mode: d == 128).
+ *   - Supported shapes: d in {64, 128} (FP4 mode: d == 128); any N >= 0.
  *     A call with B, H or N equal to zero does nothing and returns SAGE_OK.
+ *   - Ragged sequences: the quantization blocks are 128-token tiles, the
+ *     last one holding N - 128 (Np/128 - 1) tokens.  Every code buffer is
+ *     laid out for Np = N rounded up to a multiple of 128 (the rows or
+ *     columns of the missing tokens hold zero codes); its scale covers the
+ *     real tokens only; keys past N are masked out of the softmax.
  *   - Return value: SAGE_OK (0) or a negative sage_status_t.  No exception
  *     or process exit crosses the ABI.  sage_status_string() describes the
  *     most recent error of the calling thread.
  *   - Quantized buffers (sizes from sage_buffer_bytes):
  *       INT8/FP8 and FP8 modes
- *         q_codes, k_codes  int8 (FP8 mode: e4m3) [B, H, N, d]
- *         q_scales, k_scales float [B, H, N/128]    one scale per 128 tokens
+ *         q_codes, k_codes  int8 (FP8 mode: e4m3) [B, H, Np, d]
+ *         q_scales, k_scales float [B, H, Np/128]   one scale per 128 tokens
  *         k_mean            float [B, H, d]
- *         v_codes           e4m3  [B, H, d, N]      V transposed
+ *         v_codes           e4m3  [B, H, d, Np]     V transposed
  *         v_scales          float [B, H, d]         one scale per channel
  *       FP4 mode
- *         q_codes, k_codes  e2m1x2 [B, H, N, d/2]   low nibble = even channel
- *         q_scales, k_scales float [B, H, N/128]    tile scale g
+ *         q_codes, k_codes  e2m1x2 [B, H, Np, d/2]  low nibble = even channel
+ *         q_scales, k_scales float [B, H, Np/128]   tile scale g
  *         q_sf, k_sf        ue4m3 per 16 channels, tensor-core layout (below)
- *         v_codes           e2m1x2 [B, H, d, N/2]   V transposed, low nibble =
+ *         v_codes           e2m1x2 [B, H, d, Np/2]  V transposed, low nibble =
  *                                                    even token
- *         v_scales          float [B, H, N/128]     tile scale g
+ *         v_scales          float [B, H, Np/128]    tile scale g
  *         v_sf              ue4m3 per 16 tokens, tensor-core layout (below)
  *       Tensor-core scale layout: for each (b, h, 128-token tile t, 64-wide
  *       chunk c of the contraction axis) one 512-byte block; inside it byte

@@ -151,10 +151,12 @@ int check_common(int dtype, int mode, int64_t B, int64_t H, int64_t N, int64_t d
   if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d must be 64 or 128");
   if (mode == SAGE_MODE_FP4 && d != 128)
     return fail(SAGE_ERR_UNSUPPORTED, "FP4 mode supports d == 128 only");
-  if (N % 128 != 0) return fail(SAGE_ERR_UNSUPPORTED, "N must be a multiple of 128");
   if (!*empty) {
+    // code buffers hold N rounded up to whole 128-token tiles per head
+    const int64_t Np = (N + 127) / 128 * 128;
     if (B * H > 65535) return fail(SAGE_ERR_UNSUPPORTED, "B*H must be <= 65535");
-    if (B * H * N > 2147483647LL) return fail(SAGE_ERR_UNSUPPORTED, "B*H*N must be < 2^31");
+    if (B * H * Np > 2147483647LL)
+      return fail(SAGE_ERR_UNSUPPORTED, "B*H*N (N rounded up to a multiple of 128) must be < 2^31");
   }
   return SAGE_OK;
 }
@@ -199,8 +201,12 @@ EncodeFn encode_fn(const char** detail) {
   return fn;
 }
 
-size_t ws_ksum_bytes(int64_t BH, int64_t N, int64_t d) { return (size_t)(BH * (N / 128) * d * 8); }
-size_t ws_vmax_bytes(int64_t BH, int64_t N, int64_t d) { return (size_t)(BH * (N / 128) * d * 4); }
+size_t ws_ksum_bytes(int64_t BH, int64_t N, int64_t d) {
+  return (size_t)(BH * ((N + 127) / 128) * d * 8);
+}
+size_t ws_vmax_bytes(int64_t BH, int64_t N, int64_t d) {
+  return (size_t)(BH * ((N + 127) / 128) * d * 4);
+}
 
 }  // namespace
 
@@ -315,7 +321,8 @@ size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, i
     case SAGE_BUF_Q_CODES:
     case SAGE_BUF_K_CODES:
     case SAGE_BUF_V_CODES:
-      return (size_t)(fp4 ? BH * N * d / 2 : BH * N * d);
+      // padded to whole 128-token tiles (the padding holds zero codes)
+      return (size_t)(fp4 ? BH * nt * 128 * d / 2 : BH * nt * 128 * d);
     case SAGE_BUF_Q_SCALES:
     case SAGE_BUF_K_SCALES:
       return (size_t)(BH * nt * 4);

@@ -191,17 +191,18 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Max of 64 scores and a running value.  MASKED: columns col0 + i > r are
-// ignored (causal diagonal tile).
+// Max of 64 scores and a running value.  MASKED: columns col0 + i > lim
+// are ignored (the causal diagonal tile, lim = the row; the last tile of a
+// ragged sequence, lim = its last key).
 template <bool MASKED>
-__device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float acc) {
+__device__ __forceinline__ float max64(const uint32_t* s, int col0, int lim, float acc) {
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     float x = __uint_as_float(s[k]), y = __uint_as_float(s[k + 8]);
     if (MASKED) {
-      x = (col0 + k <= r) ? x : -INFINITY;
-      y = (col0 + k + 8 <= r) ? y : -INFINITY;
+      x = (col0 + k <= lim) ? x : -INFINITY;
+      y = (col0 + k + 8 <= lim) ? y : -INFINITY;
     }
     a[k] = fmaxf(x, y);
   }
@@ -211,8 +212,8 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
     for (int k = 0; k < 8; ++k) {
       float x = __uint_as_float(s[i + k]), y = __uint_as_float(s[i + 8 + k]);
       if (MASKED) {
-        x = (col0 + i + k <= r) ? x : -INFINITY;
-        y = (col0 + i + 8 + k <= r) ? y : -INFINITY;
+        x = (col0 + i + k <= lim) ? x : -INFINITY;
+        y = (col0 + i + 8 + k <= lim) ? y : -INFINITY;
       }
       a[k] = fmax3(a[k], x, y);
     }
@@ -225,7 +226,7 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
 //   s16 = ue4m3(448 amax16); code = e2m1(P~ * 2688 / s16) (0 when s16 = 0).
 template <bool MASKED>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
-                                             int r, uint32_t (&p)[4], uint32_t* sf2) {
+                                             int lim, uint32_t (&p)[4], uint32_t* sf2) {
   const float2 c2 = make_float2(c, c);
   const float2 n2 = make_float2(neg, neg);
   float x[32];
@@ -238,10 +239,10 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
         __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), c2, n2);
     float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
     if (MASKED) {
-      f0 = (col0 + i + 0 <= r) ? f0 : 0.f;
-      f1 = (col0 + i + 1 <= r) ? f1 : 0.f;
-      f2 = (col0 + i + 2 <= r) ? f2 : 0.f;
-      f3 = (col0 + i + 3 <= r) ? f3 : 0.f;
+      f0 = (col0 + i + 0 <= lim) ? f0 : 0.f;
+      f1 = (col0 + i + 1 <= lim) ? f1 : 0.f;
+      f2 = (col0 + i + 2 <= lim) ? f2 : 0.f;
+      f3 = (col0 + i + 3 <= lim) ? f3 : 0.f;
     }
     acc0 = __fadd2_rn(acc0, make_float2(f0, f1));
     acc1 = __fadd2_rn(acc1, make_float2(f2, f3));
@@ -285,21 +286,20 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
 // the chunk's row sum and its two scale bytes.
 template <bool MASKED>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int q, float c, float neg,
-                                           int r, uint32_t prow, uint32_t* sf2) {
+                                           int r, int lim, uint32_t prow, uint32_t* sf2) {
   uint32_t p[4];
-  const float sum = exp_quant32<MASKED>(s, c, neg, 32 * q, r, p, sf2);
+  const float sum = exp_quant32<MASKED>(s, c, neg, 32 * q, lim, p, sf2);
   st_shared_v4(prow + (((uint32_t)q ^ (uint32_t)((r >> 1) & 3)) << 4), p[0], p[1], p[2], p[3]);
   return sum;
 }
 
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
-template <bool CAUSAL>
-__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int bh,
-                                         const int ntiles, const uint32_t tmem, const Bars& bar,
-                                         uint8_t* smem, volatile int* abort_flag,
-                                         uint32_t* status, const float* __restrict__ q_scales,
-                                         const float* __restrict__ k_scales,
-                                         const float scale_log2) {
+// RAGGED (non-causal launches of a sequence whose last tile is partial): the
+// last key tile masks keys n_tail .. 127.
+template <bool CAUSAL, bool RAGGED>
+__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
+                                         const uint32_t tmem, const Bars& bar, uint8_t* smem,
+                                         volatile int* abort_flag, uint32_t* status) {
   using L = Layout;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -324,7 +324,10 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     const float m_j = m_s[(2 * b) * 128 + r];
     const float alpha = m_s[(2 * b + 1) * 128 + r];
     const float neg = -m_j;
+    // masked tiles: the causal diagonal and the last tile of a ragged sequence
     const bool diag = CAUSAL && (j == qt);
+    const bool masked = diag || (RAGGED && j == nkv - 1);
+    const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes + 64u * h;
     uint32_t sa[32], sb[32];
     tmem_ld32(S, sa);
@@ -341,10 +344,10 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
       return;
     const uint32_t prow = smem_u32(smem + L::OFF_P + b * L::TILE + r * 64);
     uint32_t sf_lo, sf_hi;
-    float sum = diag ? exp_chunk<true>(sa, 2 * h, c, neg, r, prow, &sf_lo)
-                     : exp_chunk<false>(sa, 2 * h, c, neg, r, prow, &sf_lo);
-    sum += diag ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, prow, &sf_hi)
-                : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, prow, &sf_hi);
+    float sum = masked ? exp_chunk<true>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo)
+                       : exp_chunk<false>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo);
+    sum += masked ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi)
+                  : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi);
     // the row's four group scales of this 64-key block, in the tensor-core
     // layout: byte 16 (r % 32) + 4 (r / 32) + s of the block's 512 bytes
     st_shared_u32(smem_u32(smem + L::OFF_SFP + b * L::SF + h * 512 + 16 * (r & 31) + 4 * (r >> 5)),
@@ -359,8 +362,9 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 
 // Stats warpgroup: row max / running max per key tile, level-2 fold (one
 // tile behind), epilogue.
-template <bool CAUSAL, typename OutT>
-__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh,
+template <bool CAUSAL, typename OutT, bool RAGGED>
+__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int n_tail,
+                                           const int bh,
                                            const int H, const int G, const int N,
                                            const int ntiles, const uint32_t tmem, const Bars& bar,
                                            uint8_t* smem, volatile int* abort_flag,
@@ -424,6 +428,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       return;
     tc_fence_after();
     const bool diag = CAUSAL && (j == qt);
+    const bool masked = diag || (RAGGED && j == nkv - 1);
+    const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes;
     float mx = -INFINITY;
 #pragma unroll
@@ -433,7 +439,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      mx = diag ? max64<true>(&s[0][0], 64 * hh, r, mx) : max64<false>(&s[0][0], 64 * hh, r, mx);
+      mx = masked ? max64<true>(&s[0][0], 64 * hh, lim, mx)
+                  : max64<false>(&s[0][0], 64 * hh, lim, mx);
     }
     const float m_j = fmaxf(m, mx * c);
     const float alpha = ex2(m - m_j);
@@ -454,6 +461,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
                   mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)))
     return;
   const float inv_l = 1.f / (l_s[r] + l_s[128 + r]);
+  // rows past the end of a ragged sequence are padding: not stored
+  if (qt * 128 + r >= N) return;
   OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
 #pragma unroll
   for (int cv = 0; cv < D; cv += 8) {
@@ -467,7 +476,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   }
 }
 
-template <bool CAUSAL, typename OutT>
+template <bool CAUSAL, typename OutT, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -482,7 +491,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = N / 128;
+  // N tokens in ntiles 128-token tiles (codes padded to Np = 128 ntiles);
+  // the last tile holds n_tail of them
+  const int ntiles = (N + 127) / 128;
+  const int Np = ntiles * 128;
+  const int n_tail = N - (ntiles - 1) * 128;
   const int bh = blockIdx.y;
   // K/V head of this query head (grouped-query attention: G query heads per
   // K/V head; G = 1 is plain multi-head attention)
@@ -549,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (elect_one()) {
         const int64_t tile0 = (int64_t)bhk * ntiles;
         mbar_arrive_expect_tx(bar.q_full, L::TILE + L::SF);
-        tma_load_2d(sQ, &tm_q, 0, bh * N + qt * 128, bar.q_full);
+        tma_load_2d(sQ, &tm_q, 0, bh * Np + qt * 128, bar.q_full);
         bulk_load(sSFQ, q_sf + ((int64_t)bh * ntiles + qt) * L::SF, L::SF, bar.q_full);
         for (int j = 0; j < nkv; ++j) {
           const int sk = j % L::KS;
@@ -557,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                kDevTimeoutMma))
             break;
           mbar_arrive_expect_tx(&bar.k_full[sk], L::TILE + L::SF);
-          tma_load_2d(sK + sk * L::TILE, &tm_k, 0, bhk * N + j * 128, &bar.k_full[sk]);
+          tma_load_2d(sK + sk * L::TILE, &tm_k, 0, bhk * Np + j * 128, &bar.k_full[sk]);
           bulk_load(sSFK + sk * L::SF, k_sf + (tile0 + j) * L::SF, L::SF, &bar.k_full[sk]);
           const int sv = j % L::VS;
           if (!mbar_wait<true>(&bar.v_empty[sv], ((j / L::VS) & 1) ^ 1, abort_flag, status,
@@ -657,11 +670,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<CAUSAL>(wg - 1, qt, nkv, bh, ntiles, tmem, bar, smem, abort_flag, status, q_scales,
-                     k_scales, scale_log2);
+    exp_loop<CAUSAL, RAGGED>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<CAUSAL, OutT>(qt, nkv, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
+    stats_loop<CAUSAL, OutT, RAGGED>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
                              q_scales, k_scales, v_scales, out, scale_log2);
   }
 
@@ -673,14 +685,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool CAUSAL, typename OutT>
+template <bool CAUSAL, typename OutT, bool RAGGED = false>
 cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, cudaStream_t st) {
   using L = Layout;
-  auto kern = attn_fp4_kernel<CAUSAL, OutT>;
+  auto kern = attn_fp4_kernel<CAUSAL, OutT, RAGGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  const int ntiles = (int)(a.N / 128);
+  const int ntiles = (int)((a.N + 127) / 128);
   dim3 grid((unsigned)ntiles, (unsigned)(a.B * a.H));
   kern<<<grid, kThreads, L::SMEM, st>>>(
       tq, tk, tv, a.q_scales, a.k_scales, a.v_scales, static_cast<const uint8_t*>(a.q_sf),
@@ -699,7 +711,7 @@ cudaError_t launch_attn_fp4(const AttnArgs& a, cudaStream_t st, const char** det
   }
   const uint64_t BH = (uint64_t)(a.B * a.H);
   const uint64_t BHK = (uint64_t)(a.B * a.Hkv);
-  const uint64_t N = (uint64_t)a.N;
+  const uint64_t N = (uint64_t)((a.N + 127) / 128 * 128);  // codes padded to whole tiles
   CUtensorMap tq, tk, tv;
   // Q, K: [B*H*N rows, 64 bytes]; V^T: [B*H*128 rows (channels), N/2 bytes]
   if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q_codes, 64, BH * N, 64, 64, 128,
@@ -712,6 +724,10 @@ cudaError_t launch_attn_fp4(const AttnArgs& a, cudaStream_t st, const char** det
   if (a.causal)
     return a.dtype == 1 ? launch_typed<true, __nv_bfloat16>(a, tq, tk, tv, st)
                         : launch_typed<true, __half>(a, tq, tk, tv, st);
+  // causal launches mask the partial last tile through the diagonal already
+  if (a.N % 128 != 0)
+    return a.dtype == 1 ? launch_typed<false, __nv_bfloat16, true>(a, tq, tk, tv, st)
+                        : launch_typed<false, __half, true>(a, tq, tk, tv, st);
   return a.dtype == 1 ? launch_typed<false, __nv_bfloat16>(a, tq, tk, tv, st)
                       : launch_typed<false, __half>(a, tq, tk, tv, st);
 }

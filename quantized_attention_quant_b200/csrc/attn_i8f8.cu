@@ -201,19 +201,20 @@ __device__ __forceinline__ float ldg_early(const float* p) {
 // A score as read from TMEM: the float 1.5 * 2^23 + A (exact).
 __device__ __forceinline__ float biased(uint32_t a) { return __uint_as_float(a); }
 
-// Max of 64 scores and a running value.  MASKED: columns col0 + i > r are
-// ignored (causal diagonal tile): they read as 0, below every biased INT8
-// score, or -inf for the plain FP32 scores of the FP8 Q K^T.
+// Max of 64 scores and a running value.  MASKED: columns col0 + i > lim are
+// ignored (the causal diagonal tile, lim = the row; the last tile of a
+// ragged sequence, lim = its last key): they read as 0, below every biased
+// INT8 score, or -inf for the plain FP32 scores of the FP8 Q K^T.
 template <bool MASKED, bool QF8>
-__device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float acc) {
+__device__ __forceinline__ float max64(const uint32_t* s, int col0, int lim, float acc) {
   constexpr float kLow = QF8 ? -INFINITY : 0.f;
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     float x = biased(s[k]), y = biased(s[k + 8]);
     if (MASKED) {
-      x = (col0 + k <= r) ? x : kLow;
-      y = (col0 + k + 8 <= r) ? y : kLow;
+      x = (col0 + k <= lim) ? x : kLow;
+      y = (col0 + k + 8 <= lim) ? y : kLow;
     }
     a[k] = fmaxf(x, y);
   }
@@ -223,8 +224,8 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
     for (int k = 0; k < 8; ++k) {
       float x = biased(s[i + k]), y = biased(s[i + 8 + k]);
       if (MASKED) {
-        x = (col0 + i + k <= r) ? x : kLow;
-        y = (col0 + i + 8 + k <= r) ? y : kLow;
+        x = (col0 + i + k <= lim) ? x : kLow;
+        y = (col0 + i + 8 + k <= lim) ? y : kLow;
       }
       a[k] = fmax3(a[k], x, y);
     }
@@ -236,7 +237,7 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int r, float
 // scores are plain FP32 (no bias to remove).
 template <bool MASKED, bool QF8>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
-                                             int r, uint32_t (&p)[8]) {
+                                             int lim, uint32_t (&p)[8]) {
   const float2 c2 = make_float2(c, c);
   const float2 n2 = make_float2(neg, neg);
   const float2 mb = make_float2(-kBias, -kBias);
@@ -254,10 +255,10 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
     const float2 t23 = __ffma2_rn(x23, c2, n2);
     float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
     if (MASKED) {
-      f0 = (col0 + i + 0 <= r) ? f0 : 0.f;
-      f1 = (col0 + i + 1 <= r) ? f1 : 0.f;
-      f2 = (col0 + i + 2 <= r) ? f2 : 0.f;
-      f3 = (col0 + i + 3 <= r) ? f3 : 0.f;
+      f0 = (col0 + i + 0 <= lim) ? f0 : 0.f;
+      f1 = (col0 + i + 1 <= lim) ? f1 : 0.f;
+      f2 = (col0 + i + 2 <= lim) ? f2 : 0.f;
+      f3 = (col0 + i + 3 <= lim) ? f3 : 0.f;
     }
     acc0 = __fadd2_rn(acc0, make_float2(f0, f1));
     acc1 = __fadd2_rn(acc1, make_float2(f2, f3));
@@ -285,16 +286,18 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
 // P~V MMA); returns the chunk's row sum.
 template <bool MASKED, bool QF8>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int cc, float c, float neg,
-                                           int r, uint32_t pcol) {
+                                           int lim, uint32_t pcol) {
   uint32_t p[8];
-  const float sum = exp_quant32<MASKED, QF8>(s, c, neg, 32 * cc, r, p);
+  const float sum = exp_quant32<MASKED, QF8>(s, c, neg, 32 * cc, lim, p);
   tmem_st8(pcol, p);
   return sum;
 }
 
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
-template <int D, bool CAUSAL, bool QF8>
-__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv,
+// RAGGED (non-causal launches of a sequence whose last tile is partial): the
+// last key tile masks keys n_tail .. 127.
+template <int D, bool CAUSAL, bool QF8, bool RAGGED>
+__device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
                                          const uint32_t tmem, const Bars& bar, uint8_t* smem,
                                          volatile int* abort_flag, uint32_t* status) {
   using L = Layout<D>;
@@ -336,7 +339,11 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     const float m_j = m_s[(2 * b) * 128 + r];
     const float alpha = m_s[(2 * b + 1) * 128 + r];
     const float neg = kLog2_448 - m_j;  // yields 448 P~ directly
+    // masked tiles: the causal diagonal (keys up to the row) and the last
+    // tile of a ragged sequence (keys up to n_tail - 1)
     const bool diag = CAUSAL && (j == qt);
+    const bool masked = diag || (RAGGED && j == nkv - 1);
+    const int lim = diag ? r : n_tail - 1;
     const int sbuf = j % L::SB;
     const uint32_t S = tmem + lanes + 128u * sbuf + 64u * h;
     const uint32_t P = tmem + lanes + L::COL_P + 32u * b + 16u * h;
@@ -358,11 +365,11 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    float sum = diag ? exp_chunk<true, QF8>(sa, 2 * h, c, neg, r, P)
-                     : exp_chunk<false, QF8>(sa, 2 * h, c, neg, r, P);
+    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, c, neg, lim, P)
+                       : exp_chunk<false, QF8>(sa, 2 * h, c, neg, lim, P);
     if (r == 0 && h == 0) SAGE_TR(14, j);
-    sum += diag ? exp_chunk<true, QF8>(sb, 2 * h + 1, c, neg, r, P + 8)
-                : exp_chunk<false, QF8>(sb, 2 * h + 1, c, neg, r, P + 8);
+    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, c, neg, lim, P + 8)
+                  : exp_chunk<false, QF8>(sb, 2 * h + 1, c, neg, lim, P + 8);
     l = fmaf(alpha, l, sum);
     if (r == 0 && h == 0) SAGE_TR(10, j);
     tmem_wait_st();
@@ -377,9 +384,9 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 
 // Stats warpgroup: row max / running max per key tile, level-2 fold,
 // epilogue.
-template <int D, bool CAUSAL, typename OutT, bool QF8>
-__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int bh,
-                                           const int H, const int G, const int N,
+template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED>
+__device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int n_tail,
+                                           const int bh, const int H, const int G, const int N,
                                            const int ntiles, const uint32_t tmem, const Bars& bar,
                                            uint8_t* smem, volatile int* abort_flag,
                                            uint32_t* status, const float* __restrict__ q_scales,
@@ -442,6 +449,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     tc_fence_after();
     if (r == 0) SAGE_TR(4, j);
     const bool diag = CAUSAL && (j == qt);
+    const bool masked = diag || (RAGGED && j == nkv - 1);
+    const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
     float mx = QF8 ? -INFINITY : 0.f;
 #pragma unroll
@@ -451,8 +460,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      mx = diag ? max64<true, QF8>(&s[0][0], 64 * hh, r, mx)
-                : max64<false, QF8>(&s[0][0], 64 * hh, r, mx);
+      mx = masked ? max64<true, QF8>(&s[0][0], 64 * hh, lim, mx)
+                  : max64<false, QF8>(&s[0][0], 64 * hh, lim, mx);
     }
     // c >= 0, so the max of the scaled scores is the scaled max
     const float m_j = fmaxf(m, (QF8 ? mx : mx - kBias) * c);
@@ -476,6 +485,8 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     return;
   const float inv_l = 1.f / (l_s[r] + l_s[128 + r]);
   const float* vs = v_scales + (int64_t)kv_head(bh, H, G) * D;
+  // rows past the end of a ragged sequence are padding: not stored
+  if (qt * 128 + r >= N) return;
   OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
 #pragma unroll
   for (int cv = 0; cv < D; cv += 8) {
@@ -489,7 +500,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   }
 }
 
-template <int D, bool CAUSAL, typename OutT, bool QF8>
+template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -503,7 +514,11 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = N / 128;
+  // N tokens in ntiles 128-token tiles (codes padded to Np = 128 ntiles);
+  // the last tile holds n_tail of them
+  const int ntiles = (N + 127) / 128;
+  const int Np = ntiles * 128;
+  const int n_tail = N - (ntiles - 1) * 128;
   const int bh = blockIdx.y;
   // K/V head of this query head (grouped-query attention: G query heads per
   // K/V head; G = 1 is plain multi-head attention)
@@ -569,14 +584,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       // ---------------------------------------------------------- producer
       if (elect_one()) {
         mbar_arrive_expect_tx(bar.q_full, L::Q_BYTES);
-        tma_load_2d(sQ, &tm_q, 0, bh * N + qt * 128, bar.q_full);
+        tma_load_2d(sQ, &tm_q, 0, bh * Np + qt * 128, bar.q_full);
         for (int j = 0; j < nkv; ++j) {
           const int sk = j % L::KS;
           if (!mbar_wait<true>(&bar.k_empty[sk], ((j / L::KS) & 1) ^ 1, abort_flag, status,
                                kDevTimeoutMma))
             break;
           mbar_arrive_expect_tx(&bar.k_full[sk], L::K_BYTES);
-          tma_load_2d(sK + sk * L::K_BYTES, &tm_k, 0, bhk * N + j * 128, &bar.k_full[sk]);
+          tma_load_2d(sK + sk * L::K_BYTES, &tm_k, 0, bhk * Np + j * 128, &bar.k_full[sk]);
           const int sv = j % L::VS;
           if (!mbar_wait<true>(&bar.v_empty[sv], ((j / L::VS) & 1) ^ 1, abort_flag, status,
                                kDevTimeoutMma))
@@ -675,10 +690,10 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL, QF8>(wg - 1, qt, nkv, tmem, bar, smem, abort_flag, status);
+    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<D, CAUSAL, OutT, QF8>(qt, nkv, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
+    stats_loop<D, CAUSAL, OutT, QF8, RAGGED>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
                                 q_scales, k_scales, v_scales, out, scale_log2);
   }
 
@@ -694,14 +709,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
 #endif
 }
 
-template <int D, bool CAUSAL, typename OutT, bool QF8>
+template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED = false>
 cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, cudaStream_t st) {
   using L = Layout<D>;
-  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, QF8>;
+  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, QF8, RAGGED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
-  const int ntiles = (int)(a.N / 128);
+  const int ntiles = (int)((a.N + 127) / 128);
   dim3 grid((unsigned)ntiles, (unsigned)(a.B * a.H));
   kern<<<grid, kThreadsAttn, L::SMEM, st>>>(tq, tk, tv, a.q_scales, a.k_scales, a.v_scales,
                                            reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H,
@@ -716,6 +731,10 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap
     return a.dtype == 1 ? launch_typed<D, true, __nv_bfloat16, QF8>(a, tq, tk, tv, st)
                         : launch_typed<D, true, __half, QF8>(a, tq, tk, tv, st);
   }
+  // causal launches mask the partial last tile through the diagonal already
+  if (a.N % 128 != 0)
+    return a.dtype == 1 ? launch_typed<D, false, __nv_bfloat16, QF8, true>(a, tq, tk, tv, st)
+                        : launch_typed<D, false, __half, QF8, true>(a, tq, tk, tv, st);
   return a.dtype == 1 ? launch_typed<D, false, __nv_bfloat16, QF8>(a, tq, tk, tv, st)
                       : launch_typed<D, false, __half, QF8>(a, tq, tk, tv, st);
 }
@@ -725,7 +744,7 @@ cudaError_t launch_d(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap
 cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** detail) {
   const uint64_t BH = (uint64_t)(a.B * a.H);
   const uint64_t BHK = (uint64_t)(a.B * a.Hkv);
-  const uint64_t N = (uint64_t)a.N;
+  const uint64_t N = (uint64_t)((a.N + 127) / 128 * 128);  // codes padded to whole tiles
   const uint64_t D = (uint64_t)a.d;
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_swz =

@@ -57,7 +57,8 @@ struct PrepassPtrs {
   const void* q;
   const void* k;
   const void* v;
-  int N;
+  int N;   // tokens per head
+  int Np;  // N rounded up to whole 128-token tiles: the token stride of every code buffer
   void* q_codes;
   float* q_scales;
   uint8_t* q_sf;
@@ -211,16 +212,33 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
+// Index of a 16-byte vector of a [128][D] tile, with padding tokens (nv and
+// up) moved onto the last real token: loads stay unconditional, so they can
+// all be in flight at once; the caller zeroes what it read for padding.
+template <int D, bool RAGGED>
+__device__ __forceinline__ int clamp_vec(int vec, int nv) {
+  if (!RAGGED) return vec;
+  const int t = vec / (D / 8);
+  return t < nv ? vec : (nv - 1) * (D / 8) + vec % (D / 8);
+}
+
 // Copies one 128-token tile [128][D] of T into shared memory with 16-byte
-// loads (consecutive threads, consecutive vectors).
-template <typename T, int D>
-__device__ __forceinline__ void stage_tile(const T* __restrict__ src, T* tile) {
+// loads (consecutive threads, consecutive vectors).  Tokens nv..127 (past
+// the end of a ragged sequence) are not read and stage as zeros.
+template <typename T, int D, bool RAGGED>
+__device__ __forceinline__ void stage_tile(const T* __restrict__ src, T* tile, int nv) {
   constexpr int VPT = 128 * D / 8 / kThreads;
   const uint4* s = reinterpret_cast<const uint4*>(src);
   uint4* d = reinterpret_cast<uint4*>(tile);
   uint4 v[VPT];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) v[i] = __ldg(s + threadIdx.x + i * kThreads);
+  for (int i = 0; i < VPT; ++i) {
+    // every load issued (a padding token re-reads a real one), then zeroed
+    const int vec = threadIdx.x + i * kThreads;
+    const bool pad = RAGGED && vec / (D / 8) >= nv;
+    v[i] = __ldg(s + clamp_vec<D, RAGGED>(vec, nv));
+    if (pad) v[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
   for (int i = 0; i < VPT; ++i) d[threadIdx.x + i * kThreads] = v[i];
 }
@@ -231,16 +249,16 @@ __device__ __forceinline__ void stage_tile(const T* __restrict__ src, T* tile) {
 // order with an FP64 sum.  V: each thread keeps the max of |V| over its
 // vectors (8 channels each) and merges it into a shared per-channel max
 // (non-negative floats order like their bit patterns).
-template <typename T, int D>
-__device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int chunk,
+template <typename T, int D, bool RAGGED>
+__device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int chunk, int nv,
                                            bool do_k, bool do_v, T* tile, uint32_t* vmax_s) {
   constexpr int VPT = 128 * D / 8 / kThreads;
-  const int nchunks = p.N / 128;
+  const int nchunks = (RAGGED ? p.Np : p.N) / 128;
   const int t = threadIdx.x;
   const int64_t row0 = bh * p.N + (int64_t)chunk * 128;
   const int64_t out = (bh * nchunks + chunk) * D;
   if (do_v && t < D) vmax_s[t] = 0u;
-  if (do_k) stage_tile<T, D>(reinterpret_cast<const T*>(p.k) + row0 * D, tile);
+  if (do_k) stage_tile<T, D, RAGGED>(reinterpret_cast<const T*>(p.k) + row0 * D, tile, nv);
   __syncthreads();
   if (do_v) {
     const T* src = reinterpret_cast<const T*>(p.v) + row0 * D;
@@ -248,8 +266,9 @@ __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int
     float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
+      const int vec = t + i * kThreads;
       float x[8];
-      load8(src + (t + i * kThreads) * 8, x);
+      load8(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);  // a re-read real token changes no max
 #pragma unroll
       for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(x[e]));
     }
@@ -259,9 +278,10 @@ __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int
   __syncthreads();
   if (t < D) {
     if (do_k) {
+      // the chunk's tokens in order (its first nv tokens)
       double acc = 0.0;
 #pragma unroll 16
-      for (int i = 0; i < 128; ++i) acc += (double)static_cast<float>(tile[i * D + t]);
+      for (int i = 0; i < nv; ++i) acc += (double)static_cast<float>(tile[i * D + t]);
       p.ksum[out + t] = acc;
     }
     if (do_v) p.vmax[out + t] = __uint_as_float(vmax_s[t]);
@@ -306,10 +326,10 @@ __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int
 // Two passes over the 128-token tile: the amax pass keeps nothing, the code
 // pass reads the tile again (from L1/L2), so the role needs few registers and
 // many CTAs fit on an SM.  A thread's vectors all cover the same 8 channels.
-template <typename T, int D, bool FP8>
+template <typename T, int D, bool FP8, bool RAGGED>
 __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const float* mean,
                                                 uint8_t* __restrict__ dst, float* scale_out,
-                                                float* red) {
+                                                float* red, int nv) {
   constexpr int VPT = 128 * D / 8 / kThreads;  // 16-byte vectors per thread
   const int c0 = (threadIdx.x % (D / 8)) * 8;
   // x - mu as x + (-mu): the same single rounding
@@ -330,11 +350,15 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
       }
     }
   };
+  // tokens nv..127 (padding of a ragged sequence) re-read a real token, so
+  // the block maximum is unchanged, and get code 0
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
+    // a padding vector re-reads a real one: it changes no maximum
+    const int vec = threadIdx.x + i * kThreads;
     float x[8];
-    load8(src + (threadIdx.x + i * kThreads) * 8, x);
+    load8(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
     smooth(x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
@@ -348,10 +372,11 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
     uint2 w = make_uint2(0u, 0u);
     if (s != 0.f) {
       float x[8];
-      load8(src + vec * 8, x);
+      load8(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
       smooth(x);
       w = FP8 ? fp8_codes8(x, s, rs) : int8_codes8(x, s, rs);
     }
+    if (RAGGED && vec / (D / 8) >= nv) w = make_uint2(0u, 0u);
     *reinterpret_cast<uint2*>(dst + vec * 8) = w;
   }
   if (threadIdx.x == 0) *scale_out = s;
@@ -366,11 +391,14 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
 // through one e4m3x2 conversion each, and the two 16-bit results must match
 // (else the unit is redone on IEEE quotients); the matching result is the
 // two codes, already packed.
-template <typename T, int D>
+template <typename T, int D, bool RAGGED>
 __device__ __forceinline__ void role_quant_v_fp8(const T* __restrict__ src,
                                                  const float* __restrict__ vs,
-                                                 uint8_t* __restrict__ dst, int N, T* tile) {
-  stage_tile<T, D>(src, tile);
+                                                 uint8_t* __restrict__ dst, int N, T* tile,
+                                                 int nv) {
+  // padding tokens stage as zeros and so get code 0; N is the row length of
+  // V^T (the padded token count)
+  stage_tile<T, D, RAGGED>(src, tile, nv);
   __syncthreads();
   constexpr int UNITS = (D / 2) * 4;  // channel pairs x 32-token groups
   const float2 lo2 = make_float2(kBracketLo, kBracketLo);
@@ -459,11 +487,11 @@ __device__ __forceinline__ int64_t sf_offset(int64_t bh, int ntiles, int tile, i
 
 // Q or smoothed K of one tile: g = amax/2688, per 16 channels
 // s16 = ue4m3(amax16 / (6 g)), code = e2m1(x / (s16 g)).
-template <typename T, int D>
+template <typename T, int D, bool RAGGED>
 __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src, const float* mean,
                                                       uint8_t* __restrict__ codes, float* g_out,
                                                       uint8_t* __restrict__ sf, int64_t bh,
-                                                      int ntiles, int tile, float* red) {
+                                                      int ntiles, int tile, float* red, int nv) {
   constexpr int G = D / 16;                // groups per row
   constexpr int GPT = 128 * G / kThreads;  // groups per thread
   float x[GPT][16];
@@ -472,9 +500,12 @@ __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src,
   for (int i = 0; i < GPT; ++i) {
     const int grp = threadIdx.x + i * kThreads;
     const int r = grp / G, gc = grp % G;
+    // a padding row re-reads the last real row (loads stay unconditional)
+    // and is zeroed below: code 0, scale 0
+    const int rr = (!RAGGED || r < nv) ? r : nv - 1;
     float a[8], b[8];
-    load8(src + r * D + gc * 16, a);
-    load8(src + r * D + gc * 16 + 8, b);
+    load8(src + rr * D + gc * 16, a);
+    load8(src + rr * D + gc * 16 + 8, b);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       x[i][e] = a[e];
@@ -484,6 +515,10 @@ __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src,
       const float* mu = mean + gc * 16;
 #pragma unroll
       for (int e = 0; e < 16; ++e) x[i][e] = __fsub_rn(x[i][e], __ldg(mu + e));
+    }
+    if (RAGGED && r >= nv) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) x[i][e] = 0.f;
     }
 #pragma unroll
     for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
@@ -518,12 +553,12 @@ __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src,
 
 // V of one tile for FP4: staged in shared memory in its input type; each
 // thread handles (channel, 16-token group) pairs.
-template <typename T, int D>
+template <typename T, int D, bool RAGGED>
 __device__ __forceinline__ void role_quant_fp4_v(const T* __restrict__ src, int N,
                                                  uint8_t* __restrict__ vt_codes, float* g_out,
                                                  uint8_t* __restrict__ v_sf, int64_t bh,
                                                  int ntiles, int tile, T (*xs)[D + 2],
-                                                 float* red) {
+                                                 float* red, int nv) {
   constexpr int VPT = 128 * D / 8 / kThreads;
   constexpr int PAIRS = D * 8;  // channels x 16-token groups
   float amax = 0.f;
@@ -531,11 +566,15 @@ __device__ __forceinline__ void role_quant_fp4_v(const T* __restrict__ src, int 
   for (int i = 0; i < VPT; ++i) {
     const int vec = threadIdx.x + i * kThreads;
     const int t = vec / (D / 8), c0 = (vec % (D / 8)) * 8;
+    // a padding token re-reads a real one (no change to the max) and
+    // stages as zeros
+    const bool pad = RAGGED && t >= nv;
+    const int cv = clamp_vec<D, RAGGED>(vec, nv);
     float x[8];
-    load8(src + vec * 8, x);
+    load8(src + cv * 8, x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      xs[t][c0 + e] = src[vec * 8 + e];
+      xs[t][c0 + e] = pad ? static_cast<T>(0.f) : src[cv * 8 + e];
       amax = fmaxf(amax, fabsf(x[e]));
     }
   }
@@ -583,7 +622,9 @@ __device__ __forceinline__ void role_quant_fp4_v(const T* __restrict__ src, int 
 // compiled in, so each launch gets the register and shared-memory footprint
 // of its own roles (and the occupancy that goes with it).
 #define SAGE_ROLE(r) if constexpr (((MASK >> (r)) & 1) != 0)
-template <typename T, int D, int MASK>
+// RAGGED: N is not a multiple of 128, so the last tile is partial (without
+// it every guard on padding tokens compiles away).
+template <typename T, int D, int MASK, bool RAGGED>
 __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles roles) {
   // one staging buffer, sized for the largest role of the mask (a CTA runs
   // one role)
@@ -603,69 +644,76 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   // roles bh_kv (a CTA leaves as a whole, before any barrier)
   const bool q_role = role == kQuantQ8 || role == kQuantQ4 || role == kQuantQF8;
   if (bh >= (q_role ? p.bh_q : p.bh_kv)) return;
-  const int ntiles = p.N / 128;
-  const int64_t row0 = bh * p.N + (int64_t)tile * 128;
+  // (without RAGGED, Np == N: the same offsets as before padding existed)
+  const int ntiles = (RAGGED ? p.Np : p.N) / 128;
+  const int nv = RAGGED ? min(128, p.N - tile * 128) : 128;  // real tokens of this tile
+  const int64_t row0 = bh * p.N + (int64_t)tile * 128;       // input rows
+  const int64_t crow0 = RAGGED ? bh * p.Np + (int64_t)tile * 128 : row0;  // code rows
+  const int Np = RAGGED ? p.Np : p.N;
   switch (role) {
     case kQuantQ8:
       SAGE_ROLE(kQuantQ8)
-      role_quant_8bit<T, D, false>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
-                                   reinterpret_cast<uint8_t*>(p.q_codes) + row0 * D,
-                                   p.q_scales + bh * ntiles + tile, red);
+      role_quant_8bit<T, D, false, RAGGED>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+                                   reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * D,
+                                   p.q_scales + bh * ntiles + tile, red, nv);
       break;
     case kQuantK8:
       SAGE_ROLE(kQuantK8)
-      role_quant_8bit<T, D, false>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
-                                   reinterpret_cast<uint8_t*>(p.k_codes) + row0 * D,
-                                   p.k_scales + bh * ntiles + tile, red);
+      role_quant_8bit<T, D, false, RAGGED>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+                                   reinterpret_cast<uint8_t*>(p.k_codes) + crow0 * D,
+                                   p.k_scales + bh * ntiles + tile, red, nv);
       break;
     case kQuantQF8:
       SAGE_ROLE(kQuantQF8)
-      role_quant_8bit<T, D, true>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
-                                  reinterpret_cast<uint8_t*>(p.q_codes) + row0 * D,
-                                  p.q_scales + bh * ntiles + tile, red);
+      role_quant_8bit<T, D, true, RAGGED>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+                                  reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * D,
+                                  p.q_scales + bh * ntiles + tile, red, nv);
       break;
     case kQuantKF8:
       SAGE_ROLE(kQuantKF8)
-      role_quant_8bit<T, D, true>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
-                                  reinterpret_cast<uint8_t*>(p.k_codes) + row0 * D,
-                                  p.k_scales + bh * ntiles + tile, red);
+      role_quant_8bit<T, D, true, RAGGED>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+                                  reinterpret_cast<uint8_t*>(p.k_codes) + crow0 * D,
+                                  p.k_scales + bh * ntiles + tile, red, nv);
       break;
     case kQuantV8:
       SAGE_ROLE(kQuantV8)
-      role_quant_v_fp8<T, D>(reinterpret_cast<const T*>(p.v) + row0 * D, p.v_scales + bh * D,
-                             reinterpret_cast<uint8_t*>(p.v_codes) + bh * D * (int64_t)p.N +
+      role_quant_v_fp8<T, D, RAGGED>(reinterpret_cast<const T*>(p.v) + row0 * D, p.v_scales + bh * D,
+                             reinterpret_cast<uint8_t*>(p.v_codes) + bh * D * (int64_t)Np +
                                  (int64_t)tile * 128,
-                             p.N, reinterpret_cast<T*>(smem_raw));
+                             Np, reinterpret_cast<T*>(smem_raw), nv);
       break;
     case kQuantQ4:
       SAGE_ROLE(kQuantQ4)
-      role_quant_fp4_tokens<T, D>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
-                                  reinterpret_cast<uint8_t*>(p.q_codes) + row0 * (D / 2),
-                                  p.q_scales + bh * ntiles + tile, p.q_sf, bh, ntiles, tile, red);
+      role_quant_fp4_tokens<T, D, RAGGED>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+                                  reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * (D / 2),
+                                  p.q_scales + bh * ntiles + tile, p.q_sf, bh, ntiles, tile, red,
+                                  nv);
       break;
     case kQuantK4:
       SAGE_ROLE(kQuantK4)
-      role_quant_fp4_tokens<T, D>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
-                                  reinterpret_cast<uint8_t*>(p.k_codes) + row0 * (D / 2),
-                                  p.k_scales + bh * ntiles + tile, p.k_sf, bh, ntiles, tile, red);
+      role_quant_fp4_tokens<T, D, RAGGED>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+                                  reinterpret_cast<uint8_t*>(p.k_codes) + crow0 * (D / 2),
+                                  p.k_scales + bh * ntiles + tile, p.k_sf, bh, ntiles, tile, red,
+                                  nv);
       break;
     case kQuantV4:
       SAGE_ROLE(kQuantV4)
-      role_quant_fp4_v<T, D>(reinterpret_cast<const T*>(p.v) + row0 * D, p.N,
+      role_quant_fp4_v<T, D, RAGGED>(reinterpret_cast<const T*>(p.v) + row0 * D, Np,
                              reinterpret_cast<uint8_t*>(p.v_codes), p.v_scales + bh * ntiles + tile,
-                             p.v_sf, bh, ntiles, tile, reinterpret_cast<T(*)[D + 2]>(smem_raw), red);
+                             p.v_sf, bh, ntiles, tile, reinterpret_cast<T(*)[D + 2]>(smem_raw), red,
+                             nv);
       break;
     case kStatsK:
       SAGE_ROLE(kStatsK)
-      role_stats<T, D>(p, bh, tile, true, false, reinterpret_cast<T*>(smem_raw), vmax_s);
+      role_stats<T, D, RAGGED>(p, bh, tile, nv, true, false, reinterpret_cast<T*>(smem_raw), vmax_s);
       break;
     case kStatsKV:
       SAGE_ROLE(kStatsKV)
-      role_stats<T, D>(p, bh, tile, true, true, reinterpret_cast<T*>(smem_raw), vmax_s);
+      role_stats<T, D, RAGGED>(p, bh, tile, nv, true, true, reinterpret_cast<T*>(smem_raw), vmax_s);
       break;
     case kStatsV:
       SAGE_ROLE(kStatsV)
-      role_stats<T, D>(p, bh, tile, false, true, reinterpret_cast<T*>(smem_raw), vmax_s);
+      role_stats<T, D, RAGGED>(p, bh, tile, nv, false, true, reinterpret_cast<T*>(smem_raw), vmax_s);
       break;
     default:
       break;
@@ -680,10 +728,16 @@ constexpr int bit(int r) { return 1 << r; }
 // counts
 template <typename T, int D, int MA, int MB>
 cudaError_t run_plan(const PrepassPtrs& p, Roles a, Roles b, cudaStream_t st) {
-  const int ntiles = p.N / 128;
+  const int ntiles = p.Np / 128;
   const int64_t BH = p.bh_q > p.bh_kv ? p.bh_q : p.bh_kv;
-  if (a.n) prepass_kernel<T, D, MA><<<dim3(ntiles, (unsigned)BH, a.n), kThreads, 0, st>>>(p, a);
-  if (b.n) prepass_kernel<T, D, MB><<<dim3(ntiles, (unsigned)BH, b.n), kThreads, 0, st>>>(p, b);
+  const dim3 grid_a(ntiles, (unsigned)BH, a.n), grid_b(ntiles, (unsigned)BH, b.n);
+  if (p.N % 128 != 0) {
+    if (a.n) prepass_kernel<T, D, MA, true><<<grid_a, kThreads, 0, st>>>(p, a);
+    if (b.n) prepass_kernel<T, D, MB, true><<<grid_b, kThreads, 0, st>>>(p, b);
+  } else {
+    if (a.n) prepass_kernel<T, D, MA, false><<<grid_a, kThreads, 0, st>>>(p, a);
+    if (b.n) prepass_kernel<T, D, MB, false><<<grid_b, kThreads, 0, st>>>(p, b);
+  }
   return cudaGetLastError();
 }
 
@@ -703,6 +757,7 @@ PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
   p.q = a.q;
   p.k = a.k;
   p.N = (int)a.N;
+  p.Np = (int)((a.N + 127) / 128 * 128);
   p.q_codes = a.q_codes;
   p.q_scales = a.q_scales;
   p.q_sf = static_cast<uint8_t*>(a.q_sf);
@@ -720,6 +775,7 @@ PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
 void add_v(PrepassPtrs& p, const QuantVArgs& a) {
   p.v = a.v;
   p.N = (int)a.N;
+  p.Np = (int)((a.N + 127) / 128 * 128);
   p.v_codes = a.v_codes;
   p.v_scales = a.v_scales;
   p.v_sf = static_cast<uint8_t*>(a.v_sf);

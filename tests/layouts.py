@@ -2,7 +2,9 @@
 
 Pure indexing (no arithmetic of the method): turns the raw byte buffers that
 the C ABI fills into the arrays the oracle returns, so that the two can be
-compared element by element.
+compared element by element.  Code buffers hold Np = N rounded up to a
+multiple of 128 tokens per head; the decoders return the first N (padded()
+gives the padding itself, which must be zero).
 """
 
 import numpy as np
@@ -12,8 +14,28 @@ def _np(t):
     return t.detach().cpu().numpy()
 
 
+def np_of(N):
+    return -(-N // 128) * 128
+
+
 def int8_codes(buf, B, H, N, d):
-    return _np(buf).view(np.int8).reshape(B, H, N, d)
+    return _np(buf).view(np.int8).reshape(B, H, np_of(N), d)[:, :, :N]
+
+
+def token_codes(buf, B, H, N, d):
+    """Q/K 8-bit codes [B, H, N, d] (padding dropped)."""
+    return _np(buf).reshape(B, H, np_of(N), d)[:, :, :N]
+
+
+def vt_codes(buf, B, H, d, N):
+    """V^T 8-bit codes [B, H, d, N] (padding dropped)."""
+    return _np(buf).reshape(B, H, d, np_of(N))[..., :N]
+
+
+def padded_tokens(buf, B, H, N):
+    """The padding of a token-major code buffer: tokens N .. Np-1 of every
+    head (all bytes of those rows)."""
+    return _np(buf).reshape(B, H, np_of(N), -1)[:, :, N:]
 
 
 def f32(buf, *shape):
@@ -47,13 +69,13 @@ def sf_rows(buf, BH, ntiles, nchunk, rows_used):
 
 def qk_sf(buf, B, H, N, d):
     """Q/K FP4 scales -> [B, H, N, d/16] (the oracle's layout)."""
-    nt = N // 128
+    nt = -(-N // 128)
     r = sf_rows(buf, B * H, nt, d // 64, 128)                   # [BH, t, 128, d/16]
-    return r.reshape(B, H, N, d // 16)
+    return r.reshape(B, H, nt * 128, d // 16)[:, :, :N]
 
 
 def v_sf(buf, B, H, N, d):
-    """V FP4 scales -> [B, H, d, N/16] (the oracle's layout)."""
-    nt = N // 128
+    """V FP4 scales -> [B, H, d, ceil(N/16)] (the oracle's layout)."""
+    nt = -(-N // 128)
     r = sf_rows(buf, B * H, nt, 2, d)                           # [BH, t, d, 8]
-    return r.transpose(0, 2, 1, 3).reshape(B, H, d, N // 16)
+    return r.transpose(0, 2, 1, 3).reshape(B, H, d, nt * 8)[..., :-(-N // 16)]

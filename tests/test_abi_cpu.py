@@ -68,7 +68,7 @@ def call_attn(lib, **kw):
     (dict(B=-1), -1, "negative"),
     (dict(d=96), -2, "head dim"),
     (dict(mode=1, d=64, qsf=FAKE, ksf=FAKE, vsf=FAKE), -2, "FP4"),
-    (dict(N=200), -2, "multiple of 128"),
+    (dict(B=1, H=1, N=2 ** 31 - 100), -2, "2^31"),     # rounded up past 2^31
     (dict(qc=None), -1, "q_codes is NULL"),
     (dict(o=FAKE + 4), -2, "aligned"),
     (dict(qsf=FAKE), -1, "must be NULL"),
@@ -120,5 +120,5 @@ def test_gqa_empty_and_shape_errors(lib):
     assert gqa(lib, B=0) == 0
     assert gqa(lib, N=0) == 0
     assert gqa(lib, H=0, Hkv=0) == 0
-    s = gqa(lib, N=200)
-    assert s == -2 and "multiple of 128" in lib.sage_status_string(s).decode()
+    s = gqa(lib, B=1, H=8, Hkv=2, N=2 ** 28)
+    assert s == -2 and "2^31" in lib.sage_status_string(s).decode()

@@ -98,6 +98,36 @@ def test_fp8_qk_random(cuda_device, N, dtype, d, causal):
     assert sage.device_status() == 0
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp8", "fp4"])
+@pytest.mark.parametrize("N", [1, 77, 200, 1000])
+def test_ragged_lengths(cuda_device, N, mode, causal):
+    # N not a multiple of 128: the last tile is partial (keys past N masked,
+    # rows past N not stored); d = 64 where the mode allows it
+    d = 128 if mode == "fp4" else (64 if N % 2 else 128)
+    q, k, v = rand_qkv(2, 2, N, d, "f16", seed=700 + N + causal)
+    dev = torch.device("cuda")
+    out = sage.sage_attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=causal, mode=mode)
+    torch.cuda.synchronize()
+    assert sage.device_status() == 0
+    check_against_oracle(to_numpy32(out), q, k, v, causal, 1 / math.sqrt(d), mode, "f16")
+
+
+def test_ragged_output_stays_in_bounds(cuda_device):
+    # O of a ragged sequence is written for its N rows only: a buffer with a
+    # sentinel tail right after O keeps the sentinel
+    B, H, N, d = 1, 2, 200, 128
+    q, k, v = rand_qkv(B, H, N, d, "bf16", seed=801)
+    dev = torch.device("cuda")
+    n = B * H * N * d
+    buf = torch.full((n + 4096,), 3.0, dtype=torch.bfloat16, device=dev)
+    o = buf[:n].view(B, H, N, d)
+    sage.sage_attn_fwd(q.to(dev), k.to(dev), v.to(dev), out=o)
+    torch.cuda.synchronize()
+    assert torch.all(buf[n:] == 3.0)
+    check_against_oracle(to_numpy32(o), q, k, v, False, 1 / math.sqrt(d), "int8_fp8", "bf16")
+
+
 def test_fp4_zero_q_gives_mean_v(cuda_device):
     # Q = 0 -> every score 0 -> P~ = 1 -> s16 = 448, code e2m1(6) = 6, whose
     # value 6 * 448 / 2688 is exactly 1 -> O = mean of the FP4-dequantized V

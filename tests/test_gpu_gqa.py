@@ -35,6 +35,7 @@ CASES = [  # (B, H, Hkv, N, d)
     (1, 4, 1, 256, 128),     # multi-query
     (2, 6, 3, 256, 64),
     (1, 2, 2, 128, 64),      # Hkv == H: plain multi-head attention
+    (2, 4, 2, 333, 128),     # a ragged length
 ]
 
 

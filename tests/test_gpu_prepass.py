@@ -36,15 +36,20 @@ def check_int8(q, k, v, heads=None, mode="int8_fp8"):
     qk = sage.sage_quant_qk(q.to(dev), k.to(dev), mode)
     vq = sage.sage_quant_v(v.to(dev), mode)
     torch.cuda.synchronize()
-    nt = N // 128
-    codes = L.u8 if mode == "fp8" else L.int8_codes
+    nt = -(-N // 128)
+    codes = L.token_codes if mode == "fp8" else L.int8_codes
     g = dict(q_codes=codes(qk["q_codes"], B, H, N, d),
              q_scales=L.f32(qk["q_scales"], B, H, nt),
              k_codes=codes(qk["k_codes"], B, H, N, d),
              k_scales=L.f32(qk["k_scales"], B, H, nt),
              k_mean=L.f32(qk["k_mean"], B, H, d),
-             v_codes=L.u8(vq["v_codes"], B, H, d, N),
+             v_codes=L.vt_codes(vq["v_codes"], B, H, d, N),
              v_scales=L.f32(vq["v_scales"], B, H, d))
+    # the padding of a ragged sequence holds zero codes
+    Np = L.np_of(N)
+    assert not L.padded_tokens(qk["q_codes"], B, H, N).any()
+    assert not L.padded_tokens(qk["k_codes"], B, H, N).any()
+    assert not L._np(vq["v_codes"]).reshape(B, H, d, Np)[..., N:].any()
     heads = heads or [(b, h) for b in range(B) for h in range(H)]
     for (b, h) in heads:
         qs, ks, vs = (to_numpy32(t[b:b + 1, h:h + 1]) for t in (q, k, v))
@@ -64,17 +69,22 @@ def check_fp4(q, k, v, heads=None):
     qk = sage.sage_quant_qk(q.to(dev), k.to(dev), "fp4")
     vq = sage.sage_quant_v(v.to(dev), "fp4")
     torch.cuda.synchronize()
-    nt = N // 128
-    g = dict(q_codes=L.unpack_fp4(qk["q_codes"], B, H, N, d),
+    nt = -(-N // 128)
+    Np = L.np_of(N)
+    g = dict(q_codes=L.unpack_fp4(qk["q_codes"], B, H, Np, d)[:, :, :N],
              q_sf=L.qk_sf(qk["q_sf"], B, H, N, d),
              q_g=L.f32(qk["q_scales"], B, H, nt),
-             k_codes=L.unpack_fp4(qk["k_codes"], B, H, N, d),
+             k_codes=L.unpack_fp4(qk["k_codes"], B, H, Np, d)[:, :, :N],
              k_sf=L.qk_sf(qk["k_sf"], B, H, N, d),
              k_g=L.f32(qk["k_scales"], B, H, nt),
              k_mean=L.f32(qk["k_mean"], B, H, d),
-             v_codes=L.unpack_fp4(vq["v_codes"], B, H, d, N),
+             v_codes=L.unpack_fp4(vq["v_codes"], B, H, d, Np)[..., :N],
              v_sf=L.v_sf(vq["v_sf"], B, H, N, d),
              v_g=L.f32(vq["v_scales"], B, H, nt))
+    # the padding of a ragged sequence holds zero codes
+    assert not L.padded_tokens(qk["q_codes"], B, H, N).any()
+    assert not L.padded_tokens(qk["k_codes"], B, H, N).any()
+    assert not L.unpack_fp4(vq["v_codes"], B, H, d, Np)[..., N:].any()
     heads = heads or [(b, h) for b in range(B) for h in range(H)]
     for (b, h) in heads:
         qs, ks, vs = (to_numpy32(t[b:b + 1, h:h + 1]) for t in (q, k, v))
@@ -144,6 +154,17 @@ def test_fp8_qk_encoder_exhaustive(cuda_device):
     assert np.all(L.f32(qk["q_scales"], 1, 1, nblk) == 1.0)
     codes = L.u8(qk["q_codes"], 1, 1, nblk * 128, 64)[0, 0].reshape(nblk, 128, 64)
     assert np.array_equal(codes[:, 1:, :].reshape(-1)[:x.size], enc.e4m3_encode(x))
+
+
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp8", "fp4"])
+@pytest.mark.parametrize("N", [1, 77, 200, 300])
+def test_prepass_ragged(cuda_device, mode, N):
+    d = 128 if mode == "fp4" else 64
+    q, k, v = rand_qkv(2, 3, N, d, "bf16", seed=600 + N)
+    if mode == "fp4":
+        check_fp4(q, k, v)
+    else:
+        check_int8(q, k, v, mode=mode)
 
 
 def test_fp8_v_encoder_exhaustive(cuda_device):
