@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float* __restrict__ k_scales, const float* __restrict__ v_scales,
                     const uint8_t* __restrict__ q_sf, const uint8_t* __restrict__ k_sf,
                     const uint8_t* __restrict__ v_sf, OutT* __restrict__ out, int N, int H,
-                    int G, float scale_log2, uint32_t* status) {
+                    int G, float scale_log2, int head_major, uint32_t* status) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -496,11 +496,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = (N + 127) / 128;
   const int Np = ntiles * 128;
   const int n_tail = N - (ntiles - 1) * 128;
-  const int bh = blockIdx.y;
+  // grid order: see head_major_grid
+  const int bh = head_major ? (int)blockIdx.x : (int)blockIdx.y;
+  const int tile_rank = head_major ? (int)blockIdx.y : (int)blockIdx.x;
   // K/V head of this query head (grouped-query attention: G query heads per
   // K/V head; G = 1 is plain multi-head attention)
   const int bhk = kv_head(bh, H, G);
-  const int qt = CAUSAL ? (ntiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy first
+  const int qt = CAUSAL ? (ntiles - 1 - tile_rank) : tile_rank;  // heavy first
   const int nkv = CAUSAL ? qt + 1 : ntiles;
 
   Bars bar = carve_bars(smem);
@@ -693,12 +695,14 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((a.N + 127) / 128);
-  dim3 grid((unsigned)ntiles, (unsigned)(a.B * a.H));
+  const int hm = head_major_grid(a);
+  const dim3 grid = hm ? dim3((unsigned)(a.B * a.H), (unsigned)ntiles)
+                       : dim3((unsigned)ntiles, (unsigned)(a.B * a.H));
   kern<<<grid, kThreads, L::SMEM, st>>>(
       tq, tk, tv, a.q_scales, a.k_scales, a.v_scales, static_cast<const uint8_t*>(a.q_sf),
       static_cast<const uint8_t*>(a.k_sf), static_cast<const uint8_t*>(a.v_sf),
       reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H, (int)(a.H / a.Hkv), a.sm_scale * kLog2e,
-      a.status);
+      hm, a.status);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,14 @@ namespace sage {
 __device__ long long g_sage_trace[16][512];
 __shared__ long long s_sage_trace[16][64];
 #define SAGE_TRACED_CTA (blockIdx.x == 7 && blockIdx.y == 1)
+// per-CTA timeline: [start, first Q K^T issue, epilogue start, end] in
+// globaltimer ns, and the SM, for the first 16384 CTAs
+__device__ unsigned long long g_sage_cta[16384][5];
+#define SAGE_CTA_ID (blockIdx.y * gridDim.x + blockIdx.x)
+#define SAGE_CTA_TR(slot)                                                     \
+  do {                                                                        \
+    if (SAGE_CTA_ID < 16384) g_sage_cta[SAGE_CTA_ID][slot] = globaltimer();  \
+  } while (0)
 #define SAGE_TR(ev, j)                                                                  \
   do {                                                                                  \
     if (SAGE_TRACED_CTA && (j) < 64) {                                                  \
@@ -78,6 +86,9 @@ __shared__ long long s_sage_trace[16][64];
 #else
 #define SAGE_TR(ev, j) \
   do {                 \
+  } while (0)
+#define SAGE_CTA_TR(slot) \
+  do {                    \
   } while (0)
 #endif
 
@@ -111,7 +122,8 @@ struct Layout {
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
   static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots] dequant factor of the tile
-  static constexpr int END = OFF_C + 16;
+  static constexpr int OFF_VS = OFF_C + 128;         // s_V[D] of the head (bulk-copied with Q)
+  static constexpr int END = OFF_VS + 4 * D;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t QK_SBO = 8 * D;  // 8 rows of D bytes
@@ -484,7 +496,11 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
                   mbar_wait(bar.l_ready, 0, abort_flag, status, kDevTimeoutSoftmax)))
     return;
   const float inv_l = 1.f / (l_s[r] + l_s[128 + r]);
-  const float* vs = v_scales + (int64_t)kv_head(bh, H, G) * D;
+  // s_V arrived in shared memory with Q (q_full has long completed)
+  if (!__all_sync(0xffffffffu, mbar_wait(bar.q_full, 0, abort_flag, status, kDevTimeoutEpi)))
+    return;
+  const float* vs = reinterpret_cast<const float*>(smem + L::OFF_VS);
+  if (r == 0) SAGE_CTA_TR(2);
   // rows past the end of a ragged sequence are padding: not stored
   if (qt * 128 + r >= N) return;
   OutT* dst = out + ((int64_t)bh * N + (int64_t)qt * 128 + r) * D;
@@ -494,7 +510,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 v = o2[cv / 2 + e];
-      w4[e] = pack2<OutT>(v.x * __ldg(vs + cv + 2 * e) * inv_l, v.y * __ldg(vs + cv + 2 * e + 1) * inv_l);
+      w4[e] = pack2<OutT>(v.x * vs[cv + 2 * e] * inv_l, v.y * vs[cv + 2 * e + 1] * inv_l);
     }
     *reinterpret_cast<uint4*>(dst + cv) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
@@ -507,7 +523,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scales,
                      const float* __restrict__ k_scales, const float* __restrict__ v_scales,
                      OutT* __restrict__ out, int N, int H, int G, float scale_log2,
-                     uint32_t* status) {
+                     int head_major, uint32_t* status) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -519,13 +535,25 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
   const int ntiles = (N + 127) / 128;
   const int Np = ntiles * 128;
   const int n_tail = N - (ntiles - 1) * 128;
-  const int bh = blockIdx.y;
+  // head-major grids (x = head) dispatch every head's heaviest causal tile
+  // first: longest-first over the whole grid; tile-major grids (x = tile)
+  // keep the concurrently running CTAs on few heads (K/V reuse in L2)
+  const int bh = head_major ? (int)blockIdx.x : (int)blockIdx.y;
+  const int tile_rank = head_major ? (int)blockIdx.y : (int)blockIdx.x;
   // K/V head of this query head (grouped-query attention: G query heads per
   // K/V head; G = 1 is plain multi-head attention)
   const int bhk = kv_head(bh, H, G);
-  const int qt = CAUSAL ? (ntiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;  // heavy first
+  const int qt = CAUSAL ? (ntiles - 1 - tile_rank) : tile_rank;  // heavy first
   const int nkv = CAUSAL ? qt + 1 : ntiles;
 
+#ifdef SAGE_TRACE
+  if (threadIdx.x == 0) {
+    SAGE_CTA_TR(0);
+    unsigned smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    if (SAGE_CTA_ID < 16384) g_sage_cta[SAGE_CTA_ID][4] = smid;
+  }
+#endif
   Bars bar = carve_bars<D>(smem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_ABORT);
@@ -583,8 +611,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (elect_one()) {
-        mbar_arrive_expect_tx(bar.q_full, L::Q_BYTES);
+        mbar_arrive_expect_tx(bar.q_full, L::Q_BYTES + 4 * D);
         tma_load_2d(sQ, &tm_q, 0, bh * Np + qt * 128, bar.q_full);
+        bulk_load(smem + L::OFF_VS, v_scales + (int64_t)bhk * D, 4 * D, bar.q_full);
         for (int j = 0; j < nkv; ++j) {
           const int sk = j % L::KS;
           if (!mbar_wait<true>(&bar.k_empty[sk], ((j / L::KS) & 1) ^ 1, abort_flag, status,
@@ -617,6 +646,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
             return false;
           tc_fence_after();
           SAGE_TR(8, j);
+          if (j == 0) SAGE_CTA_TR(1);
           const uint64_t kdesc =
               make_sdesc(smem_u32(sK + sk * L::K_BYTES), L::QK_SBO, 16, L::QK_SWZ);
 #pragma unroll
@@ -703,6 +733,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) SAGE_CTA_TR(3);
 #ifdef SAGE_TRACE
   if (SAGE_TRACED_CTA && threadIdx.x < 64)
     for (int e = 0; e < 16; ++e) g_sage_trace[e][threadIdx.x] = s_sage_trace[e][threadIdx.x];
@@ -717,10 +748,13 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((a.N + 127) / 128);
-  dim3 grid((unsigned)ntiles, (unsigned)(a.B * a.H));
+  const int hm = head_major_grid(a);
+  const dim3 grid = hm ? dim3((unsigned)(a.B * a.H), (unsigned)ntiles)
+                       : dim3((unsigned)ntiles, (unsigned)(a.B * a.H));
   kern<<<grid, kThreadsAttn, L::SMEM, st>>>(tq, tk, tv, a.q_scales, a.k_scales, a.v_scales,
                                            reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H,
-                                           (int)(a.H / a.Hkv), a.sm_scale * kLog2e, a.status);
+                                           (int)(a.H / a.Hkv), a.sm_scale * kLog2e, hm,
+                                           a.status);
   return cudaGetLastError();
 }
 
@@ -766,5 +800,8 @@ cudaError_t launch_attn_i8f8(const AttnArgs& a, cudaStream_t st, const char** de
 #ifdef SAGE_TRACE
 extern "C" int sage_trace_read(long long* host) {
   return (int)cudaMemcpyFromSymbol(host, sage::g_sage_trace, sizeof(long long) * 16 * 512);
+}
+extern "C" int sage_trace_read_cta(unsigned long long* host) {
+  return (int)cudaMemcpyFromSymbol(host, sage::g_sage_cta, sizeof(unsigned long long) * 16384 * 5);
 }
 #endif

@@ -70,7 +70,7 @@ struct AttnArgs {
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st);
-// Q, K and V together (the pre-pass of sage_attn_fwd): three launches.
+// Q, K and V together (the pre-pass of sage_attn_fwd): two launches.
 cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st);
 
 // Returns cudaSuccess, or an error; `detail` receives a message on failure
@@ -82,6 +82,20 @@ cudaError_t launch_attn_fp4(const AttnArgs& a, cudaStream_t st, const char** det
 // bh = b * H + h, with G query heads per key/value head (G = 1: multi-head).
 __host__ __device__ __forceinline__ int kv_head(int bh, int H, int G) {
   return (bh / H) * (H / G) + (bh % H) / G;
+}
+
+// Grid order of the attention kernels.  Causal query tiles differ in work
+// (tile t sees t + 1 key tiles); CTAs start in grid order, so a head-major
+// grid (every head's heaviest tile first) runs longest-first over the whole
+// launch, which keeps the tail short.  It also spreads the running CTAs over
+// all heads, so it is used only while every head's K and V codes fit in L2
+// together (at most 64 MB); otherwise the grid stays tile-major, where the
+// running CTAs share the K/V tiles of a few heads.
+inline int head_major_grid(const AttnArgs& a) {
+  if (!a.causal) return 0;
+  const int64_t np = (a.N + 127) / 128 * 128;
+  const int64_t kv_bytes = 2 * a.B * a.Hkv * np * a.d;  // 8-bit K and V codes
+  return kv_bytes <= (int64_t(64) << 20) ? 1 : 0;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (the
