@@ -15,7 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsage_b200.so")
-SOURCES = ["api.cu", "quant.cu", "attn_i8f8.cu", "attn_fp4.cu"]
+SOURCES = ["api.cu", "quant.cu", "attn_i8f8.cu", "attn_i8f8_persist.cu", "attn_fp4.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-cudart", "static",
          "--expt-relaxed-constexpr"]

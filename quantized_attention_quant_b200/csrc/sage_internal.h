@@ -98,10 +98,29 @@ inline int head_major_grid(const AttnArgs& a) {
   return kv_bytes <= (int64_t(64) << 20) ? 1 : 0;
 }
 
+// The INT8/FP8 attention runs as a persistent kernel (one CTA per SM
+// working through a list of (query tile, b*h) items) when the items are
+// short: a CTA's start-up and epilogue then cost as much as a few key tiles,
+// and the persistent kernel overlaps them with the next item.  Long items
+// keep one CTA each, which the hardware balances itself.
+int sm_count();
+inline bool use_persistent_attention(const AttnArgs& a) {
+  const int64_t ntiles = (a.N + 127) / 128;
+  const int64_t mean_tiles = a.causal ? (ntiles + 1) / 2 : ntiles;
+  return mean_tiles <= 64 && ntiles * a.B * a.H > sm_count();
+}
+cudaError_t launch_attn_i8f8_persist(const AttnArgs& a, cudaStream_t st, const char** detail);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (the
 // library does not link libcuda).  Returns false with a message on failure.
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t dim0,
                     uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
                     CUtensorMapSwizzle swz, const char** detail);
+// The same for a 3-D tensor (box depth 1 in dimension 2).
+bool encode_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t dim0,
+                    uint64_t dim1, uint64_t dim2, uint64_t stride1_bytes, uint64_t stride2_bytes,
+                    uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz, const char** detail);
+// Streaming multiprocessors of the current device (cached per device):
+// declared above.
 
 }  // namespace sage

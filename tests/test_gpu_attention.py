@@ -260,3 +260,28 @@ def test_bounded_wait_expires_and_context_survives(cuda_device):
     torch.cuda.synchronize()
     check_against_oracle(to_numpy32(o), q, k, v, True, 1 / math.sqrt(128), "int8_fp8", "bf16")
     assert sage.device_status() == 0
+
+
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp8"])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("N,d", [(512, 128), (300, 64), (1000, 128)])
+def test_persistent_kernel_matches_one_item_per_cta(cuda_device, mode, causal, N, d):
+    """Many short work items run on the persistent INT8/FP8 kernel (one CTA
+    per SM working through a list of (query tile, head) items); a launch
+    with few items runs one CTA per item.  Both compute the same arithmetic
+    in the same order, so the heads they share must agree bit for bit; the
+    large launch is also held to the oracle on sampled heads."""
+    H = 80                                   # 80 heads x >= 3 tiles > 148 items
+    q, k, v = rand_qkv(1, H, N, d, "bf16", seed=900 + N + d + causal)
+    dev = torch.device("cuda")
+    big = sage.sage_attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=causal, mode=mode)
+    sub = [0, 37, 79]
+    small = sage.sage_attn_fwd(q[:, sub].contiguous().to(dev), k[:, sub].contiguous().to(dev),
+                               v[:, sub].contiguous().to(dev), causal=causal, mode=mode)
+    torch.cuda.synchronize()
+    assert sage.device_status() == 0
+    assert torch.equal(big[:, sub], small)
+    for h in (0, 79):
+        sel = (slice(0, 1), slice(h, h + 1))
+        check_against_oracle(to_numpy32(big[sel]), q[sel], k[sel], v[sel], causal,
+                             1 / math.sqrt(d), mode, "bf16")

@@ -90,3 +90,18 @@ def test_gqa_rejects_bad_head_counts(cuda_device):
     dev = torch.device("cuda")
     with pytest.raises(sage.SageError, match="Hkv"):
         sage.sage_attn_fwd_gqa(q.to(dev), k.to(dev), v.to(dev))
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_gqa_persistent_kernel(cuda_device, causal):
+    """Enough short items for the persistent INT8/FP8 kernel: GQA still
+    equals the multi-head pass on repeated K/V bit for bit."""
+    B, H, Hkv, N, d = 2, 48, 12, 384, 128
+    q, k, v = gqa_inputs(B, H, Hkv, N, d, "bf16", seed=77 + causal)
+    dev = torch.device("cuda")
+    qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
+    o = sage.sage_attn_fwd_gqa(qg, kg, vg, causal=causal)
+    o_rep = sage.sage_attn_fwd(qg, repeat_heads(kg, 4), repeat_heads(vg, 4), causal=causal)
+    torch.cuda.synchronize()
+    assert sage.device_status() == 0
+    assert torch.equal(o, o_rep)
