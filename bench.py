@@ -192,11 +192,12 @@ def run_sage(args):
             raise RuntimeError(lib.sage_status_string(s).decode())
 
     def step(ev_attn=None):
-        check(lib.sage_quant_qk(q.data_ptr(), k.data_ptr(), dt, B, H, N, d, mode,
-                                P["q_codes"], P["q_scales"], P["q_sf"], P["k_codes"],
-                                P["k_scales"], P["k_sf"], P["k_mean"], sptr))
-        check(lib.sage_quant_v(v.data_ptr(), dt, B, H, N, d, mode, P["v_codes"], P["v_scales"],
-                               P["v_sf"], sptr))
+        # both pre-passes (the V pass overlapped with the Q/K pass), then
+        # the attention kernel on the codes
+        check(lib.sage_quant_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), dt, B, H, N, d, mode,
+                                 P["q_codes"], P["q_scales"], P["q_sf"], P["k_codes"],
+                                 P["k_scales"], P["k_sf"], P["k_mean"], P["v_codes"],
+                                 P["v_scales"], P["v_sf"], sptr))
         if ev_attn:
             ev_attn[0].record(stream)
         check(lib.sage_attn_fwd_quantized(mode, P["q_codes"], P["q_scales"], P["q_sf"],
@@ -206,7 +207,7 @@ def run_sage(args):
         if ev_attn:
             ev_attn[1].record(stream)
 
-    # sage_quant_qk: 2 launches; sage_quant_v: 2 (FP8) or 1 (FP4); attention: 1
+    # sage_quant_qkv: 2 (Q/K) + 2 (V in FP8) or 1 (V in FP4); attention: 1
     launches_per_step = 2 + (1 if w.mode == "fp4" else 2) + 1
 
     uuid = None
@@ -297,7 +298,8 @@ def run_sage(args):
         "prepass_ms": round(t_step - t_attn, 4),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": "attn_i8f8_kernel" if w.mode != "fp4" else "attn_fp4_kernel",
+                     "kernel": attention_kernel(w, torch.cuda.get_device_properties(dev)
+                                                .multi_processor_count),
                      "peak_source": f"{src} bf16 burst x{ratio:g} (nominal dense ratio)",
                      "work": "4 d ops per visible (q,k) pair"},
         "e2e": {"value": round(e2e_val, 2), "unit": "TOPS",
@@ -312,6 +314,18 @@ def run_sage(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def attention_kernel(w, sms):
+    """The attention kernel the library runs for this workload: FP4, or
+    INT8/FP8 one CTA per (query tile, head), or INT8/FP8 persistent when the
+    items are short (the rule of use_persistent_attention in the library)."""
+    if w.mode == "fp4":
+        return "attn_fp4_kernel"
+    ntiles = -(-w.N // 128)
+    mean = (ntiles + 1) // 2 if w.causal else ntiles
+    return ("attn_i8f8_persist_kernel" if mean <= 64 and ntiles * w.B * w.H > sms
+            else "attn_i8f8_kernel")
 
 
 def read_traffic(workload):

@@ -128,6 +128,17 @@ int sage_quant_v(const void* v, int dtype,
                  int64_t B, int64_t H, int64_t N, int64_t d, int mode,
                  void* v_codes, float* v_scales, void* v_sf, sage_stream_t stream);
 
+/* The Q/K and V pre-passes in one call, with the arguments of both (Q, K
+ * and V share B, H, N, d).  The two are independent: the V pre-pass runs on
+ * a library-owned second stream, forked from `stream` and joined back to
+ * it with events (stream capture records the fork and the join), so the
+ * two overlap on the GPU.  Results are those of the two separate calls. */
+int sage_quant_qkv(const void* q, const void* k, const void* v, int dtype,
+                   int64_t B, int64_t H, int64_t N, int64_t d, int mode,
+                   void* q_codes, float* q_scales, void* q_sf,
+                   void* k_codes, float* k_scales, void* k_sf, float* k_mean,
+                   void* v_codes, float* v_scales, void* v_sf, sage_stream_t stream);
+
 /* Attention on already-quantized operands (the buffers written by the two
  * pre-pass calls); writes O [B, H, N, d] in `dtype`.  causal != 0 applies
  * the top-left-aligned causal mask (query t sees keys 0..t).  sm_scale is

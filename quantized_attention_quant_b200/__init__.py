@@ -10,6 +10,7 @@ Entry points (same names as the C ABI in include/sage.h):
 
     sage_quant_qk(q, k, mode="int8_fp8")      -> dict of code/scale tensors
     sage_quant_v(v, mode="int8_fp8")          -> dict of code/scale tensors
+    sage_quant_qkv(q, k, v, mode="int8_fp8")  -> (Q/K dict, V dict), the two overlapped
     sage_attn_fwd_quantized(qk, vq, mode, causal, sm_scale, out_dtype) -> O
     sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8") -> O
     sage_attn_fwd_gqa(q, k, v, ...)           -> O  (K/V with fewer heads than Q)
@@ -19,7 +20,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["sage_quant_qk", "sage_quant_v", "sage_attn_fwd", "sage_attn_fwd_gqa",
+__all__ = ["sage_quant_qk", "sage_quant_v", "sage_quant_qkv", "sage_attn_fwd", "sage_attn_fwd_gqa",
            "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
            "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS",
            "selftest_bounded_wait"]
@@ -34,7 +35,8 @@ BUF = {name: i for i, name in enumerate(
      "v_codes", "v_scales", "v_sf"])}
 
 # every symbol include/sage.h declares
-EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd_quantized",
+EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv",
+           "sage_attn_fwd_quantized",
            "sage_attn_fwd", "sage_attn_fwd_gqa", "sage_attn_fwd_noalloc",
            "sage_get_last_device_status",
            "sage_selftest_bounded_wait", "sage_status_string", "sage_version"]
@@ -66,6 +68,9 @@ def library():
                                   vp, fp, vp, vp, fp, vp, fp, vp]
     lib.sage_quant_v.restype = i32
     lib.sage_quant_v.argtypes = [vp, i32, i64, i64, i64, i64, i32, vp, fp, vp, vp]
+    lib.sage_quant_qkv.restype = i32
+    lib.sage_quant_qkv.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i32,
+                                   vp, fp, vp, vp, fp, vp, fp, vp, fp, vp, vp]
     lib.sage_attn_fwd_quantized.restype = i32
     lib.sage_attn_fwd_quantized.argtypes = [i32, vp, fp, vp, vp, fp, vp, vp, fp, vp, vp, i32,
                                             i64, i64, i64, i64, i32, ctypes.c_float, vp]
@@ -160,6 +165,25 @@ def sage_quant_v(v, mode="int8_fp8"):
         _ptr(v), _dtype_code(v), B, H, N, d, MODES[mode],
         _f(bufs["v_codes"]), _f(bufs["v_scales"]), _f(bufs["v_sf"]), _stream()))
     return bufs
+
+
+def sage_quant_qkv(q, k, v, mode="int8_fp8"):
+    """Both pre-passes in one call (the V pass overlaps the Q/K pass on a
+    library stream).  Returns (qk, vq) as sage_quant_qk and sage_quant_v do."""
+    B, H, N, d = _shape(q)
+    if _shape(k) != (B, H, N, d) or _shape(v) != (B, H, N, d):
+        raise ValueError("q, k, v must have the same shape")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must have the same dtype")
+    qk = _alloc(mode, ["q_codes", "q_scales", "q_sf", "k_codes", "k_scales", "k_sf", "k_mean"],
+                B, H, N, d, q.device)
+    vq = _alloc(mode, ["v_codes", "v_scales", "v_sf"], B, H, N, d, v.device)
+    _check(library().sage_quant_qkv(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, H, N, d, MODES[mode],
+        _f(qk["q_codes"]), _f(qk["q_scales"]), _f(qk["q_sf"]),
+        _f(qk["k_codes"]), _f(qk["k_scales"]), _f(qk["k_sf"]), _f(qk["k_mean"]),
+        _f(vq["v_codes"]), _f(vq["v_scales"]), _f(vq["v_sf"]), _stream()))
+    return qk, vq
 
 
 def sage_attn_fwd_quantized(qk, vq, shape, mode="int8_fp8", causal=False, sm_scale=None,

@@ -129,6 +129,60 @@ int workspace(cudaStream_t st, size_t need, void** out, uint32_t** counters) {
   return SAGE_OK;
 }
 
+// A second stream per device.  The pre-pass is two independent chains:
+// Q codes + K statistics then K codes, and V statistics then V codes; the
+// V chain runs on this stream, forked from and joined back to the caller's
+// stream by events (a pattern stream capture records as a fork and a join).
+// The two chains use disjoint parts of the workspace (K sums and counters
+// vs. V maxima and counters).
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;  // one fork/join at a time: the events are shared
+};
+std::map<int, SideStream*> g_side;
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  SideStream*& ss = g_side[dev];
+  if (!ss) {
+    auto* n = new SideStream;
+    if ((e = cudaStreamCreateWithFlags(&n->s, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&n->fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&n->join, cudaEventDisableTiming)) != cudaSuccess) {
+      delete n;
+      return fail_cuda(e, "side stream setup");
+    }
+    ss = n;
+  }
+  *out = ss;
+  return SAGE_OK;
+}
+
+// Q/K chain on st, V chain on the side stream; st continues after both.
+int prepass_forked(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st) {
+  SideStream* ss = nullptr;
+  const int got = side_stream(&ss);
+  if (got != SAGE_OK) return got;
+  std::lock_guard<std::mutex> lk(ss->mu);
+  cudaError_t e;
+  if ((e = cudaEventRecord(ss->fork, st)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess)
+    return fail_cuda(e, "pre-pass fork");
+  if ((e = launch_quant_v(va, ss->s)) != cudaSuccess) return fail_cuda(e, "quant_v launch");
+  if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess)
+    return fail_cuda(e, "pre-pass join");
+  // the caller's stream waits for the V chain even if the Q/K launch fails
+  const cudaError_t eq = launch_quant_qk(qa, st);
+  if ((e = cudaStreamWaitEvent(st, ss->join, 0)) != cudaSuccess)
+    return fail_cuda(e, "pre-pass join");
+  if (eq != cudaSuccess) return fail_cuda(eq, "quant_qk launch");
+  return SAGE_OK;
+}
+
 struct WorkspaceReleaser {
   ~WorkspaceReleaser() {
     // Best effort at unload; during process teardown the runtime may already
@@ -329,8 +383,8 @@ int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtyp
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax), cnt};
-  cudaError_t e = launch_prepass(qa, va, st);
-  if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
+  SAGE_TRY(prepass_forked(qa, va, st));
+  cudaError_t e = cudaSuccess;
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
@@ -431,6 +485,47 @@ int sage_quant_v(const void* v, int dtype, int64_t B, int64_t H, int64_t N, int6
   cudaError_t e = launch_quant_v(a, st);
   if (e != cudaSuccess) return fail_cuda(e, "quant_v launch");
   return SAGE_OK;
+}
+
+int sage_quant_qkv(const void* q, const void* k, const void* v, int dtype, int64_t B, int64_t H,
+                   int64_t N, int64_t d, int mode, void* q_codes, float* q_scales, void* q_sf,
+                   void* k_codes, float* k_scales, void* k_sf, float* k_mean, void* v_codes,
+                   float* v_scales, void* v_sf, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  SAGE_TRY(check_ptr(q, "q", true));
+  SAGE_TRY(check_ptr(k, "k", true));
+  SAGE_TRY(check_ptr(v, "v", true));
+  SAGE_TRY(check_ptr(q_codes, "q_codes", true));
+  SAGE_TRY(check_ptr(q_scales, "q_scales", true));
+  SAGE_TRY(check_ptr(k_codes, "k_codes", true));
+  SAGE_TRY(check_ptr(k_scales, "k_scales", true));
+  SAGE_TRY(check_ptr(k_mean, "k_mean", true));
+  SAGE_TRY(check_ptr(v_codes, "v_codes", true));
+  SAGE_TRY(check_ptr(v_scales, "v_scales", true));
+  if (mode == SAGE_MODE_FP4) {
+    SAGE_TRY(check_ptr(q_sf, "q_sf", true));
+    SAGE_TRY(check_ptr(k_sf, "k_sf", true));
+    SAGE_TRY(check_ptr(v_sf, "v_sf", true));
+  } else {
+    SAGE_TRY(check_unused(q_sf, "q_sf"));
+    SAGE_TRY(check_unused(k_sf, "k_sf"));
+    SAGE_TRY(check_unused(v_sf, "v_sf"));
+  }
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  uint32_t* cnt = nullptr;
+  const size_t ks = align_up(ws_ksum_bytes(B * H, N, d));
+  SAGE_TRY(workspace(st, ks + ws_vmax_bytes(B * H, N, d), &ws, &cnt));
+  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d, H, q_codes, q_scales, q_sf,
+                 k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws), cnt};
+  QuantVArgs va{v, dtype, mode, B, H, N, d, v_codes, v_scales, v_sf,
+                static_cast<double*>(ws), reinterpret_cast<float*>(static_cast<char*>(ws) + ks),
+                cnt};
+  return prepass_forked(qa, va, st);
 }
 
 int sage_attn_fwd_quantized(int mode, const void* q_codes, const float* q_scales, const void* q_sf,
@@ -634,8 +729,8 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax), cnt};
-  cudaError_t e = launch_prepass(qa, va, st);
-  if (e != cudaSuccess) return fail_cuda(e, "pre-pass launch");
+  SAGE_TRY(prepass_forked(qa, va, st));
+  cudaError_t e = cudaSuccess;
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),

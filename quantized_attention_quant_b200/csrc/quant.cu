@@ -808,20 +808,5 @@ cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st) {
                                     Roles{0, {}}, st);
 }
 
-cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st) {
-  PrepassPtrs p = ptrs_qk(qa);
-  add_v(p, va);
-  if (qa.mode == kModeInt8Fp8)
-    return dispatch<bit(kQuantQ8) | bit(kStatsKV), bit(kQuantK8) | bit(kQuantV8)>(
-        p, qa.dtype, qa.d, Roles{2, {kQuantQ8, kStatsKV}},
-        Roles{2, {kQuantK8, kQuantV8}}, st);
-  if (qa.mode == kModeFp8)
-    return dispatch<bit(kQuantQF8) | bit(kStatsKV), bit(kQuantKF8) | bit(kQuantV8)>(
-        p, qa.dtype, qa.d, Roles{2, {kQuantQF8, kStatsKV}},
-        Roles{2, {kQuantKF8, kQuantV8}}, st);
-  return dispatch<bit(kQuantQ4) | bit(kQuantV4) | bit(kStatsK), bit(kQuantK4)>(
-      p, qa.dtype, qa.d, Roles{3, {kQuantQ4, kQuantV4, kStatsK}},
-      Roles{1, {kQuantK4}}, st);
-}
 
 }  // namespace sage

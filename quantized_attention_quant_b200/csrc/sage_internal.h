@@ -70,8 +70,6 @@ struct AttnArgs {
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st);
-// Q, K and V together (the pre-pass of sage_attn_fwd): two launches.
-cudaError_t launch_prepass(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st);
 
 // Returns cudaSuccess, or an error; `detail` receives a message on failure
 // of something other than a CUDA call (e.g. tensor-map encoding).

@@ -285,3 +285,32 @@ def test_persistent_kernel_matches_one_item_per_cta(cuda_device, mode, causal, N
         sel = (slice(0, 1), slice(h, h + 1))
         check_against_oracle(to_numpy32(big[sel]), q[sel], k[sel], v[sel], causal,
                              1 / math.sqrt(d), mode, "bf16")
+
+
+def test_cuda_graph_capture_and_replay(cuda_device):
+    # sage_attn_fwd inside a captured CUDA graph: the pre-pass fork/join to
+    # the library's second stream is recorded too; replays match eager runs
+    B, H, N, d = 1, 4, 640, 128
+    q, k, v = rand_qkv(B, H, N, d, "bf16", seed=1300)
+    dev = torch.device("cuda")
+    qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
+    out = torch.empty_like(qg)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        sage.sage_attn_fwd(qg, kg, vg, causal=True, out=out)   # warm-up: workspace, streams
+    s.synchronize()
+    eager = out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        sage.sage_attn_fwd(qg, kg, vg, causal=True, out=out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    qg.copy_(rand_qkv(B, H, N, d, "bf16", seed=1301)[0].to(dev))
+    g.replay()
+    torch.cuda.synchronize()
+    ref = sage.sage_attn_fwd(qg, kg, vg, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert sage.device_status() == 0

@@ -212,3 +212,18 @@ def test_prepass_full_workloads(cuda_device, name):
         check_fp4(q, k, v, heads)
     else:
         check_int8(q, k, v, heads)
+
+
+@pytest.mark.parametrize("mode,N,d", [("int8_fp8", 384, 128), ("fp8", 300, 64), ("fp4", 200, 128)])
+def test_quant_qkv_equals_separate_calls(cuda_device, mode, N, d):
+    # the V pre-pass forked onto the library's second stream gives the same
+    # bytes as the two separate calls
+    q, k, v = rand_qkv(2, 3, N, d, "bf16", seed=1200 + N)
+    dev = torch.device("cuda")
+    qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
+    qk1, vq1 = sage.sage_quant_qkv(qg, kg, vg, mode)
+    qk2 = sage.sage_quant_qk(qg, kg, mode)
+    vq2 = sage.sage_quant_v(vg, mode)
+    torch.cuda.synchronize()
+    for a, b in list(zip(qk1.values(), qk2.values())) + list(zip(vq1.values(), vq2.values())):
+        assert (a is None and b is None) or torch.equal(a, b)
