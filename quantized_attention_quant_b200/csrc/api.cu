@@ -163,7 +163,13 @@ int side_stream(SideStream** out) {
 }
 
 // Q/K chain on st, V chain on the side stream; st continues after both.
+// Sequences short enough for the cluster-fused pre-pass take one launch on st.
 int prepass_forked(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st) {
+  if (fused_prepass_fits(qa)) {
+    const cudaError_t e = launch_prepass_fused(qa, va, st);
+    if (e != cudaSuccess) return fail_cuda(e, "fused pre-pass launch");
+    return SAGE_OK;
+  }
   SideStream* ss = nullptr;
   const int got = side_stream(&ss);
   if (got != SAGE_OK) return got;
@@ -383,6 +389,7 @@ int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtyp
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax), cnt};
+  qa.status = di->status;
   SAGE_TRY(prepass_forked(qa, va, st));
   cudaError_t e = cudaSuccess;
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
@@ -525,6 +532,7 @@ int sage_quant_qkv(const void* q, const void* k, const void* v, int dtype, int64
   QuantVArgs va{v, dtype, mode, B, H, N, d, v_codes, v_scales, v_sf,
                 static_cast<double*>(ws), reinterpret_cast<float*>(static_cast<char*>(ws) + ks),
                 cnt};
+  qa.status = di->status;
   return prepass_forked(qa, va, st);
 }
 
@@ -729,6 +737,7 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                 at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax), cnt};
+  qa.status = di->status;
   SAGE_TRY(prepass_forked(qa, va, st));
   cudaError_t e = cudaSuccess;
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),

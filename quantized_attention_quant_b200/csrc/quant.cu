@@ -78,9 +78,11 @@ struct PrepassPtrs {
 
 constexpr int kMaxHeads = 65536;
 
-template <typename T>
+// Eight elements as FP32 from global memory (read-only path) or, SHARED,
+// from shared memory.
+template <typename T, bool SHARED = false>
 __device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
-  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  uint4 u = SHARED ? *reinterpret_cast<const uint4*>(p) : __ldg(reinterpret_cast<const uint4*>(p));
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -326,7 +328,9 @@ __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int
 // Two passes over the 128-token tile: the amax pass keeps nothing, the code
 // pass reads the tile again (from L1/L2), so the role needs few registers and
 // many CTAs fit on an SM.  A thread's vectors all cover the same 8 channels.
-template <typename T, int D, bool FP8, bool RAGGED>
+// SHARED: the tile and the mean are in shared memory (the cluster-fused
+// pre-pass), else in global memory.
+template <typename T, int D, bool FP8, bool RAGGED, bool SHARED = false>
 __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const float* mean,
                                                 uint8_t* __restrict__ dst, float* scale_out,
                                                 float* red, int nv) {
@@ -335,8 +339,10 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
   // x - mu as x + (-mu): the same single rounding
   float nmu[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (mean) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(mean + c0));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(mean + c0 + 4));
+    const float4 a = SHARED ? *reinterpret_cast<const float4*>(mean + c0)
+                            : __ldg(reinterpret_cast<const float4*>(mean + c0));
+    const float4 b = SHARED ? *reinterpret_cast<const float4*>(mean + c0 + 4)
+                            : __ldg(reinterpret_cast<const float4*>(mean + c0 + 4));
     nmu[0] = -a.x; nmu[1] = -a.y; nmu[2] = -a.z; nmu[3] = -a.w;
     nmu[4] = -b.x; nmu[5] = -b.y; nmu[6] = -b.z; nmu[7] = -b.w;
   }
@@ -358,7 +364,7 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
     // a padding vector re-reads a real one: it changes no maximum
     const int vec = threadIdx.x + i * kThreads;
     float x[8];
-    load8(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
+    load8<T, SHARED>(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
     smooth(x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
@@ -372,7 +378,7 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
     uint2 w = make_uint2(0u, 0u);
     if (s != 0.f) {
       float x[8];
-      load8(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
+      load8<T, SHARED>(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
       smooth(x);
       w = FP8 ? fp8_codes8(x, s, rs) : int8_codes8(x, s, rs);
     }
@@ -391,21 +397,17 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
 // through one e4m3x2 conversion each, and the two 16-bit results must match
 // (else the unit is redone on IEEE quotients); the matching result is the
 // two codes, already packed.
-template <typename T, int D, bool RAGGED>
-__device__ __forceinline__ void role_quant_v_fp8(const T* __restrict__ src,
-                                                 const float* __restrict__ vs,
-                                                 uint8_t* __restrict__ dst, int N, T* tile,
-                                                 int nv) {
-  // padding tokens stage as zeros and so get code 0; N is the row length of
-  // V^T (the padded token count)
-  stage_tile<T, D, RAGGED>(src, tile, nv);
-  __syncthreads();
+// The encoding of one staged tile (shared memory, padding tokens zero); vs:
+// the head's s_V (global or shared memory).
+template <typename T, int D>
+__device__ __forceinline__ void encode_v_fp8_tile(const T* tile, const float* vs,
+                                                  uint8_t* __restrict__ dst, int N) {
   constexpr int UNITS = (D / 2) * 4;  // channel pairs x 32-token groups
   const float2 lo2 = make_float2(kBracketLo, kBracketLo);
   const float2 hi2 = make_float2(kBracketHi, kBracketHi);
   for (int u = threadIdx.x; u < UNITS; u += kThreads) {
     const int cp = u % (D / 2), grp = u / (D / 2);
-    const float s0 = __ldg(vs + 2 * cp), s1 = __ldg(vs + 2 * cp + 1);
+    const float s0 = vs[2 * cp], s1 = vs[2 * cp + 1];
     const float r0 = recip_or_zero(s0), r1 = recip_or_zero(s1);
     const uint32_t* col = reinterpret_cast<const uint32_t*>(tile) + (grp * 32) * (D / 2) + cp;
     auto pair_of = [&](int tok, float& x0, float& x1) {
@@ -468,6 +470,18 @@ __device__ __forceinline__ void role_quant_v_fp8(const T* __restrict__ src,
       *reinterpret_cast<uint4*>(d1 + 16 * half) = v1;
     }
   }
+}
+
+template <typename T, int D, bool RAGGED>
+__device__ __forceinline__ void role_quant_v_fp8(const T* __restrict__ src,
+                                                 const float* __restrict__ vs,
+                                                 uint8_t* __restrict__ dst, int N, T* tile,
+                                                 int nv) {
+  // padding tokens stage as zeros and so get code 0; N is the row length of
+  // V^T (the padded token count)
+  stage_tile<T, D, RAGGED>(src, tile, nv);
+  __syncthreads();
+  encode_v_fp8_tile<T, D>(tile, vs, dst, N);
 }
 
 // -------------------------------------------------------------------- FP4
@@ -721,6 +735,140 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
 }
 #undef SAGE_ROLE
 
+// ------------------------------------------------ the cluster-fused pre-pass
+// For the 8-bit modes and heads of at most 8 tiles (1024 tokens), where the
+// two-launch chains are bound by launch latency: one launch encodes Q, K and
+// V.  A cluster of 8 CTAs per (b*h, tensor) holds the head's tiles in shared
+// memory, one tile per CTA (one bulk copy each), and reduces the head
+// statistics through distributed shared memory in the order the two-launch
+// path uses (FP64 K sums per tile in token order, then tiles in order; the
+// |V| maximum), so the codes are the same bits; each input is read once.
+// grid (8, max(B*Hq, B*Hkv), 3): z = 0 Q codes, 1 K mean + K codes, 2 V scales
+// + V codes; a cluster spans x only, so all its CTAs share (b*h, tensor).
+constexpr int kFusedCluster = 8;
+
+template <typename T, int D, bool FP8, bool RAGGED>
+__global__ void __cluster_dims__(kFusedCluster, 1, 1) __launch_bounds__(kThreads)
+    prepass_fused_kernel(PrepassPtrs p, uint32_t* status) {
+  __shared__ __align__(128) T tile[128 * D];
+  __shared__ uint64_t bar;
+  __shared__ double ksum_s[D];
+  __shared__ uint32_t vmax_s[D];
+  __shared__ __align__(16) float stat_s[D];  // the head's K mean or s_V
+  __shared__ float red[kThreads / 32];
+  __shared__ int abort_flag;
+  const int role = blockIdx.z;
+  const int64_t bh = blockIdx.y;
+  // whole clusters leave here (before any cluster barrier)
+  if (bh >= (role == 0 ? p.bh_q : p.bh_kv)) return;
+  const int t = threadIdx.x;
+  const int g = (int)cluster_ctarank();  // this CTA's tile
+  const int Np = RAGGED ? p.Np : p.N;
+  const int ntiles = Np / 128;
+  const bool has = g < ntiles;
+  const int nv = RAGGED ? min(128, p.N - g * 128) : 128;  // its real tokens (when has)
+  const T* src = reinterpret_cast<const T*>(role == 0 ? p.q : role == 1 ? p.k : p.v) +
+                 (bh * p.N + (int64_t)g * 128) * D;
+
+  if (t == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (t < D) vmax_s[t] = 0u;
+  __syncthreads();
+  if (t == 0 && has) {
+    const uint32_t bytes = (uint32_t)(nv * D * (int)sizeof(T));
+    mbar_arrive_expect_tx(&bar, bytes);
+    bulk_load(tile, src, bytes, &bar);
+  }
+  // padding tokens of a partial last tile stage as zeros (V codes read them)
+  if (RAGGED && has && nv < 128) {
+    uint4* pad = reinterpret_cast<uint4*>(tile + nv * D);
+    for (int i = t; i < (128 - nv) * D / 8; i += kThreads) pad[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  // every thread observes the copy's completion before it reads the tile
+  if (has) mbar_wait(&bar, 0, &abort_flag, status, kDevTimeoutTma);
+
+  if (role == 0) {
+    if (has)
+      role_quant_8bit<T, D, FP8, RAGGED, true>(
+          tile, nullptr, reinterpret_cast<uint8_t*>(p.q_codes) + (bh * Np + g * 128) * D,
+          p.q_scales + bh * ntiles + g, red, nv);
+  } else if (role == 1) {
+    // FP64 sum of the tile's tokens in order, channel t
+    if (has && t < D) {
+      double acc = 0.0;
+#pragma unroll 16
+      for (int k = 0; k < nv; ++k) acc += (double)static_cast<float>(tile[k * D + t]);
+      ksum_s[t] = acc;
+    }
+    cluster_sync();
+    if (t < D) {
+      // every CTA folds the tiles of the head in tile order: the same mean
+      double part[kFusedCluster];
+#pragma unroll
+      for (int r = 0; r < kFusedCluster; ++r)
+        part[r] = r < ntiles ? ld_dsmem_f64(dsmem_addr(&ksum_s[t], (uint32_t)r)) : 0.0;
+      double acc = 0.0;
+#pragma unroll
+      for (int r = 0; r < kFusedCluster; ++r)
+        if (r < ntiles) acc += part[r];
+      const float mean = __double2float_rn(__ddiv_rn(acc, (double)p.N));
+      stat_s[t] = mean;
+      if (g == 0) p.k_mean[bh * D + t] = mean;
+    }
+    // no CTA leaves while others read its partials
+    cluster_sync();
+    if (has)
+      role_quant_8bit<T, D, FP8, RAGGED, true>(
+          tile, stat_s, reinterpret_cast<uint8_t*>(p.k_codes) + (bh * Np + g * 128) * D,
+          p.k_scales + bh * ntiles + g, red, nv);
+  } else {
+    if (has) {
+      // |V| maximum per channel (a thread keeps 8 channels; a padding token
+      // re-reads a real one, so no maximum changes)
+      constexpr int VPT = 128 * D / 8 / kThreads;
+      const int c0 = (t % (D / 8)) * 8;
+      float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) {
+        float x[8];
+        load8<T, true>(tile + clamp_vec<D, RAGGED>(t + j * kThreads, nv) * 8, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(x[e]));
+      }
+      // non-negative floats order like their bit patterns
+#pragma unroll
+      for (int e = 0; e < 8; ++e) atomicMax(vmax_s + c0 + e, __float_as_uint(m[e]));
+    }
+    cluster_sync();
+    if (t < D) {
+      uint32_t mb[kFusedCluster];
+#pragma unroll
+      for (int r = 0; r < kFusedCluster; ++r) mb[r] = ld_dsmem_u32(dsmem_addr(&vmax_s[t], (uint32_t)r));
+      float mx = 0.f;
+#pragma unroll
+      for (int r = 0; r < kFusedCluster; ++r) mx = fmaxf(mx, __uint_as_float(mb[r]));
+      const float sv = __fdiv_rn(mx, 448.f);  // s_V = fp32(amax / 448)
+      stat_s[t] = sv;
+      if (g == 0) p.v_scales[bh * D + t] = sv;
+    }
+    cluster_sync();
+    if (has)
+      encode_v_fp8_tile<T, D>(tile, stat_s,
+                              reinterpret_cast<uint8_t*>(p.v_codes) + bh * D * (int64_t)Np +
+                                  (int64_t)g * 128,
+                              Np);
+  }
+  // after an expired wait, let the copy land before the CTA leaves
+  __syncthreads();
+  if (t == 0 && has && abort_flag) {
+    volatile int no_abort = 0;
+    mbar_wait(&bar, 0, &no_abort, status, kDevTimeoutTma);
+  }
+}
+
 constexpr int bit(int r) { return 1 << r; }
 
 // kernel A (roles a; its statistics CTAs also fold the head statistics),
@@ -784,7 +932,44 @@ void add_v(PrepassPtrs& p, const QuantVArgs& a) {
   p.bh_kv = a.B * a.H;  // QuantVArgs counts K/V heads in H
 }
 
+template <typename T, int D, bool FP8>
+cudaError_t run_fused(const PrepassPtrs& p, uint32_t* status, cudaStream_t st) {
+  const int64_t BH = p.bh_q > p.bh_kv ? p.bh_q : p.bh_kv;
+  const dim3 grid(kFusedCluster, (unsigned)BH, 3);
+  if (p.N % 128 != 0)
+    prepass_fused_kernel<T, D, FP8, true><<<grid, kThreads, 0, st>>>(p, status);
+  else
+    prepass_fused_kernel<T, D, FP8, false><<<grid, kThreads, 0, st>>>(p, status);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+bool fused_prepass_fits(const QuantQKArgs& a) {
+  const int64_t ntiles = (a.N + 127) / 128;
+  const int64_t BH = a.B * a.H;
+  return a.mode != kModeFp4 && a.status != nullptr && ntiles > 0 &&
+         ntiles <= kFusedCluster && BH <= 65535 &&
+         (a.d == 64 || a.d == 128);
+}
+
+cudaError_t launch_prepass_fused(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st) {
+  PrepassPtrs p = ptrs_qk(qa);
+  add_v(p, va);
+  const bool fp8 = qa.mode == kModeFp8;
+  if (qa.dtype == 1) {
+    if (qa.d == 128)
+      return fp8 ? run_fused<__nv_bfloat16, 128, true>(p, qa.status, st)
+                 : run_fused<__nv_bfloat16, 128, false>(p, qa.status, st);
+    return fp8 ? run_fused<__nv_bfloat16, 64, true>(p, qa.status, st)
+               : run_fused<__nv_bfloat16, 64, false>(p, qa.status, st);
+  }
+  if (qa.d == 128)
+    return fp8 ? run_fused<__half, 128, true>(p, qa.status, st)
+               : run_fused<__half, 128, false>(p, qa.status, st);
+  return fp8 ? run_fused<__half, 64, true>(p, qa.status, st)
+             : run_fused<__half, 64, false>(p, qa.status, st);
+}
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
   const PrepassPtrs p = ptrs_qk(a);

@@ -30,6 +30,7 @@ struct QuantQKArgs {
   double* ws_ksum;  // [B*H, N/128, d] FP64 chunk partial sums (workspace)
   uint32_t* ws_cnt;  // [2][65536] per-head statistics counters: zero before the
                      // call, zero again after it (workspace)
+  uint32_t* status = nullptr;  // device status word (bounded waits of the fused pre-pass)
 };
 
 struct QuantVArgs {
@@ -70,6 +71,10 @@ struct AttnArgs {
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st);
 cudaError_t launch_quant_v(const QuantVArgs& a, cudaStream_t st);
+// The whole 8-bit pre-pass (Q, K and V) in one cluster launch, for sequences
+// whose K / V head slices fit in one cluster's shared memory.
+bool fused_prepass_fits(const QuantQKArgs& a);
+cudaError_t launch_prepass_fused(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st);
 
 // Returns cudaSuccess, or an error; `detail` receives a message on failure
 // of something other than a CUDA call (e.g. tensor-map encoding).

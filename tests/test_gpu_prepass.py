@@ -28,13 +28,18 @@ def rand_qkv(B, H, N, d, dtype, seed, k_bias=3.0):
     return [torch.from_numpy(x).to(TDT[dtype]) for x in (q, k, v)]
 
 
-def check_int8(q, k, v, heads=None, mode="int8_fp8"):
+def check_int8(q, k, v, heads=None, mode="int8_fp8", fused=False):
     """Run the INT8/FP8 (or FP8 Q/K) pre-pass on the GPU; compare (sampled)
-    heads."""
+    heads.  fused: through sage_quant_qkv (one call for Q, K and V, the
+    cluster-fused kernel where the sequence fits in it), else through the
+    separate Q/K and V calls (two launches each)."""
     B, H, N, d = q.shape
     dev = torch.device("cuda")
-    qk = sage.sage_quant_qk(q.to(dev), k.to(dev), mode)
-    vq = sage.sage_quant_v(v.to(dev), mode)
+    if fused:
+        qk, vq = sage.sage_quant_qkv(q.to(dev), k.to(dev), v.to(dev), mode)
+    else:
+        qk = sage.sage_quant_qk(q.to(dev), k.to(dev), mode)
+        vq = sage.sage_quant_v(v.to(dev), mode)
     torch.cuda.synchronize()
     nt = -(-N // 128)
     codes = L.token_codes if mode == "fp8" else L.int8_codes
@@ -214,10 +219,29 @@ def test_prepass_full_workloads(cuda_device, name):
         check_int8(q, k, v, heads)
 
 
-@pytest.mark.parametrize("mode,N,d", [("int8_fp8", 384, 128), ("fp8", 300, 64), ("fp4", 200, 128)])
+# (N, d): through the cluster-fused kernel (8 CTAs, one tile each): one
+# token (seven CTAs without a tile), a partial tile, a partial eighth tile,
+# eight whole tiles; past it (two-launch chains on two streams): one token
+# more, and the llm length
+FUSED_SIZES = [(1, 64), (77, 128), (1000, 64), (1024, 128), (1025, 64), (4096, 128)]
+
+
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp8"])
+@pytest.mark.parametrize("N,d", FUSED_SIZES)
+def test_quant_qkv_matches_oracle(cuda_device, mode, N, d):
+    """sage_quant_qkv (the path sage_attn_fwd takes) is bit-identical to the
+    oracle on every head."""
+    q, k, v = rand_qkv(1, 3, N, d, "bf16" if d == 128 else "f16", seed=1400 + N + d)
+    check_int8(q, k, v, mode=mode, fused=True)
+
+
+@pytest.mark.parametrize("mode,N,d", [("int8_fp8", 384, 128), ("fp8", 300, 64), ("fp4", 200, 128),
+                                      ("int8_fp8", 1024, 128), ("fp8", 1000, 64),
+                                      ("int8_fp8", 1025, 128)])
 def test_quant_qkv_equals_separate_calls(cuda_device, mode, N, d):
-    # the V pre-pass forked onto the library's second stream gives the same
-    # bytes as the two separate calls
+    # sage_quant_qkv (the cluster-fused kernel, or past its size the V chain
+    # forked onto the library's second stream) gives the same bytes as the
+    # two separate calls
     q, k, v = rand_qkv(2, 3, N, d, "bf16", seed=1200 + N)
     dev = torch.device("cuda")
     qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
