@@ -208,9 +208,9 @@ def run_sage(args):
             ev_attn[1].record(stream)
 
     # sage_quant_qkv: one cluster-fused launch in the 8-bit modes up to 8
-    # tiles (1024 tokens) per head, else 2 (Q/K) + 2 (V in FP8) or 1 (V in
-    # FP4); attention: 1
-    if w.mode != "fp4" and -(-N // 128) <= 8:
+    # tiles (1024 tokens) per head and 16 heads, else 2 (Q/K) + 2 (V in FP8)
+    # or 1 (V in FP4); attention: 1
+    if w.mode != "fp4" and -(-N // 128) <= 8 and B * H <= 16:
         launches_per_step = 1 + 1
     else:
         launches_per_step = 2 + (1 if w.mode == "fp4" else 2) + 1

@@ -15,6 +15,7 @@ Distributions (normal laws written N(0, sigma); the K bias is one value per
   llm    Q, K ~ N(0,1) with 4 random channels per head scaled by 20 in both
          Q and K (the same channel set for Q and K of a head);
          bias ~ N(0,2); V ~ N(0,1)
+  short  as llm (a batch of 1024-token sequences)
   video  Q, K, V ~ N(0,1); bias ~ N(0,4)
   long   Q, K, V ~ Student-t(nu=4) / sqrt(2) (unit variance); bias ~ N(0,2)
   fp4    Q, K ~ N(0,1); bias ~ N(0,3); V ~ N(0,1)
@@ -64,6 +65,8 @@ WORKLOADS = {
     "long_fp8": Workload("long_fp8", 1, 16, 32768, 128, False, "bf16", "fp8", 3, "student_t",
                          2.0),
     "llm_fp8": Workload("llm_fp8", 1, 32, 4096, 128, True, "bf16", "fp8", 1, "llm_outliers", 2.0),
+    # a batch of short LLM prefills (the llm value laws), 200 MB of inputs
+    "short": Workload("short", 8, 32, 1024, 128, True, "bf16", "int8_fp8", 5, "llm_outliers", 2.0),
 }
 
 

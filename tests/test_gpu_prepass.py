@@ -207,16 +207,20 @@ def test_fp4_prepass_edge_values(cuda_device):
     check_fp4(q, k, v)
 
 
-@pytest.mark.parametrize("name", ["tiny", "llm", "video", "long", "fp4"])
-def test_prepass_full_workloads(cuda_device, name):
-    """The pre-pass over the full workload tensors, checked on sampled heads."""
+@pytest.mark.parametrize("name", ["tiny", "llm", "video", "long", "fp4", "short"])
+@pytest.mark.parametrize("fused", [False, True])
+def test_prepass_full_workloads(cuda_device, name, fused):
+    """The pre-pass over the full workload tensors, checked on sampled heads;
+    fused: through sage_quant_qkv (the launch bench.py times)."""
     w = WORKLOADS[name]
     q, k, v = make_qkv(w)
     heads = [(0, 0), (w.B - 1, w.H - 1)]
     if w.mode == "fp4":
+        if fused:
+            pytest.skip("FP4 has no sage_quant_qkv-only path")
         check_fp4(q, k, v, heads)
     else:
-        check_int8(q, k, v, heads)
+        check_int8(q, k, v, heads, fused=fused)
 
 
 # (N, d): through the cluster-fused kernel (8 CTAs, one tile each): one
@@ -233,6 +237,13 @@ def test_quant_qkv_matches_oracle(cuda_device, mode, N, d):
     oracle on every head."""
     q, k, v = rand_qkv(1, 3, N, d, "bf16" if d == 128 else "f16", seed=1400 + N + d)
     check_int8(q, k, v, mode=mode, fused=True)
+
+
+# (B, H): 16 heads (the most the fused kernel takes), 17 (the chains)
+@pytest.mark.parametrize("B,H", [(2, 8), (1, 17)])
+def test_quant_qkv_head_limit(cuda_device, B, H):
+    q, k, v = rand_qkv(B, H, 200, 128, "bf16", seed=1500 + H)
+    check_int8(q, k, v, fused=True)
 
 
 @pytest.mark.parametrize("mode,N,d", [("int8_fp8", 384, 128), ("fp8", 300, 64), ("fp4", 200, 128),
