@@ -129,10 +129,17 @@ int sage_quant_v(const void* v, int dtype,
                  void* v_codes, float* v_scales, void* v_sf, sage_stream_t stream);
 
 /* The Q/K and V pre-passes in one call, with the arguments of both (Q, K
- * and V share B, H, N, d).  The two are independent: the V pre-pass runs on
- * a library-owned second stream, forked from `stream` and joined back to
- * it with events (stream capture records the fork and the join), so the
- * two overlap on the GPU.  Results are those of the two separate calls. */
+ * and V share B, H, N, d).  Results are those of the two separate calls, bit
+ * for bit.  Two launch forms:
+ *   - 8-bit modes with N <= 1024 and B * H <= 16: one launch on `stream`
+ *     (clusters of 8 CTAs per head and tensor hold the head in shared memory
+ *     and reduce the K mean and V scales across the cluster).  Its wait for
+ *     the input copy is bounded: if it expires, the codes are not valid and
+ *     sage_get_last_device_status reports SAGE_ERR_DEVICE_TIMEOUT.
+ *   - otherwise the two pre-passes are independent: the V pre-pass runs on
+ *     a library-owned second stream, forked from `stream` and joined back to
+ *     it with events (stream capture records the fork and the join), so the
+ *     two overlap on the GPU. */
 int sage_quant_qkv(const void* q, const void* k, const void* v, int dtype,
                    int64_t B, int64_t H, int64_t N, int64_t d, int mode,
                    void* q_codes, float* q_scales, void* q_sf,
@@ -155,7 +162,8 @@ int sage_attn_fwd_quantized(int mode,
 
 /* The whole forward pass: pre-pass into a library-owned workspace (grown
  * on demand with stream-ordered allocation, one per device, freed at
- * unload), then the attention kernel.  sm_scale <= 0 means 1/sqrt(d). */
+ * unload; the pre-pass takes the launch forms of sage_quant_qkv), then the
+ * attention kernel.  sm_scale <= 0 means 1/sqrt(d). */
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype,
                   int64_t B, int64_t H, int64_t N, int64_t d,
                   int causal, float sm_scale, int mode, sage_stream_t stream);
