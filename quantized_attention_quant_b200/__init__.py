@@ -168,8 +168,10 @@ def sage_quant_v(v, mode="int8_fp8"):
 
 
 def sage_quant_qkv(q, k, v, mode="int8_fp8"):
-    """Both pre-passes in one call (the V pass overlaps the Q/K pass on a
-    library stream).  Returns (qk, vq) as sage_quant_qk and sage_quant_v do."""
+    """Both pre-passes in one call: one cluster-fused launch for short heads
+    in the 8-bit modes, else the V pass overlapped with the Q/K pass on a
+    library stream.  Returns (qk, vq) as sage_quant_qk and sage_quant_v do,
+    bit for bit."""
     B, H, N, d = _shape(q)
     if _shape(k) != (B, H, N, d) or _shape(v) != (B, H, N, d):
         raise ValueError("q, k, v must have the same shape")

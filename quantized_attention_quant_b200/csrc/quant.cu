@@ -11,14 +11,18 @@
 // abstract (FP8 V), SageAttention3 abstract (FP4 with one FP8 scale per 16
 // elements), all on the dblp author page on taxoreview.com.
 //
-// Launch structure (one 256-thread CTA per 128-token tile and role):
+// Launch structure of the chains (one 256-thread CTA per 128-token tile and
+// role):
 //   kernel A  roles that need no head-wide statistic: Q codes, FP4 V codes,
 //             and the per-chunk K sums / V maxima.  The last statistics CTA
 //             of each (b, h) (a per-head counter tells it) folds the chunk
 //             partials in chunk order into the K mean and the per-channel V
 //             scale, then resets the counter;
 //   kernel B  roles that need them: smoothed K codes, FP8 V codes.
-// sage_attn_fwd runs all roles of Q, K and V in these two launches.
+// The Q/K pre-pass is one A -> B chain, the V pre-pass another (in FP4 mode
+// a single launch); sage_quant_qkv and sage_attn_fwd run the two chains on
+// two streams, or, for short heads in the 8-bit modes, the one launch of the
+// cluster-fused kernel at the end of this file.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

@@ -287,10 +287,14 @@ def test_persistent_kernel_matches_one_item_per_cta(cuda_device, mode, causal, N
                              1 / math.sqrt(d), mode, "bf16")
 
 
-def test_cuda_graph_capture_and_replay(cuda_device):
-    # sage_attn_fwd inside a captured CUDA graph: the pre-pass fork/join to
-    # the library's second stream is recorded too; replays match eager runs
-    B, H, N, d = 1, 4, 640, 128
+# N = 640: the cluster-fused pre-pass (one launch); N = 1280: the two
+# pre-pass chains, the V chain forked onto the library's second stream
+@pytest.mark.parametrize("N", [640, 1280])
+def test_cuda_graph_capture_and_replay(cuda_device, N):
+    # sage_attn_fwd inside a captured CUDA graph (with the chains, the
+    # fork/join to the library's second stream is recorded too); replays
+    # match eager runs
+    B, H, d = 1, 4, 128
     q, k, v = rand_qkv(B, H, N, d, "bf16", seed=1300)
     dev = torch.device("cuda")
     qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
