@@ -601,3 +601,79 @@ def test_ragged_identity_and_close_to_exact(mode):
         b = att.exact_attention(q, k, v, causal, 0.125)
         cos = np.sum(a * b) / np.sqrt(np.sum(a * a) * np.sum(b * b))
         assert cos >= (0.97 if mode == "fp4" else 0.995)
+
+
+# ------------------------------------------------------ FP4 P~ encoder ----
+# Pins of quant_p_fp4 itself (SageAttention3 abstract: FP4 values with one FP8
+# scale per 16 elements; the P~ reading is s16 = ue4m3(448 amax16) with the
+# static tile scale 1/2688).  The restatement below writes both grids out
+# and takes the nearest value (ties to the even code, saturating), sharing
+# nothing with oracle/encoders.py.
+
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+# UE4M3 codes 0..0x7E: eight subnormals k 2^-9, then (1 + m/8) 2^(e-7)
+UE4M3_GRID = np.array([k * 2.0 ** -9 for k in range(8)] +
+                      [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8)][:-1])
+
+
+def nearest_even(grid, x):
+    x = np.minimum(np.asarray(x, np.float64), grid[-1])
+    dist = np.abs(x[..., None] - grid)
+    cand = dist == dist.min(axis=-1, keepdims=True)
+    even = cand & (np.arange(len(grid)) % 2 == 0)
+    pick = np.where(even.any(axis=-1), even.argmax(axis=-1), cand.argmax(axis=-1))
+    return grid[pick]
+
+
+def brute_quant_p_fp4(pt):
+    R, C = pt.shape
+    out = np.zeros((R, C))
+    for r in range(R):
+        for g0 in range(0, C, 16):
+            blk = pt[r, g0:g0 + 16]
+            s16 = nearest_even(UE4M3_GRID, blk.max() * 448.0)
+            den = s16 / 2688.0
+            if den > 0:
+                out[r, g0:g0 + 16] = nearest_even(E2M1_GRID, blk / den) * s16
+    return out
+
+
+def test_fp4_p_encoder_matches_grid_restatement():
+    g = np.random.default_rng(90)
+    pt = np.exp(-np.abs(g.standard_normal((6, 128))) * 3.0)
+    pt[0, 5] = 1.0                                   # a row max
+    pt[1, 16:32] = 0.0                               # an all-zero group
+    pt[2, 32:48] *= 2.0 ** -20                       # a group with a subnormal scale
+    # values planted at e2m1 midpoints of their group (both ends must round
+    # to the even code)
+    den = nearest_even(UE4M3_GRID, pt[3, 64:80].max() * 448.0) / 2688.0
+    for j, mid in enumerate([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]):
+        if mid * den < pt[3, 64:80].max():
+            pt[3, 65 + j] = mid * den
+    assert np.array_equal(att.quant_p_fp4(pt), brute_quant_p_fp4(pt))
+
+
+def test_fp4_p_encoder_closed_forms():
+    # the row max P~ = 1: s16 = ue4m3(448) = 448, t = 6 P~ -> code 6, and the
+    # value 6 * 448 times the tile scale 1/2688 is exactly 1
+    pt = np.full((1, 32), 0.3)
+    pt[0, 7] = 1.0
+    v = att.quant_p_fp4(pt)
+    assert v[0, 7] * att.P_FP4_G == 1.0
+    # an all-zero group stays zero; other groups do not see it
+    pt2 = pt.copy()
+    pt2[0, 16:] = 0.0
+    v2 = att.quant_p_fp4(pt2)
+    assert np.all(v2[0, 16:] == 0.0)
+    assert np.array_equal(v2[0, :16], v[0, :16])
+
+
+def test_fp4_p_encoder_power_of_two_scaling():
+    # both grids are the same in every normal binade: scaling a group by 2^-k
+    # (scale still normal: 448 amax 2^-k >= 2^-6) scales its values by 2^-k
+    g = np.random.default_rng(91)
+    pt = np.exp(-np.abs(g.standard_normal((4, 64))) * 2.0)
+    pt[:, 0] = 1.0
+    base = att.quant_p_fp4(pt)
+    for k in range(1, 9):
+        assert np.array_equal(att.quant_p_fp4(pt * 2.0 ** -k), base * 2.0 ** -k)
