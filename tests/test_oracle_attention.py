@@ -677,3 +677,20 @@ def test_fp4_p_encoder_power_of_two_scaling():
     base = att.quant_p_fp4(pt)
     for k in range(1, 9):
         assert np.array_equal(att.quant_p_fp4(pt * 2.0 ** -k), base * 2.0 ** -k)
+
+
+def test_fp8_p_encoder_matches_grid_restatement():
+    # quant_p_fp8 is the e4m3 value of 448 P~ (the non-negative e4m3 grid is
+    # the UE4M3 grid above): the row max P~ = 1 is 448, and every value is the
+    # nearest grid point, ties to the even code (planted midpoints included)
+    g = np.random.default_rng(92)
+    pt = np.exp(-np.abs(g.standard_normal((4, 128))) * 4.0)
+    pt[0, 0] = 1.0
+    mids = 0.5 * (UE4M3_GRID[1:] + UE4M3_GRID[:-1])
+    mids = mids[(mids / 448.0) * 448.0 == mids] / 448.0   # 448 P~ lands on the midpoint
+    assert len(mids) > 60
+    pt[1, :len(mids[::2])] = mids[::2]
+    pt[2, :len(mids[1::2])] = mids[1::2]
+    got = att.quant_p_fp8(pt)
+    assert got[0, 0] == 448.0
+    assert np.array_equal(got, nearest_even(UE4M3_GRID, pt * 448.0))
