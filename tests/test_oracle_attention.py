@@ -694,3 +694,79 @@ def test_fp8_p_encoder_matches_grid_restatement():
     got = att.quant_p_fp8(pt)
     assert got[0, 0] == 448.0
     assert np.array_equal(got, nearest_even(UE4M3_GRID, pt * 448.0))
+
+
+# ------------------------------------------------ FP4 Q/K/V pre-pass encoders ----
+# The FP32 formula of the FP4 encodings restated step by step on the grids
+# above (SageAttention3 abstract; the reading of the scale chain:
+# g = fp32(amax_tile / 2688), s16 = ue4m3(fp32(amax16 / fp32(6 g))),
+# code = e2m1(fp32(x / fp32(s16 g)))); values compared, not code bits.
+
+def brute_fp4_tile(blk):
+    """blk float32 [L, W], 16-groups along W: (values [L, W], scales [L, W/16], g)."""
+    f32 = np.float32
+    g = f32(f32(np.abs(blk).max()) / f32(2688))
+    six_g = f32(f32(6) * g)
+    L, W = blk.shape
+    vals = np.zeros((L, W))
+    scales = np.zeros((L, W // 16))
+    for l in range(L):
+        for m in range(W // 16):
+            grp = blk[l, 16 * m:16 * m + 16]
+            r = f32(f32(np.abs(grp).max()) / six_g) if six_g != 0 else f32(0)
+            s = nearest_even(UE4M3_GRID, float(r))
+            scales[l, m] = s
+            den = f32(f32(s) * g)
+            if den != 0:
+                t = (grp / den).astype(np.float32).astype(np.float64)
+                vals[l, 16 * m:16 * m + 16] = np.sign(t) * nearest_even(E2M1_GRID, np.abs(t))
+    return vals, scales, g
+
+
+def e2m1_value(codes):
+    c = codes.astype(np.int64)
+    return np.where(c & 8, -1.0, 1.0) * E2M1_GRID[c & 7]
+
+
+def test_fp4_token_encoder_matches_grid_restatement():
+    x = rnd((1, 1, 256, 64), 23, 2.0)
+    x[0, 0, 5, 16:32] = 0.0                          # an all-zero group
+    x[0, 0, 9, 0:16] *= np.float32(2.0 ** -12)       # a group far below the tile max
+    # exact e2m1 ties, x / fp32(s16 g) on a midpoint, planted under the
+    # group max of a few groups of the first tile (each takes the even code;
+    # a scale chain rounded differently breaks them the other way)
+    f32 = np.float32
+    tile_g = f32(f32(np.abs(x[0, 0, :128]).max()) / f32(2688))
+    planted = 0
+    for r in (20, 33, 77):
+        for m in range(4):
+            grp = x[0, 0, r, 16 * m:16 * m + 16]
+            s = nearest_even(UE4M3_GRID, float(f32(f32(np.abs(grp).max()) / f32(f32(6) * tile_g))))
+            den = f32(f32(s) * tile_g)
+            for j, mid in enumerate([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]):
+                xv = f32(f32(mid) * den)
+                if abs(xv) < np.abs(grp).max() and f32(xv / den) == f32(mid):
+                    x[0, 0, r, 16 * m + 1 + j] = -xv if j % 2 else xv
+                    planted += 1
+    assert planted > 40
+    codes, sf, g = pp.quant_fp4_tokens(x)
+    for t in range(2):
+        blk = x[0, 0, 128 * t:128 * (t + 1)].astype(np.float32)
+        vals, scales, gt = brute_fp4_tile(blk)
+        assert g[0, 0, t] == gt
+        assert np.array_equal(UE4M3_GRID[sf[0, 0, 128 * t:128 * (t + 1)]], scales)
+        assert np.array_equal(e2m1_value(codes[0, 0, 128 * t:128 * (t + 1)]), vals)
+
+
+def test_fp4_v_encoder_matches_grid_restatement():
+    # V: 16-groups over tokens, written transposed; tile = 128 tokens x d
+    v = rnd((1, 1, 256, 32), 24)
+    v[0, 0, 40:56, 7] = 0.0                          # an all-zero token group of one channel
+    codes, sf, g = pp.quant_v_fp4(v)
+    vt = v[0, 0].T.astype(np.float32)                # [d, N]
+    for t in range(2):
+        blk = vt[:, 128 * t:128 * (t + 1)]
+        vals, scales, gt = brute_fp4_tile(blk)
+        assert g[0, 0, t] == gt
+        assert np.array_equal(UE4M3_GRID[sf[0, 0, :, 8 * t:8 * (t + 1)]], scales)
+        assert np.array_equal(e2m1_value(codes[0, 0, :, 128 * t:128 * (t + 1)]), vals)
