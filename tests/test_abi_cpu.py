@@ -122,3 +122,19 @@ def test_gqa_empty_and_shape_errors(lib):
     assert gqa(lib, H=0, Hkv=0) == 0
     s = gqa(lib, B=1, H=8, Hkv=2, N=2 ** 28)
     assert s == -2 and "2^31" in lib.sage_status_string(s).decode()
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    # no CPU fallback: without libsage_b200.so every entry point raises
+    import torch
+    import quantized_attention_quant_b200 as sage
+    monkeypatch.setattr(sage, "library_path", "/nonexistent/libsage_b200.so")
+    monkeypatch.setattr(sage, "_lib", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        sage.library()
+    with pytest.raises(RuntimeError, match="no fallback"):
+        sage.buffer_bytes("int8_fp8", "q_codes", 1, 1, 128, 64)
+    # and host tensors are refused rather than computed on the CPU
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sage.sage_attn_fwd(q, q, q)
