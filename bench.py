@@ -2,13 +2,18 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl sage|reference]
 
-One step = the whole hot path over one batch: the Q/K pre-pass
-(sage_quant_qk), the V pre-pass (sage_quant_v) and the fused attention
-kernel (sage_attn_fwd_quantized), inputs resident in HBM.  L2 is flushed (a 256 MiB device write) between
+One step = the whole hot path over one batch: the Q/K and V pre-passes
+(sage_quant_qkv) and the fused attention kernel (sage_attn_fwd_quantized),
+inputs resident in HBM.  L2 is flushed (a 256 MiB device write) between
 timed steps; each step is bracketed by CUDA events on the launching stream.
 Metric: effective TOPS = 4*B*H*N^2*d / t (summed over ranks; weak scaling,
 each rank processes its own batch of heads with no collective on the data
 path).  Prints one JSON line on rank 0.
+
+The default workload is n16k (B=2 H=32 N=16384 d=128, non-causal, bf16,
+INT8 Q/K with FP8 P~ and V); the same shape in FP4 mode (the fp4 workload)
+is timed after it, kernel-only, and reported under "also"
+(--also none skips it).
 
 --impl reference times the CPU oracle (NumPy FP64, the method restated) on
 the host cores, on a bounded sample of the same workload per step.
@@ -30,7 +35,8 @@ sys.path.insert(0, ROOT)
 from quantized_attention_quant_b200.workloads import WORKLOADS, make_qkv  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
-DEFAULT_WORKLOAD = "llm"
+DEFAULT_WORKLOAD = "n16k"
+DEFAULT_ALSO = {"n16k": "fp4"}
 
 
 def parse():
@@ -41,7 +47,16 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--impl", default="sage", choices=["sage", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--also", default=None,
+                   help="comma-separated workloads timed after the main one (kernel-only "
+                        "lines under 'also'); 'none' for none")
     a = p.parse_args()
+    if a.also is None:
+        a.also = DEFAULT_ALSO.get(a.workload, "none")
+    a.also = [x for x in a.also.split(",") if x and x != "none"]
+    for x in a.also:
+        if x not in WORKLOADS:
+            p.error(f"unknown workload in --also: {x}")
     if a.warmup < 3:
         a.warmup = 3
     return a
@@ -56,6 +71,25 @@ def work_ops(w, heads):
     """Algorithmic tensor-core operations: 4 d per visible pair (2d for
     Q K^T, 2d for P~V)."""
     return 4.0 * w.d * visible_pairs(w) * heads
+
+
+def prepass_bytes(w, heads):
+    """Algorithmic HBM bytes of the pre-pass: read Q, K, V once (2 B per
+    element each), write the three code tensors (1 B per element in the
+    8-bit modes, 0.5 B + one UE4M3 scale per 16 elements in FP4 mode)."""
+    elem = heads * w.N * w.d
+    write = 1.0 if w.mode != "fp4" else 0.5 + 1.0 / 16
+    return elem * 3 * (2.0 + write)
+
+
+def percentile(xs, p):
+    xs = sorted(xs)
+    if not xs:
+        return None
+    i = (len(xs) - 1) * p / 100.0
+    lo = int(math.floor(i))
+    hi = min(lo + 1, len(xs) - 1)
+    return xs[lo] + (xs[hi] - xs[lo]) * (i - lo)
 
 
 def measured_peaks():
@@ -149,9 +183,146 @@ def job_throughput(ops_per_rank, world, t_ms):
     return ops_per_rank * world / (t_ms * 1e-3) / 1e12
 
 
-def run_sage(args):
-    import ctypes
+class Runner:
+    """The timed step of one workload on one rank: device inputs, the code
+    buffers, and the two library calls of a step."""
 
+    def __init__(self, w, dev):
+        import torch
+
+        import quantized_attention_quant_b200 as sage
+        self.torch, self.sage = torch, sage
+        self.lib = sage.library()
+        self.w, self.dev = w, dev
+        self.mode = sage.MODES[w.mode]
+        self.dt = sage.DTYPES[w.dtype]
+        qh, kh, vh = make_qkv(w)
+        self.host = [t.pin_memory() for t in (qh, kh, vh)]
+        self.q, self.k, self.v = (t.to(dev) for t in self.host)
+        self.o = torch.empty_like(self.q)
+        names = ["q_codes", "q_scales", "q_sf", "k_codes", "k_scales", "k_sf", "k_mean",
+                 "v_codes", "v_scales", "v_sf"]
+        self.bufs = {}
+        for n in names:
+            nb = sage.buffer_bytes(w.mode, n, w.B, w.H, w.N, w.d)
+            self.bufs[n] = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+        self.P = {n: (b.data_ptr() if b is not None else None) for n, b in self.bufs.items()}
+        self.stream = torch.cuda.current_stream(dev)
+
+    def check(self, s):
+        if s != 0:
+            raise RuntimeError(self.lib.sage_status_string(s).decode())
+
+    def step(self, ev_mid=None):
+        """Both pre-passes (the V pass overlapped with the Q/K pass), then the
+        attention kernel on the codes; ev_mid is recorded between them."""
+        import ctypes
+        w, P, sptr = self.w, self.P, self.stream.cuda_stream
+        self.check(self.lib.sage_quant_qkv(
+            self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), self.dt, w.B, w.H, w.N, w.d,
+            self.mode, P["q_codes"], P["q_scales"], P["q_sf"], P["k_codes"], P["k_scales"],
+            P["k_sf"], P["k_mean"], P["v_codes"], P["v_scales"], P["v_sf"], sptr))
+        if ev_mid is not None:
+            ev_mid.record(self.stream)
+        self.check(self.lib.sage_attn_fwd_quantized(
+            self.mode, P["q_codes"], P["q_scales"], P["q_sf"], P["k_codes"], P["k_scales"],
+            P["k_sf"], P["v_codes"], P["v_scales"], P["v_sf"], self.o.data_ptr(), self.dt,
+            w.B, w.H, w.N, w.d, int(w.causal), ctypes.c_float(w.sm_scale), sptr))
+
+    def launches_per_step(self):
+        """sage_quant_qkv: one cluster-fused launch in the 8-bit modes up to 8
+        tiles (1024 tokens) per head and 16 heads, else 2 (Q/K) + 2 (V in the
+        8-bit modes) or 1 (V in FP4); attention: 1."""
+        w = self.w
+        if w.mode != "fp4" and -(-w.N // 128) <= 8 and w.B * w.H <= 16:
+            return 1 + 1
+        return 2 + (1 if w.mode == "fp4" else 2) + 1
+
+    def time(self, steps, warmup, flush):
+        """Per timed step: (step ms, pre-pass ms, attention ms), CUDA events
+        on the launching stream, L2 flushed before every step."""
+        torch = self.torch
+        for _ in range(warmup):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e0, e1, e2 in ev:
+            flush.zero_()                  # outside the events
+            e0.record(self.stream)
+            self.step(e1)
+            e2.record(self.stream)
+        torch.cuda.synchronize()
+        return [(a.elapsed_time(c), a.elapsed_time(b), b.elapsed_time(c)) for a, b, c in ev]
+
+    def time_e2e(self, steps, flush):
+        """The public sage_attn_fwd with pinned host inputs copied in and O
+        copied back to the host, every step inside the events."""
+        torch, sage, w, dev = self.torch, self.sage, self.w, self.dev
+        qh, kh, vh = self.host
+        oh = torch.empty_like(qh).pin_memory()
+        for _ in range(2):
+            oh.copy_(sage.sage_attn_fwd(qh.to(dev, non_blocking=True),
+                                        kh.to(dev, non_blocking=True),
+                                        vh.to(dev, non_blocking=True), w.causal, None,
+                                        w.mode).to("cpu", non_blocking=True))
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            qd = qh.to(dev, non_blocking=True)
+            kd = kh.to(dev, non_blocking=True)
+            vd = vh.to(dev, non_blocking=True)
+            od = sage.sage_attn_fwd(qd, kd, vd, w.causal, None, w.mode)
+            oh.copy_(od, non_blocking=True)
+            e1.record(self.stream)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        elem = w.B * w.H * w.N * w.d
+        return ms, 3 * elem * 2, elem * 2
+
+    def free(self):
+        del self.q, self.k, self.v, self.o, self.bufs, self.host
+        self.torch.cuda.empty_cache()
+
+
+def summarize(w, world, times, sms, dev_name=None):
+    """Throughput, percentiles and the attention roofline of a list of
+    (step, pre-pass, attention) times (already the max over ranks)."""
+    steps = [t[0] for t in times]
+    pre = [t[1] for t in times]
+    attn = [t[2] for t in times]
+    t_step, t_pre, t_attn = (sum(x) / len(x) for x in (steps, pre, attn))
+    heads = w.B * w.H
+    peaks, src = measured_peaks()
+    ratio = 4.0 if w.mode == "fp4" else 2.0             # vs bf16, nominal dense ratios
+    peak = peaks["bf16_tflops"] * ratio
+    achieved = work_ops(w, heads) / (t_attn * 1e-3) / 1e12
+    pre_gbs = prepass_bytes(w, heads) / (t_pre * 1e-3) / 1e9
+    return {
+        "value": round(job_throughput(w.ops, world, t_step), 2),
+        "value_done": round(job_throughput(work_ops(w, heads), world, t_step), 2),
+        "ms_per_step": round(t_step, 4),
+        "step_ms_p50": round(percentile(steps, 50), 4),
+        "step_ms_p95": round(percentile(steps, 95), 4),
+        "attn_kernel_ms": round(t_attn, 4),
+        "attn_kernel_ms_p50": round(percentile(attn, 50), 4),
+        "attn_kernel_ms_p95": round(percentile(attn, 95), 4),
+        "prepass_ms": round(t_pre, 4),
+        "prepass_gbs": round(pre_gbs, 1),
+        "prepass_hbm_frac": round(pre_gbs / peaks["hbm_gbs"], 4),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": read_traffic(w.name),
+                     "kernel": attention_kernel(w, sms),
+                     "peak_source": f"{src} bf16 burst x{ratio:g} (nominal dense ratio)",
+                     "work": "4 d ops per visible (q,k) pair"},
+    }
+
+
+def run_sage(args):
     import torch
     import torch.distributed as dist
 
@@ -162,58 +333,12 @@ def run_sage(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    lib = sage.library()
+    sage.library()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     w0 = WORKLOADS[args.workload]
     w = rank_workload(w0, rank)
-    B, H, N, d = w.B, w.H, w.N, w.d
-    mode = sage.MODES[w.mode]
-    dt = sage.DTYPES[w.dtype]
-
-    qh, kh, vh = make_qkv(w)
-    qh, kh, vh = qh.pin_memory(), kh.pin_memory(), vh.pin_memory()
-    q, k, v = qh.to(dev), kh.to(dev), vh.to(dev)
-    o = torch.empty_like(q)
-
-    def buf(name):
-        n = sage.buffer_bytes(w.mode, name, B, H, N, d)
-        return torch.empty(n, dtype=torch.uint8, device=dev) if n else None
-
-    names = ["q_codes", "q_scales", "q_sf", "k_codes", "k_scales", "k_sf", "k_mean",
-             "v_codes", "v_scales", "v_sf"]
-    bufs = {n: buf(n) for n in names}
-    P = {n: (bufs[n].data_ptr() if bufs[n] is not None else None) for n in names}
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    sptr = stream.cuda_stream
-    sm_scale = w.sm_scale
-
-    def check(s):
-        if s != 0:
-            raise RuntimeError(lib.sage_status_string(s).decode())
-
-    def step(ev_attn=None):
-        # both pre-passes (the V pass overlapped with the Q/K pass), then
-        # the attention kernel on the codes
-        check(lib.sage_quant_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), dt, B, H, N, d, mode,
-                                 P["q_codes"], P["q_scales"], P["q_sf"], P["k_codes"],
-                                 P["k_scales"], P["k_sf"], P["k_mean"], P["v_codes"],
-                                 P["v_scales"], P["v_sf"], sptr))
-        if ev_attn:
-            ev_attn[0].record(stream)
-        check(lib.sage_attn_fwd_quantized(mode, P["q_codes"], P["q_scales"], P["q_sf"],
-                                          P["k_codes"], P["k_scales"], P["k_sf"], P["v_codes"],
-                                          P["v_scales"], P["v_sf"], o.data_ptr(), dt, B, H, N, d,
-                                          int(w.causal), ctypes.c_float(sm_scale), sptr))
-        if ev_attn:
-            ev_attn[1].record(stream)
-
-    # sage_quant_qkv: one cluster-fused launch in the 8-bit modes up to 8
-    # tiles (1024 tokens) per head and 16 heads, else 2 (Q/K) + 2 (V in FP8)
-    # or 1 (V in FP4); attention: 1
-    if w.mode != "fp4" and -(-N // 128) <= 8 and B * H <= 16:
-        launches_per_step = 1 + 1
-    else:
-        launches_per_step = 2 + (1 if w.mode == "fp4" else 2) + 1
+    run = Runner(w, dev)
 
     uuid = None
     try:
@@ -222,96 +347,71 @@ def run_sage(args):
         pass
     clocks = ClockSampler(uuid)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    times = run.time(args.steps, args.warmup, flush)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()                      # L2 flush between timed steps (outside the events)
-        ev[i][0].record(stream)
-        step(ea[i])
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    attn_ms = [a.elapsed_time(b) for a, b in ea]
     status = sage.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status}")
-
-    # end to end through the public API: pinned host inputs in, O back to host
-    oh = torch.empty_like(qh).pin_memory()
-    for _ in range(2):
-        oh.copy_(sage.sage_attn_fwd(qh.to(dev, non_blocking=True), kh.to(dev, non_blocking=True),
-                                    vh.to(dev, non_blocking=True), w.causal, None, w.mode).to(
-                                        "cpu", non_blocking=True))
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(max(3, args.steps // 4)):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        qd = qh.to(dev, non_blocking=True)
-        kd = kh.to(dev, non_blocking=True)
-        vd = vh.to(dev, non_blocking=True)
-        od = sage.sage_attn_fwd(qd, kd, vd, w.causal, None, w.mode)
-        oh.copy_(od, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms.append(e0.elapsed_time(e1))
+    e2e_ms, h2d, d2h = run.time_e2e(max(3, args.steps // 4), flush)
     clk = clocks.stop()
 
-    # max over ranks
-    t_step = sum(step_ms) / len(step_ms)
-    t_attn = sum(attn_ms) / len(attn_ms)
-    t_e2e = sum(e2e_ms) / len(e2e_ms)
-    t_step, t_attn, t_e2e = max_over_ranks([t_step, t_attn, t_e2e], world, dev)
-
-    heads = B * H
-    value = job_throughput(w.ops, world, t_step)        # 4 B H N^2 d, all ranks
-    e2e_val = job_throughput(w.ops, world, t_e2e)
-    peaks, src = measured_peaks()
-    ratio = 4.0 if w.mode == "fp4" else 2.0             # vs bf16, nominal dense ratios
-    peak = peaks["bf16_tflops"] * ratio
-    achieved = work_ops(w, heads) / (t_attn * 1e-3) / 1e12
-    traffic = read_traffic(args.workload)
-    elem = B * H * N * d
+    # max over ranks, step by step
+    flat = [x for t in times for x in t] + [sum(e2e_ms) / len(e2e_ms)]
+    flat = max_over_ranks(flat, world, dev)
+    times = [tuple(flat[3 * i:3 * i + 3]) for i in range(len(times))]
+    t_e2e = flat[-1]
+    summ = summarize(w0, world, times, sms)
     out = {
         "metric": "attention fwd effective TOPS (4*B*H*N^2*d/t)",
-        "value": round(value, 2),
+        "value": summ.pop("value"),
         "unit": "TOPS",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(t_step, 4),
+        "ms_per_step": summ.pop("ms_per_step"),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": {"fp4": "fp4e2m1", "fp8": "fp8e4m3"}.get(w.mode, "int8+fp8e4m3"),
         "data": "synthetic",
         "config": config_of(w0, world),
-        "attn_kernel_ms": round(t_attn, 4),
-        "prepass_ms": round(t_step - t_attn, 4),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": attention_kernel(w, torch.cuda.get_device_properties(dev)
-                                                .multi_processor_count),
-                     "peak_source": f"{src} bf16 burst x{ratio:g} (nominal dense ratio)",
-                     "work": "4 d ops per visible (q,k) pair"},
-        "e2e": {"value": round(e2e_val, 2), "unit": "TOPS",
-                "h2d_bytes_per_step": 3 * elem * 2, "d2h_bytes_per_step": elem * 2},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk,
     }
+    out.update(summ)
+    out["value_done_note"] = ("value counts 4*B*H*N^2*d as the metric is written; value_done "
+                              "counts 4*d per visible (q,k) pair (half of it, plus the "
+                              "diagonal, in causal runs)")
+    out["e2e"] = {"value": round(job_throughput(w0.ops, world, t_e2e), 2), "unit": "TOPS",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    out["gpu_launches"] = run.launches_per_step() * args.steps
+    out["clocks"] = clk
+    run.free()
+
+    # further workloads, kernel-only (the same timed step)
+    also = []
+    for name in args.also:
+        wa = rank_workload(WORKLOADS[name], rank)
+        ra = Runner(wa, dev)
+        if world > 1:
+            dist.barrier()
+        ta = ra.time(args.steps, args.warmup, flush)
+        flat = max_over_ranks([x for t in ta for x in t], world, dev)
+        ta = [tuple(flat[3 * i:3 * i + 3]) for i in range(len(ta))]
+        sa = summarize(WORKLOADS[name], world, ta, sms)
+        sa["config"] = config_of(WORKLOADS[name], world)
+        sa["gpu_launches"] = ra.launches_per_step() * args.steps
+        also.append(sa)
+        ra.free()
+    status = sage.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    if also:
+        out["also"] = also
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w0, budget_s=12.0)
     if world > 1:
@@ -360,13 +460,17 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_sample(w, heads, rows=None):
-    """Run the oracle (emulated path) on the given heads; returns seconds."""
+def oracle_sample(w, heads, rows=None, exact=False):
+    """Run the oracle on the given heads -- the emulated quantized path, or
+    with exact=True the FP64 exact attention; returns seconds."""
     from oracle import attention as att
     from quantized_attention_quant_b200.workloads import to_numpy32
     q, k, v = (to_numpy32(t) for t in make_qkv(w, heads))
     t0 = time.perf_counter()
-    att.emulated_sage_attention(q, k, v, w.causal, w.sm_scale, mode=w.mode, rows=rows)
+    if exact:
+        att.exact_attention(q, k, v, w.causal, w.sm_scale, rows=rows)
+    else:
+        att.emulated_sage_attention(q, k, v, w.causal, w.sm_scale, mode=w.mode, rows=rows)
     return time.perf_counter() - t0
 
 
@@ -382,20 +486,37 @@ def sample_rows(w):
     return rows, len(rows) * w.N
 
 
-def cpu_baseline(w, budget_s=12.0):
-    rows, pairs = sample_rows(w)
+def _oracle_rate(w, rows, pairs, budget_s, exact=False):
+    """Heads run within the budget and the oracle's rate on them (TOPS of
+    the metric's 4 d ops per pair)."""
     t = 0.0
-    done = 0
     h = 0
     while t < budget_s and h < w.B * w.H:
-        t += oracle_sample(w, [(h // w.H, h % w.H)], rows)
-        done += pairs
+        t += oracle_sample(w, [(h // w.H, h % w.H)], rows, exact=exact)
         h += 1
-    ops = 4.0 * w.d * done
+    return h, 4.0 * w.d * pairs * h / t / 1e12, t
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle on the host cores: the emulated quantized path (the
+    baseline), the exact FP64 attention beside it, and the emulated path
+    again on one BLAS thread."""
+    rows, pairs = sample_rows(w)
+    h, value, t = _oracle_rate(w, rows, pairs, budget_s)
+    _, exact, _ = _oracle_rate(w, rows, pairs, budget_s / 4, exact=True)
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"):
+            _, single, _ = _oracle_rate(w, rows, pairs, budget_s / 4)
+    except ImportError:
+        pass
     desc = (f"{h} head(s), {'all' if rows is None else len(rows)} query rows each, "
             f"emulated quantized path (pre-pass of the sampled heads included)")
-    return {"value": round(ops / t / 1e12, 6), "unit": "TOPS", "cores": blas_threads(),
-            "kind": "oracle", "sample": desc, "seconds": round(t, 2)}
+    return {"value": round(value, 6), "unit": "TOPS", "cores": blas_threads(),
+            "kind": "oracle", "sample": desc, "seconds": round(t, 2),
+            "exact_fp64_value": round(exact, 6),
+            "emulated_1_thread_value": None if single is None else round(single, 6)}
 
 
 def run_reference(args):

@@ -139,7 +139,10 @@ int sage_quant_v(const void* v, int dtype,
  *   - otherwise the two pre-passes are independent: the V pre-pass runs on
  *     a library-owned second stream, forked from `stream` and joined back to
  *     it with events (stream capture records the fork and the join), so the
- *     two overlap on the GPU. */
+ *     two overlap on the GPU.  That second stream is one per device, shared
+ *     by every caller stream: callers on different streams that reach this
+ *     point at the same time have their V pre-passes serialised on it (the
+ *     results are unaffected; only the overlap between them is lost). */
 int sage_quant_qkv(const void* q, const void* k, const void* v, int dtype,
                    int64_t B, int64_t H, int64_t N, int64_t d, int mode,
                    void* q_codes, float* q_scales, void* q_sf,
@@ -161,9 +164,10 @@ int sage_attn_fwd_quantized(int mode,
                             int causal, float sm_scale, sage_stream_t stream);
 
 /* The whole forward pass: pre-pass into a library-owned workspace (grown
- * on demand with stream-ordered allocation, one per device, freed at
- * unload; the pre-pass takes the launch forms of sage_quant_qkv), then the
- * attention kernel.  sm_scale <= 0 means 1/sqrt(d). */
+ * on demand with stream-ordered allocation, one per (device, stream),
+ * freed at unload; the pre-pass takes the launch forms of sage_quant_qkv),
+ * then the attention kernel.  sm_scale <= 0 means 1/sqrt(d).  An allocation
+ * failure returns SAGE_ERR_CUDA before any kernel is launched. */
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype,
                   int64_t B, int64_t H, int64_t N, int64_t d,
                   int causal, float sm_scale, int mode, sage_stream_t stream);
@@ -197,11 +201,20 @@ int sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, int 
  *   - A shape whose scratch exceeds the array is rejected with
  *     SAGE_ERR_UNSUPPORTED and a message giving both sizes (about 3.1 bytes
  *     per element of Q in INT8/FP8 mode: B*H*N*d up to about 21 million).
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - The first call on a device does its one-time set-up with that device
+ *     current: it looks up the array's device address and creates the
+ *     library's second stream (and two events) that the pre-pass forks onto
+ *     for long sequences.  Make that first call, of any shape, before any
+ *     stream capture; later calls create nothing.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind: calls whose GPU work overlaps (different streams, or threads)
- *     race on it and must be serialised by the caller. */
+ *     race on it and must be serialised by the caller.  Each call clears the
+ *     statistics counters it uses (a stream-ordered memset, which allocates
+ *     nothing) before its pre-pass, so an overlap spoils only the calls that
+ *     overlapped.
+ *   - The second stream is shared by every caller stream of a device: two
+ *     callers that run this pre-pass at once on different streams have their
+ *     V chains serialised (results are unaffected). */
 #define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int dtype,
                           int64_t B, int64_t H, int64_t N, int64_t d,

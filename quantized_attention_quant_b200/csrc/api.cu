@@ -660,19 +660,27 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // never a device address).
 std::map<int, void*> g_noalloc_addr;
 
+// One-time set-up per device: the array's device address, and the side
+// stream (with its fork/join events) that the two-launch pre-pass uses, so
+// that no later call of any shape creates a CUDA object.
 int noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
-  std::lock_guard<std::mutex> lk(g_mu);
-  auto it = g_noalloc_addr.find(dev);
-  if (it != g_noalloc_addr.end()) {
-    *out = it->second;
-    return SAGE_OK;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_noalloc_addr.find(dev);
+    if (it != g_noalloc_addr.end()) {
+      *out = it->second;
+      return SAGE_OK;
+    }
   }
+  SideStream* ss = nullptr;
+  SAGE_TRY(side_stream(&ss));
   void* p = nullptr;
   e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(no-allocation scratch)");
+  std::lock_guard<std::mutex> lk(g_mu);
   g_noalloc_addr[dev] = p;
   *out = p;
   return SAGE_OK;
@@ -727,8 +735,15 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
     return sage_buffer_bytes(mode, w, B, H, N, d) ? base + off[w] : nullptr;
   };
   // Every scratch byte the kernels read is written earlier in the same call
-  // (codes, scales, statistics partials), except the per-head counters:
-  // zero in the loaded image, and returned to zero by every pre-pass.
+  // (codes, scales, statistics partials), except the per-head counters of
+  // the statistics pass.  A pre-pass leaves them at zero, but a call that
+  // overlapped another one on the GPU may not have: clear the counters of
+  // the heads in use (K, then V) first, in stream order, so that one such
+  // race cannot spoil the calls after it.
+  cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)(B * H) * sizeof(uint32_t), st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(cnt + kMaxStatHeads, 0, (size_t)(B * H) * sizeof(uint32_t), st);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaMemsetAsync(no-allocation counters)");
   QuantQKArgs qa{q, k, dtype, mode, B, H, N, d, H,
                  at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
                  at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
@@ -739,7 +754,6 @@ int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, 
                 reinterpret_cast<float*>(base + off_vmax), cnt};
   qa.status = di->status;
   SAGE_TRY(prepass_forked(qa, va, st));
-  cudaError_t e = cudaSuccess;
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),

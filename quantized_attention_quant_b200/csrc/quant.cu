@@ -84,7 +84,7 @@ struct PrepassPtrs {
   int64_t bh_kv;  // K/V heads (B * Hkv; fewer than bh_q under grouped-query attention)
 };
 
-constexpr int kMaxHeads = 65536;
+constexpr int kMaxHeads = kMaxStatHeads;
 
 // Eight elements as FP32 from global memory (read-only path) or, SHARED,
 // from shared memory.

@@ -46,8 +46,10 @@ struct QuantVArgs {
   uint32_t* ws_cnt;  // as in QuantQKArgs
 };
 
-// Bytes of the per-head counters at the start of every workspace.
-constexpr size_t kStatsCounterBytes = size_t(2) * 65536 * 4;
+// The per-head counters at the start of every workspace: K counters at
+// [0, kMaxStatHeads), V counters at [kMaxStatHeads, 2 kMaxStatHeads).
+constexpr int kMaxStatHeads = 65536;
+constexpr size_t kStatsCounterBytes = size_t(2) * kMaxStatHeads * 4;
 
 struct AttnArgs {
   int mode;

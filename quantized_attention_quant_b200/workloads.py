@@ -19,6 +19,7 @@ Distributions (normal laws written N(0, sigma); the K bias is one value per
   video  Q, K, V ~ N(0,1); bias ~ N(0,4)
   long   Q, K, V ~ Student-t(nu=4) / sqrt(2) (unit variance); bias ~ N(0,2)
   fp4    Q, K ~ N(0,1); bias ~ N(0,3); V ~ N(0,1)
+  n16k   the fp4 laws and shape in the 8-bit modes
 """
 
 from dataclasses import dataclass, replace
@@ -67,6 +68,10 @@ WORKLOADS = {
     "llm_fp8": Workload("llm_fp8", 1, 32, 4096, 128, True, "bf16", "fp8", 1, "llm_outliers", 2.0),
     # a batch of short LLM prefills (the llm value laws), 200 MB of inputs
     "short": Workload("short", 8, 32, 1024, 128, True, "bf16", "int8_fp8", 5, "llm_outliers", 2.0),
+    # the fp4 shape and value laws (16k tokens, d = 128, non-causal) through
+    # the 8-bit modes: INT8 Q/K (and FP8 Q/K) with FP8 P~ and V
+    "n16k": Workload("n16k", 2, 32, 16384, 128, False, "bf16", "int8_fp8", 6, "normal", 3.0),
+    "n16k_fp8": Workload("n16k_fp8", 2, 32, 16384, 128, False, "bf16", "fp8", 6, "normal", 3.0),
 }
 
 

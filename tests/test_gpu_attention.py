@@ -223,7 +223,8 @@ def test_side_stream(cuda_device):
 
 
 FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", None), ("long_causal", None),
-        ("fp4", None), ("long_fp8", None), ("llm_fp8", None), ("short", None)]
+        ("fp4", None), ("long_fp8", None), ("llm_fp8", None), ("short", None),
+        ("n16k", 0.999), ("n16k_fp8", None)]
 
 
 @pytest.mark.parametrize("name,cos_floor", FULL)

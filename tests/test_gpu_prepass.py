@@ -207,7 +207,7 @@ def test_fp4_prepass_edge_values(cuda_device):
     check_fp4(q, k, v)
 
 
-@pytest.mark.parametrize("name", ["tiny", "llm", "video", "long", "fp4", "short"])
+@pytest.mark.parametrize("name", ["tiny", "llm", "video", "long", "fp4", "short", "n16k"])
 @pytest.mark.parametrize("fused", [False, True])
 def test_prepass_full_workloads(cuda_device, name, fused):
     """The pre-pass over the full workload tensors, checked on sampled heads;

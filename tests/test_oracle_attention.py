@@ -176,6 +176,54 @@ def test_fp8_v_properties():
             assert np.all(err[big] <= row[big] * 2.0 ** -4 * (1 + 1e-6))
 
 
+def test_fp8_v_scale_pinned():
+    """s_V of a channel is amax over ALL N tokens of the head, over 448, and
+    the codes follow from it: planted values make every expected scale and
+    code a closed form.  Channel c's largest |V| is 448 * 2^e_c and sits in
+    the second 128-token block, whose maximum differs from the first
+    block's; the other planted values are 2^e_c times exact e4m3 grid
+    points.  A 447 divisor, a per-block amax, or a max over the channel axis
+    instead of the token axis each break the closed form."""
+    N, d = 256, 8
+    grid = np.array([96.0, -40.0, 13.0, 0.5, -2.0 ** -6, 2.0 ** -9], np.float64)  # e4m3 values
+    codes_of = {96.0: 0x6C, -40.0: 0xE2, 13.0: 0x55, 0.5: 0x30, -2.0 ** -6: 0x88,
+                2.0 ** -9: 0x01}
+    for val, code in codes_of.items():                    # the grid points, decoded
+        assert float(enc.e4m3_decode(np.array([code], np.uint8))[0]) == val
+    v = np.zeros((1, 2, N, d), np.float32)
+    expect_s = np.zeros((1, 2, d), np.float32)
+    expect_codes = np.zeros((1, 2, d, N), np.uint8)
+    for h in range(2):
+        for c in range(d):
+            e = c - 4 + 3 * h                                # scales 2^-4 .. 2^6
+            s_c = 2.0 ** e
+            expect_s[0, h, c] = s_c
+            t_max = 128 + (37 * c + 11 * h) % 128            # in the second block
+            v[0, h, t_max, c] = -448.0 * s_c if c % 2 else 448.0 * s_c
+            expect_codes[0, h, c, t_max] = 0xFE if c % 2 else 0x7E
+            for i, g in enumerate(grid):                     # first block: max 96 * s_c
+                t = (5 * c + 3 * i) % 128
+                v[0, h, t, c] = g * s_c
+                expect_codes[0, h, c, t] = codes_of[g]
+    # the per-channel scale is 2^e exactly, so every planted code is exact
+    codes, s = pp.quant_v_fp8(v)
+    assert s.dtype == np.float32
+    np.testing.assert_array_equal(s.view(np.uint32), expect_s.view(np.uint32))
+    np.testing.assert_array_equal(codes, expect_codes)
+    # a value that is not a power of two times 448: s = fp32(amax / 448), the
+    # correctly rounded quotient, checked against exact rational arithmetic
+    from fractions import Fraction
+    w = np.zeros((1, 1, N, 1), np.float32)
+    w[0, 0, 200, 0] = np.float32(1000.0)
+    w[0, 0, 10, 0] = np.float32(-3.0)
+    _, s2 = pp.quant_v_fp8(w)
+    q = Fraction(1000) / 448
+    cand = [np.nextafter(s2[0, 0, 0], np.float32(-np.inf)), s2[0, 0, 0],
+            np.nextafter(s2[0, 0, 0], np.float32(np.inf))]
+    dist = [abs(Fraction(float(x)) - q) for x in cand]
+    assert dist[1] < dist[0] and dist[1] < dist[2]
+
+
 def test_fp4_tokens_properties():
     x = rnd((1, 1, 256, 64), 21, 2.0)
     codes, sf, g = pp.quant_fp4_tokens(x)
