@@ -14,8 +14,11 @@ traffic" for the tiled online softmax):
   (causal: only keys t_k <= t_q):
     A      = q_codes . k_codes^T                (exact integer / exact FP64;
                                                  FP8 Q/K mode: e4m3 codes)
-    S      = A * s_Q * s_K * sm_scale           (FP4: A * g_Q * g_K * sm_scale,
-                                                 block scales inside A)
+    S      = A * s_Q * s_K * sm_scale           (s_Q of the query's token,
+                                                 s_K of the key's 32-token
+                                                 block; FP4: A * g_Q * g_K *
+                                                 sm_scale, block scales
+                                                 inside A)
     m_new  = max(m, rowmax S)
     alpha  = exp(m - m_new)
     P~     = exp(S - m_new)                     (<= 1)
@@ -330,8 +333,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                     qd = qk["q_codes"][b, h].astype(np.float64)
                     kd = qk["k_codes"][b, h].astype(np.float64)
                 vd = e4m3_decode(vc[b, h]).T                      # [N, d]
-                s_row = qk["q_scales"][b, h].astype(np.float64)[tile_of]
-                s_key = qk["k_scales"][b, h].astype(np.float64)[tile_of]
+                s_row = qk["q_scales"][b, h].astype(np.float64)[np.arange(N) // pp.Q_GROUP]
+                s_key = qk["k_scales"][b, h].astype(np.float64)[np.arange(N) // pp.K_GROUP]
                 v_fold = np.broadcast_to(vs[b, h].astype(np.float64) / P_FP8_SCALE, (ntiles, d))
                 res = _tile_loop(qd, kd, vd, s_row, s_key, v_fold, quant_p_fp8,
                                  causal, sm_scale, rows, amb,

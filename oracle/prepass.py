@@ -14,10 +14,13 @@ Readings of the pages (they give the method only at abstract level):
    fixed order: per 128-token chunk a partial sum in token order, then the
    chunk partials in chunk order; mean = fp32(total / N).
 2. Q is not smoothed (Q smoothing is the SageAttention2 extension).
-3. INT8 Q/K: one FP32 scale per 128-token block of one (b, h), covering all
+3. INT8 Q/K: one FP32 scale per block of tokens of one (b, h), covering all
    d channels: s = fp32(amax / 127); code = clamp(rne(fp32(x / s)), +-127);
    an all-zero block gets s = 0 and codes 0.  For K, x = fp32(K) - mean is a
-   single FP32 subtraction.
+   single FP32 subtraction.  Block sizes (the SageAttention2 abstract's
+   "hardware-friendly thread-level granularity", read for a kernel in which
+   one thread owns one query row and dequantizes 32 keys at a time): Q one
+   token (Q_GROUP), K 32 tokens (K_GROUP).
 4. FP8 V (SageAttention2 abstract): per channel over all N tokens of a
    (b, h): s_V = fp32(amax / 448); code = e4m3(fp32(V / s_V)).  Written
    transposed, [B, H, d, N], so that the P~V contraction (over tokens) reads
@@ -31,11 +34,13 @@ Readings of the pages (they give the method only at abstract level):
 6. FP8 Q/K (the kernel-comparison blog, "How SageAttention uses
    quantization for more throughput": queries and keys go to INT8 or FP8):
    the INT8 scheme of reading 3 with the e4m3 grid in place of the
-   integers: per 128-token block s = fp32(amax / 448); code =
-   e4m3(fp32(x / s)) (round to nearest even, saturating); an all-zero
-   block gets s = 0 and codes 0.  K is smoothed first, as in reading 1.
-7. Ragged sequences (N not a multiple of 128): the last 128-token block is
-   shorter and its scale covers its tokens only; the K mean and the V
+   integers, with the same blocks (Q per token, K per 32 tokens):
+   s = fp32(amax / 448); code = e4m3(fp32(x / s)) (round to nearest even,
+   saturating); an all-zero block gets s = 0 and codes 0.  K is smoothed
+   first, as in reading 1.
+7. Ragged sequences (N not a multiple of 128): the last block (of 32 K
+   tokens, or 128 tokens in FP4 mode) may be shorter and its scale covers
+   its tokens only; the K mean and the V
    scales divide by / range over the N real tokens; in FP4 mode a partial
    16-element group (V over tokens, P~ over keys) counts its missing
    elements as zeros, which change neither its maximum nor any code.
@@ -46,7 +51,9 @@ import numpy as np
 from .encoders import (e4m3_encode, e2m1_encode, ue4m3_encode, ue4m3_decode,
                        int8_quantize)
 
-BLOCK = 128      # tokens per quantization block / tile
+BLOCK = 128      # tokens per tile (FP4 tile scales, K-mean chunks, V tiles)
+Q_GROUP = 1      # tokens per Q scale in the 8-bit modes (one query row)
+K_GROUP = 32     # tokens per K scale in the 8-bit modes (32 keys)
 FP4_VEC = 16     # elements per FP4 micro-block
 FP4_G_DIV = np.float32(2688.0)   # 448 * 6
 FP8_DIV = np.float32(448.0)
@@ -80,18 +87,18 @@ def smooth_k(k, mean):
     return (np.asarray(k, np.float32) - np.asarray(mean, np.float32)[:, :, None, :]).astype(np.float32)
 
 
-def quant_int8_blocks(x):
-    """Per-128-token-block symmetric INT8 (reading 3).
+def quant_int8_blocks(x, tokens=BLOCK):
+    """Symmetric INT8 with one scale per block of `tokens` tokens (reading 3).
 
     x: float32 [B, H, N, d].  Returns (codes int8 [B,H,N,d],
-    scales float32 [B,H,ceil(N/128)]).
+    scales float32 [B,H,ceil(N/tokens)]).
     """
     x = np.asarray(x, np.float32)
     B, H, N, d = x.shape
-    nb = -(-N // BLOCK)
+    nb = -(-N // tokens)
     codes = np.zeros((B, H, N, d), np.int8)
     scales = np.zeros((B, H, nb), np.float32)
-    for i, (s, e) in enumerate(_blocks(N)):
+    for i, (s, e) in enumerate(_blocks(N, tokens)):
         blk = x[:, :, s:e, :]
         amax = np.abs(blk).max(axis=(2, 3)).astype(np.float32)
         sc = (amax / INT8_DIV).astype(np.float32)
@@ -100,18 +107,18 @@ def quant_int8_blocks(x):
     return codes, scales
 
 
-def quant_fp8_blocks(x):
-    """Per-128-token-block FP8 e4m3 (reading 6).
+def quant_fp8_blocks(x, tokens=BLOCK):
+    """FP8 e4m3 with one scale per block of `tokens` tokens (reading 6).
 
     x: float32 [B, H, N, d].  Returns (codes uint8 e4m3 [B,H,N,d],
-    scales float32 [B,H,ceil(N/128)]).
+    scales float32 [B,H,ceil(N/tokens)]).
     """
     x = np.asarray(x, np.float32)
     B, H, N, d = x.shape
-    nb = -(-N // BLOCK)
+    nb = -(-N // tokens)
     codes = np.zeros((B, H, N, d), np.uint8)
     scales = np.zeros((B, H, nb), np.float32)
-    for i, (s, e) in enumerate(_blocks(N)):
+    for i, (s, e) in enumerate(_blocks(N, tokens)):
         blk = x[:, :, s:e, :]
         amax = np.abs(blk).max(axis=(2, 3)).astype(np.float32)
         sc = (amax / FP8_DIV).astype(np.float32)
@@ -125,22 +132,24 @@ def quant_fp8_blocks(x):
 def quant_qk_fp8(q, k):
     """FP8 Q/K mode pre-pass (reading 6; K smoothed as in reading 1).
 
-    Returns dict with q_codes, q_scales, k_codes, k_scales, k_mean.
+    Returns dict with q_codes, q_scales [B,H,N] (one per token), k_codes,
+    k_scales [B,H,ceil(N/32)], k_mean.
     """
     mean = k_channel_mean(k)
-    qc, qs = quant_fp8_blocks(np.asarray(q, np.float32))
-    kc, ks = quant_fp8_blocks(smooth_k(k, mean))
+    qc, qs = quant_fp8_blocks(np.asarray(q, np.float32), Q_GROUP)
+    kc, ks = quant_fp8_blocks(smooth_k(k, mean), K_GROUP)
     return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean)
 
 
 def quant_qk_int8(q, k):
-    """INT8 mode pre-pass for Q and K.
+    """INT8 mode pre-pass for Q and K (readings 1 and 3).
 
-    Returns dict with q_codes, q_scales, k_codes, k_scales, k_mean.
+    Returns dict with q_codes, q_scales [B,H,N] (one per token), k_codes,
+    k_scales [B,H,ceil(N/32)], k_mean.
     """
     mean = k_channel_mean(k)
-    qc, qs = quant_int8_blocks(np.asarray(q, np.float32))
-    kc, ks = quant_int8_blocks(smooth_k(k, mean))
+    qc, qs = quant_int8_blocks(np.asarray(q, np.float32), Q_GROUP)
+    kc, ks = quant_int8_blocks(smooth_k(k, mean), K_GROUP)
     return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean)
 
 

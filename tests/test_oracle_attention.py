@@ -146,14 +146,85 @@ def test_int8_blocks_properties():
             assert scales[0, h, i] == np.float32(np.float32(np.abs(blk).max()) / np.float32(127))
 
 
+@pytest.mark.parametrize("tokens", [1, 32])
+def test_int8_blocks_small_groups(tokens):
+    # the block rule holds for any group size: one scale per `tokens` tokens
+    # (the last group of a ragged head shorter), amax / 127, codes within
+    # half a step, the group max on +-127
+    x = rnd((1, 2, 77, 64), 117 + tokens, 2.0)
+    x[0, 1, 32:64] = 0.0                                 # zero groups
+    codes, scales = pp.quant_int8_blocks(x, tokens)
+    assert scales.shape == (1, 2, -(-77 // tokens))
+    for h in range(2):
+        for i in range(scales.shape[2]):
+            s, e = i * tokens, min((i + 1) * tokens, 77)
+            blk = x[0, h, s:e].astype(np.float64)
+            sc = float(scales[0, h, i])
+            if np.abs(blk).max() == 0:
+                assert sc == 0 and np.all(codes[0, h, s:e] == 0)
+                continue
+            assert np.abs(codes[0, h, s:e]).max() == 127
+            # the code is decided on the FP32 quotient, which may sit up to
+            # 127 * 2^-24 past a half step
+            assert np.all(np.abs(blk - codes[0, h, s:e] * sc) <= sc * (0.5 + 128 * 2.0 ** -24))
+
+
+def test_int8_qk_scales_pinned():
+    """Q takes one scale per token, smoothed K one per 32 tokens: planted
+    values make every scale and code a closed form.  Token t of Q has amax
+    127 * 2^e_t.  K is planted in (+x, -x) token pairs of one channel, so
+    every channel mean is exactly 0 and smoothing changes nothing; its
+    32-token block b has amax 127 * 2^f_b and its other values are
+    +-60 * 2^f_b.  A 128-token Q block, a 128-token or per-token K block, or
+    a 126 divisor each break the closed form."""
+    N, d = 128, 16
+    q = np.zeros((1, 1, N, d), np.float32)
+    k = np.zeros((1, 1, N, d), np.float32)
+    eq = (np.arange(N) % 7) - 3                          # per-token exponents -3..3
+    ek = np.array([-2, 1, 0, 3])                         # per-32-token-block exponents
+    want_qc = np.zeros((N, d), np.int8)
+    want_kc = np.zeros((N, d), np.int8)
+    for t in range(N):
+        c = t % d
+        q[0, 0, t, c] = 127.0 * 2.0 ** eq[t]
+        q[0, 0, t, (c + 5) % d] = -45.0 * 2.0 ** eq[t]
+        want_qc[t, c], want_qc[t, (c + 5) % d] = 127, -45
+        ck = (t // 2) % d
+        mag = 127 if t % 32 in (4, 5) else 60
+        sgn = 1 if t % 2 == 0 else -1
+        k[0, 0, t, ck] = sgn * mag * 2.0 ** ek[t // 32]
+        want_kc[t, ck] = sgn * mag
+    r = pp.quant_qk_int8(q, k)
+    assert np.all(r["k_mean"] == 0)
+    assert r["q_scales"].shape == (1, 1, N) and r["k_scales"].shape == (1, 1, 4)
+    np.testing.assert_array_equal(r["q_scales"][0, 0], (2.0 ** eq).astype(np.float32))
+    np.testing.assert_array_equal(r["q_codes"][0, 0], want_qc)
+    np.testing.assert_array_equal(r["k_scales"][0, 0], (2.0 ** ek).astype(np.float32))
+    np.testing.assert_array_equal(r["k_codes"][0, 0], want_kc)
+
+
 def test_quant_qk_smooths_k_only():
     q, k = rnd((1, 1, 256, 32), 18), rnd((1, 1, 256, 32), 19) + np.float32(10)
     r = pp.quant_qk_int8(q, k)
-    c2, s2 = pp.quant_int8_blocks(q)
+    c2, s2 = pp.quant_int8_blocks(q, 1)
     assert np.array_equal(r["q_codes"], c2) and np.array_equal(r["q_scales"], s2)
-    kc, ks = pp.quant_int8_blocks(k.astype(np.float32) - r["k_mean"][:, :, None, :])
+    kc, ks = pp.quant_int8_blocks(k.astype(np.float32) - r["k_mean"][:, :, None, :], 32)
     assert np.array_equal(r["k_codes"], kc) and np.array_equal(r["k_scales"], ks)
     assert np.all(np.abs(r["k_mean"] - 10) < 0.5)
+    assert r["q_scales"].shape == (1, 1, 256) and r["k_scales"].shape == (1, 1, 8)
+
+
+def test_query_rows_quantized_independently():
+    # one scale per query token: a huge value planted in one query row
+    # changes no other row's codes or output (bit for bit)
+    q, k, v = rnd((1, 1, 256, 32), 30), rnd((1, 1, 256, 32), 31), rnd((1, 1, 256, 32), 32)
+    o = att.emulated_sage_attention(q, k, v, True, 0.2)
+    q2 = q.copy()
+    q2[0, 0, 100, 3] = np.float32(1000.0)
+    o2 = att.emulated_sage_attention(q2, k, v, True, 0.2)
+    rows = np.arange(256) != 100
+    assert np.array_equal(o[0, 0, rows], o2[0, 0, rows])
+    assert not np.array_equal(o[0, 0, 100], o2[0, 0, 100])
 
 
 def test_fp8_v_properties():
@@ -478,10 +549,11 @@ def test_fp8_blocks_properties():
 def test_quant_qk_fp8_smooths_k_only():
     q, k = rnd((1, 1, 256, 32), 91), rnd((1, 1, 256, 32), 92) + np.float32(10)
     r = pp.quant_qk_fp8(q, k)
-    c2, s2 = pp.quant_fp8_blocks(q)
+    c2, s2 = pp.quant_fp8_blocks(q, 1)
     assert np.array_equal(r["q_codes"], c2) and np.array_equal(r["q_scales"], s2)
-    kc, ks = pp.quant_fp8_blocks(k.astype(np.float32) - r["k_mean"][:, :, None, :])
+    kc, ks = pp.quant_fp8_blocks(k.astype(np.float32) - r["k_mean"][:, :, None, :], 32)
     assert np.array_equal(r["k_codes"], kc) and np.array_equal(r["k_scales"], ks)
+    assert r["q_scales"].shape == (1, 1, 256) and r["k_scales"].shape == (1, 1, 8)
 
 
 @pytest.mark.parametrize("N", [256, 139])
