@@ -6,11 +6,13 @@
  *   - K is smoothed by subtracting its per-channel mean over tokens
  *     (SageAttention abstract, dblp author page on taxoreview.com: accurate
  *     8-bit attention; softmax is unchanged by a per-row shift);
- *   - Q and K are quantized per 128-token block to INT8 or FP8
+ *   - Q and K are quantized per block of tokens to INT8 or FP8
  *     ("Flash Attention vs Sage Attention: Kernel Comparison", section "How
- *     SageAttention uses quantization for more throughput"), or to FP4 with
- *     one UE4M3 scale per 16 elements (SageAttention3 abstract: FP4 tensor
- *     cores of Blackwell GPUs);
+ *     SageAttention uses quantization for more throughput") -- one scale
+ *     per query token and one per 32 keys, the granularity of the kernel's
+ *     threads (SageAttention2 abstract: "hardware-friendly thread-level
+ *     granularity") -- or to FP4 with one UE4M3 scale per 16 elements
+ *     (SageAttention3 abstract: FP4 tensor cores of Blackwell GPUs);
  *   - Q K^T runs on the tensor cores and is dequantized by the product of
  *     the scales;
  *   - an online (flash-style) softmax follows (kernel-comparison blog,
@@ -29,18 +31,20 @@
  *     `stream`; the library never synchronises it.
  *   - Supported shapes: d in {64, 128} (FP4 mode: d == 128); any N >= 0.
  *     A call with B, H or N equal to zero does nothing and returns SAGE_OK.
- *   - Ragged sequences: the quantization blocks are 128-token tiles, the
- *     last one holding N - 128 (Np/128 - 1) tokens.  Every code buffer is
- *     laid out for Np = N rounded up to a multiple of 128 (the rows or
- *     columns of the missing tokens hold zero codes); its scale covers the
- *     real tokens only; keys past N are masked out of the softmax.
+ *   - Ragged sequences: every code buffer is laid out for Np = N rounded
+ *     up to a multiple of 128 (the rows or columns of the missing tokens
+ *     hold zero codes); the last quantization block (32 K tokens, a 128-token
+ *     tile in FP4 mode) may be partial and its scale covers the real tokens
+ *     only; a block of missing tokens has scale 0; keys past N are masked
+ *     out of the softmax.
  *   - Return value: SAGE_OK (0) or a negative sage_status_t.  No exception
  *     or process exit crosses the ABI.  sage_status_string() describes the
  *     most recent error of the calling thread.
  *   - Quantized buffers (sizes from sage_buffer_bytes):
  *       INT8/FP8 and FP8 modes
  *         q_codes, k_codes  int8 (FP8 mode: e4m3) [B, H, Np, d]
- *         q_scales, k_scales float [B, H, Np/128]   one scale per 128 tokens
+ *         q_scales          float [B, H, Np]        one scale per token
+ *         k_scales          float [B, H, Np/32]     one scale per 32 tokens
  *         k_mean            float [B, H, d]
  *         v_codes           e4m3  [B, H, d, Np]     V transposed
  *         v_scales          float [B, H, d]         one scale per channel
@@ -80,8 +84,9 @@ typedef enum {
 } sage_status_t;
 
 /* INT8_FP8: INT8 Q/K, FP8 P~ and V.  FP4: FP4 Q/K/P~/V.  FP8: FP8 Q/K
- * (e4m3, per-block scale amax/448), FP8 P~ and V; its Q K^T accumulates in
- * FP32 on the tensor cores instead of exactly in INT32. */
+ * (e4m3, block scale amax/448 with the INT8 mode's blocks), FP8 P~ and V;
+ * its Q K^T accumulates in FP32 on the tensor cores instead of exactly in
+ * INT32. */
 typedef enum { SAGE_MODE_INT8_FP8 = 0, SAGE_MODE_FP4 = 1, SAGE_MODE_FP8 = 2 } sage_mode_t;
 typedef enum { SAGE_DTYPE_F16 = 0, SAGE_DTYPE_BF16 = 1 } sage_dtype_t;
 
@@ -97,8 +102,9 @@ size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, i
 
 /* Q/K pre-pass: K channel mean (FP64 accumulation: per 128-token chunk in
  * token order, then over chunks; mean = fp32(sum / N)), K smoothing
- * (one FP32 subtraction), then per-128-token-block quantization of Q and
- * of smoothed K.
+ * (one FP32 subtraction), then block quantization of Q (8-bit modes: one
+ * scale per token) and of smoothed K (8-bit modes: one scale per 32
+ * tokens), amax taken over the block's tokens and all d channels.
  *   INT8 mode: s = fp32(amax / 127); code = clamp(rne(fp32(x / s)), +-127);
  *              q_sf, k_sf must be NULL.
  *   FP8 mode:  s = fp32(amax / 448); code = e4m3(fp32(x / s)); q_sf, k_sf

@@ -419,8 +419,11 @@ size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, i
       // padded to whole 128-token tiles (the padding holds zero codes)
       return (size_t)(fp4 ? BH * nt * 128 * d / 2 : BH * nt * 128 * d);
     case SAGE_BUF_Q_SCALES:
+      // 8-bit modes: one scale per token; FP4: one tile scale per 128 tokens
+      return (size_t)(fp4 ? BH * nt * 4 : BH * nt * 128 * 4);
     case SAGE_BUF_K_SCALES:
-      return (size_t)(BH * nt * 4);
+      // 8-bit modes: one scale per 32 tokens; FP4: one tile scale per 128
+      return (size_t)(fp4 ? BH * nt * 4 : BH * nt * 4 * 4);
     case SAGE_BUF_Q_SF:
     case SAGE_BUF_K_SF:
       return fp4 ? (size_t)(BH * nt * ((d + 63) / 64) * 512) : 0;

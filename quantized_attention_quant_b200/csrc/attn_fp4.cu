@@ -42,8 +42,15 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "exp2_poly.cuh"
 #include "sage_internal.h"
 #include "sage_ptx.cuh"
+
+// Of every 8 groups of 4 scores in the exp pass, how many take 2^t from the
+// FMA-pipe polynomial (exp2_poly.cuh) instead of the SFU.
+#ifndef SAGE_FP4_EXP_POLY_GROUPS
+#define SAGE_FP4_EXP_POLY_GROUPS 2
+#endif
 
 namespace sage {
 namespace {
@@ -237,7 +244,13 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
         __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), c2, n2);
     const float2 t23 =
         __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), c2, n2);
-    float f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
+    float f0, f1, f2, f3;
+    if (((i >> 2) * SAGE_FP4_EXP_POLY_GROUPS) % 8 < SAGE_FP4_EXP_POLY_GROUPS) {
+      const float2 e01 = exp2_poly2(t01), e23 = exp2_poly2(t23);
+      f0 = e01.x, f1 = e01.y, f2 = e23.x, f3 = e23.y;
+    } else {
+      f0 = ex2(t01.x), f1 = ex2(t01.y), f2 = ex2(t23.x), f3 = ex2(t23.y);
+    }
     if (MASKED) {
       f0 = (col0 + i + 0 <= lim) ? f0 : 0.f;
       f1 = (col0 + i + 1 <= lim) ? f1 : 0.f;

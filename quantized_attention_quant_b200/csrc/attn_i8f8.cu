@@ -9,7 +9,9 @@
 //   per query row, over 128-key tiles j (causal: j <= query tile):
 //     A      = q_codes . k_codes_j^T                 (tcgen05 kind::i8, exact;
 //                                                     FP8 Q/K: kind::f8f6f4, FP32)
-//     t      = A * (s_Q s_Kj sm_scale log2 e)        (log2 domain)
+//     t      = A * (s_Q s_K sm_scale log2 e)         (log2 domain; s_Q of the
+//                                                     query token, s_K of the
+//                                                     key's 32-key block)
 //     m_j    = max(m_{j-1}, rowmax t); alpha_j = 2^(m_{j-1} - m_j)
 //     p      = e4m3(448 * 2^(t - m_j))               (448 P~, quantized)
 //     l      = alpha_j l + sum 448 P~                (unquantized P~)
@@ -21,15 +23,13 @@
 // the throughput limit (the tensor core finishes a 128x128 tile in far fewer
 // cycles than the SFU needs for its 16K exponentials; one warp per SM
 // sub-partition keeps the SFU only about half busy, two about 80 %), so two
-// warpgroups share every tile.  The scores stay biased floats end to end:
-// an integer add or an int-to-float conversion per score costs the exp
-// pass about a third of its SFU rate.  Warp roles (512 threads):
+// warpgroups share every tile.  Warp roles (512 threads):
 //   warpgroup 0: warp 0 TMA producer (Q once, K_j and V_j^T rings),
 //                warp 1 TMEM allocator and single-thread tcgen05 issuer
 //   warpgroups 1, 2 ("exp"): key columns 0..63 / 64..127 of every tile.
 //                Thread = query row = TMEM lane.  448 P~ as e4m3 codes into
-//                a TMEM tile (the A operand of the P~V MMA, read from TMEM),
-//                the row sum, and the bias written back into S.
+//                a TMEM tile (the A operand of the P~V MMA, read from TMEM)
+//                and the row sum.
 //   warpgroup 3 ("stats"): per key tile the row max, the running max m_j and
 //                alpha_j (published for both exp warpgroups), then the level-2
 //                fold of the tile's FP32 partial into the running FP32
@@ -39,15 +39,18 @@
 // P~[0] 384..415, P~[1] 416..447 (four e4m3 codes per column, keys
 // 64h .. 64h+63 in columns 16h .. 16h+15).  Key tile j uses S[j % SB],
 // PV[j % 2] (folded two tiles behind) and P~[j % 2].  The exp warpgroups
-// read their S columns first, write the bias back and release S at once,
-// so the next Q K^T runs while they work on the exponentials; the MMA
-// thread issues it ahead of the P~V of the previous tile.  Before each
-// Q K^T the S columns hold the bit pattern of 1.5 * 2^23; the INT8 MMA
-// accumulates onto it, so a score reads back as the float
-// 1.5*2^23 + A exactly (|A| <= 127^2*128 < 2^22) with no conversion
-// instruction.  The FP8 Q/K variant (QF8; the kernel-comparison blog's
-// "INT8 or FP8" queries and keys) runs the same pipeline with an FP32
-// Q K^T that overwrites S, so it has no bias to write back or remove.
+// read their S columns first and release S at once, so the next Q K^T runs
+// while they work on the exponentials; the MMA thread issues it ahead of
+// the P~V of the previous tile.  Each Q K^T overwrites S: the INT8 scores
+// are INT32, which the exp warpgroups turn into floats with one integer add
+// each (score() in attn_i8f8_common.cuh; TMEM stores are about a third as
+// fast as loads, so writing a float bias back into S for the next MMA to
+// accumulate onto cost more); the stats warpgroup takes the row maximum on
+// the integers.  The FP8 Q/K variant (QF8; the kernel-comparison blog's
+// "INT8 or FP8" queries and keys) runs the same pipeline with FP32 scores.
+// Dequantization: the Q scale is the row's (one per token), the K scale the
+// 32-key chunk's (one per 32 keys), so every thread applies one factor per
+// chunk of 32 scores it holds.
 // Every barrier wait is bounded; an expired wait sets the device status
 // word and makes every role leave its loop.
 
@@ -98,7 +101,7 @@ struct Layout {
   static constexpr int OFF_ABORT = OFF_MISC + 528;
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
-  static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots] dequant factor of the tile
+  static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots][4] s_K sm_scale log2 e per 32 keys
   static constexpr int OFF_VS = OFF_C + 128;         // s_V[D] of the head (bulk-copied with Q)
   static constexpr int END = OFF_VS + 4 * D;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
@@ -117,9 +120,9 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;
   uint64_t* v_empty;
-  uint64_t* s_init;    // [1] exp -> MMA: the S buffers hold the bias
-  uint64_t* s_full;    // [SB] MMA -> stats: S[b] holds bias + Q K_j^T
-  uint64_t* s_ready;   // [SB] exp -> MMA: S[b] read and re-biased
+  uint64_t* s_init;    // [1] exp -> MMA: the exp warpgroups are running
+  uint64_t* s_full;    // [SB] MMA -> stats: S[b] holds Q K_j^T
+  uint64_t* s_ready;   // [SB] exp -> MMA: S[b] read
   uint64_t* m_full;    // [2] stats -> exp: m_j, alpha_j of tile j (slot j % 2)
   uint64_t* p_full;    // [2] exp -> MMA: P~[b] written
   uint64_t* p_empty;   // [2] MMA -> exp: P~[b] read by the P~V MMA
@@ -157,7 +160,9 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
 // last key tile masks keys n_tail .. 127.
 template <int D, bool CAUSAL, bool QF8, bool RAGGED>
 __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
-                                         const uint32_t tmem, const Bars& bar, uint8_t* smem,
+                                         const int bh, const int ntiles,
+                                         const float* __restrict__ q_scales, const uint32_t tmem,
+                                         const Bars& bar, uint8_t* smem,
                                          volatile int* abort_flag, uint32_t* status) {
   using L = Layout<D>;
   const int warp = threadIdx.x >> 5;
@@ -168,17 +173,11 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
   const float* m_s = reinterpret_cast<const float*>(smem + L::OFF_M);
   const float* c_s = reinterpret_cast<const float*>(smem + L::OFF_C);
   float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
+  // this row's Q scale (one per token); padding rows of a ragged tile read
+  // the scale 0 the pre-pass wrote there
+  const float qs = __ldg(q_scales + ((int64_t)bh * ntiles + qt) * 128 + r);
 
-  // the first Q K^T into each S buffer accumulates onto the bias (the FP8
-  // Q K^T overwrites S instead)
-  if (!QF8) {
-#pragma unroll
-    for (int b = 0; b < L::SB; ++b) {
-      tmem_fill32(tmem + lanes + 128u * b + 64u * h, kBiasBits);
-      tmem_fill32(tmem + lanes + 128u * b + 64u * h + 32u, kBiasBits);
-    }
-    tmem_wait_st();
-  }
+  // (every Q K^T overwrites S: nothing to prepare in TMEM)
   tc_fence_before();
   mbar_arrive(bar.s_init);
 
@@ -194,7 +193,9 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
       return;
     tc_fence_after();
     if (r == 0) SAGE_TR(h, j);
-    const float c = c_s[b];
+    // dequant factors of this warpgroup's two 32-key chunks (the stats
+    // warpgroup forms its maximum from the same products)
+    const float ca = qs * c_s[4 * b + 2 * h], cb = qs * c_s[4 * b + 2 * h + 1];
     const float m_j = m_s[(2 * b) * 128 + r];
     const float alpha = m_s[(2 * b + 1) * 128 + r];
     const float neg = kLog2_448 - m_j;  // yields 448 P~ directly
@@ -212,23 +213,18 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     tmem_wait_ld_regs(sa);
     reg_fence(sb);
     if (r == 0 && h == 0) SAGE_TR(13, j);
-    // S read: the bias back, and S free for the next Q K^T into it
-    if (!QF8) {
-      tmem_fill32(S, kBiasBits);
-      tmem_fill32(S + 32, kBiasBits);
-      tmem_wait_st();
-    }
+    // S read: free for the next Q K^T into it
     tc_fence_before();
     mbar_arrive(&bar.s_ready[sbuf]);
     // P~[b] is free once the P~V MMA of tile j - 2 has read it
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, c, neg, lim, P)
-                       : exp_chunk<false, QF8>(sa, 2 * h, c, neg, lim, P);
+    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, ca, neg, lim, P)
+                       : exp_chunk<false, QF8>(sa, 2 * h, ca, neg, lim, P);
     if (r == 0 && h == 0) SAGE_TR(14, j);
-    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, c, neg, lim, P + 8)
-                  : exp_chunk<false, QF8>(sb, 2 * h + 1, c, neg, lim, P + 8);
+    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8)
+                  : exp_chunk<false, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8);
     l = fmaf(alpha, l, sum);
     if (r == 0 && h == 0) SAGE_TR(10, j);
     tmem_wait_st();
@@ -260,8 +256,9 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
   float* m_s = reinterpret_cast<float*>(smem + L::OFF_M);
   const float* l_s = reinterpret_cast<const float*>(smem + L::OFF_L);
-  const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
-  const float* ksp = k_scales + (int64_t)kv_head(bh, H, G) * ntiles;
+  // this row's Q scale; the K/V head's K scales, four per key tile
+  const float qs = __ldg(q_scales + ((int64_t)bh * ntiles + qt) * 128 + r);
+  const float* ksp = k_scales + (int64_t)kv_head(bh, H, G) * ntiles * 4;
 
   float2 o2[D / 2];
 #pragma unroll
@@ -296,11 +293,14 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   // exp warpgroups wait for) never queues behind the P~V product of tile j.
   float alpha_hist[2] = {0.f, 0.f};
   float* c_s = reinterpret_cast<float*>(smem + L::OFF_C);
-  float ks_cur = ldg_early(ksp);
+  float4 ks_cur = ldg4_early(ksp);
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
-    const float c = qs * ks_cur * scale_log2;
-    const float ks_nxt = j + 1 < nkv ? ldg_early(ksp + j + 1) : 0.f;
+    // s_K sm_scale log2 e of the tile's four 32-key chunks; a row's factor
+    // is its Q scale times that (the exp warpgroups form the same products)
+    const float kl[4] = {ks_cur.x * scale_log2, ks_cur.y * scale_log2, ks_cur.z * scale_log2,
+                         ks_cur.w * scale_log2};
+    const float4 ks_nxt = j + 1 < nkv ? ldg4_early(ksp + 4 * (j + 1)) : make_float4(0.f, 0.f, 0.f, 0.f);
     const int sbuf = j % L::SB;
     if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[sbuf], (j / L::SB) & 1, abort_flag,
                                            status, kDevTimeoutMma)))
@@ -311,7 +311,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     const bool masked = diag || (RAGGED && j == nkv - 1);
     const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
-    float mx = QF8 ? -INFINITY : 0.f;
+    float mx = -INFINITY;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       uint32_t s[2][32];
@@ -319,16 +319,23 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      mx = masked ? max64<true, QF8>(&s[0][0], 64 * hh, lim, mx)
-                  : max64<false, QF8>(&s[0][0], 64 * hh, lim, mx);
+      // each chunk's factor is >= 0, so its scaled max is the max scaled
+      mx = masked ? scaled_max64<true, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                            qs * kl[2 * hh + 1], mx)
+                  : scaled_max64<false, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                             qs * kl[2 * hh + 1], mx);
     }
-    // c >= 0, so the max of the scaled scores is the scaled max
-    const float m_j = fmaxf(m, (QF8 ? mx : mx - kBias) * c);
+    const float m_j = fmaxf(m, mx);
     const float alpha = ex2(m - m_j);
     m = m_j;
     m_s[(2 * b) * 128 + r] = m_j;
     m_s[(2 * b + 1) * 128 + r] = alpha;
-    if (r == 0) c_s[b] = c;
+    if (r == 0) {
+      c_s[4 * b] = kl[0];
+      c_s[4 * b + 1] = kl[1];
+      c_s[4 * b + 2] = kl[2];
+      c_s[4 * b + 3] = kl[3];
+    }
     if (r == 0) SAGE_TR(5, j);
     // S[b] has been read: the exp warpgroups may overwrite it with P~ codes
     tc_fence_before();
@@ -476,7 +483,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         constexpr uint32_t idesc_pv = make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, D);
         const uint64_t qdesc = make_sdesc(smem_u32(sQ), L::QK_SBO, 16, L::QK_SWZ);
         bool ok = mbar_wait(bar.q_full, 0, abort_flag, status, kDevTimeoutTma);
-        // S[j % SB] = bias + Q K_j^T
+        // S[j % SB] = Q K_j^T
         auto qk = [&](int j) -> bool {
           const int sk = j % L::KS;
           const int sbuf = j % L::SB;
@@ -492,7 +499,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               mma_f8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk,
                         kk > 0);
             else
-              mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
+              mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk,
+                        kk > 0);
           }
           mma_commit(&bar.s_full[sbuf]);
           mma_commit(&bar.k_empty[sk]);
@@ -557,7 +565,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
+    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, qt, nkv, n_tail, bh, ntiles, q_scales, tmem, bar,
+                                     smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
     stats_loop<D, CAUSAL, OutT, QF8, RAGGED>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,

@@ -42,7 +42,7 @@ struct Layout {
   static constexpr int OFF_ABORT = OFF_MISC + 528;
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [3 items][2 halves][128] row sums
-  static constexpr int OFF_C = OFF_L + 6 * 128 * 4;  // [2 slots] dequant factor of the tile
+  static constexpr int OFF_C = OFF_L + 6 * 128 * 4;  // [2 slots][4] s_K sm_scale log2 e per 32 keys
   static constexpr int OFF_VS = OFF_C + 128;         // [3][D] s_V of an item (bulk-copied)
   static constexpr int END = OFF_VS + 3 * 4 * D;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
@@ -66,9 +66,9 @@ struct Bars {
   uint64_t* k_empty;
   uint64_t* v_full;
   uint64_t* v_empty;
-  uint64_t* s_init;    // [1] exp -> MMA: the S buffers hold the bias
-  uint64_t* s_full;    // [SB] MMA -> stats: S[b] holds bias + Q K_j^T
-  uint64_t* s_ready;   // [SB] exp -> MMA: S[b] read and re-biased
+  uint64_t* s_init;    // [1] exp -> MMA: the exp warpgroups are running
+  uint64_t* s_full;    // [SB] MMA -> stats: S[b] holds Q K_j^T
+  uint64_t* s_ready;   // [SB] exp -> MMA: S[b] read
   uint64_t* m_full;    // [2] stats -> exp: m_j, alpha_j of tile j (slot j % 2)
   uint64_t* p_full;    // [2] exp -> MMA: P~[b] written
   uint64_t* p_empty;   // [2] MMA -> exp: P~[b] read by the P~V MMA
@@ -151,7 +151,8 @@ struct Cursor {
 // partial): the last key tile of an item masks keys n_tail .. 127.
 template <int D, bool CAUSAL, bool QF8, bool RAGGED>
 __device__ __forceinline__ void exp_loop(const int h, const Sched& sch, const int T,
-                                         const int n_tail, const uint32_t tmem, const Bars& bar,
+                                         const int n_tail, const float* __restrict__ q_scales,
+                                         const uint32_t tmem, const Bars& bar,
                                          uint8_t* smem, volatile int* abort_flag,
                                          uint32_t* status) {
   using L = Layout<D>;
@@ -164,16 +165,7 @@ __device__ __forceinline__ void exp_loop(const int h, const Sched& sch, const in
   const float* c_s = reinterpret_cast<const float*>(smem + L::OFF_C);
   float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
 
-  // the first Q K^T into each S buffer accumulates onto the bias (the FP8
-  // Q K^T overwrites S instead)
-  if (!QF8) {
-#pragma unroll
-    for (int b = 0; b < L::SB; ++b) {
-      tmem_fill32(tmem + lanes + 128u * b + 64u * h, kBiasBits);
-      tmem_fill32(tmem + lanes + 128u * b + 64u * h + 32u, kBiasBits);
-    }
-    tmem_wait_st();
-  }
+  // (every Q K^T overwrites S: nothing to prepare in TMEM)
   tc_fence_before();
   mbar_arrive(bar.s_init);
 
@@ -181,17 +173,21 @@ __device__ __forceinline__ void exp_loop(const int h, const Sched& sch, const in
   cur.load(sch, blockIdx.x, 0);
   // l restarts at every item by itself: the first tile's alpha is 0
   float l = 0.f;
+  float qs = 0.f;  // this row's Q scale in the current item
   for (int g = 0; g < T; ++g, cur.next(sch, blockIdx.x)) {
     const int j = cur.j;
     const int b = g & 1;
     const uint32_t ph = (g >> 1) & 1;
+    if (j == 0) qs = __ldg(q_scales + ((int64_t)cur.bh * sch.ntiles + cur.qt) * 128 + r);
     // m_full(g) is published by the stats warpgroup after it waited for
     // s_full(g) and read S[b]: it orders this warpgroup after the Q K^T too
     if (!__all_sync(0xffffffffu,
                     mbar_wait(&bar.m_full[b], ph, abort_flag, status, kDevTimeoutEpi)))
       return;
     tc_fence_after();
-    const float c = c_s[b];
+    // dequant factors of this warpgroup's two 32-key chunks (the stats
+    // warpgroup forms its maximum from the same products)
+    const float ca = qs * c_s[4 * b + 2 * h], cb = qs * c_s[4 * b + 2 * h + 1];
     const float m_j = m_s[(2 * b) * 128 + r];
     const float alpha = m_s[(2 * b + 1) * 128 + r];
     const float neg = kLog2_448 - m_j;  // yields 448 P~ directly
@@ -208,22 +204,17 @@ __device__ __forceinline__ void exp_loop(const int h, const Sched& sch, const in
     tmem_ld32(S + 32, sb);
     tmem_wait_ld_regs(sa);
     reg_fence(sb);
-    // S read: the bias back, and S free for the next Q K^T into it
-    if (!QF8) {
-      tmem_fill32(S, kBiasBits);
-      tmem_fill32(S + 32, kBiasBits);
-      tmem_wait_st();
-    }
+    // S read: free for the next Q K^T into it
     tc_fence_before();
     mbar_arrive(&bar.s_ready[sbuf]);
     // P~[b] is free once the P~V MMA of tile g - 2 has read it
     if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, c, neg, lim, P)
-                       : exp_chunk<false, QF8>(sa, 2 * h, c, neg, lim, P);
-    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, c, neg, lim, P + 8)
-                  : exp_chunk<false, QF8>(sb, 2 * h + 1, c, neg, lim, P + 8);
+    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, ca, neg, lim, P)
+                       : exp_chunk<false, QF8>(sa, 2 * h, ca, neg, lim, P);
+    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8)
+                  : exp_chunk<false, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8);
     l = fmaf(alpha, l, sum);
     tmem_wait_st();
     tc_fence_before();
@@ -348,7 +339,8 @@ __device__ __forceinline__ void stats_loop(const Sched& sch, const int T, const 
   float alpha_hist[2] = {0.f, 0.f};
   Cursor<CAUSAL> mc;  // tile whose max is taken
   mc.load(sch, blockIdx.x, 0);
-  float m = -INFINITY, qs = 0.f, ks_cur = 0.f;
+  float m = -INFINITY, qs = 0.f;
+  float4 ks_cur = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* ksp = k_scales;
   // one pass: the max of tile g (g < T), then the fold of tile g - PVB
   for (int g = 0; g < T + L::PVB; ++g) {
@@ -359,12 +351,16 @@ __device__ __forceinline__ void stats_loop(const Sched& sch, const int T, const 
       if (j == 0) {
         // a new item: its Q scale, its head's K scales, a fresh running max
         m = -INFINITY;
-        qs = __ldg(q_scales + (int64_t)mc.bh * ntiles + mc.qt);
-        ksp = k_scales + (int64_t)kv_head(mc.bh, H, G) * ntiles;
-        ks_cur = __ldg(ksp);
+        qs = __ldg(q_scales + ((int64_t)mc.bh * ntiles + mc.qt) * 128 + r);
+        ksp = k_scales + (int64_t)kv_head(mc.bh, H, G) * ntiles * 4;
+        ks_cur = __ldg(reinterpret_cast<const float4*>(ksp));
       }
-      const float c = qs * ks_cur * scale_log2;
-      const float ks_nxt = j + 1 < mc.nkv ? ldg_early(ksp + j + 1) : 0.f;
+      // s_K sm_scale log2 e of the tile's four 32-key chunks; a row's factor
+      // is its Q scale times that (the exp warpgroups form the same products)
+      const float kl[4] = {ks_cur.x * scale_log2, ks_cur.y * scale_log2, ks_cur.z * scale_log2,
+                           ks_cur.w * scale_log2};
+      const float4 ks_nxt =
+          j + 1 < mc.nkv ? ldg4_early(ksp + 4 * (j + 1)) : make_float4(0.f, 0.f, 0.f, 0.f);
       const int sbuf = g % L::SB;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[sbuf], (g / L::SB) & 1, abort_flag,
                                              status, kDevTimeoutMma)))
@@ -374,7 +370,7 @@ __device__ __forceinline__ void stats_loop(const Sched& sch, const int T, const 
       const bool masked = diag || (RAGGED && j == mc.nkv - 1);
       const int lim = diag ? r : n_tail - 1;
       const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
-      float mx = QF8 ? -INFINITY : 0.f;
+      float mx = -INFINITY;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t s[2][32];
@@ -382,16 +378,23 @@ __device__ __forceinline__ void stats_loop(const Sched& sch, const int T, const 
         tmem_ld32(S + 64 * hh + 32, s[1]);
         tmem_wait_ld_regs(s[0]);
         reg_fence(s[1]);
-        mx = masked ? max64<true, QF8>(&s[0][0], 64 * hh, lim, mx)
-                    : max64<false, QF8>(&s[0][0], 64 * hh, lim, mx);
+        // each chunk's factor is >= 0, so its scaled max is the max scaled
+        mx = masked ? scaled_max64<true, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                              qs * kl[2 * hh + 1], mx)
+                    : scaled_max64<false, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                               qs * kl[2 * hh + 1], mx);
       }
-      // c >= 0, so the max of the scaled scores is the scaled max
-      const float m_j = fmaxf(m, (QF8 ? mx : mx - kBias) * c);
+      const float m_j = fmaxf(m, mx);
       alpha = ex2(m - m_j);
       m = m_j;
       m_s[(2 * b) * 128 + r] = m_j;
       m_s[(2 * b + 1) * 128 + r] = alpha;
-      if (r == 0) c_s[b] = c;
+      if (r == 0) {
+        c_s[4 * b] = kl[0];
+        c_s[4 * b + 1] = kl[1];
+        c_s[4 * b + 2] = kl[2];
+        c_s[4 * b + 3] = kl[3];
+      }
       // S[b] has been read: the exp warpgroups may overwrite it with P~ codes
       tc_fence_before();
       mbar_arrive(&bar.m_full[b]);
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
         constexpr uint32_t idesc_pv = make_idesc(1 /*F32*/, 0 /*e4m3*/, 0 /*e4m3*/, 128, D);
         Cursor<CAUSAL> qc;  // item of the next Q K^T
         qc.load(sch, c, 0);
-        // S[g % SB] = bias + Q K_g^T (Q of the tile's item)
+        // S[g % SB] = Q K_g^T (Q of the tile's item)
         auto qk = [&](int g) -> bool {
           const int sk = g % L::KS;
           const int sbuf = g % L::SB;
@@ -579,7 +582,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
               mma_f8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk,
                         kk > 0);
             else
-              mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk, 1);
+              mma_i8_ss(tmem + (uint32_t)sbuf * 128u, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk,
+                        kk > 0);
           }
           mma_commit(&bar.s_full[sbuf]);
           mma_commit(&bar.k_empty[sk]);
@@ -647,7 +651,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, sch, T, n_tail, tmem, bar, smem, abort_flag, status);
+    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, sch, T, n_tail, q_scales, tmem, bar, smem, abort_flag,
+                                     status);
   } else {
     setmaxnreg_inc<kRegsStats>();
     stats_loop<D, CAUSAL, OutT, QF8, RAGGED>(sch, T, n_tail, H, G, tmem, bar, smem, abort_flag,

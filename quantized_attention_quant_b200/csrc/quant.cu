@@ -332,18 +332,28 @@ __device__ __forceinline__ void role_stats(const PrepassPtrs& p, int64_t bh, int
 
 // ------------------------------------------------------- INT8 / FP8 Q / K
 // Load, (smooth), block amax, s = amax / 127, codes = clamp(rne(x / s))
-// (FP8: s = amax / 448, codes = e4m3(x / s)).
-// Two passes over the 128-token tile: the amax pass keeps nothing, the code
-// pass reads the tile again (from L1/L2), so the role needs few registers and
-// many CTAs fit on an SM.  A thread's vectors all cover the same 8 channels.
+// (FP8: s = amax / 448, codes = e4m3(x / s)).  Blocks of GROUP tokens:
+// GROUP = 1 (Q: one scale per query row) or 32 (K: one scale per 32 keys).
+// Two passes over the 128-token tile: the amax pass keeps one maximum per
+// vector, the code pass reads the tile again (from L1/L2), so the role needs
+// few registers and many CTAs fit on an SM.  A thread's vectors all cover
+// the same 8 channels: vector i of thread t holds token t / (D/8) + TPI i.
 // SHARED: the tile and the mean are in shared memory (the cluster-fused
-// pre-pass), else in global memory.
-template <typename T, int D, bool FP8, bool RAGGED, bool SHARED = false>
+// pre-pass), else in global memory.  scale_out: the tile's first scale
+// (128 per tile for GROUP = 1, 4 for GROUP = 32); red: 4 * kThreads / 32
+// floats of shared memory.
+template <typename T, int D, bool FP8, bool RAGGED, int GROUP, bool SHARED = false>
 __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const float* mean,
                                                 uint8_t* __restrict__ dst, float* scale_out,
                                                 float* red, int nv) {
+  static_assert(GROUP == 1 || GROUP == 32, "Q scales per token, K scales per 32 tokens");
   constexpr int VPT = 128 * D / 8 / kThreads;  // 16-byte vectors per thread
-  const int c0 = (threadIdx.x % (D / 8)) * 8;
+  constexpr int VPTOK = D / 8;                 // vectors per token
+  constexpr int TPI = kThreads / VPTOK;        // tokens between a thread's vectors
+  constexpr int VPB = 32 / TPI;                // a thread's vectors per 32-token block
+  static_assert(VPB * TPI == 32 && VPT / VPB == 4, "four 32-token blocks per tile");
+  const int tok0 = threadIdx.x / VPTOK;
+  const int c0 = (threadIdx.x % VPTOK) * 8;
   // x - mu as x + (-mu): the same single rounding
   float nmu[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (mean) {
@@ -364,36 +374,76 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
       }
     }
   };
-  // tokens nv..127 (padding of a ragged sequence) re-read a real token, so
-  // the block maximum is unchanged, and get code 0
-  float amax = 0.f;
+  // tokens nv..127 (padding of a ragged sequence) re-read the last real
+  // token, so no maximum of a block holding real tokens changes; they get
+  // code 0, and a block of padding only gets scale 0
+  float amax[VPT];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
-    // a padding vector re-reads a real one: it changes no maximum
     const int vec = threadIdx.x + i * kThreads;
     float x[8];
     load8<T, SHARED>(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
     smooth(x);
+    float a = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+    for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
+    amax[i] = a;
   }
-  amax = block_max(amax, red);
-  const float s = __fdiv_rn(amax, FP8 ? 448.f : 127.f);
-  const float rs = recip_or_zero(s);
+  float s[GROUP == 1 ? VPT : 4];
+  if constexpr (GROUP == 1) {
+    // one token's vectors sit in VPTOK consecutive lanes
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      float a = amax[i];
+#pragma unroll
+      for (int o = VPTOK / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      const int tok = tok0 + TPI * i;
+      s[i] = (RAGGED && tok >= nv) ? 0.f : __fdiv_rn(a, FP8 ? 448.f : 127.f);
+      if (threadIdx.x % VPTOK == 0) scale_out[tok] = s[i];
+    }
+  } else {
+    // the four block maxima over the whole CTA
+    float bm[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float a = amax[VPB * b];
+#pragma unroll
+      for (int v = 1; v < VPB; ++v) a = fmaxf(a, amax[VPB * b + v]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      bm[b] = a;
+    }
+    const int w = threadIdx.x >> 5;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) red[4 * w + b] = bm[b];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      float a = red[b];
+#pragma unroll
+      for (int i = 1; i < kThreads / 32; ++i) a = fmaxf(a, red[4 * i + b]);
+      s[b] = (RAGGED && 32 * b >= nv) ? 0.f : __fdiv_rn(a, FP8 ? 448.f : 127.f);
+    }
+    if (threadIdx.x < 4) scale_out[threadIdx.x] = s[threadIdx.x];
+  }
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vec = threadIdx.x + i * kThreads;
+    const float si = s[GROUP == 1 ? i : i / VPB];
     uint2 w = make_uint2(0u, 0u);
-    if (s != 0.f) {
+    if (si != 0.f) {
+      const float rs = recip_or_zero(si);
       float x[8];
       load8<T, SHARED>(src + clamp_vec<D, RAGGED>(vec, nv) * 8, x);
       smooth(x);
-      w = FP8 ? fp8_codes8(x, s, rs) : int8_codes8(x, s, rs);
+      w = FP8 ? fp8_codes8(x, si, rs) : int8_codes8(x, si, rs);
     }
-    if (RAGGED && vec / (D / 8) >= nv) w = make_uint2(0u, 0u);
+    if (RAGGED && vec / VPTOK >= nv) w = make_uint2(0u, 0u);
     *reinterpret_cast<uint2*>(dst + vec * 8) = w;
   }
-  if (threadIdx.x == 0) *scale_out = s;
 }
 
 // ---------------------------------------------------------------- FP8 V
@@ -658,7 +708,7 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   constexpr int SMEM_BYTES = V4_BYTES > TILE_BYTES ? V4_BYTES : TILE_BYTES;
   __shared__ __align__(16) uint8_t smem_raw[SMEM_BYTES];
   __shared__ uint32_t vmax_s[D];
-  __shared__ float red[kThreads / 32];
+  __shared__ float red[4 * (kThreads / 32)];
   const int role = roles.r[blockIdx.z];
   const int64_t bh = roles.reverse ? (int64_t)(gridDim.y - 1 - blockIdx.y) : (int64_t)blockIdx.y;
   const int tile = roles.reverse ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
@@ -675,27 +725,29 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   switch (role) {
     case kQuantQ8:
       SAGE_ROLE(kQuantQ8)
-      role_quant_8bit<T, D, false, RAGGED>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+      role_quant_8bit<T, D, false, RAGGED, 1>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
                                    reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * D,
-                                   p.q_scales + bh * ntiles + tile, red, nv);
+                                   p.q_scales + crow0, red, nv);
       break;
     case kQuantK8:
       SAGE_ROLE(kQuantK8)
-      role_quant_8bit<T, D, false, RAGGED>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+      role_quant_8bit<T, D, false, RAGGED, 32>(reinterpret_cast<const T*>(p.k) + row0 * D,
+                                   p.k_mean + bh * D,
                                    reinterpret_cast<uint8_t*>(p.k_codes) + crow0 * D,
-                                   p.k_scales + bh * ntiles + tile, red, nv);
+                                   p.k_scales + crow0 / 32, red, nv);
       break;
     case kQuantQF8:
       SAGE_ROLE(kQuantQF8)
-      role_quant_8bit<T, D, true, RAGGED>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
+      role_quant_8bit<T, D, true, RAGGED, 1>(reinterpret_cast<const T*>(p.q) + row0 * D, nullptr,
                                   reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * D,
-                                  p.q_scales + bh * ntiles + tile, red, nv);
+                                  p.q_scales + crow0, red, nv);
       break;
     case kQuantKF8:
       SAGE_ROLE(kQuantKF8)
-      role_quant_8bit<T, D, true, RAGGED>(reinterpret_cast<const T*>(p.k) + row0 * D, p.k_mean + bh * D,
+      role_quant_8bit<T, D, true, RAGGED, 32>(reinterpret_cast<const T*>(p.k) + row0 * D,
+                                  p.k_mean + bh * D,
                                   reinterpret_cast<uint8_t*>(p.k_codes) + crow0 * D,
-                                  p.k_scales + bh * ntiles + tile, red, nv);
+                                  p.k_scales + crow0 / 32, red, nv);
       break;
     case kQuantV8:
       SAGE_ROLE(kQuantV8)
@@ -763,7 +815,7 @@ __global__ void __cluster_dims__(kFusedCluster, 1, 1) __launch_bounds__(kThreads
   __shared__ double ksum_s[D];
   __shared__ uint32_t vmax_s[D];
   __shared__ __align__(16) float stat_s[D];  // the head's K mean or s_V
-  __shared__ float red[kThreads / 32];
+  __shared__ float red[4 * (kThreads / 32)];
   __shared__ int abort_flag;
   const int role = blockIdx.z;
   const int64_t bh = blockIdx.y;
@@ -800,9 +852,9 @@ __global__ void __cluster_dims__(kFusedCluster, 1, 1) __launch_bounds__(kThreads
 
   if (role == 0) {
     if (has)
-      role_quant_8bit<T, D, FP8, RAGGED, true>(
+      role_quant_8bit<T, D, FP8, RAGGED, 1, true>(
           tile, nullptr, reinterpret_cast<uint8_t*>(p.q_codes) + (bh * Np + g * 128) * D,
-          p.q_scales + bh * ntiles + g, red, nv);
+          p.q_scales + bh * Np + g * 128, red, nv);
   } else if (role == 1) {
     // FP64 sum of the tile's tokens in order, channel t
     if (has && t < D) {
@@ -829,9 +881,9 @@ __global__ void __cluster_dims__(kFusedCluster, 1, 1) __launch_bounds__(kThreads
     // no CTA leaves while others read its partials
     cluster_sync();
     if (has)
-      role_quant_8bit<T, D, FP8, RAGGED, true>(
+      role_quant_8bit<T, D, FP8, RAGGED, 32, true>(
           tile, stat_s, reinterpret_cast<uint8_t*>(p.k_codes) + (bh * Np + g * 128) * D,
-          p.k_scales + bh * ntiles + g, red, nv);
+          p.k_scales + (bh * Np + g * 128) / 32, red, nv);
   } else {
     if (has) {
       // |V| maximum per channel (a thread keeps 8 channels; a padding token

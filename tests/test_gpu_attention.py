@@ -184,10 +184,11 @@ def test_int8_fp8_onehot_selects_rows(cuda_device):
                          ).to(torch.bfloat16)
     vq = sage.sage_quant_v(v.to(dev))
     qk = {"q_codes": torch.from_numpy(qc.view(np.uint8).ravel()).to(dev),
-          "q_scales": torch.ones(1, dtype=torch.float32, device=dev).view(torch.uint8),
+          # one Q scale per token, one K scale per 32 keys, all 1
+          "q_scales": torch.ones(N, dtype=torch.float32, device=dev).view(torch.uint8),
           "q_sf": None,
           "k_codes": torch.from_numpy(kc.view(np.uint8).ravel()).to(dev),
-          "k_scales": torch.ones(1, dtype=torch.float32, device=dev).view(torch.uint8),
+          "k_scales": torch.ones(N // 32, dtype=torch.float32, device=dev).view(torch.uint8),
           "k_sf": None}
     o = to_numpy32(sage.sage_attn_fwd_quantized(qk, vq, (B, H, N, d), sm_scale=0.05))
     from oracle import prepass as pp

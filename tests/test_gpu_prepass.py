@@ -41,17 +41,21 @@ def check_int8(q, k, v, heads=None, mode="int8_fp8", fused=False):
         qk = sage.sage_quant_qk(q.to(dev), k.to(dev), mode)
         vq = sage.sage_quant_v(v.to(dev), mode)
     torch.cuda.synchronize()
-    nt = -(-N // 128)
+    Np = L.np_of(N)
+    nk = -(-N // 32)
     codes = L.token_codes if mode == "fp8" else L.int8_codes
+    qsc = L.f32(qk["q_scales"], B, H, Np)          # one per token
+    ksc = L.f32(qk["k_scales"], B, H, Np // 32)    # one per 32 tokens
+    # padding tokens (and K blocks of padding only) have scale 0
+    assert not qsc[:, :, N:].any() and not ksc[:, :, nk:].any()
     g = dict(q_codes=codes(qk["q_codes"], B, H, N, d),
-             q_scales=L.f32(qk["q_scales"], B, H, nt),
+             q_scales=qsc[:, :, :N],
              k_codes=codes(qk["k_codes"], B, H, N, d),
-             k_scales=L.f32(qk["k_scales"], B, H, nt),
+             k_scales=ksc[:, :, :nk],
              k_mean=L.f32(qk["k_mean"], B, H, d),
              v_codes=L.vt_codes(vq["v_codes"], B, H, d, N),
              v_scales=L.f32(vq["v_scales"], B, H, d))
     # the padding of a ragged sequence holds zero codes
-    Np = L.np_of(N)
     assert not L.padded_tokens(qk["q_codes"], B, H, N).any()
     assert not L.padded_tokens(qk["k_codes"], B, H, N).any()
     assert not L._np(vq["v_codes"]).reshape(B, H, d, Np)[..., N:].any()
@@ -142,23 +146,25 @@ def test_fp8_qk_prepass_edge_values(cuda_device):
 
 
 def test_fp8_qk_encoder_exhaustive(cuda_device):
-    # every finite fp16 value of magnitude <= 448 as Q, with a 448 in each
-    # 128-token block (so s = 1 and the code is exactly e4m3(x))
+    # every finite fp16 value of magnitude <= 448 as Q, with a 448 in channel
+    # 0 of every token (Q has one scale per token, so s = 1 and the code is
+    # exactly e4m3(x))
     x = np.arange(1 << 16, dtype=np.uint16).view(np.float16).astype(np.float32)
     x = x[np.isfinite(x) & (np.abs(x) <= 448)]
-    per = 127 * 64                            # values per block (one row keeps the 448)
-    nblk = -(-x.size // per)
-    blocks = np.zeros((nblk, 128, 64), np.float32)
-    flat = np.zeros(nblk * per, np.float32)
+    per = 63                                  # values per token (channel 0 keeps the 448)
+    ntok = -(-x.size // per)
+    ntok = -(-ntok // 128) * 128
+    rows = np.zeros((ntok, 64), np.float32)
+    flat = np.zeros(ntok * per, np.float32)
     flat[:x.size] = x
-    blocks[:, 1:, :] = flat.reshape(nblk, 127, 64)
-    blocks[:, 0, 0] = 448.0
-    q = torch.from_numpy(blocks.reshape(1, 1, nblk * 128, 64)).to(torch.float16)
+    rows[:, 1:] = flat.reshape(ntok, per)
+    rows[:, 0] = 448.0
+    q = torch.from_numpy(rows.reshape(1, 1, ntok, 64)).to(torch.float16)
     qk = sage.sage_quant_qk(q.cuda(), q.cuda(), "fp8")
     torch.cuda.synchronize()
-    assert np.all(L.f32(qk["q_scales"], 1, 1, nblk) == 1.0)
-    codes = L.u8(qk["q_codes"], 1, 1, nblk * 128, 64)[0, 0].reshape(nblk, 128, 64)
-    assert np.array_equal(codes[:, 1:, :].reshape(-1)[:x.size], enc.e4m3_encode(x))
+    assert np.all(L.f32(qk["q_scales"], 1, 1, ntok) == 1.0)
+    codes = L.u8(qk["q_codes"], 1, 1, ntok, 64)[0, 0]
+    assert np.array_equal(codes[:, 1:].reshape(-1)[:x.size], enc.e4m3_encode(x))
 
 
 @pytest.mark.parametrize("mode", ["int8_fp8", "fp8", "fp4"])
