@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--impl", default="sage", choices=["sage", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ubench", action="store_true",
+                   help="run the microbenchmarks of include/sage_ubench.h instead (one JSON line)")
     p.add_argument("--also", default=None,
                    help="comma-separated workloads timed after the main one (kernel-only "
                         "lines under 'also'); 'none' for none")
@@ -550,9 +552,44 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_ubench():
+    """The microbenchmarks behind the kernels' design (libsage_ubench.so):
+    tcgen05 MMA throughput per kind, accumulator and tile width, and the
+    SFU exponential rate, FP32 against packed FP16x2."""
+    import ctypes
+
+    import torch
+
+    from quantized_attention_quant_b200 import build as qb
+    qb.build()
+    torch.cuda.init()
+    lib = ctypes.CDLL(qb.UBENCH_LIB)
+    lib.sage_ubench_mma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.POINTER(ctypes.c_double)]
+    lib.sage_ubench_exp.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.POINTER(ctypes.c_double)]
+    out = {"ubench": "tcgen05 MMA and SFU exponential rates", "mma_tops": {}, "exp_per_clk_per_sm": {}}
+    kinds = {"f8f6f4_e4m3_f32acc": 0, "f8f6f4_e4m3_f16acc": 1, "i8_s32acc": 2}
+    for name, kind in kinds.items():
+        for n in (128, 256):
+            v = ctypes.c_double(0.0)
+            st = lib.sage_ubench_mma(kind, n, 8192, 5, ctypes.byref(v))
+            out["mma_tops"][f"{name}_M128_N{n}_K32"] = round(v.value, 1) if st == 0 else f"status {st}"
+    for name, mode in (("ex2_f32", 0), ("ex2_f16x2", 1)):
+        for threads in (128, 256, 512):
+            v = ctypes.c_double(0.0)
+            st = lib.sage_ubench_exp(mode, threads, 4096, ctypes.byref(v))
+            out["exp_per_clk_per_sm"][f"{name}_{threads}thr"] = round(v.value, 2) if st == 0 \
+                else f"status {st}"
+    out["device"] = torch.cuda.get_device_name(0)
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.ubench:
+        run_ubench()
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_sage(args)

@@ -239,6 +239,16 @@ int sage_get_last_device_status(void);
  * stays usable.  No counterpart on the pages: a failure-detection check. */
 int sage_selftest_bounded_wait(sage_stream_t stream);
 
+/* Failure injection for tests: the next `count` workspace allocations (the
+ * stream-ordered growth of the workspace of sage_attn_fwd, sage_attn_fwd_gqa
+ * and the pre-pass calls) fail as if the allocation call had failed, without
+ * making it: the entry point returns SAGE_ERR_CUDA with a message naming the
+ * injected failure and launches nothing, and the workspace stays
+ * unallocated, so a later call allocates it again.  count = 0 clears the
+ * injection; a negative count is SAGE_ERR_INVALID_ARG.  No counterpart on
+ * the pages: a failure-detection check made on the host. */
+int sage_debug_fail_allocations(int count);
+
 /* Human-readable text of a status, with the detail of the calling thread's
  * most recent error when `status` is that error. */
 const char* sage_status_string(int status);

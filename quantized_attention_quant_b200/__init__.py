@@ -39,7 +39,8 @@ EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv
            "sage_attn_fwd_quantized",
            "sage_attn_fwd", "sage_attn_fwd_gqa", "sage_attn_fwd_noalloc",
            "sage_get_last_device_status",
-           "sage_selftest_bounded_wait", "sage_status_string", "sage_version"]
+           "sage_selftest_bounded_wait", "sage_status_string", "sage_version",
+           "sage_debug_fail_allocations"]
 
 _lib = None
 
@@ -91,6 +92,8 @@ def library():
     lib.sage_status_string.argtypes = [i32]
     lib.sage_version.restype = ctypes.c_char_p
     lib.sage_version.argtypes = []
+    lib.sage_debug_fail_allocations.restype = i32
+    lib.sage_debug_fail_allocations.argtypes = [i32]
     _lib = lib
     return lib
 

@@ -103,6 +103,10 @@ struct Workspace {
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
+// Workspace allocations still to fail on purpose (sage_debug_fail_allocations):
+// the failure is made on the host, in place of the allocation call.
+int g_fail_allocs = 0;
+
 int workspace(cudaStream_t st, size_t need, void** out, uint32_t** counters) {
   need += kStatsCounterBytes;
   int dev = 0;
@@ -118,6 +122,11 @@ int workspace(cudaStream_t st, size_t need, void** out, uint32_t** counters) {
       w.bytes = 0;
     }
     const size_t grow = need + need / 4;
+    if (g_fail_allocs > 0) {
+      --g_fail_allocs;
+      return fail(SAGE_ERR_CUDA,
+                  "cudaMallocAsync(workspace): injected failure (sage_debug_fail_allocations)");
+    }
     e = cudaMallocAsync(&w.ptr, grow, st);
     if (e != cudaSuccess) return fail_cuda(e, "cudaMallocAsync(workspace)");
     w.bytes = grow;
@@ -170,6 +179,7 @@ int prepass_forked(const QuantQKArgs& qa, const QuantVArgs& va, cudaStream_t st)
     if (e != cudaSuccess) return fail_cuda(e, "fused pre-pass launch");
     return SAGE_OK;
   }
+
   SideStream* ss = nullptr;
   const int got = side_stream(&ss);
   if (got != SAGE_OK) return got;
@@ -636,6 +646,13 @@ const char* sage_status_string(int status) {
 }
 
 const char* sage_version(void) { return "sage-b200 0.1 (sm_100a)"; }
+
+int sage_debug_fail_allocations(int count) {
+  if (count < 0) return fail(SAGE_ERR_INVALID_ARG, "count must be >= 0");
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_fail_allocs = count;
+  return SAGE_OK;
+}
 
 }  // extern "C"
 

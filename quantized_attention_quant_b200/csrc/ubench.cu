@@ -1,0 +1,210 @@
+// ubench.cu -- measurement kernels behind the design choices of the
+// attention kernels (libsage_ubench.so, include/sage_ubench.h):
+//   - tcgen05 MMA throughput per kind, accumulator type and tile width N
+//     (is an FP16 accumulator faster than FP32 for FP8 P~V, as the
+//     SageAttention2++ page reports for its GPUs; how much narrower is an
+//     N = 128 tile than N = 256);
+//   - SFU exponential throughput, FP32 against packed FP16x2.
+// One CTA per SM; every wait is bounded (a timeout sets a flag the host
+// reads and returns as an error).  No other code of the library uses this.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/sage_ubench.h"
+#include "sage_ptx.cuh"
+
+namespace sage {
+namespace {
+
+// M = 128, K = 32 (8-bit operands: 32 bytes of K per row), N = 128 or 256;
+// operands zero in shared memory (the rate does not depend on the values).
+template <int KIND, int N>
+__global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, uint32_t* flag) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ uint64_t bar;
+  __shared__ uint32_t slot;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  // A: 128 rows, B: N rows, 128 bytes each (128-byte swizzle atoms)
+  for (int i = threadIdx.x; i < (128 + N) * 128 / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(smem)[i] = 0u;
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(&slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = slot;
+  if (warp == 0 && elect_one()) {
+    constexpr uint32_t idesc = KIND == SAGE_UBENCH_F8_F32 ? make_idesc(1, 0, 0, 128, N)
+                             : KIND == SAGE_UBENCH_F8_F16 ? make_idesc(0, 0, 0, 128, N)
+                                                          : make_idesc(2, 1, 1, 128, N);
+    const uint64_t a = make_sdesc(smem_u32(smem), 1024, 16, Swz::k128);
+    const uint64_t b = make_sdesc(smem_u32(smem + 128 * 128), 1024, 16, Swz::k128);
+    for (int i = 0; i < iters; ++i) {
+      if (KIND == SAGE_UBENCH_I8_S32) mma_i8_ss(tmem, a, b, idesc, i > 0);
+      else mma_f8_ss(tmem, a, b, idesc, i > 0);
+    }
+    mma_commit(&bar);
+    volatile int no_abort = 0;
+    mbar_wait(&bar, 0, &no_abort, flag, 1u);  // an expired wait sets *flag
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// 8 independent exponentials per thread and round, each fed by the
+// previous round (y = 2^(y - 1) converges to 1): FP32 ex2, or packed
+// FP16x2 ex2 (two values per instruction).
+template <int MODE>
+__global__ void exp_rate_kernel(int iters, float* sink, long long* cycles) {
+  const long long t0 = clock64();
+  float acc = 0.f;
+  if (MODE == SAGE_UBENCH_EXP_F32) {
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = 1.0f + 0.001f * (float)(threadIdx.x + i);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float r;
+        asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y[i] - 1.0f));
+        y[i] = r;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc += y[i];
+  } else {
+    uint32_t y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = 0x3C003C00u;  // (1, 1) in f16x2
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint32_t d, r;
+        asm volatile("sub.f16x2 %0, %1, %2;" : "=r"(d) : "r"(y[i]), "r"(0x3C003C00u));
+        asm volatile("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(d));
+        y[i] = r;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc += (float)(y[i] & 0xFFFFu);
+  }
+  const long long t1 = clock64();
+  sink[blockIdx.x * blockDim.x + threadIdx.x] = acc;
+  if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
+}
+
+int sms_of_device(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? 0 : -1;
+}
+
+template <int KIND, int N>
+int run_mma(int iters, int reps, double* tops) {
+  int sms = 0;
+  if (sms_of_device(&sms) != 0) return SAGE_UBENCH_ERR_CUDA;
+  auto k = mma_rate_kernel<KIND, N>;
+  const int smem = (128 + N) * 128 + 1024;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SAGE_UBENCH_ERR_CUDA;
+  uint32_t* flag = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  int status = SAGE_UBENCH_ERR_CUDA;
+  float ms = 0.f;
+  if (cudaMalloc(&flag, 4) != cudaSuccess) return SAGE_UBENCH_ERR_CUDA;
+  if (cudaMemset(flag, 0, 4) == cudaSuccess && cudaEventCreate(&e0) == cudaSuccess &&
+      cudaEventCreate(&e1) == cudaSuccess) {
+    k<<<sms, 128, smem>>>(iters, flag);  // warm-up
+    cudaEventRecord(e0);
+    for (int r = 0; r < reps; ++r) k<<<sms, 128, smem>>>(iters, flag);
+    cudaEventRecord(e1);
+    uint32_t h = 0;
+    if (cudaEventSynchronize(e1) == cudaSuccess && cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess &&
+        cudaMemcpy(&h, flag, 4, cudaMemcpyDeviceToHost) == cudaSuccess)
+      status = h ? SAGE_UBENCH_ERR_TIMEOUT : SAGE_UBENCH_OK;
+  }
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  cudaFree(flag);
+  if (status == SAGE_UBENCH_OK)
+    *tops = 2.0 * 128 * N * 32 * (double)iters * sms * reps / (ms * 1e-3) / 1e12;
+  return status;
+}
+
+template <int MODE>
+int run_exp(int threads, int iters, double* per_clk) {
+  int sms = 0;
+  if (sms_of_device(&sms) != 0) return SAGE_UBENCH_ERR_CUDA;
+  float* sink = nullptr;
+  long long* cyc = nullptr;
+  int status = SAGE_UBENCH_ERR_CUDA;
+  if (cudaMalloc(&sink, (size_t)sms * threads * 4) == cudaSuccess &&
+      cudaMalloc(&cyc, (size_t)sms * 8) == cudaSuccess) {
+    exp_rate_kernel<MODE><<<sms, threads>>>(iters, sink, cyc);  // warm-up
+    exp_rate_kernel<MODE><<<sms, threads>>>(iters, sink, cyc);
+    long long* h = new long long[sms];
+    if (cudaMemcpy(h, cyc, (size_t)sms * 8, cudaMemcpyDeviceToHost) == cudaSuccess) {
+      double c = 0;
+      for (int i = 0; i < sms; ++i) c += (double)h[i];
+      c /= sms;
+      const double values = (double)threads * 8 * iters * (MODE == SAGE_UBENCH_EXP_F32 ? 1 : 2);
+      *per_clk = values / c;
+      status = SAGE_UBENCH_OK;
+    }
+    delete[] h;
+  }
+  cudaFree(sink);
+  cudaFree(cyc);
+  return status;
+}
+
+}  // namespace
+}  // namespace sage
+
+extern "C" {
+
+int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops) {
+  using namespace sage;
+  if (!tops || iters <= 0 || reps <= 0 || (n != 128 && n != 256)) return SAGE_UBENCH_ERR_ARG;
+  switch (kind) {
+    case SAGE_UBENCH_F8_F32:
+      return n == 128 ? run_mma<SAGE_UBENCH_F8_F32, 128>(iters, reps, tops)
+                      : run_mma<SAGE_UBENCH_F8_F32, 256>(iters, reps, tops);
+    case SAGE_UBENCH_F8_F16:
+      return n == 128 ? run_mma<SAGE_UBENCH_F8_F16, 128>(iters, reps, tops)
+                      : run_mma<SAGE_UBENCH_F8_F16, 256>(iters, reps, tops);
+    case SAGE_UBENCH_I8_S32:
+      return n == 128 ? run_mma<SAGE_UBENCH_I8_S32, 128>(iters, reps, tops)
+                      : run_mma<SAGE_UBENCH_I8_S32, 256>(iters, reps, tops);
+    default:
+      return SAGE_UBENCH_ERR_ARG;
+  }
+}
+
+int sage_ubench_exp(int mode, int threads, int iters, double* per_clk_per_sm) {
+  using namespace sage;
+  if (!per_clk_per_sm || iters <= 0 || threads <= 0 || threads > 1024 || threads % 32)
+    return SAGE_UBENCH_ERR_ARG;
+  if (mode == SAGE_UBENCH_EXP_F32) return run_exp<SAGE_UBENCH_EXP_F32>(threads, iters, per_clk_per_sm);
+  if (mode == SAGE_UBENCH_EXP_F16X2)
+    return run_exp<SAGE_UBENCH_EXP_F16X2>(threads, iters, per_clk_per_sm);
+  return SAGE_UBENCH_ERR_ARG;
+}
+
+}  // extern "C"

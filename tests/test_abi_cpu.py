@@ -35,6 +35,36 @@ def test_exports_match_header(lib):
     assert lib.sage_version().decode().startswith("sage-b200")
 
 
+def test_ubench_library_exports_its_header():
+    # the microbenchmark library exports every function include/sage_ubench.h
+    # declares, and rejects bad arguments before touching a device
+    import ctypes
+
+    from quantized_attention_quant_b200 import build as qb
+    qb.build()
+    text = open(os.path.join(ROOT, "include", "sage_ubench.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+    assert names == ["sage_ubench_exp", "sage_ubench_mma"]
+    ub = ctypes.CDLL(qb.UBENCH_LIB)
+    for n in names:
+        assert hasattr(ub, n), n
+    v = ctypes.c_double(0.0)
+    ub.sage_ubench_mma.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(ctypes.c_double)]
+    ub.sage_ubench_exp.argtypes = [ctypes.c_int] * 3 + [ctypes.POINTER(ctypes.c_double)]
+    assert ub.sage_ubench_mma(0, 96, 10, 1, ctypes.byref(v)) == -1      # N must be 128 or 256
+    assert ub.sage_ubench_mma(7, 128, 10, 1, ctypes.byref(v)) == -1     # unknown kind
+    assert ub.sage_ubench_exp(0, 100, 10, ctypes.byref(v)) == -1        # not whole warps
+    assert ub.sage_ubench_exp(5, 128, 10, ctypes.byref(v)) == -1        # unknown mode
+
+
+def test_allocation_failure_injection_arguments(lib):
+    # the injection is a host-side counter: no device call
+    assert lib.sage_debug_fail_allocations(2) == 0
+    assert lib.sage_debug_fail_allocations(0) == 0
+    assert lib.sage_debug_fail_allocations(-1) == -1
+
+
 def test_buffer_bytes(lib):
     import quantized_attention_quant_b200 as q
     B, H, N, d = 2, 3, 256, 128

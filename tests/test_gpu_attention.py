@@ -223,7 +223,10 @@ def test_side_stream(cuda_device):
     assert torch.equal(ref, out)
 
 
-FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", None), ("long_causal", None),
+# cosine floor against exact attention where the quantization scheme itself
+# reaches 0.999 (per-token Q and per-32-key K scales); elsewhere the test holds
+# the GPU to the emulated oracle's own cosine
+FULL = [("tiny", 0.999), ("llm", None), ("video", 0.999), ("long", 0.999), ("long_causal", 0.999),
         ("fp4", None), ("long_fp8", None), ("llm_fp8", None), ("short", None),
         ("n16k", 0.999), ("n16k_fp8", None)]
 
@@ -320,3 +323,35 @@ def test_cuda_graph_capture_and_replay(cuda_device, N):
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
     assert sage.device_status() == 0
+
+
+def test_workspace_allocation_failure_is_reported(cuda_device):
+    """A failed workspace allocation (made to fail on the host, in place of
+    the allocation call) comes back as SAGE_ERR_CUDA naming the failure;
+    nothing is launched, and the next call allocates and computes."""
+    lib = sage.library()
+    # larger than anything the other tests run on a pooled stream, so the
+    # stream's workspace has to grow
+    B, H, N, d = 1, 8, 4096, 128
+    q, k, v = rand_qkv(B, H, N, d, "bf16", seed=1700)
+    dev = torch.device("cuda")
+    qg, kg, vg = q.to(dev), k.to(dev), v.to(dev)
+    s = torch.cuda.Stream()
+    out = torch.full_like(qg, 7.0)
+    assert lib.sage_debug_fail_allocations(1) == 0
+    with torch.cuda.stream(s):
+        with pytest.raises(sage.SageError) as err:
+            sage.sage_attn_fwd(qg, kg, vg, out=out)
+    assert err.value.status == -3 and "injected failure" in str(err.value)
+    s.synchronize()
+    assert torch.all(out == 7.0)            # no kernel ran
+    with torch.cuda.stream(s):
+        sage.sage_attn_fwd(qg, kg, vg, out=out)
+    s.synchronize()
+    assert sage.device_status() == 0
+    rows = np.r_[0:8, 1000, 2047, 4095]
+    hs = [0, H - 1]
+    check_against_oracle(to_numpy32(out)[:, hs][:, :, rows], q[:, hs], k[:, hs], v[:, hs], False,
+                         1 / math.sqrt(d), "int8_fp8", "bf16", rows=rows)
+    assert lib.sage_debug_fail_allocations(-1) == -1
+    assert lib.sage_debug_fail_allocations(0) == 0
