@@ -569,12 +569,14 @@ def run_ubench():
     lib.sage_ubench_exp.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.POINTER(ctypes.c_double)]
     out = {"ubench": "tcgen05 MMA and SFU exponential rates", "mma_tops": {}, "exp_per_clk_per_sm": {}}
-    kinds = {"f8f6f4_e4m3_f32acc": 0, "f8f6f4_e4m3_f16acc": 1, "i8_s32acc": 2}
-    for name, kind in kinds.items():
+    kinds = {"f8f6f4_e4m3_f32acc": (0, 32), "f8f6f4_e4m3_f16acc": (1, 32), "i8_s32acc": (2, 32),
+             "mxf4nvf4_e2m1_ue4m3x16_f32acc": (3, 64)}
+    for name, (kind, kdim) in kinds.items():
         for n in (128, 256):
             v = ctypes.c_double(0.0)
             st = lib.sage_ubench_mma(kind, n, 8192, 5, ctypes.byref(v))
-            out["mma_tops"][f"{name}_M128_N{n}_K32"] = round(v.value, 1) if st == 0 else f"status {st}"
+            out["mma_tops"][f"{name}_M128_N{n}_K{kdim}"] = round(v.value, 1) if st == 0 \
+                else f"status {st}"
     for name, mode in (("ex2_f32", 0), ("ex2_f16x2", 1)):
         for threads in (128, 256, 512):
             v = ctypes.c_double(0.0)

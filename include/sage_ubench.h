@@ -25,16 +25,20 @@ enum {
 enum {
   SAGE_UBENCH_F8_F32 = 0,  /* kind::f8f6f4, e4m3 x e4m3, FP32 accumulator */
   SAGE_UBENCH_F8_F16 = 1,  /* kind::f8f6f4, e4m3 x e4m3, FP16 accumulator */
-  SAGE_UBENCH_I8_S32 = 2   /* kind::i8, s8 x s8, INT32 accumulator        */
+  SAGE_UBENCH_I8_S32 = 2,  /* kind::i8, s8 x s8, INT32 accumulator        */
+  SAGE_UBENCH_NVF4 = 3     /* kind::mxf4nvf4.block_scale.block16, e2m1 x
+                              e2m1 with UE4M3 scales per 16 elements of K
+                              (in TMEM), FP32 accumulator                  */
 };
 
 /* Exponential variants measured by sage_ubench_exp. */
 enum { SAGE_UBENCH_EXP_F32 = 0, SAGE_UBENCH_EXP_F16X2 = 1 };
 
 /* Dense MMA throughput: one CTA per SM issues `iters` MMAs of M = 128,
- * N = n (128 or 256), K = 32 from shared memory onto one TMEM accumulator,
- * `reps` launches timed with CUDA events.  *tops receives 2 M N K iters
- * SMs reps / time, in 10^12 operations per second.  The SageAttention2++
+ * N = n (128 or 256), K = 32 (K = 64 for SAGE_UBENCH_NVF4) from shared
+ * memory onto one TMEM accumulator, `reps` launches timed with CUDA
+ * events.  *tops receives 2 M N K iters SMs reps / time, in 10^12
+ * operations per second.  The SageAttention2++
  * page reports an FP8 MMA with FP16 accumulation twice as fast as with
  * FP32 on its GPUs; this measures the same question on this one. */
 int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops);

@@ -171,14 +171,22 @@ __device__ __forceinline__ void exp_loop(const int h, const Sched& sch, const in
 
   Cursor<CAUSAL> cur;
   cur.load(sch, blockIdx.x, 0);
+  const int nitems = sch.count(blockIdx.x);
+  // this row's Q scale in the current item; the next item's is loaded at
+  // the start of the current item's last tile, a tile ahead of its use
+  float qs = ldg_early(q_scales + ((int64_t)cur.bh * sch.ntiles + cur.qt) * 128 + r);
+  float qs_next = 0.f;
   // l restarts at every item by itself: the first tile's alpha is 0
   float l = 0.f;
-  float qs = 0.f;  // this row's Q scale in the current item
   for (int g = 0; g < T; ++g, cur.next(sch, blockIdx.x)) {
     const int j = cur.j;
     const int b = g & 1;
     const uint32_t ph = (g >> 1) & 1;
-    if (j == 0) qs = __ldg(q_scales + ((int64_t)cur.bh * sch.ntiles + cur.qt) * 128 + r);
+    if (j == cur.nkv - 1 && cur.it + 1 < nitems) {
+      Cursor<CAUSAL> nx;
+      nx.load(sch, blockIdx.x, cur.it + 1);
+      qs_next = ldg_early(q_scales + ((int64_t)nx.bh * sch.ntiles + nx.qt) * 128 + r);
+    }
     // m_full(g) is published by the stats warpgroup after it waited for
     // s_full(g) and read S[b]: it orders this warpgroup after the Q K^T too
     if (!__all_sync(0xffffffffu,
@@ -225,6 +233,7 @@ __device__ __forceinline__ void exp_loop(const int h, const Sched& sch, const in
       const int lb = cur.it % 3;
       l_s[(lb * 2 + h) * 128 + r] = l;
       mbar_arrive(&bar.l_ready[lb]);
+      qs = qs_next;
     }
   }
 }
@@ -339,28 +348,37 @@ __device__ __forceinline__ void stats_loop(const Sched& sch, const int T, const 
   float alpha_hist[2] = {0.f, 0.f};
   Cursor<CAUSAL> mc;  // tile whose max is taken
   mc.load(sch, blockIdx.x, 0);
-  float m = -INFINITY, qs = 0.f;
-  float4 ks_cur = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* ksp = k_scales;
+  const int nitems = sch.count(blockIdx.x);
+  // this row's Q scale and the K/V head's K scales (four per key tile) of
+  // the current item; the next item's are loaded at the start of the
+  // current item's last tile, a tile ahead of their use
+  const float* ksp = k_scales + (int64_t)kv_head(mc.bh, H, G) * ntiles * 4;
+  const float* ksp_next = ksp;
+  float qs = ldg_early(q_scales + ((int64_t)mc.bh * ntiles + mc.qt) * 128 + r);
+  float qs_next = 0.f;
+  float4 ks_cur = ldg4_early(ksp);
+  float m = -INFINITY;
   // one pass: the max of tile g (g < T), then the fold of tile g - PVB
   for (int g = 0; g < T + L::PVB; ++g) {
     float alpha = 0.f;
     if (g < T) {
       const int j = mc.j;
       const int b = g & 1;
-      if (j == 0) {
-        // a new item: its Q scale, its head's K scales, a fresh running max
-        m = -INFINITY;
-        qs = __ldg(q_scales + ((int64_t)mc.bh * ntiles + mc.qt) * 128 + r);
-        ksp = k_scales + (int64_t)kv_head(mc.bh, H, G) * ntiles * 4;
-        ks_cur = __ldg(reinterpret_cast<const float4*>(ksp));
-      }
+      if (j == 0) m = -INFINITY;  // a new item: a fresh running max
       // s_K sm_scale log2 e of the tile's four 32-key chunks; a row's factor
       // is its Q scale times that (the exp warpgroups form the same products)
       const float kl[4] = {ks_cur.x * scale_log2, ks_cur.y * scale_log2, ks_cur.z * scale_log2,
                            ks_cur.w * scale_log2};
-      const float4 ks_nxt =
-          j + 1 < mc.nkv ? ldg4_early(ksp + 4 * (j + 1)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 ks_nxt = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j + 1 < mc.nkv) {
+        ks_nxt = ldg4_early(ksp + 4 * (j + 1));
+      } else if (mc.it + 1 < nitems) {
+        Cursor<CAUSAL> nx;
+        nx.load(sch, blockIdx.x, mc.it + 1);
+        ksp_next = k_scales + (int64_t)kv_head(nx.bh, H, G) * ntiles * 4;
+        ks_nxt = ldg4_early(ksp_next);
+        qs_next = ldg_early(q_scales + ((int64_t)nx.bh * ntiles + nx.qt) * 128 + r);
+      }
       const int sbuf = g % L::SB;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[sbuf], (g / L::SB) & 1, abort_flag,
                                              status, kDevTimeoutMma)))
@@ -399,6 +417,10 @@ __device__ __forceinline__ void stats_loop(const Sched& sch, const int T, const 
       tc_fence_before();
       mbar_arrive(&bar.m_full[b]);
       ks_cur = ks_nxt;
+      if (j == mc.nkv - 1) {
+        qs = qs_next;
+        ksp = ksp_next;
+      }
       mc.next(sch, blockIdx.x);
     }
     if (g >= L::PVB) {

@@ -1,6 +1,7 @@
 // ubench.cu -- measurement kernels behind the design choices of the
 // attention kernels (libsage_ubench.so, include/sage_ubench.h):
-//   - tcgen05 MMA throughput per kind, accumulator type and tile width N
+//   - tcgen05 MMA throughput per kind (8-bit, and block-scaled FP4),
+//     accumulator type and tile width N
 //     (is an FP16 accumulator faster than FP32 for FP8 P~V, as the
 //     SageAttention2++ page reports for its GPUs; how much narrower is an
 //     N = 128 tile than N = 256);
@@ -18,8 +19,12 @@
 namespace sage {
 namespace {
 
-// M = 128, K = 32 (8-bit operands: 32 bytes of K per row), N = 128 or 256;
-// operands zero in shared memory (the rate does not depend on the values).
+// M = 128, N = 128 or 256; K = 32 for the 8-bit kinds (32 bytes of K per
+// row), 64 for block-scaled FP4 (E2M1 operands, one UE4M3 scale per 16
+// elements of K, the scales in TMEM); operands and scales zero (the rate
+// does not depend on the values).
+template <int KIND>
+constexpr int kUbenchK = KIND == SAGE_UBENCH_NVF4 ? 64 : 32;
 template <int KIND, int N>
 __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, uint32_t* flag) {
   extern __shared__ uint8_t smem_raw[];
@@ -36,22 +41,45 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, uint32_t* f
   for (int i = threadIdx.x; i < (128 + N) * 128 / 4; i += blockDim.x)
     reinterpret_cast<uint32_t*>(smem)[i] = 0u;
   fence_proxy_async_smem();
+  // the accumulator in columns 0 .. N-1; FP4 scale factors of A from
+  // column kColSfA, of B from kColSfB
+  constexpr uint32_t kColSfA = 384, kColSfB = 416;
   if (warp == 0) {
-    tmem_alloc(&slot, 256);
+    tmem_alloc(&slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = slot;
+  if (KIND == SAGE_UBENCH_NVF4) {
+    // zero scale factors: each warp its 32 lanes of columns 384 .. 447
+    const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    const uint32_t lanes = (uint32_t)(warp * 32) << 16;
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) tmem_st8(tmem + lanes + kColSfA + (uint32_t)c, z);
+    tmem_wait_st();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
   if (warp == 0 && elect_one()) {
     constexpr uint32_t idesc = KIND == SAGE_UBENCH_F8_F32 ? make_idesc(1, 0, 0, 128, N)
                              : KIND == SAGE_UBENCH_F8_F16 ? make_idesc(0, 0, 0, 128, N)
+                             : KIND == SAGE_UBENCH_NVF4   ? make_idesc_nvf4(128, N)
                                                           : make_idesc(2, 1, 1, 128, N);
-    const uint64_t a = make_sdesc(smem_u32(smem), 1024, 16, Swz::k128);
-    const uint64_t b = make_sdesc(smem_u32(smem + 128 * 128), 1024, 16, Swz::k128);
+    // 8-bit kinds: 128-byte rows, 128-byte swizzle; FP4: 64-byte rows
+    // (128 E2M1 elements, two K steps), 64-byte swizzle, first K step
+    const uint64_t a = KIND == SAGE_UBENCH_NVF4
+                           ? make_sdesc(smem_u32(smem), 8 * 64, 16, Swz::k64)
+                           : make_sdesc(smem_u32(smem), 1024, 16, Swz::k128);
+    const uint64_t b = KIND == SAGE_UBENCH_NVF4
+                           ? make_sdesc(smem_u32(smem + 128 * 128), 8 * 64, 16, Swz::k64)
+                           : make_sdesc(smem_u32(smem + 128 * 128), 1024, 16, Swz::k128);
     for (int i = 0; i < iters; ++i) {
       if (KIND == SAGE_UBENCH_I8_S32) mma_i8_ss(tmem, a, b, idesc, i > 0);
+      else if (KIND == SAGE_UBENCH_NVF4)
+        mma_nvf4_ss(tmem, a, b, idesc, tmem + kColSfA, tmem + kColSfB, i > 0);
       else mma_f8_ss(tmem, a, b, idesc, i > 0);
     }
     mma_commit(&bar);
@@ -63,7 +91,7 @@ __global__ void __launch_bounds__(128, 1) mma_rate_kernel(int iters, uint32_t* f
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -143,7 +171,7 @@ int run_mma(int iters, int reps, double* tops) {
   if (e1) cudaEventDestroy(e1);
   cudaFree(flag);
   if (status == SAGE_UBENCH_OK)
-    *tops = 2.0 * 128 * N * 32 * (double)iters * sms * reps / (ms * 1e-3) / 1e12;
+    *tops = 2.0 * 128 * N * kUbenchK<KIND> * (double)iters * sms * reps / (ms * 1e-3) / 1e12;
   return status;
 }
 
@@ -192,6 +220,9 @@ int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops) {
     case SAGE_UBENCH_I8_S32:
       return n == 128 ? run_mma<SAGE_UBENCH_I8_S32, 128>(iters, reps, tops)
                       : run_mma<SAGE_UBENCH_I8_S32, 256>(iters, reps, tops);
+    case SAGE_UBENCH_NVF4:
+      return n == 128 ? run_mma<SAGE_UBENCH_NVF4, 128>(iters, reps, tops)
+                      : run_mma<SAGE_UBENCH_NVF4, 256>(iters, reps, tops);
     default:
       return SAGE_UBENCH_ERR_ARG;
   }

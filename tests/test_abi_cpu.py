@@ -54,6 +54,7 @@ def test_ubench_library_exports_its_header():
     ub.sage_ubench_exp.argtypes = [ctypes.c_int] * 3 + [ctypes.POINTER(ctypes.c_double)]
     assert ub.sage_ubench_mma(0, 96, 10, 1, ctypes.byref(v)) == -1      # N must be 128 or 256
     assert ub.sage_ubench_mma(7, 128, 10, 1, ctypes.byref(v)) == -1     # unknown kind
+    assert ub.sage_ubench_mma(3, 64, 10, 1, ctypes.byref(v)) == -1      # FP4 kind: N 128 or 256 too
     assert ub.sage_ubench_exp(0, 100, 10, ctypes.byref(v)) == -1        # not whole warps
     assert ub.sage_ubench_exp(5, 128, 10, ctypes.byref(v)) == -1        # unknown mode
 
