@@ -19,6 +19,8 @@ traffic" for the tiled online softmax):
                                                  block; FP4: A * g_Q * g_K *
                                                  sm_scale, block scales
                                                  inside A)
+             (+ dS[query block, key] * sm_scale with Q smoothing: the
+              SageAttention2 abstract's smoothed Q, prepass reading 2)
     m_new  = max(m, rowmax S)
     alpha  = exp(m - m_new)
     P~     = exp(S - m_new)                     (<= 1)
@@ -198,7 +200,7 @@ def fp4_p_ambiguity(pt, eps):
 # --------------------------------------------------------------------------
 
 def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows=None,
-               p_ambiguity=None, qk_acc_rel=0.0):
+               p_ambiguity=None, qk_acc_rel=0.0, s_bias=None):
     """Online softmax + two-level P~V accumulation for one (b, h).
 
     qd [N, d], kd [N, d]: decoded code values (exact FP64).
@@ -219,6 +221,8 @@ def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows
     the largest dS so far (Dm), so each P~ by a factor within exp(+-(dS +
     Dm)): the code decisions get that much extra room, and the row sum (thus
     O / l) a relative deviation of at most expm1(2 Dm).
+    s_bias: optional [ceil(N/128), N] score bias of Q smoothing (dS, in the
+    units of A * s_Q * s_K): row r's scores gain s_bias[r // 128] * sm_scale.
     Returns O [len(rows), d] in FP64 (before the output rounding), and the
     bound when p_ambiguity is given.
     """
@@ -237,6 +241,8 @@ def _tile_loop(qd, kd, vd, s_row, s_key, v_fold, p_quant, causal, sm_scale, rows
         r_act = rows[act]
         A = qk_product(qd[r_act], kd[ks:ke])       # exact
         S = A * s_row[r_act, None] * s_key[None, ks:ke] * sm_scale
+        if s_bias is not None:
+            S = S + s_bias[r_act // BLOCK, ks:ke].astype(np.float64) * sm_scale
         if causal:
             S = np.where(np.arange(ks, ke)[None, :] <= r_act[:, None], S, -np.inf)
         m_new = np.maximum(m[act], S.max(axis=1))
@@ -278,7 +284,8 @@ def _identity(x):
 
 
 def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8",
-                            quantizers="faithful", rows=None, ambiguity_eps=None):
+                            quantizers="faithful", rows=None, ambiguity_eps=None,
+                            smooth_q=False):
     """Step-by-step emulation of the quantized forward pass, FP64 O [B,H,N,d].
 
     mode: "int8_fp8" (INT8 Q/K, FP8 P~ and V), "fp8" (FP8 Q/K, P~ and V) or
@@ -294,6 +301,11 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     INT8/FP8 and FP8 mode; the UE4M3 group scales and e2m1 codes in FP4 mode.
     In FP8 mode the bound also covers the FP32 accumulation of Q K^T
     (FP8_QK_ACC_REL).
+    smooth_q: Q smoothing (prepass reading 2): Q loses its per-block mean
+    before quantization and every score of the block gains dS * sm_scale.
+    With quantizers="identity" the smoothed Q' and the smoothed K' enter
+    unrounded beside the FP32 dS, so the result is exact attention up to the
+    FP32 roundings of Q', K' and dS.
     """
     q = np.asarray(q, np.float32)
     k = np.asarray(k, np.float32)
@@ -307,12 +319,18 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     tile_of = np.arange(N) // BLOCK
 
     if quantizers == "identity":
+        qi, ki, bias = q, k, None
+        if smooth_q:
+            ki = pp.smooth_k(k, pp.k_channel_mean(k))
+            qm = pp.q_block_mean(q)
+            qi, bias = pp.smooth_q(q, qm), pp.smoothing_bias(qm, ki)
         for b in range(B):
             for h in range(H):
                 ones_n = np.ones(N)
-                out[b, h] = _tile_loop(q[b, h].astype(np.float64), k[b, h].astype(np.float64),
+                out[b, h] = _tile_loop(qi[b, h].astype(np.float64), ki[b, h].astype(np.float64),
                                        v[b, h].astype(np.float64), ones_n, ones_n,
-                                       np.ones((ntiles, d)), _identity, causal, sm_scale, rows)
+                                       np.ones((ntiles, d)), _identity, causal, sm_scale, rows,
+                                       s_bias=None if bias is None else bias[b, h])
         return out
     if quantizers != "faithful":
         raise ValueError(quantizers)
@@ -322,7 +340,7 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
         bound = np.zeros_like(out) if ambiguity_eps is not None else None
         amb = ((lambda pt, extra: fp8_p_ambiguity(pt, ambiguity_eps + extra))
                if bound is not None else None)
-        qk = pp.quant_qk_fp8(q, k) if fp8_qk else pp.quant_qk_int8(q, k)
+        qk = pp.quant_qk_fp8(q, k, smooth_q) if fp8_qk else pp.quant_qk_int8(q, k, smooth_q)
         vc, vs = pp.quant_v_fp8(v)
         for b in range(B):
             for h in range(H):
@@ -338,7 +356,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                 v_fold = np.broadcast_to(vs[b, h].astype(np.float64) / P_FP8_SCALE, (ntiles, d))
                 res = _tile_loop(qd, kd, vd, s_row, s_key, v_fold, quant_p_fp8,
                                  causal, sm_scale, rows, amb,
-                                 FP8_QK_ACC_REL if fp8_qk else 0.0)
+                                 FP8_QK_ACC_REL if fp8_qk else 0.0,
+                                 qk["dS"][b, h] if smooth_q else None)
                 if bound is None:
                     out[b, h] = res
                 else:
@@ -349,7 +368,7 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
         bound = np.zeros_like(out) if ambiguity_eps is not None else None
         amb = ((lambda pt, extra: fp4_p_ambiguity(pt, ambiguity_eps + extra))
                if bound is not None else None)
-        qk = pp.quant_qk_fp4(q, k)
+        qk = pp.quant_qk_fp4(q, k, smooth_q)
         vc, vsf, vg = pp.quant_v_fp4(v)
         for b in range(B):
             for h in range(H):
@@ -363,7 +382,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
                 s_key = qk["k_g"][b, h].astype(np.float64)[tile_of]
                 v_fold = (vg[b, h].astype(np.float64) * P_FP4_G)[:, None] * np.ones((1, d))
                 res = _tile_loop(qd, kd, vdt.T, s_row, s_key, v_fold, quant_p_fp4,
-                                 causal, sm_scale, rows, amb)
+                                 causal, sm_scale, rows, amb,
+                                 s_bias=qk["dS"][b, h] if smooth_q else None)
                 if bound is None:
                     out[b, h] = res
                 else:
@@ -372,6 +392,8 @@ def emulated_sage_attention(q, k, v, causal=False, sm_scale=None, mode="int8_fp8
     raise ValueError(mode)
 
 
-def sage_attention_output(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", dtype="bf16"):
+def sage_attention_output(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", dtype="bf16",
+                          smooth_q=False):
     """Emulated O rounded to the input dtype ('bf16' or 'f16'), as float32."""
-    return round_to_dtype(emulated_sage_attention(q, k, v, causal, sm_scale, mode), dtype)
+    return round_to_dtype(emulated_sage_attention(q, k, v, causal, sm_scale, mode,
+                                                  smooth_q=smooth_q), dtype)

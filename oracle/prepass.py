@@ -13,7 +13,16 @@ Readings of the pages (they give the method only at abstract level):
    softmax -- and O -- is unchanged.  The mean is accumulated in FP64 in a
    fixed order: per 128-token chunk a partial sum in token order, then the
    chunk partials in chunk order; mean = fp32(total / N).
-2. Q is not smoothed (Q smoothing is the SageAttention2 extension).
+2. Q smoothing (SageAttention2 abstract: "we propose a method to smooth
+   Q"), optional (smooth_q): per (b, h) and per 128-token block of queries
+   (the query tile), qbar = fp32(mean of the block's tokens), accumulated in
+   FP64 in token order; Q' = fp32(Q) - qbar (one FP32 subtraction) is what
+   gets quantized.  What qbar removes comes back as a bias on every score of
+   the block: dS[blk, j] = qbar[blk] . k'_j with k'_j = fp32(K_j) - mean_K
+   the smoothed key (reading 1) before quantization, evaluated in FP64 with
+   the d products added in channel order (each product of two FP32 values
+   is exact in FP64, so one rounding per addition) and rounded once to
+   FP32.  Without it Q is quantized as it is.
 3. INT8 Q/K: one FP32 scale per block of tokens of one (b, h), covering all
    d channels: s = fp32(amax / 127); code = clamp(rne(fp32(x / s)), +-127);
    an all-zero block gets s = 0 and codes 0.  For K, x = fp32(K) - mean is a
@@ -87,6 +96,49 @@ def smooth_k(k, mean):
     return (np.asarray(k, np.float32) - np.asarray(mean, np.float32)[:, :, None, :]).astype(np.float32)
 
 
+def q_block_mean(q):
+    """Per-(b, h, 128-token block, channel) mean of Q, reading 2.
+
+    FP64 sum in token order over the block's tokens (a ragged last block:
+    its tokens only), divided by their count, rounded to FP32.  Returns
+    float32 [B, H, ceil(N/128), d].
+    """
+    q = np.asarray(q, np.float64)
+    B, H, N, d = q.shape
+    out = np.zeros((B, H, -(-N // BLOCK), d), np.float32)
+    for i, (s, e) in enumerate(_blocks(N)):
+        part = np.zeros((B, H, d), np.float64)
+        for t in range(s, e):
+            part += q[:, :, t, :]
+        out[:, :, i, :] = (part / np.float64(e - s)).astype(np.float32)
+    return out
+
+
+def smooth_q(q, qmean):
+    """fp32(Q) - qbar of the token's block, one FP32 subtraction per element."""
+    q = np.asarray(q, np.float32)
+    N = q.shape[2]
+    return (q - np.asarray(qmean, np.float32)[:, :, np.arange(N) // BLOCK, :]).astype(np.float32)
+
+
+def smoothing_bias(qmean, k_smoothed):
+    """dS[b, h, blk, j] = qbar[b, h, blk] . k'[b, h, j] (reading 2).
+
+    qmean float32 [B, H, nb, d]; k_smoothed float32 [B, H, N, d].  FP64
+    accumulation in channel order c = 0 .. d-1 (every product of two FP32
+    values is exact in FP64), rounded once to FP32.  Returns float32
+    [B, H, nb, N].
+    """
+    qm = np.asarray(qmean, np.float32).astype(np.float64)
+    kk = np.asarray(k_smoothed, np.float32).astype(np.float64)
+    B, H, nb, d = qm.shape
+    N = kk.shape[2]
+    acc = np.zeros((B, H, nb, N), np.float64)
+    for c in range(d):                 # channel order
+        acc += qm[:, :, :, c, None] * kk[:, :, None, :, c]
+    return acc.astype(np.float32)
+
+
 def quant_int8_blocks(x, tokens=BLOCK):
     """Symmetric INT8 with one scale per block of `tokens` tokens (reading 3).
 
@@ -129,28 +181,44 @@ def quant_fp8_blocks(x, tokens=BLOCK):
     return codes, scales
 
 
-def quant_qk_fp8(q, k):
-    """FP8 Q/K mode pre-pass (reading 6; K smoothed as in reading 1).
+def _q_for_quant(q, k_smoothed, smooth):
+    """Q as it enters its quantizer, plus the smoothing outputs (reading 2)."""
+    if not smooth:
+        return np.asarray(q, np.float32), {}
+    qm = q_block_mean(q)
+    return smooth_q(q, qm), dict(q_mean=qm, dS=smoothing_bias(qm, k_smoothed))
+
+
+def quant_qk_fp8(q, k, smooth=False):
+    """FP8 Q/K mode pre-pass (reading 6; K smoothed as in reading 1; Q
+    smoothed as in reading 2 when `smooth`).
 
     Returns dict with q_codes, q_scales [B,H,N] (one per token), k_codes,
-    k_scales [B,H,ceil(N/32)], k_mean.
+    k_scales [B,H,ceil(N/32)], k_mean; with `smooth` also q_mean
+    [B,H,ceil(N/128),d] and dS [B,H,ceil(N/128),N].
     """
     mean = k_channel_mean(k)
-    qc, qs = quant_fp8_blocks(np.asarray(q, np.float32), Q_GROUP)
-    kc, ks = quant_fp8_blocks(smooth_k(k, mean), K_GROUP)
-    return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean)
+    ks_in = smooth_k(k, mean)
+    q_in, extra = _q_for_quant(q, ks_in, smooth)
+    qc, qs = quant_fp8_blocks(q_in, Q_GROUP)
+    kc, ks = quant_fp8_blocks(ks_in, K_GROUP)
+    return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean, **extra)
 
 
-def quant_qk_int8(q, k):
-    """INT8 mode pre-pass for Q and K (readings 1 and 3).
+def quant_qk_int8(q, k, smooth=False):
+    """INT8 mode pre-pass for Q and K (readings 1 and 3; Q smoothed as in
+    reading 2 when `smooth`).
 
     Returns dict with q_codes, q_scales [B,H,N] (one per token), k_codes,
-    k_scales [B,H,ceil(N/32)], k_mean.
+    k_scales [B,H,ceil(N/32)], k_mean; with `smooth` also q_mean
+    [B,H,ceil(N/128),d] and dS [B,H,ceil(N/128),N].
     """
     mean = k_channel_mean(k)
-    qc, qs = quant_int8_blocks(np.asarray(q, np.float32), Q_GROUP)
-    kc, ks = quant_int8_blocks(smooth_k(k, mean), K_GROUP)
-    return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean)
+    ks_in = smooth_k(k, mean)
+    q_in, extra = _q_for_quant(q, ks_in, smooth)
+    qc, qs = quant_int8_blocks(q_in, Q_GROUP)
+    kc, ks = quant_int8_blocks(ks_in, K_GROUP)
+    return dict(q_codes=qc, q_scales=qs, k_codes=kc, k_scales=ks, k_mean=mean, **extra)
 
 
 def quant_v_fp8(v):
@@ -218,11 +286,15 @@ def quant_fp4_tokens(x):
     return codes, sf, g
 
 
-def quant_qk_fp4(q, k):
+def quant_qk_fp4(q, k, smooth=False):
+    """FP4 mode pre-pass for Q and K (readings 1 and 5; Q smoothed as in
+    reading 2 when `smooth`)."""
     mean = k_channel_mean(k)
-    qc, qsf, qg = quant_fp4_tokens(np.asarray(q, np.float32))
-    kc, ksf, kg = quant_fp4_tokens(smooth_k(k, mean))
-    return dict(q_codes=qc, q_sf=qsf, q_g=qg, k_codes=kc, k_sf=ksf, k_g=kg, k_mean=mean)
+    ks_in = smooth_k(k, mean)
+    q_in, extra = _q_for_quant(q, ks_in, smooth)
+    qc, qsf, qg = quant_fp4_tokens(q_in)
+    kc, ksf, kg = quant_fp4_tokens(ks_in)
+    return dict(q_codes=qc, q_sf=qsf, q_g=qg, k_codes=kc, k_sf=ksf, k_g=kg, k_mean=mean, **extra)
 
 
 def quant_v_fp4(v):
