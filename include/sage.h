@@ -93,8 +93,18 @@ typedef enum { SAGE_DTYPE_F16 = 0, SAGE_DTYPE_BF16 = 1 } sage_dtype_t;
 typedef enum {
   SAGE_BUF_Q_CODES = 0, SAGE_BUF_Q_SCALES, SAGE_BUF_Q_SF,
   SAGE_BUF_K_CODES, SAGE_BUF_K_SCALES, SAGE_BUF_K_SF, SAGE_BUF_K_MEAN,
-  SAGE_BUF_V_CODES, SAGE_BUF_V_SCALES, SAGE_BUF_V_SF
+  SAGE_BUF_V_CODES, SAGE_BUF_V_SCALES, SAGE_BUF_V_SF,
+  /* Q smoothing (8-bit modes): the per-block Q means, FP32
+   * [B, H, ceil(N/128), d], and the score bias, FP32
+   * [B, H, ceil(N/128), 128 ceil(N/128)] */
+  SAGE_BUF_Q_MEAN, SAGE_BUF_DS
 } sage_buffer_t;
+
+/* OR'ed into the mode of sage_attn_fwd / sage_attn_fwd_gqa: Q smoothing
+ * (SageAttention2 abstract, "we propose a method to smooth Q"; see
+ * sage_quant_qk_smooth).  8-bit modes only (SAGE_ERR_UNSUPPORTED with
+ * FP4). */
+#define SAGE_FLAG_SMOOTH_Q 0x100
 
 /* Bytes of one quantized buffer for the given mode and shape (0 for a
  * buffer the mode does not use, e.g. *_SF outside FP4 mode). */
@@ -121,6 +131,27 @@ int sage_quant_qk(const void* q, const void* k, int dtype,
                   void* q_codes, float* q_scales, void* q_sf,
                   void* k_codes, float* k_scales, void* k_sf,
                   float* k_mean, sage_stream_t stream);
+
+/* The Q/K pre-pass with Q smoothing, 8-bit modes (SAGE_MODE_INT8_FP8,
+ * SAGE_MODE_FP8; SAGE_ERR_UNSUPPORTED for FP4).  Before Q is quantized,
+ * each (b, h) and 128-token block of queries loses its mean:
+ *   qbar = fp32(FP64 sum of the block's tokens in token order / count)
+ *   (the last block of a ragged sequence: its own tokens), written to
+ *   q_mean [B, H, ceil(N/128), d];
+ *   Q' = fp32(Q) - qbar (one FP32 subtraction) is quantized as Q is in
+ *   sage_quant_qk.
+ * What qbar takes out comes back as a bias on the block's scores,
+ *   ds[b, h, blk, j] = fp32( sum over c in order of qbar[blk, c] *
+ *                           (fp32(K[j, c]) - k_mean[c]) ),
+ * the sum in FP64 (every product exact), written to
+ * ds [B, H, ceil(N/128), 128 ceil(N/128)] (keys past N hold 0); it costs
+ * B H N^2 d / 128 FP64 multiply-adds.  K, its mean and its codes are as in
+ * sage_quant_qk.  Everything is bit-identical to the CPU oracle.  Buffer
+ * sizes: sage_buffer_bytes with SAGE_BUF_Q_MEAN and SAGE_BUF_DS. */
+int sage_quant_qk_smooth(const void* q, const void* k, int dtype,
+                         int64_t B, int64_t H, int64_t N, int64_t d, int mode,
+                         void* q_codes, float* q_scales, void* k_codes, float* k_scales,
+                         float* k_mean, float* q_mean, float* ds, sage_stream_t stream);
 
 /* V pre-pass.
  *   INT8_FP8 and FP8 modes: s_V[c] = fp32(amax_c / 448) over all N tokens
@@ -169,11 +200,25 @@ int sage_attn_fwd_quantized(int mode,
                             int64_t B, int64_t H, int64_t N, int64_t d,
                             int causal, float sm_scale, sage_stream_t stream);
 
+/* Attention with Q smoothing on the buffers of sage_quant_qk_smooth and
+ * sage_quant_v (8-bit modes): every score of query block blk and key j is
+ * dequantized as in sage_attn_fwd_quantized and gains ds[b, h, blk, j]
+ * sm_scale before the online softmax.  Other arguments and errors as in
+ * sage_attn_fwd_quantized. */
+int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q_scales,
+                                   const void* k_codes, const float* k_scales,
+                                   const void* v_codes, const float* v_scales, const float* ds,
+                                   void* o, int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
+                                   int causal, float sm_scale, sage_stream_t stream);
+
 /* The whole forward pass: pre-pass into a library-owned workspace (grown
  * on demand with stream-ordered allocation, one per (device, stream),
  * freed at unload; the pre-pass takes the launch forms of sage_quant_qkv),
  * then the attention kernel.  sm_scale <= 0 means 1/sqrt(d).  An allocation
- * failure returns SAGE_ERR_CUDA before any kernel is launched. */
+ * failure returns SAGE_ERR_CUDA before any kernel is launched.  mode may
+ * carry SAGE_FLAG_SMOOTH_Q (8-bit modes): the pre-pass is then that of
+ * sage_quant_qk_smooth (chained form only) and the attention that of
+ * sage_attn_fwd_quantized_smooth. */
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype,
                   int64_t B, int64_t H, int64_t N, int64_t d,
                   int causal, float sm_scale, int mode, sage_stream_t stream);
@@ -221,6 +266,8 @@ int sage_attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, int 
  *   - The second stream is shared by every caller stream of a device: two
  *     callers that run this pre-pass at once on different streams have their
  *     V chains serialised (results are unaffected). */
+/* (mode as in sage_attn_fwd, without SAGE_FLAG_SMOOTH_Q: a mode carrying
+ * it is SAGE_ERR_INVALID_ARG here.) */
 #define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, int dtype,
                           int64_t B, int64_t H, int64_t N, int64_t d,

@@ -14,6 +14,9 @@ Entry points (same names as the C ABI in include/sage.h):
     sage_attn_fwd_quantized(qk, vq, mode, causal, sm_scale, out_dtype) -> O
     sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8") -> O
     sage_attn_fwd_gqa(q, k, v, ...)           -> O  (K/V with fewer heads than Q)
+    sage_quant_qk_smooth(q, k, mode)          -> dict, with Q smoothing (q_mean, ds)
+    sage_attn_fwd_quantized_smooth(qk, vq, shape, mode, ...) -> O, with Q smoothing
+    (sage_attn_fwd(..., smooth_q=True) runs the whole pass with Q smoothing)
 """
 
 import ctypes
@@ -22,6 +25,7 @@ import os
 
 __all__ = ["sage_quant_qk", "sage_quant_v", "sage_quant_qkv", "sage_attn_fwd", "sage_attn_fwd_gqa",
            "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
+           "sage_quant_qk_smooth", "sage_attn_fwd_quantized_smooth", "SMOOTH_Q",
            "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS",
            "selftest_bounded_wait"]
 
@@ -29,14 +33,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libsage_b200.so")
 
 MODES = {"int8_fp8": 0, "fp4": 1, "fp8": 2}
+SMOOTH_Q = 0x100  # SAGE_FLAG_SMOOTH_Q, OR'ed into the mode of sage_attn_fwd
 DTYPES = {"f16": 0, "bf16": 1}
 BUF = {name: i for i, name in enumerate(
     ["q_codes", "q_scales", "q_sf", "k_codes", "k_scales", "k_sf", "k_mean",
-     "v_codes", "v_scales", "v_sf"])}
+     "v_codes", "v_scales", "v_sf", "q_mean", "ds"])}
 
 # every symbol include/sage.h declares
 EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv",
-           "sage_attn_fwd_quantized",
+           "sage_attn_fwd_quantized", "sage_quant_qk_smooth", "sage_attn_fwd_quantized_smooth",
            "sage_attn_fwd", "sage_attn_fwd_gqa", "sage_attn_fwd_noalloc",
            "sage_get_last_device_status",
            "sage_selftest_bounded_wait", "sage_status_string", "sage_version",
@@ -67,6 +72,12 @@ def library():
     lib.sage_quant_qk.restype = i32
     lib.sage_quant_qk.argtypes = [vp, vp, i32, i64, i64, i64, i64, i32,
                                   vp, fp, vp, vp, fp, vp, fp, vp]
+    lib.sage_quant_qk_smooth.restype = i32
+    lib.sage_quant_qk_smooth.argtypes = [vp, vp, i32, i64, i64, i64, i64, i32,
+                                         vp, fp, vp, fp, fp, fp, fp, vp]
+    lib.sage_attn_fwd_quantized_smooth.restype = i32
+    lib.sage_attn_fwd_quantized_smooth.argtypes = [i32, vp, fp, vp, fp, vp, fp, fp, vp, i32,
+                                                   i64, i64, i64, i64, i32, ctypes.c_float, vp]
     lib.sage_quant_v.restype = i32
     lib.sage_quant_v.argtypes = [vp, i32, i64, i64, i64, i64, i32, vp, fp, vp, vp]
     lib.sage_quant_qkv.restype = i32
@@ -160,6 +171,22 @@ def sage_quant_qk(q, k, mode="int8_fp8"):
     return bufs
 
 
+def sage_quant_qk_smooth(q, k, mode="int8_fp8"):
+    """Q/K pre-pass with Q smoothing (8-bit modes).  Returns {q_codes,
+    q_scales, k_codes, k_scales, k_mean, q_mean, ds} as raw uint8 tensors
+    laid out as include/sage.h describes."""
+    B, H, N, d = _shape(q)
+    if _shape(k) != (B, H, N, d) or k.dtype != q.dtype:
+        raise ValueError("q and k must have the same shape and dtype")
+    bufs = _alloc(mode, ["q_codes", "q_scales", "k_codes", "k_scales", "k_mean", "q_mean", "ds"],
+                  B, H, N, d, q.device)
+    _check(library().sage_quant_qk_smooth(
+        _ptr(q), _ptr(k), _dtype_code(q), B, H, N, d, MODES[mode],
+        _f(bufs["q_codes"]), _f(bufs["q_scales"]), _f(bufs["k_codes"]), _f(bufs["k_scales"]),
+        _f(bufs["k_mean"]), _f(bufs["q_mean"]), _f(bufs["ds"]), _stream()))
+    return bufs
+
+
 def sage_quant_v(v, mode="int8_fp8"):
     """V pre-pass.  Returns {v_codes, v_scales, v_sf} as raw uint8 tensors."""
     B, H, N, d = _shape(v)
@@ -209,14 +236,35 @@ def sage_attn_fwd_quantized(qk, vq, shape, mode="int8_fp8", causal=False, sm_sca
     return out
 
 
-def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None):
+def sage_attn_fwd_quantized_smooth(qk, vq, shape, mode="int8_fp8", causal=False, sm_scale=None,
+                                   out_dtype=None, out=None):
+    """Attention with Q smoothing on the dicts of sage_quant_qk_smooth and
+    sage_quant_v."""
+    import torch
+    B, H, N, d = shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=out_dtype or torch.bfloat16,
+                          device=qk["q_codes"].device)
+    _check(library().sage_attn_fwd_quantized_smooth(
+        MODES[mode], _f(qk["q_codes"]), _f(qk["q_scales"]), _f(qk["k_codes"]),
+        _f(qk["k_scales"]), _f(vq["v_codes"]), _f(vq["v_scales"]), _f(qk["ds"]),
+        _ptr(out), _dtype_code(out), B, H, N, d, int(bool(causal)), float(sm_scale), _stream()))
+    return out
+
+
+def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None,
+                  smooth_q=False):
     """O = softmax(Q K^T sm_scale) V through the quantized path; O has q's dtype.
     K and V with fewer heads than Q (grouped-query attention) go to
-    sage_attn_fwd_gqa."""
+    sage_attn_fwd_gqa.  smooth_q: Q smoothing (SAGE_FLAG_SMOOTH_Q, 8-bit
+    modes)."""
     import torch
     B, H, N, d = _shape(q)
     if _shape(k)[1] != H:
-        return sage_attn_fwd_gqa(q, k, v, causal=causal, sm_scale=sm_scale, mode=mode, out=out)
+        return sage_attn_fwd_gqa(q, k, v, causal=causal, sm_scale=sm_scale, mode=mode, out=out,
+                                 smooth_q=smooth_q)
     if _shape(k) != (B, H, N, d) or _shape(v) != (B, H, N, d):
         raise ValueError("q, k, v must have the same shape")
     if not (q.dtype == k.dtype == v.dtype):
@@ -225,11 +273,13 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=Non
         out = torch.empty_like(q)
     _check(library().sage_attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, N, d,
-        int(bool(causal)), float(sm_scale or 0.0), MODES[mode], _stream()))
+        int(bool(causal)), float(sm_scale or 0.0), MODES[mode] | (SMOOTH_Q if smooth_q else 0),
+        _stream()))
     return out
 
 
-def sage_attn_fwd_gqa(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None):
+def sage_attn_fwd_gqa(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None,
+                      smooth_q=False):
     """Grouped-query attention: q is [B, H, N, d], k and v are [B, Hkv, N, d]
     with Hkv dividing H; query head h reads key/value head h // (H // Hkv)."""
     import torch
@@ -243,7 +293,8 @@ def sage_attn_fwd_gqa(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out
         out = torch.empty_like(q)
     _check(library().sage_attn_fwd_gqa(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, Hkv, N, d,
-        int(bool(causal)), float(sm_scale or 0.0), MODES[mode], _stream()))
+        int(bool(causal)), float(sm_scale or 0.0), MODES[mode] | (SMOOTH_Q if smooth_q else 0),
+        _stream()))
     return out
 
 

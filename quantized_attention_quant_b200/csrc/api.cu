@@ -351,8 +351,10 @@ int check_kv_heads(int64_t H, int64_t Hkv) {
 
 // Q-side buffers are per query head, K/V-side ones per key/value head
 int64_t heads_of(int which, int64_t H, int64_t Hkv) {
-  return which == SAGE_BUF_Q_CODES || which == SAGE_BUF_Q_SCALES || which == SAGE_BUF_Q_SF ? H
-                                                                                          : Hkv;
+  return which == SAGE_BUF_Q_CODES || which == SAGE_BUF_Q_SCALES || which == SAGE_BUF_Q_SF ||
+                 which == SAGE_BUF_Q_MEAN || which == SAGE_BUF_DS
+             ? H
+             : Hkv;
 }
 
 // The whole pipeline (pre-pass, then attention) with every buffer carved
@@ -361,8 +363,12 @@ int64_t heads_of(int which, int64_t H, int64_t Hkv) {
 int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,
                   int64_t H, int64_t Hkv, int64_t N, int64_t d, int causal, float sm_scale,
                   int mode, sage_stream_t stream) {
+  const bool smooth = (mode & SAGE_FLAG_SMOOTH_Q) != 0;
+  mode &= ~SAGE_FLAG_SMOOTH_Q;
   bool empty = false;
   SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  if (smooth && mode == SAGE_MODE_FP4)
+    return fail(SAGE_ERR_UNSUPPORTED, "Q smoothing (SAGE_FLAG_SMOOTH_Q) needs an 8-bit mode");
   SAGE_TRY(check_kv_heads(H, Hkv));
   SAGE_TRY(check_ptr(q, "q", true));
   SAGE_TRY(check_ptr(k, "k", true));
@@ -384,6 +390,10 @@ int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtyp
   total += align_up(ws_ksum_bytes(B * Hkv, N, d));
   const size_t off_vmax = total;
   total += align_up(ws_vmax_bytes(B * Hkv, N, d));
+  const size_t off_qmean = total;
+  if (smooth) total += align_up(sage_buffer_bytes(mode, SAGE_BUF_Q_MEAN, B, H, N, d));
+  const size_t off_ds = total;
+  if (smooth) total += align_up(sage_buffer_bytes(mode, SAGE_BUF_DS, B, H, N, d));
   void* ws = nullptr;
   uint32_t* cnt = nullptr;
   SAGE_TRY(workspace(st, total, &ws, &cnt));
@@ -400,12 +410,17 @@ int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtyp
                 reinterpret_cast<double*>(base + off_ksum),
                 reinterpret_cast<float*>(base + off_vmax), cnt};
   qa.status = di->status;
+  if (smooth) {
+    qa.q_mean = reinterpret_cast<float*>(base + off_qmean);
+    qa.ds = reinterpret_cast<float*>(base + off_ds);
+  }
   SAGE_TRY(prepass_forked(qa, va, st));
   cudaError_t e = cudaSuccess;
   AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
               at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
               at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
               o, dtype, B, H, N, d, Hkv, causal != 0, sm_scale, di->status};
+  aa.ds = qa.ds;
   const char* detail = nullptr;
   e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
   if (detail) return fail(SAGE_ERR_CUDA, detail);
@@ -443,6 +458,10 @@ size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, i
       return (size_t)(fp4 ? BH * nt * 4 : BH * d * 4);
     case SAGE_BUF_V_SF:
       return fp4 ? (size_t)(BH * nt * 2 * 512) : 0;
+    case SAGE_BUF_Q_MEAN:
+      return fp4 ? 0 : (size_t)(BH * nt * d * 4);
+    case SAGE_BUF_DS:
+      return fp4 ? 0 : (size_t)(BH * nt * nt * 128 * 4);
     default:
       return 0;
   }
@@ -478,6 +497,38 @@ int sage_quant_qk(const void* q, const void* k, int dtype, int64_t B, int64_t H,
                 k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws), cnt};
   cudaError_t e = launch_quant_qk(a, st);
   if (e != cudaSuccess) return fail_cuda(e, "quant_qk launch");
+  return SAGE_OK;
+}
+
+int sage_quant_qk_smooth(const void* q, const void* k, int dtype, int64_t B, int64_t H, int64_t N,
+                         int64_t d, int mode, void* q_codes, float* q_scales, void* k_codes,
+                         float* k_scales, float* k_mean, float* q_mean, float* ds,
+                         sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  if (mode == SAGE_MODE_FP4) return fail(SAGE_ERR_UNSUPPORTED, "Q smoothing needs an 8-bit mode");
+  SAGE_TRY(check_ptr(q, "q", true));
+  SAGE_TRY(check_ptr(k, "k", true));
+  SAGE_TRY(check_ptr(q_codes, "q_codes", true));
+  SAGE_TRY(check_ptr(q_scales, "q_scales", true));
+  SAGE_TRY(check_ptr(k_codes, "k_codes", true));
+  SAGE_TRY(check_ptr(k_scales, "k_scales", true));
+  SAGE_TRY(check_ptr(k_mean, "k_mean", true));
+  SAGE_TRY(check_ptr(q_mean, "q_mean", true));
+  SAGE_TRY(check_ptr(ds, "ds", true));
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  uint32_t* cnt = nullptr;
+  SAGE_TRY(workspace(st, ws_ksum_bytes(B * H, N, d), &ws, &cnt));
+  QuantQKArgs a{q, k, dtype, mode, B, H, N, d, H, q_codes, q_scales, nullptr,
+                k_codes, k_scales, nullptr, k_mean, static_cast<double*>(ws), cnt};
+  a.q_mean = q_mean;
+  a.ds = ds;
+  cudaError_t e = launch_quant_qk(a, st);
+  if (e != cudaSuccess) return fail_cuda(e, "quant_qk_smooth launch");
   return SAGE_OK;
 }
 
@@ -583,6 +634,38 @@ int sage_attn_fwd_quantized(int mode, const void* q_codes, const float* q_scales
   const char* detail = nullptr;
   cudaError_t e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(a, st, &detail)
                                         : launch_attn_i8f8(a, st, &detail);
+  if (detail) return fail(SAGE_ERR_CUDA, detail);
+  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  return SAGE_OK;
+}
+
+int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q_scales,
+                                   const void* k_codes, const float* k_scales,
+                                   const void* v_codes, const float* v_scales, const float* ds,
+                                   void* o, int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
+                                   int causal, float sm_scale, sage_stream_t stream) {
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
+  if (mode == SAGE_MODE_FP4) return fail(SAGE_ERR_UNSUPPORTED, "Q smoothing needs an 8-bit mode");
+  SAGE_TRY(check_ptr(q_codes, "q_codes", true));
+  SAGE_TRY(check_ptr(q_scales, "q_scales", true));
+  SAGE_TRY(check_ptr(k_codes, "k_codes", true));
+  SAGE_TRY(check_ptr(k_scales, "k_scales", true));
+  SAGE_TRY(check_ptr(v_codes, "v_codes", true));
+  SAGE_TRY(check_ptr(v_scales, "v_scales", true));
+  SAGE_TRY(check_ptr(ds, "ds", true));
+  SAGE_TRY(check_ptr(o, "o", true));
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
+    return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be positive and finite");
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  AttnArgs a{mode, q_codes, q_scales, nullptr, k_codes, k_scales, nullptr, v_codes, v_scales,
+             nullptr, o, dtype, B, H, N, d, H, causal != 0, sm_scale, di->status};
+  a.ds = ds;
+  const char* detail = nullptr;
+  cudaError_t e = launch_attn_i8f8(a, st, &detail);
   if (detail) return fail(SAGE_ERR_CUDA, detail);
   if (e != cudaSuccess) return fail_cuda(e, "attention launch");
   return SAGE_OK;

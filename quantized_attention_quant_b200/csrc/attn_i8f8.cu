@@ -103,7 +103,9 @@ struct Layout {
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
   static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots][4] s_K sm_scale log2 e per 32 keys
   static constexpr int OFF_VS = OFF_C + 128;         // s_V[D] of the head (bulk-copied with Q)
-  static constexpr int END = OFF_VS + 4 * D;
+  // Q smoothing: the score bias of key tile j (log2 units) in slot j % 4
+  static constexpr int OFF_BIAS = OFF_VS + 4 * D;
+  static constexpr int END = OFF_BIAS + 4 * 128 * 4;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t QK_SBO = 8 * D;  // 8 rows of D bytes
@@ -130,6 +132,7 @@ struct Bars {
   uint64_t* pv_empty;  // [PVB] stats -> MMA: PV[b] read
   uint64_t* l_ready;   // [1] exp -> stats: final row sums
   uint64_t* drain;     // MMA drain on abort
+  uint64_t* bias_full; // [2] stats -> stats: a tile's bias is in shared memory (Q smoothing)
 };
 
 template <int D>
@@ -152,13 +155,14 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.pv_empty = r.pv_full + L::PVB;
   r.l_ready = r.pv_empty + L::PVB;
   r.drain = r.l_ready + 1;
+  r.bias_full = r.drain + 1;
   return r;
 }
 
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
 // RAGGED (non-causal launches of a sequence whose last tile is partial): the
 // last key tile masks keys n_tail .. 127.
-template <int D, bool CAUSAL, bool QF8, bool RAGGED>
+template <int D, bool CAUSAL, bool QF8, bool RAGGED, bool SMOOTH>
 __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
                                          const int bh, const int ntiles,
                                          const float* __restrict__ q_scales, const uint32_t tmem,
@@ -220,11 +224,13 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, ca, neg, lim, P)
-                       : exp_chunk<false, QF8>(sa, 2 * h, ca, neg, lim, P);
+    // Q smoothing: this tile's key biases (m_full(j) orders them too)
+    const float* bias = reinterpret_cast<const float*>(smem + L::OFF_BIAS) + (j & 3) * 128 + 64 * h;
+    float sum = masked ? exp_chunk<true, QF8, SMOOTH>(sa, 2 * h, ca, neg, lim, P, bias)
+                       : exp_chunk<false, QF8, SMOOTH>(sa, 2 * h, ca, neg, lim, P, bias);
     if (r == 0 && h == 0) SAGE_TR(14, j);
-    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8)
-                  : exp_chunk<false, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8);
+    sum += masked ? exp_chunk<true, QF8, SMOOTH>(sb, 2 * h + 1, cb, neg, lim, P + 8, bias + 32)
+                  : exp_chunk<false, QF8, SMOOTH>(sb, 2 * h + 1, cb, neg, lim, P + 8, bias + 32);
     l = fmaf(alpha, l, sum);
     if (r == 0 && h == 0) SAGE_TR(10, j);
     tmem_wait_st();
@@ -239,7 +245,7 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 
 // Stats warpgroup: row max / running max per key tile, level-2 fold,
 // epilogue.
-template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED>
+template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED, bool SMOOTH>
 __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int n_tail,
                                            const int bh, const int H, const int G, const int N,
                                            const int ntiles, const uint32_t tmem, const Bars& bar,
@@ -247,6 +253,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
                                            uint32_t* status, const float* __restrict__ q_scales,
                                            const float* __restrict__ k_scales,
                                            const float* __restrict__ v_scales,
+                                           const float* __restrict__ ds,
                                            OutT* __restrict__ out, const float scale_log2) {
   using L = Layout<D>;
   const int warp = threadIdx.x >> 5;
@@ -294,6 +301,21 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float alpha_hist[2] = {0.f, 0.f};
   float* c_s = reinterpret_cast<float*>(smem + L::OFF_C);
   float4 ks_cur = ldg4_early(ksp);
+  // Q smoothing: this query block's score bias.  Thread r writes key
+  // 128 j + r of tile j (log2 units) into slot j % 4 of the shared bias
+  // buffer one tile ahead, after publishing tile j - 1's maximum, and
+  // arrives on bias_full[j % 2]; the whole buffer is then read by every row's
+  // maximum and, after m_full, by the exp warpgroups.  A slot is rewritten
+  // for tile j + 4 only once both exp warpgroups and every stats thread are
+  // past tile j (the s_full wait of tile j + 3 comes first).
+  const float* dsr = SMOOTH ? ds + ((int64_t)bh * ntiles + qt) * (int64_t)(ntiles * 128) : nullptr;
+  float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);
+  float d_nxt = 0.f;
+  if (SMOOTH) {
+    bias_s[r] = ldg_early(dsr + r) * scale_log2;
+    mbar_arrive(&bar.bias_full[0]);
+    if (nkv > 1) d_nxt = ldg_early(dsr + 128 + r);
+  }
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
     // s_K sm_scale log2 e of the tile's four 32-key chunks; a row's factor
@@ -311,6 +333,10 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     const bool masked = diag || (RAGGED && j == nkv - 1);
     const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
+    const float* bias = bias_s + (j & 3) * 128;
+    if (SMOOTH && !__all_sync(0xffffffffu, mbar_wait(&bar.bias_full[b], (j >> 1) & 1, abort_flag,
+                                                     status, kDevTimeoutSoftmax)))
+      return;
     float mx = -INFINITY;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -319,11 +345,21 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      // each chunk's factor is >= 0, so its scaled max is the max scaled
-      mx = masked ? scaled_max64<true, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
-                                            qs * kl[2 * hh + 1], mx)
-                  : scaled_max64<false, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
-                                             qs * kl[2 * hh + 1], mx);
+      if (SMOOTH) {
+        // biased scores: the maximum of the sums
+        const float c0 = qs * kl[2 * hh], c1 = qs * kl[2 * hh + 1];
+        mx = masked ? fmax3(mx, max32_biased<true, QF8>(s[0], 64 * hh, lim, c0, bias + 64 * hh),
+                            max32_biased<true, QF8>(s[1], 64 * hh + 32, lim, c1, bias + 64 * hh + 32))
+                    : fmax3(mx, max32_biased<false, QF8>(s[0], 64 * hh, lim, c0, bias + 64 * hh),
+                            max32_biased<false, QF8>(s[1], 64 * hh + 32, lim, c1,
+                                                     bias + 64 * hh + 32));
+      } else {
+        // each chunk's factor is >= 0, so its scaled max is the max scaled
+        mx = masked ? scaled_max64<true, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                              qs * kl[2 * hh + 1], mx)
+                    : scaled_max64<false, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                               qs * kl[2 * hh + 1], mx);
+      }
     }
     const float m_j = fmaxf(m, mx);
     const float alpha = ex2(m - m_j);
@@ -340,6 +376,12 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     // S[b] has been read: the exp warpgroups may overwrite it with P~ codes
     tc_fence_before();
     mbar_arrive(&bar.m_full[b]);
+    if (SMOOTH && j + 1 < nkv) {
+      // the next tile's bias, and the one after it from global memory
+      bias_s[((j + 1) & 3) * 128 + r] = d_nxt * scale_log2;
+      mbar_arrive(&bar.bias_full[b ^ 1]);
+      if (j + 2 < nkv) d_nxt = ldg_early(dsr + 128 * (j + 2) + r);
+    }
     if (j >= L::PVB && !fold(j - L::PVB, alpha_hist[j % L::PVB])) return;
     alpha_hist[j % L::PVB] = alpha;
     ks_cur = ks_nxt;
@@ -369,14 +411,14 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   }
 }
 
-template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED>
+template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED, bool SMOOTH>
 __global__ void __launch_bounds__(kThreadsAttn, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scales,
                      const float* __restrict__ k_scales, const float* __restrict__ v_scales,
-                     OutT* __restrict__ out, int N, int H, int G, float scale_log2,
-                     int head_major, uint32_t* status) {
+                     const float* __restrict__ ds, OutT* __restrict__ out, int N, int H, int G,
+                     float scale_log2, int head_major, uint32_t* status) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -429,6 +471,8 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     mbar_init(bar.s_init, 256);
     mbar_init(bar.l_ready, 256);
     mbar_init(bar.drain, 1);
+    mbar_init(&bar.bias_full[0], 128);
+    mbar_init(&bar.bias_full[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -565,12 +609,13 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, qt, nkv, n_tail, bh, ntiles, q_scales, tmem, bar,
+    exp_loop<D, CAUSAL, QF8, RAGGED, SMOOTH>(wg - 1, qt, nkv, n_tail, bh, ntiles, q_scales, tmem, bar,
                                      smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<D, CAUSAL, OutT, QF8, RAGGED>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
-                                q_scales, k_scales, v_scales, out, scale_log2);
+    stats_loop<D, CAUSAL, OutT, QF8, RAGGED, SMOOTH>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar,
+                                                     smem, abort_flag, status, q_scales, k_scales,
+                                                     v_scales, ds, out, scale_log2);
   }
 
   tc_fence_before();
@@ -589,14 +634,15 @@ template <int D, bool CAUSAL, typename OutT, bool QF8, bool RAGGED = false>
 cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, cudaStream_t st) {
   using L = Layout<D>;
-  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, QF8, RAGGED>;
+  auto kern = a.ds ? attn_i8f8_kernel<D, CAUSAL, OutT, QF8, RAGGED, true>
+                   : attn_i8f8_kernel<D, CAUSAL, OutT, QF8, RAGGED, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((a.N + 127) / 128);
   const int hm = head_major_grid(a);
   const dim3 grid = hm ? dim3((unsigned)(a.B * a.H), (unsigned)ntiles)
                        : dim3((unsigned)ntiles, (unsigned)(a.B * a.H));
-  kern<<<grid, kThreadsAttn, L::SMEM, st>>>(tq, tk, tv, a.q_scales, a.k_scales, a.v_scales,
+  kern<<<grid, kThreadsAttn, L::SMEM, st>>>(tq, tk, tv, a.q_scales, a.k_scales, a.v_scales, a.ds,
                                            reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H,
                                            (int)(a.H / a.Hkv), a.sm_scale * kLog2e, hm,
                                            a.status);

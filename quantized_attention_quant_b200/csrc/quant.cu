@@ -49,6 +49,8 @@ enum Role : int {
   kStatsV = 8,    // V chunk maxima
   kQuantQF8 = 9,  // FP8 (e4m3) Q codes + block scales
   kQuantKF8 = 10, // FP8 (e4m3) smoothed-K codes + block scales (needs the K mean)
+  kQuantQ8S = 11,  // INT8 codes of the smoothed Q (tile mean out) + scales + the mean
+  kQuantQF8S = 12, // FP8 codes of the smoothed Q + scales + the mean
 };
 
 struct Roles {
@@ -80,6 +82,7 @@ struct PrepassPtrs {
   double* ksum;  // [B*H, N/128, d] FP64 chunk sums of K
   float* vmax;   // [B*H, N/128, d] chunk maxima of |V|
   uint32_t* cnt;  // [2][kMaxHeads] statistics CTAs done per head (K, V); 0 between passes
+  float* q_mean;  // [B*H, Np/128, d] per-tile Q means (Q smoothing)
   int64_t bh_q;   // Q heads (B * H)
   int64_t bh_kv;  // K/V heads (B * Hkv; fewer than bh_q under grouped-query attention)
 };
@@ -446,6 +449,31 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
   }
 }
 
+// ------------------------------------------------------- smoothed Q
+// Q smoothing (SageAttention2 abstract: "we propose a method to smooth Q"):
+// the tile is staged in shared memory, thread c < D takes the FP64 sum of
+// channel c over the tile's real tokens in token order, qbar = fp32(sum /
+// count) goes to global memory and to shared memory, and the tile is
+// encoded as Q - qbar (one FP32 subtraction) with the 8-bit encoder.
+template <typename T, int D, bool FP8, bool RAGGED>
+__device__ __forceinline__ void role_quant_q_smooth(const T* __restrict__ src, float* q_mean_out,
+                                                    uint8_t* __restrict__ dst, float* scale_out,
+                                                    T* tile, float* mean_s, float* red, int nv) {
+  stage_tile<T, D, RAGGED>(src, tile, nv);
+  __syncthreads();
+  const int t = threadIdx.x;
+  if (t < D) {
+    double acc = 0.0;
+#pragma unroll 16
+    for (int i = 0; i < nv; ++i) acc += (double)static_cast<float>(tile[i * D + t]);
+    const float m = __double2float_rn(__ddiv_rn(acc, (double)nv));
+    mean_s[t] = m;
+    q_mean_out[t] = m;
+  }
+  __syncthreads();
+  role_quant_8bit<T, D, FP8, RAGGED, 1, true>(tile, mean_s, dst, scale_out, red, nv);
+}
+
 // ---------------------------------------------------------------- FP8 V
 // codes = e4m3(V / s_V[c]) written transposed into V^T.  The tile is staged
 // in shared memory; a thread then owns a channel pair and 32 consecutive
@@ -702,19 +730,22 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   // one role)
   constexpr bool kV4 = ((MASK >> kQuantV4) & 1) != 0;
   constexpr bool kTile = ((MASK >> kQuantV8) & 1) || ((MASK >> kStatsK) & 1) ||
-                         ((MASK >> kStatsKV) & 1);
+                         ((MASK >> kStatsKV) & 1) || ((MASK >> kQuantQ8S) & 1) ||
+                         ((MASK >> kQuantQF8S) & 1);
   constexpr int V4_BYTES = kV4 ? 128 * (D + 2) * (int)sizeof(T) : 16;
   constexpr int TILE_BYTES = kTile ? 128 * D * (int)sizeof(T) : 16;
   constexpr int SMEM_BYTES = V4_BYTES > TILE_BYTES ? V4_BYTES : TILE_BYTES;
   __shared__ __align__(16) uint8_t smem_raw[SMEM_BYTES];
   __shared__ uint32_t vmax_s[D];
   __shared__ float red[4 * (kThreads / 32)];
+  __shared__ __align__(16) float qmean_s[D];
   const int role = roles.r[blockIdx.z];
   const int64_t bh = roles.reverse ? (int64_t)(gridDim.y - 1 - blockIdx.y) : (int64_t)blockIdx.y;
   const int tile = roles.reverse ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   // the grid spans the larger head count: Q roles cover bh_q heads, K/V
   // roles bh_kv (a CTA leaves as a whole, before any barrier)
-  const bool q_role = role == kQuantQ8 || role == kQuantQ4 || role == kQuantQF8;
+  const bool q_role = role == kQuantQ8 || role == kQuantQ4 || role == kQuantQF8 ||
+                      role == kQuantQ8S || role == kQuantQF8S;
   if (bh >= (q_role ? p.bh_q : p.bh_kv)) return;
   // (without RAGGED, Np == N: the same offsets as before padding existed)
   const int ntiles = (RAGGED ? p.Np : p.N) / 128;
@@ -748,6 +779,20 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
                                   p.k_mean + bh * D,
                                   reinterpret_cast<uint8_t*>(p.k_codes) + crow0 * D,
                                   p.k_scales + crow0 / 32, red, nv);
+      break;
+    case kQuantQ8S:
+      SAGE_ROLE(kQuantQ8S)
+      role_quant_q_smooth<T, D, false, RAGGED>(
+          reinterpret_cast<const T*>(p.q) + row0 * D, p.q_mean + (bh * ntiles + tile) * D,
+          reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * D, p.q_scales + crow0,
+          reinterpret_cast<T*>(smem_raw), qmean_s, red, nv);
+      break;
+    case kQuantQF8S:
+      SAGE_ROLE(kQuantQF8S)
+      role_quant_q_smooth<T, D, true, RAGGED>(
+          reinterpret_cast<const T*>(p.q) + row0 * D, p.q_mean + (bh * ntiles + tile) * D,
+          reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * D, p.q_scales + crow0,
+          reinterpret_cast<T*>(smem_raw), qmean_s, red, nv);
       break;
     case kQuantV8:
       SAGE_ROLE(kQuantV8)
@@ -966,6 +1011,112 @@ cudaError_t dispatch(const PrepassPtrs& p, int dtype, int64_t d, Roles a, Roles 
                   : run_plan<__half, 64, MA, MB>(p, a, b, st);
 }
 
+// ------------------------------------------------- smoothing bias dS
+// dS[bh, blk, j] = fp32(sum_c qbar[bh, blk, c] * k'[j, c]), k' = fp32(K) -
+// mean_K of the key/value head, the sum in FP64 in channel order (products
+// of FP32 values are exact in FP64, so FMA and multiply-then-add agree):
+// the oracle's arithmetic, bit for bit.  A CTA takes 64 keys and 32 query
+// blocks of one query head; a thread a 4 x 4 register tile (keys tx + 16 i,
+// blocks ty + 8 i), reading two channels of a key or a block per 16-byte
+// shared load.  Keys past N get 0.
+constexpr int kBiasKeys = 64;
+constexpr int kBiasBlocks = 32;
+constexpr int kBiasThreads = 128;
+
+template <int D>
+constexpr int bias_smem_bytes() {
+  return (kBiasKeys + kBiasBlocks) * (D / 2) * 16;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kBiasThreads)
+    smoothing_bias_kernel(const T* __restrict__ k, const float* __restrict__ k_mean,
+                          const float* __restrict__ q_mean, float* __restrict__ ds, int N, int Np,
+                          int nblk, int H, int G) {
+  extern __shared__ __align__(16) double2 bias_smem[];
+  double2* ks = bias_smem;                              // [D/2][64]: k' of channels 2cp, 2cp+1
+  double2* qs = bias_smem + (D / 2) * kBiasKeys;        // [D/2][32]: qbar likewise
+  const int bh = (int)blockIdx.z;
+  const int bhk = kv_head(bh, H, G);
+  const int j0 = (int)blockIdx.x * kBiasKeys;
+  const int b0 = (int)blockIdx.y * kBiasBlocks;
+  const int nb = min(kBiasBlocks, nblk - b0);
+  const int t = threadIdx.x;
+  for (int i = t; i < kBiasKeys * (D / 2); i += kBiasThreads) {
+    const int key = i / (D / 2), cp = i % (D / 2);
+    const int j = j0 + key;
+    float k0 = 0.f, k1 = 0.f;
+    if (j < N) {
+      const T* row = k + ((int64_t)bhk * N + j) * D + 2 * cp;
+      const float* mu = k_mean + (int64_t)bhk * D + 2 * cp;
+      k0 = __fsub_rn(static_cast<float>(row[0]), mu[0]);
+      k1 = __fsub_rn(static_cast<float>(row[1]), mu[1]);
+    }
+    ks[cp * kBiasKeys + key] = make_double2((double)k0, (double)k1);
+  }
+  for (int i = t; i < kBiasBlocks * (D / 2); i += kBiasThreads) {
+    const int blk = i / (D / 2), cp = i % (D / 2);
+    const float* qm = q_mean + ((int64_t)bh * nblk + b0 + blk) * D + 2 * cp;
+    qs[cp * kBiasBlocks + blk] =
+        blk < nb ? make_double2((double)qm[0], (double)qm[1]) : make_double2(0.0, 0.0);
+  }
+  __syncthreads();
+  const int tx = t % 16, ty = t / 16;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+#pragma unroll 2
+  for (int cp = 0; cp < D / 2; ++cp) {
+    double2 kv[4], qv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) kv[i] = ks[cp * kBiasKeys + tx + 16 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = qs[cp * kBiasBlocks + ty + 8 * i];
+    // channel 2cp, then 2cp + 1: the channel order of every sum
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[b].x, kv[a].x, acc[a][b]);
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[b].y, kv[a].y, acc[a][b]);
+  }
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int j = j0 + tx + 16 * a;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int blk = b0 + ty + 8 * b;
+      if (blk < nblk) ds[((int64_t)bh * nblk + blk) * Np + j] = j < N ? __double2float_rn(acc[a][b]) : 0.f;
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t run_bias(const QuantQKArgs& a, cudaStream_t st) {
+  auto kern = smoothing_bias_kernel<T, D>;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bias_smem_bytes<D>());
+  if (e != cudaSuccess) return e;
+  const int Np = (int)((a.N + 127) / 128 * 128);
+  const int nblk = Np / 128;
+  const dim3 grid((unsigned)(Np / kBiasKeys), (unsigned)((nblk + kBiasBlocks - 1) / kBiasBlocks),
+                  (unsigned)(a.B * a.H));
+  kern<<<grid, kBiasThreads, bias_smem_bytes<D>(), st>>>(
+      static_cast<const T*>(a.k), a.k_mean, a.q_mean, a.ds, (int)a.N, Np, nblk, (int)a.H,
+      (int)(a.H / a.Hkv));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_smoothing_bias(const QuantQKArgs& a, cudaStream_t st) {
+  if (a.dtype == 1)
+    return a.d == 128 ? run_bias<__nv_bfloat16, 128>(a, st) : run_bias<__nv_bfloat16, 64>(a, st);
+  return a.d == 128 ? run_bias<__half, 128>(a, st) : run_bias<__half, 64>(a, st);
+}
+
 PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
   PrepassPtrs p{};
   p.q = a.q;
@@ -981,6 +1132,7 @@ PrepassPtrs ptrs_qk(const QuantQKArgs& a) {
   p.k_mean = a.k_mean;
   p.ksum = a.ws_ksum;
   p.cnt = a.ws_cnt;
+  p.q_mean = a.q_mean;
   p.bh_q = a.B * a.H;
   p.bh_kv = a.B * a.Hkv;
   return p;
@@ -1020,7 +1172,7 @@ constexpr int64_t kFusedMaxHeads = 16;
 bool fused_prepass_fits(const QuantQKArgs& a) {
   const int64_t ntiles = (a.N + 127) / 128;
   const int64_t BH = a.B * a.H;
-  return a.mode != kModeFp4 && a.status != nullptr && ntiles > 0 &&
+  return a.mode != kModeFp4 && a.status != nullptr && a.q_mean == nullptr && ntiles > 0 &&
          ntiles <= kFusedCluster && BH <= kFusedMaxHeads && (a.d == 64 || a.d == 128);
 }
 
@@ -1044,6 +1196,19 @@ cudaError_t launch_prepass_fused(const QuantQKArgs& qa, const QuantVArgs& va, cu
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
   const PrepassPtrs p = ptrs_qk(a);
+  if (a.q_mean) {
+    // Q smoothing (8-bit modes): smoothed Q codes and the means beside the K
+    // statistics, then the K codes, then the bias (it needs both means)
+    cudaError_t e;
+    if (a.mode == kModeInt8Fp8)
+      e = dispatch<bit(kQuantQ8S) | bit(kStatsK), bit(kQuantK8)>(
+          p, a.dtype, a.d, Roles{2, {kQuantQ8S, kStatsK}}, Roles{1, {kQuantK8}}, st);
+    else
+      e = dispatch<bit(kQuantQF8S) | bit(kStatsK), bit(kQuantKF8)>(
+          p, a.dtype, a.d, Roles{2, {kQuantQF8S, kStatsK}}, Roles{1, {kQuantKF8}}, st);
+    if (e != cudaSuccess) return e;
+    return launch_smoothing_bias(a, st);
+  }
   if (a.mode == kModeInt8Fp8)
     return dispatch<bit(kQuantQ8) | bit(kStatsK), bit(kQuantK8)>(
         p, a.dtype, a.d, Roles{2, {kQuantQ8, kStatsK}}, Roles{1, {kQuantK8}}, st);

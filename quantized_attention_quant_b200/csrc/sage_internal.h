@@ -31,6 +31,11 @@ struct QuantQKArgs {
   uint32_t* ws_cnt;  // [2][65536] per-head statistics counters: zero before the
                      // call, zero again after it (workspace)
   uint32_t* status = nullptr;  // device status word (bounded waits of the fused pre-pass)
+  // Q smoothing (8-bit modes): when q_mean is set, Q loses its per-128-token
+  // block mean before quantization (q_mean [B*H, N/128, d] FP32 receives
+  // it) and ds [B*H, N/128, Np] FP32 receives the score bias qbar . k'
+  float* q_mean = nullptr;
+  float* ds = nullptr;
 };
 
 struct QuantVArgs {
@@ -69,6 +74,9 @@ struct AttnArgs {
   int causal;
   float sm_scale;
   uint32_t* status;  // device status word
+  // Q smoothing: the score bias [B*H, N/128, Np] of sage_quant_qk_smooth
+  // (null: none)
+  const float* ds = nullptr;
 };
 
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st);
@@ -110,6 +118,7 @@ inline int head_major_grid(const AttnArgs& a) {
 // keep one CTA each, which the hardware balances itself.
 int sm_count();
 inline bool use_persistent_attention(const AttnArgs& a) {
+  if (a.ds) return false;  // Q smoothing runs in the one-item-per-CTA kernel
   const int64_t ntiles = (a.N + 127) / 128;
   const int64_t mean_tiles = a.causal ? (ntiles + 1) / 2 : ntiles;
   return mean_tiles <= 64 && ntiles * a.B * a.H > sm_count();

@@ -44,10 +44,11 @@ def cosine(a, b):
     return float(a @ b / math.sqrt((a @ a) * (b @ b)))
 
 
-def check_against_oracle(o_gpu, q, k, v, causal, sm_scale, mode, dtype, rows=None, cos_floor=None):
+def check_against_oracle(o_gpu, q, k, v, causal, sm_scale, mode, dtype, rows=None, cos_floor=None,
+                         smooth_q=False):
     qs, ks, vs = (to_numpy32(t) for t in (q, k, v))
     emu, amb = att.emulated_sage_attention(qs, ks, vs, causal, sm_scale, mode=mode, rows=rows,
-                                           ambiguity_eps=AMBIGUITY_EPS)
+                                           ambiguity_eps=AMBIGUITY_EPS, smooth_q=smooth_q)
     ex = att.exact_attention(qs, ks, vs, causal, sm_scale, rows=rows)
     g = o_gpu.astype(np.float64)
     err = np.abs(g - emu)
