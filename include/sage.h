@@ -94,16 +94,14 @@ typedef enum {
   SAGE_BUF_Q_CODES = 0, SAGE_BUF_Q_SCALES, SAGE_BUF_Q_SF,
   SAGE_BUF_K_CODES, SAGE_BUF_K_SCALES, SAGE_BUF_K_SF, SAGE_BUF_K_MEAN,
   SAGE_BUF_V_CODES, SAGE_BUF_V_SCALES, SAGE_BUF_V_SF,
-  /* Q smoothing (8-bit modes): the per-block Q means, FP32
-   * [B, H, ceil(N/128), d], and the score bias, FP32
-   * [B, H, ceil(N/128), 128 ceil(N/128)] */
+  /* Q smoothing: the per-block Q means, FP32 [B, H, ceil(N/128), d], and
+   * the score bias, FP32 [B, H, ceil(N/128), 128 ceil(N/128)] */
   SAGE_BUF_Q_MEAN, SAGE_BUF_DS
 } sage_buffer_t;
 
 /* OR'ed into the mode of sage_attn_fwd / sage_attn_fwd_gqa: Q smoothing
  * (SageAttention2 abstract, "we propose a method to smooth Q"; see
- * sage_quant_qk_smooth).  8-bit modes only (SAGE_ERR_UNSUPPORTED with
- * FP4). */
+ * sage_quant_qk_smooth), in every mode. */
 #define SAGE_FLAG_SMOOTH_Q 0x100
 
 /* Bytes of one quantized buffer for the given mode and shape (0 for a
@@ -132,8 +130,7 @@ int sage_quant_qk(const void* q, const void* k, int dtype,
                   void* k_codes, float* k_scales, void* k_sf,
                   float* k_mean, sage_stream_t stream);
 
-/* The Q/K pre-pass with Q smoothing, 8-bit modes (SAGE_MODE_INT8_FP8,
- * SAGE_MODE_FP8; SAGE_ERR_UNSUPPORTED for FP4).  Before Q is quantized,
+/* The Q/K pre-pass with Q smoothing, in every mode.  Before Q is quantized,
  * each (b, h) and 128-token block of queries loses its mean:
  *   qbar = fp32(FP64 sum of the block's tokens in token order / count)
  *   (the last block of a ragged sequence: its own tokens), written to
@@ -150,7 +147,8 @@ int sage_quant_qk(const void* q, const void* k, int dtype,
  * sizes: sage_buffer_bytes with SAGE_BUF_Q_MEAN and SAGE_BUF_DS. */
 int sage_quant_qk_smooth(const void* q, const void* k, int dtype,
                          int64_t B, int64_t H, int64_t N, int64_t d, int mode,
-                         void* q_codes, float* q_scales, void* k_codes, float* k_scales,
+                         void* q_codes, float* q_scales, void* q_sf,
+                         void* k_codes, float* k_scales, void* k_sf,
                          float* k_mean, float* q_mean, float* ds, sage_stream_t stream);
 
 /* V pre-pass.
@@ -201,14 +199,16 @@ int sage_attn_fwd_quantized(int mode,
                             int causal, float sm_scale, sage_stream_t stream);
 
 /* Attention with Q smoothing on the buffers of sage_quant_qk_smooth and
- * sage_quant_v (8-bit modes): every score of query block blk and key j is
- * dequantized as in sage_attn_fwd_quantized and gains ds[b, h, blk, j]
- * sm_scale before the online softmax.  Other arguments and errors as in
+ * sage_quant_v: every score of query block blk and key j is dequantized as
+ * in sage_attn_fwd_quantized and gains ds[b, h, blk, j] sm_scale before the
+ * online softmax.  Other arguments and errors as in
  * sage_attn_fwd_quantized. */
-int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q_scales,
-                                   const void* k_codes, const float* k_scales,
-                                   const void* v_codes, const float* v_scales, const float* ds,
-                                   void* o, int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
+int sage_attn_fwd_quantized_smooth(int mode,
+                                   const void* q_codes, const float* q_scales, const void* q_sf,
+                                   const void* k_codes, const float* k_scales, const void* k_sf,
+                                   const void* v_codes, const float* v_scales, const void* v_sf,
+                                   const float* ds, void* o, int dtype,
+                                   int64_t B, int64_t H, int64_t N, int64_t d,
                                    int causal, float sm_scale, sage_stream_t stream);
 
 /* The whole forward pass: pre-pass into a library-owned workspace (grown
@@ -216,7 +216,7 @@ int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q
  * freed at unload; the pre-pass takes the launch forms of sage_quant_qkv),
  * then the attention kernel.  sm_scale <= 0 means 1/sqrt(d).  An allocation
  * failure returns SAGE_ERR_CUDA before any kernel is launched.  mode may
- * carry SAGE_FLAG_SMOOTH_Q (8-bit modes): the pre-pass is then that of
+ * carry SAGE_FLAG_SMOOTH_Q: the pre-pass is then that of
  * sage_quant_qk_smooth (chained form only) and the attention that of
  * sage_attn_fwd_quantized_smooth. */
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype,

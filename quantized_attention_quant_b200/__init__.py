@@ -74,10 +74,11 @@ def library():
                                   vp, fp, vp, vp, fp, vp, fp, vp]
     lib.sage_quant_qk_smooth.restype = i32
     lib.sage_quant_qk_smooth.argtypes = [vp, vp, i32, i64, i64, i64, i64, i32,
-                                         vp, fp, vp, fp, fp, fp, fp, vp]
+                                         vp, fp, vp, vp, fp, vp, fp, fp, fp, vp]
     lib.sage_attn_fwd_quantized_smooth.restype = i32
-    lib.sage_attn_fwd_quantized_smooth.argtypes = [i32, vp, fp, vp, fp, vp, fp, fp, vp, i32,
-                                                   i64, i64, i64, i64, i32, ctypes.c_float, vp]
+    lib.sage_attn_fwd_quantized_smooth.argtypes = [i32, vp, fp, vp, vp, fp, vp, vp, fp, vp, fp,
+                                                   vp, i32, i64, i64, i64, i64, i32,
+                                                   ctypes.c_float, vp]
     lib.sage_quant_v.restype = i32
     lib.sage_quant_v.argtypes = [vp, i32, i64, i64, i64, i64, i32, vp, fp, vp, vp]
     lib.sage_quant_qkv.restype = i32
@@ -172,17 +173,18 @@ def sage_quant_qk(q, k, mode="int8_fp8"):
 
 
 def sage_quant_qk_smooth(q, k, mode="int8_fp8"):
-    """Q/K pre-pass with Q smoothing (8-bit modes).  Returns {q_codes,
-    q_scales, k_codes, k_scales, k_mean, q_mean, ds} as raw uint8 tensors
-    laid out as include/sage.h describes."""
+    """Q/K pre-pass with Q smoothing.  Returns {q_codes, q_scales, q_sf,
+    k_codes, k_scales, k_sf, k_mean, q_mean, ds} as raw uint8 tensors laid
+    out as include/sage.h describes."""
     B, H, N, d = _shape(q)
     if _shape(k) != (B, H, N, d) or k.dtype != q.dtype:
         raise ValueError("q and k must have the same shape and dtype")
-    bufs = _alloc(mode, ["q_codes", "q_scales", "k_codes", "k_scales", "k_mean", "q_mean", "ds"],
-                  B, H, N, d, q.device)
+    bufs = _alloc(mode, ["q_codes", "q_scales", "q_sf", "k_codes", "k_scales", "k_sf", "k_mean",
+                         "q_mean", "ds"], B, H, N, d, q.device)
     _check(library().sage_quant_qk_smooth(
         _ptr(q), _ptr(k), _dtype_code(q), B, H, N, d, MODES[mode],
-        _f(bufs["q_codes"]), _f(bufs["q_scales"]), _f(bufs["k_codes"]), _f(bufs["k_scales"]),
+        _f(bufs["q_codes"]), _f(bufs["q_scales"]), _f(bufs["q_sf"]),
+        _f(bufs["k_codes"]), _f(bufs["k_scales"]), _f(bufs["k_sf"]),
         _f(bufs["k_mean"]), _f(bufs["q_mean"]), _f(bufs["ds"]), _stream()))
     return bufs
 
@@ -248,8 +250,9 @@ def sage_attn_fwd_quantized_smooth(qk, vq, shape, mode="int8_fp8", causal=False,
         out = torch.empty((B, H, N, d), dtype=out_dtype or torch.bfloat16,
                           device=qk["q_codes"].device)
     _check(library().sage_attn_fwd_quantized_smooth(
-        MODES[mode], _f(qk["q_codes"]), _f(qk["q_scales"]), _f(qk["k_codes"]),
-        _f(qk["k_scales"]), _f(vq["v_codes"]), _f(vq["v_scales"]), _f(qk["ds"]),
+        MODES[mode], _f(qk["q_codes"]), _f(qk["q_scales"]), _f(qk["q_sf"]),
+        _f(qk["k_codes"]), _f(qk["k_scales"]), _f(qk["k_sf"]),
+        _f(vq["v_codes"]), _f(vq["v_scales"]), _f(vq["v_sf"]), _f(qk["ds"]),
         _ptr(out), _dtype_code(out), B, H, N, d, int(bool(causal)), float(sm_scale), _stream()))
     return out
 
@@ -258,8 +261,7 @@ def sage_attn_fwd(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=Non
                   smooth_q=False):
     """O = softmax(Q K^T sm_scale) V through the quantized path; O has q's dtype.
     K and V with fewer heads than Q (grouped-query attention) go to
-    sage_attn_fwd_gqa.  smooth_q: Q smoothing (SAGE_FLAG_SMOOTH_Q, 8-bit
-    modes)."""
+    sage_attn_fwd_gqa.  smooth_q: Q smoothing (SAGE_FLAG_SMOOTH_Q)."""
     import torch
     B, H, N, d = _shape(q)
     if _shape(k)[1] != H:

@@ -367,8 +367,6 @@ int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtyp
   mode &= ~SAGE_FLAG_SMOOTH_Q;
   bool empty = false;
   SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
-  if (smooth && mode == SAGE_MODE_FP4)
-    return fail(SAGE_ERR_UNSUPPORTED, "Q smoothing (SAGE_FLAG_SMOOTH_Q) needs an 8-bit mode");
   SAGE_TRY(check_kv_heads(H, Hkv));
   SAGE_TRY(check_ptr(q, "q", true));
   SAGE_TRY(check_ptr(k, "k", true));
@@ -459,9 +457,9 @@ size_t sage_buffer_bytes(int mode, int which, int64_t B, int64_t H, int64_t N, i
     case SAGE_BUF_V_SF:
       return fp4 ? (size_t)(BH * nt * 2 * 512) : 0;
     case SAGE_BUF_Q_MEAN:
-      return fp4 ? 0 : (size_t)(BH * nt * d * 4);
+      return (size_t)(BH * nt * d * 4);
     case SAGE_BUF_DS:
-      return fp4 ? 0 : (size_t)(BH * nt * nt * 128 * 4);
+      return (size_t)(BH * nt * nt * 128 * 4);
     default:
       return 0;
   }
@@ -501,12 +499,11 @@ int sage_quant_qk(const void* q, const void* k, int dtype, int64_t B, int64_t H,
 }
 
 int sage_quant_qk_smooth(const void* q, const void* k, int dtype, int64_t B, int64_t H, int64_t N,
-                         int64_t d, int mode, void* q_codes, float* q_scales, void* k_codes,
-                         float* k_scales, float* k_mean, float* q_mean, float* ds,
-                         sage_stream_t stream) {
+                         int64_t d, int mode, void* q_codes, float* q_scales, void* q_sf,
+                         void* k_codes, float* k_scales, void* k_sf, float* k_mean, float* q_mean,
+                         float* ds, sage_stream_t stream) {
   bool empty = false;
   SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
-  if (mode == SAGE_MODE_FP4) return fail(SAGE_ERR_UNSUPPORTED, "Q smoothing needs an 8-bit mode");
   SAGE_TRY(check_ptr(q, "q", true));
   SAGE_TRY(check_ptr(k, "k", true));
   SAGE_TRY(check_ptr(q_codes, "q_codes", true));
@@ -516,6 +513,13 @@ int sage_quant_qk_smooth(const void* q, const void* k, int dtype, int64_t B, int
   SAGE_TRY(check_ptr(k_mean, "k_mean", true));
   SAGE_TRY(check_ptr(q_mean, "q_mean", true));
   SAGE_TRY(check_ptr(ds, "ds", true));
+  if (mode == SAGE_MODE_FP4) {
+    SAGE_TRY(check_ptr(q_sf, "q_sf", true));
+    SAGE_TRY(check_ptr(k_sf, "k_sf", true));
+  } else {
+    SAGE_TRY(check_unused(q_sf, "q_sf"));
+    SAGE_TRY(check_unused(k_sf, "k_sf"));
+  }
   if (empty) return SAGE_OK;
   DeviceInfo* di = nullptr;
   SAGE_TRY(device_info(&di));
@@ -523,8 +527,8 @@ int sage_quant_qk_smooth(const void* q, const void* k, int dtype, int64_t B, int
   void* ws = nullptr;
   uint32_t* cnt = nullptr;
   SAGE_TRY(workspace(st, ws_ksum_bytes(B * H, N, d), &ws, &cnt));
-  QuantQKArgs a{q, k, dtype, mode, B, H, N, d, H, q_codes, q_scales, nullptr,
-                k_codes, k_scales, nullptr, k_mean, static_cast<double*>(ws), cnt};
+  QuantQKArgs a{q, k, dtype, mode, B, H, N, d, H, q_codes, q_scales, q_sf,
+                k_codes, k_scales, k_sf, k_mean, static_cast<double*>(ws), cnt};
   a.q_mean = q_mean;
   a.ds = ds;
   cudaError_t e = launch_quant_qk(a, st);
@@ -640,13 +644,13 @@ int sage_attn_fwd_quantized(int mode, const void* q_codes, const float* q_scales
 }
 
 int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q_scales,
-                                   const void* k_codes, const float* k_scales,
-                                   const void* v_codes, const float* v_scales, const float* ds,
-                                   void* o, int dtype, int64_t B, int64_t H, int64_t N, int64_t d,
-                                   int causal, float sm_scale, sage_stream_t stream) {
+                                   const void* q_sf, const void* k_codes, const float* k_scales,
+                                   const void* k_sf, const void* v_codes, const float* v_scales,
+                                   const void* v_sf, const float* ds, void* o, int dtype,
+                                   int64_t B, int64_t H, int64_t N, int64_t d, int causal,
+                                   float sm_scale, sage_stream_t stream) {
   bool empty = false;
   SAGE_TRY(check_common(dtype, mode, B, H, N, d, &empty));
-  if (mode == SAGE_MODE_FP4) return fail(SAGE_ERR_UNSUPPORTED, "Q smoothing needs an 8-bit mode");
   SAGE_TRY(check_ptr(q_codes, "q_codes", true));
   SAGE_TRY(check_ptr(q_scales, "q_scales", true));
   SAGE_TRY(check_ptr(k_codes, "k_codes", true));
@@ -655,17 +659,27 @@ int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q
   SAGE_TRY(check_ptr(v_scales, "v_scales", true));
   SAGE_TRY(check_ptr(ds, "ds", true));
   SAGE_TRY(check_ptr(o, "o", true));
+  if (mode == SAGE_MODE_FP4) {
+    SAGE_TRY(check_ptr(q_sf, "q_sf", true));
+    SAGE_TRY(check_ptr(k_sf, "k_sf", true));
+    SAGE_TRY(check_ptr(v_sf, "v_sf", true));
+  } else {
+    SAGE_TRY(check_unused(q_sf, "q_sf"));
+    SAGE_TRY(check_unused(k_sf, "k_sf"));
+    SAGE_TRY(check_unused(v_sf, "v_sf"));
+  }
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale))
     return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be positive and finite");
   if (empty) return SAGE_OK;
   DeviceInfo* di = nullptr;
   SAGE_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  AttnArgs a{mode, q_codes, q_scales, nullptr, k_codes, k_scales, nullptr, v_codes, v_scales,
-             nullptr, o, dtype, B, H, N, d, H, causal != 0, sm_scale, di->status};
+  AttnArgs a{mode, q_codes, q_scales, q_sf, k_codes, k_scales, k_sf, v_codes, v_scales,
+             v_sf, o, dtype, B, H, N, d, H, causal != 0, sm_scale, di->status};
   a.ds = ds;
   const char* detail = nullptr;
-  cudaError_t e = launch_attn_i8f8(a, st, &detail);
+  cudaError_t e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(a, st, &detail)
+                                        : launch_attn_i8f8(a, st, &detail);
   if (detail) return fail(SAGE_ERR_CUDA, detail);
   if (e != cudaSuccess) return fail_cuda(e, "attention launch");
   return SAGE_OK;

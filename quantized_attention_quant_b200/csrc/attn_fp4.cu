@@ -93,7 +93,9 @@ struct Layout {
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
   static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots] dequant factor of the tile
-  static constexpr int END = OFF_C + 16;
+  // Q smoothing: the score bias of key tile j (log2 units) in slot j % 4
+  static constexpr int OFF_BIAS = OFF_C + 16;
+  static constexpr int END = OFF_BIAS + 4 * 128 * 4;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t SBO = 8 * 64;  // 8 rows of 64 bytes (64-byte swizzle atom)
@@ -115,6 +117,7 @@ struct Bars {
   uint64_t* pv_empty;  // [2] stats -> MMA: PV[b] read
   uint64_t* l_ready;   // [1] exp -> stats: final row sums
   uint64_t* drain;     // MMA drain on abort
+  uint64_t* bias_full; // [2] stats -> stats: a tile's bias is in shared memory (Q smoothing)
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
@@ -135,6 +138,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.pv_empty = r.pv_full + 2;
   r.l_ready = r.pv_empty + 2;
   r.drain = r.l_ready + 1;
+  r.bias_full = r.drain + 1;
   return r;
 }
 
@@ -227,23 +231,57 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int lim, flo
   return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], acc));
 }
 
+// Q smoothing: the maximum of 32 scores that each gain a per-key bias (log2
+// units, bias[i] for key col0 + i), dequantized with factor c, and a
+// running value; masking as in max64.
+template <bool MASKED>
+__device__ __forceinline__ float max32_biased(const uint32_t* s, int col0, int lim, float c,
+                                              const float* bias, float acc) {
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const float4 bv = *reinterpret_cast<const float4*>(bias + i);
+    const float2 t01 = __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])),
+                                  c2, make_float2(bv.x, bv.y));
+    const float2 t23 = __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])),
+                                  c2, make_float2(bv.z, bv.w));
+    float v0 = t01.x, v1 = t01.y, v2 = t23.x, v3 = t23.y;
+    if (MASKED) {
+      v0 = (col0 + i + 0 <= lim) ? v0 : -INFINITY;
+      v1 = (col0 + i + 1 <= lim) ? v1 : -INFINITY;
+      v2 = (col0 + i + 2 <= lim) ? v2 : -INFINITY;
+      v3 = (col0 + i + 3 <= lim) ? v3 : -INFINITY;
+    }
+    acc = fmax3(fmax3(acc, v0, v1), v2, v3);
+  }
+  return acc;
+}
+
 // P~ for 32 scores of a row -> 16 bytes of e2m1 codes (key i in nibble i),
 // the two UE4M3 scales of its 16-key groups (bytes 0 and 1 of *sf2), and
 // the sum of the unquantized values.
 //   s16 = ue4m3(448 amax16); code = e2m1(P~ * 2688 / s16) (0 when s16 = 0).
-template <bool MASKED>
+// BIAS (Q smoothing): key col0 + i's score gains bias[i] (log2 units).
+template <bool MASKED, bool BIAS = false>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
-                                             int lim, uint32_t (&p)[4], uint32_t* sf2) {
+                                             int lim, uint32_t (&p)[4], uint32_t* sf2,
+                                             const float* bias = nullptr) {
   const float2 c2 = make_float2(c, c);
   const float2 n2 = make_float2(neg, neg);
   float x[32];
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
+    float2 n01 = n2, n23 = n2;
+    if (BIAS) {
+      const float4 bv = *reinterpret_cast<const float4*>(bias + i);
+      n01 = __fadd2_rn(make_float2(bv.x, bv.y), n2);
+      n23 = __fadd2_rn(make_float2(bv.z, bv.w), n2);
+    }
     const float2 t01 =
-        __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), c2, n2);
+        __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), c2, n01);
     const float2 t23 =
-        __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), c2, n2);
+        __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), c2, n23);
     float f0, f1, f2, f3;
     if (((i >> 2) * SAGE_FP4_EXP_POLY_GROUPS) % 8 < SAGE_FP4_EXP_POLY_GROUPS) {
       const float2 e01 = exp2_poly2(t01), e23 = exp2_poly2(t23);
@@ -297,11 +335,12 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
 // One 32-key chunk q (0..3) of row r: e2m1 codes into the 64-byte-swizzled
 // P~ tile (16-byte chunk q of row r lands at q ^ ((r >> 1) & 3)); returns
 // the chunk's row sum and its two scale bytes.
-template <bool MASKED>
+template <bool MASKED, bool BIAS = false>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int q, float c, float neg,
-                                           int r, int lim, uint32_t prow, uint32_t* sf2) {
+                                           int r, int lim, uint32_t prow, uint32_t* sf2,
+                                           const float* bias = nullptr) {
   uint32_t p[4];
-  const float sum = exp_quant32<MASKED>(s, c, neg, 32 * q, lim, p, sf2);
+  const float sum = exp_quant32<MASKED, BIAS>(s, c, neg, 32 * q, lim, p, sf2, bias);
   st_shared_v4(prow + (((uint32_t)q ^ (uint32_t)((r >> 1) & 3)) << 4), p[0], p[1], p[2], p[3]);
   return sum;
 }
@@ -309,7 +348,7 @@ __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int q, float
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
 // RAGGED (non-causal launches of a sequence whose last tile is partial): the
 // last key tile masks keys n_tail .. 127.
-template <bool CAUSAL, bool RAGGED>
+template <bool CAUSAL, bool RAGGED, bool SMOOTH>
 __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
                                          const uint32_t tmem, const Bars& bar, uint8_t* smem,
                                          volatile int* abort_flag, uint32_t* status) {
@@ -357,10 +396,12 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
       return;
     const uint32_t prow = smem_u32(smem + L::OFF_P + b * L::TILE + r * 64);
     uint32_t sf_lo, sf_hi;
-    float sum = masked ? exp_chunk<true>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo)
-                       : exp_chunk<false>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo);
-    sum += masked ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi)
-                  : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi);
+    // Q smoothing: this tile's key biases (m_full(j) orders them too)
+    const float* bias = reinterpret_cast<const float*>(smem + L::OFF_BIAS) + (j & 3) * 128 + 64 * h;
+    float sum = masked ? exp_chunk<true, SMOOTH>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo, bias)
+                       : exp_chunk<false, SMOOTH>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo, bias);
+    sum += masked ? exp_chunk<true, SMOOTH>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi, bias + 32)
+                  : exp_chunk<false, SMOOTH>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi, bias + 32);
     // the row's four group scales of this 64-key block, in the tensor-core
     // layout: byte 16 (r % 32) + 4 (r / 32) + s of the block's 512 bytes
     st_shared_u32(smem_u32(smem + L::OFF_SFP + b * L::SF + h * 512 + 16 * (r & 31) + 4 * (r >> 5)),
@@ -375,7 +416,7 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
 
 // Stats warpgroup: row max / running max per key tile, level-2 fold (one
 // tile behind), epilogue.
-template <bool CAUSAL, typename OutT, bool RAGGED>
+template <bool CAUSAL, typename OutT, bool RAGGED, bool SMOOTH>
 __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const int n_tail,
                                            const int bh,
                                            const int H, const int G, const int N,
@@ -384,6 +425,7 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
                                            uint32_t* status, const float* __restrict__ q_scales,
                                            const float* __restrict__ k_scales,
                                            const float* __restrict__ v_scales,
+                                           const float* __restrict__ ds,
                                            OutT* __restrict__ out, const float scale_log2) {
   using L = Layout;
   const int warp = threadIdx.x >> 5;
@@ -432,6 +474,19 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float alpha_hist[2] = {0.f, 0.f};
   float* c_s = reinterpret_cast<float*>(smem + L::OFF_C);
   float ks_cur = ldg_early(ksp);
+  // Q smoothing: this query block's score bias, exchanged through slot j % 4
+  // of a shared buffer one tile ahead (as in the 8-bit kernel): thread r
+  // writes key 128 j + r after publishing tile j - 1's maximum and arrives on
+  // bias_full[j % 2]; a slot is rewritten for tile j + 4 only after the
+  // s_full wait of tile j + 3, when every reader is past tile j.
+  const float* dsr = SMOOTH ? ds + ((int64_t)bh * ntiles + qt) * (int64_t)(ntiles * 128) : nullptr;
+  float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);
+  float d_nxt = 0.f;
+  if (SMOOTH) {
+    bias_s[r] = ldg_early(dsr + r) * scale_log2;
+    mbar_arrive(&bar.bias_full[0]);
+    if (nkv > 1) d_nxt = ldg_early(dsr + 128 + r);
+  }
   for (int j = 0; j < nkv; ++j) {
     const int b = j & 1;
     const float c = qs * ks_cur * scale_log2;
@@ -444,6 +499,10 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     const bool masked = diag || (RAGGED && j == nkv - 1);
     const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes;
+    if (SMOOTH && !__all_sync(0xffffffffu, mbar_wait(&bar.bias_full[b], (j >> 1) & 1, abort_flag,
+                                                     status, kDevTimeoutSoftmax)))
+      return;
+    const float* bias = bias_s + (j & 3) * 128;
     float mx = -INFINITY;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -452,10 +511,18 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      mx = masked ? max64<true>(&s[0][0], 64 * hh, lim, mx)
-                  : max64<false>(&s[0][0], 64 * hh, lim, mx);
+      if (SMOOTH) {
+        // biased scores, already scaled: the maximum of the sums
+        mx = masked ? max32_biased<true>(s[1], 64 * hh + 32, lim, c, bias + 64 * hh + 32,
+                                         max32_biased<true>(s[0], 64 * hh, lim, c, bias + 64 * hh, mx))
+                    : max32_biased<false>(s[1], 64 * hh + 32, lim, c, bias + 64 * hh + 32,
+                                          max32_biased<false>(s[0], 64 * hh, lim, c, bias + 64 * hh, mx));
+      } else {
+        mx = masked ? max64<true>(&s[0][0], 64 * hh, lim, mx)
+                    : max64<false>(&s[0][0], 64 * hh, lim, mx);
+      }
     }
-    const float m_j = fmaxf(m, mx * c);
+    const float m_j = fmaxf(m, SMOOTH ? mx : mx * c);
     const float alpha = ex2(m - m_j);
     m = m_j;
     m_s[(2 * b) * 128 + r] = m_j;
@@ -463,6 +530,12 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     if (r == 0) c_s[b] = c;
     tc_fence_before();
     mbar_arrive(&bar.m_full[b]);
+    if (SMOOTH && j + 1 < nkv) {
+      // the next tile's bias, and the one after it from global memory
+      bias_s[((j + 1) & 3) * 128 + r] = d_nxt * scale_log2;
+      mbar_arrive(&bar.bias_full[b ^ 1]);
+      if (j + 2 < nkv) d_nxt = ldg_early(dsr + 128 * (j + 2) + r);
+    }
     // the fold runs two tiles behind the max
     if (j > 1 && !fold(j - 2, alpha_hist[b])) return;
     alpha_hist[b] = alpha;
@@ -489,15 +562,16 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   }
 }
 
-template <bool CAUSAL, typename OutT, bool RAGGED>
+template <bool CAUSAL, typename OutT, bool RAGGED, bool SMOOTH>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fp4_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scales,
                     const float* __restrict__ k_scales, const float* __restrict__ v_scales,
                     const uint8_t* __restrict__ q_sf, const uint8_t* __restrict__ k_sf,
-                    const uint8_t* __restrict__ v_sf, OutT* __restrict__ out, int N, int H,
-                    int G, float scale_log2, int head_major, uint32_t* status) {
+                    const uint8_t* __restrict__ v_sf, const float* __restrict__ ds,
+                    OutT* __restrict__ out, int N, int H, int G, float scale_log2,
+                    int head_major, uint32_t* status) {
   using L = Layout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -543,6 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar.l_ready, 256);
     mbar_init(bar.drain, 1);
+    mbar_init(&bar.bias_full[0], 128);
+    mbar_init(&bar.bias_full[1], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -685,11 +761,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<CAUSAL, RAGGED>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
+    exp_loop<CAUSAL, RAGGED, SMOOTH>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
-    stats_loop<CAUSAL, OutT, RAGGED>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem, abort_flag, status,
-                             q_scales, k_scales, v_scales, out, scale_log2);
+    stats_loop<CAUSAL, OutT, RAGGED, SMOOTH>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem,
+                                             abort_flag, status, q_scales, k_scales, v_scales, ds,
+                                             out, scale_log2);
   }
 
   tc_fence_before();
@@ -704,7 +781,8 @@ template <bool CAUSAL, typename OutT, bool RAGGED = false>
 cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                          const CUtensorMap& tv, cudaStream_t st) {
   using L = Layout;
-  auto kern = attn_fp4_kernel<CAUSAL, OutT, RAGGED>;
+  auto kern = a.ds ? attn_fp4_kernel<CAUSAL, OutT, RAGGED, true>
+                   : attn_fp4_kernel<CAUSAL, OutT, RAGGED, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
   if (e != cudaSuccess) return e;
   const int ntiles = (int)((a.N + 127) / 128);
@@ -713,7 +791,7 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& tq, const CUtenso
                        : dim3((unsigned)ntiles, (unsigned)(a.B * a.H));
   kern<<<grid, kThreads, L::SMEM, st>>>(
       tq, tk, tv, a.q_scales, a.k_scales, a.v_scales, static_cast<const uint8_t*>(a.q_sf),
-      static_cast<const uint8_t*>(a.k_sf), static_cast<const uint8_t*>(a.v_sf),
+      static_cast<const uint8_t*>(a.k_sf), static_cast<const uint8_t*>(a.v_sf), a.ds,
       reinterpret_cast<OutT*>(a.o), (int)a.N, (int)a.H, (int)(a.H / a.Hkv), a.sm_scale * kLog2e,
       hm, a.status);
   return cudaGetLastError();

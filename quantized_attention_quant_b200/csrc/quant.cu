@@ -51,6 +51,7 @@ enum Role : int {
   kQuantKF8 = 10, // FP8 (e4m3) smoothed-K codes + block scales (needs the K mean)
   kQuantQ8S = 11,  // INT8 codes of the smoothed Q (tile mean out) + scales + the mean
   kQuantQF8S = 12, // FP8 codes of the smoothed Q + scales + the mean
+  kQuantQ4S = 13,  // FP4 codes of the smoothed Q + scales + the mean
 };
 
 struct Roles {
@@ -455,10 +456,9 @@ __device__ __forceinline__ void role_quant_8bit(const T* __restrict__ src, const
 // channel c over the tile's real tokens in token order, qbar = fp32(sum /
 // count) goes to global memory and to shared memory, and the tile is
 // encoded as Q - qbar (one FP32 subtraction) with the 8-bit encoder.
-template <typename T, int D, bool FP8, bool RAGGED>
-__device__ __forceinline__ void role_quant_q_smooth(const T* __restrict__ src, float* q_mean_out,
-                                                    uint8_t* __restrict__ dst, float* scale_out,
-                                                    T* tile, float* mean_s, float* red, int nv) {
+template <typename T, int D, bool RAGGED>
+__device__ __forceinline__ void stage_tile_mean(const T* __restrict__ src, float* q_mean_out,
+                                                T* tile, float* mean_s, int nv) {
   stage_tile<T, D, RAGGED>(src, tile, nv);
   __syncthreads();
   const int t = threadIdx.x;
@@ -471,6 +471,13 @@ __device__ __forceinline__ void role_quant_q_smooth(const T* __restrict__ src, f
     q_mean_out[t] = m;
   }
   __syncthreads();
+}
+
+template <typename T, int D, bool FP8, bool RAGGED>
+__device__ __forceinline__ void role_quant_q_smooth(const T* __restrict__ src, float* q_mean_out,
+                                                    uint8_t* __restrict__ dst, float* scale_out,
+                                                    T* tile, float* mean_s, float* red, int nv) {
+  stage_tile_mean<T, D, RAGGED>(src, q_mean_out, tile, mean_s, nv);
   role_quant_8bit<T, D, FP8, RAGGED, 1, true>(tile, mean_s, dst, scale_out, red, nv);
 }
 
@@ -587,7 +594,8 @@ __device__ __forceinline__ int64_t sf_offset(int64_t bh, int ntiles, int tile, i
 
 // Q or smoothed K of one tile: g = amax/2688, per 16 channels
 // s16 = ue4m3(amax16 / (6 g)), code = e2m1(x / (s16 g)).
-template <typename T, int D, bool RAGGED>
+// SHARED: the tile and the mean are in shared memory (the smoothed Q role).
+template <typename T, int D, bool RAGGED, bool SHARED = false>
 __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src, const float* mean,
                                                       uint8_t* __restrict__ codes, float* g_out,
                                                       uint8_t* __restrict__ sf, int64_t bh,
@@ -604,8 +612,8 @@ __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src,
     // and is zeroed below: code 0, scale 0
     const int rr = (!RAGGED || r < nv) ? r : nv - 1;
     float a[8], b[8];
-    load8(src + rr * D + gc * 16, a);
-    load8(src + rr * D + gc * 16 + 8, b);
+    load8<T, SHARED>(src + rr * D + gc * 16, a);
+    load8<T, SHARED>(src + rr * D + gc * 16 + 8, b);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       x[i][e] = a[e];
@@ -614,7 +622,7 @@ __device__ __forceinline__ void role_quant_fp4_tokens(const T* __restrict__ src,
     if (mean) {
       const float* mu = mean + gc * 16;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) x[i][e] = __fsub_rn(x[i][e], __ldg(mu + e));
+      for (int e = 0; e < 16; ++e) x[i][e] = __fsub_rn(x[i][e], SHARED ? mu[e] : __ldg(mu + e));
     }
     if (RAGGED && r >= nv) {
 #pragma unroll
@@ -731,7 +739,7 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   constexpr bool kV4 = ((MASK >> kQuantV4) & 1) != 0;
   constexpr bool kTile = ((MASK >> kQuantV8) & 1) || ((MASK >> kStatsK) & 1) ||
                          ((MASK >> kStatsKV) & 1) || ((MASK >> kQuantQ8S) & 1) ||
-                         ((MASK >> kQuantQF8S) & 1);
+                         ((MASK >> kQuantQF8S) & 1) || ((MASK >> kQuantQ4S) & 1);
   constexpr int V4_BYTES = kV4 ? 128 * (D + 2) * (int)sizeof(T) : 16;
   constexpr int TILE_BYTES = kTile ? 128 * D * (int)sizeof(T) : 16;
   constexpr int SMEM_BYTES = V4_BYTES > TILE_BYTES ? V4_BYTES : TILE_BYTES;
@@ -745,7 +753,7 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
   // the grid spans the larger head count: Q roles cover bh_q heads, K/V
   // roles bh_kv (a CTA leaves as a whole, before any barrier)
   const bool q_role = role == kQuantQ8 || role == kQuantQ4 || role == kQuantQF8 ||
-                      role == kQuantQ8S || role == kQuantQF8S;
+                      role == kQuantQ8S || role == kQuantQF8S || role == kQuantQ4S;
   if (bh >= (q_role ? p.bh_q : p.bh_kv)) return;
   // (without RAGGED, Np == N: the same offsets as before padding existed)
   const int ntiles = (RAGGED ? p.Np : p.N) / 128;
@@ -807,6 +815,17 @@ __global__ void __launch_bounds__(kThreads) prepass_kernel(PrepassPtrs p, Roles 
                                   reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * (D / 2),
                                   p.q_scales + bh * ntiles + tile, p.q_sf, bh, ntiles, tile, red,
                                   nv);
+      break;
+    case kQuantQ4S:
+      SAGE_ROLE(kQuantQ4S) {
+        stage_tile_mean<T, D, RAGGED>(reinterpret_cast<const T*>(p.q) + row0 * D,
+                                      p.q_mean + (bh * ntiles + tile) * D,
+                                      reinterpret_cast<T*>(smem_raw), qmean_s, nv);
+        role_quant_fp4_tokens<T, D, RAGGED, true>(
+            reinterpret_cast<const T*>(smem_raw), qmean_s,
+            reinterpret_cast<uint8_t*>(p.q_codes) + crow0 * (D / 2),
+            p.q_scales + bh * ntiles + tile, p.q_sf, bh, ntiles, tile, red, nv);
+      }
       break;
     case kQuantK4:
       SAGE_ROLE(kQuantK4)
@@ -1197,15 +1216,18 @@ cudaError_t launch_prepass_fused(const QuantQKArgs& qa, const QuantVArgs& va, cu
 cudaError_t launch_quant_qk(const QuantQKArgs& a, cudaStream_t st) {
   const PrepassPtrs p = ptrs_qk(a);
   if (a.q_mean) {
-    // Q smoothing (8-bit modes): smoothed Q codes and the means beside the K
+    // Q smoothing: smoothed Q codes and the means beside the K
     // statistics, then the K codes, then the bias (it needs both means)
     cudaError_t e;
     if (a.mode == kModeInt8Fp8)
       e = dispatch<bit(kQuantQ8S) | bit(kStatsK), bit(kQuantK8)>(
           p, a.dtype, a.d, Roles{2, {kQuantQ8S, kStatsK}}, Roles{1, {kQuantK8}}, st);
-    else
+    else if (a.mode == kModeFp8)
       e = dispatch<bit(kQuantQF8S) | bit(kStatsK), bit(kQuantKF8)>(
           p, a.dtype, a.d, Roles{2, {kQuantQF8S, kStatsK}}, Roles{1, {kQuantKF8}}, st);
+    else
+      e = dispatch<bit(kQuantQ4S) | bit(kStatsK), bit(kQuantK4)>(
+          p, a.dtype, a.d, Roles{2, {kQuantQ4S, kStatsK}}, Roles{1, {kQuantK4}}, st);
     if (e != cudaSuccess) return e;
     return launch_smoothing_bias(a, st);
   }

@@ -180,29 +180,28 @@ def test_missing_library_fails_loudly(monkeypatch):
 
 def test_smoothing_buffers_and_argument_errors(lib):
     # Q smoothing: buffer sizes, and every refusal comes before any device
-    # call (8-bit modes only; required pointers; the mode flag)
+    # call (required pointers; the FP4 scale-factor buffers; the mode flag)
     import quantized_attention_quant_b200 as q
     B, H, N, d = 2, 3, 200, 128
     nt, Np = 2, 256
     assert q.buffer_bytes("int8_fp8", "q_mean", B, H, N, d) == B * H * nt * d * 4
     assert q.buffer_bytes("fp8", "ds", B, H, N, d) == B * H * nt * Np * 4
-    assert q.buffer_bytes("fp4", "q_mean", B, H, N, d) == 0
-    assert q.buffer_bytes("fp4", "ds", B, H, N, d) == 0
-    s = lib.sage_quant_qk_smooth(FAKE, FAKE, 1, 1, 1, 128, 128, 1, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                 FAKE, FAKE, None)
-    assert s == -2 and "8-bit" in lib.sage_status_string(s).decode()
-    s = lib.sage_quant_qk_smooth(FAKE, FAKE, 1, 1, 1, 128, 128, 0, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                 None, FAKE, None)
+    assert q.buffer_bytes("fp4", "q_mean", B, H, N, d) == B * H * nt * d * 4
+    assert q.buffer_bytes("fp4", "ds", B, H, N, d) == B * H * nt * Np * 4
+    s = lib.sage_quant_qk_smooth(FAKE, FAKE, 1, 1, 1, 128, 128, 1, FAKE, FAKE, None, FAKE, FAKE,
+                                 FAKE, FAKE, FAKE, FAKE, None)
+    assert s == -1 and "q_sf is NULL" in lib.sage_status_string(s).decode()
+    s = lib.sage_quant_qk_smooth(FAKE, FAKE, 1, 1, 1, 128, 128, 0, FAKE, FAKE, None, FAKE, FAKE,
+                                 None, FAKE, None, FAKE, None)
     assert s == -1 and "q_mean is NULL" in lib.sage_status_string(s).decode()
-    s = lib.sage_attn_fwd_quantized_smooth(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1,
-                                           1, 1, 128, 128, 0, ctypes.c_float(0.1), None)
+    s = lib.sage_attn_fwd_quantized_smooth(0, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, FAKE,
+                                           None, None, FAKE, 1, 1, 1, 128, 128, 0,
+                                           ctypes.c_float(0.1), None)
     assert s == -1 and "ds is NULL" in lib.sage_status_string(s).decode()
-    s = lib.sage_attn_fwd_quantized_smooth(1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1,
-                                           1, 1, 128, 128, 0, ctypes.c_float(0.1), None)
-    assert s == -2
-    s = lib.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 128, 0, ctypes.c_float(0.0),
-                          1 | q.SMOOTH_Q, None)
-    assert s == -2 and "smoothing" in lib.sage_status_string(s).decode()
+    s = lib.sage_attn_fwd_quantized_smooth(0, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+                                           None, FAKE, FAKE, 1, 1, 1, 128, 128, 0,
+                                           ctypes.c_float(0.1), None)
+    assert s == -1 and "must be NULL" in lib.sage_status_string(s).decode()
     assert lib.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, 1, 0, 1, 128, 128, 0, ctypes.c_float(0.0),
                              q.SMOOTH_Q, None) == 0
     s = lib.sage_attn_fwd_noalloc(FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 128, 0,
