@@ -223,6 +223,23 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
                   int64_t B, int64_t H, int64_t N, int64_t d,
                   int causal, float sm_scale, int mode, sage_stream_t stream);
 
+/* The whole forward pass on HOST buffers: q, k, v and o point to host
+ * memory holding [B, H, N, d] in `dtype` (any host memory; page-locked
+ * memory lets the copies overlap the compute).  The heads are cut into
+ * about 8 chunks (none smaller than 32 MB of inputs); chunk i + 1 is copied
+ * in and chunk i - 1 copied out on two library-owned copy streams (one pair
+ * per device, shared by callers, one call at a time) while chunk i runs the
+ * pre-pass and attention of sage_attn_fwd on `stream`.  Heads are
+ * independent, so O equals sage_attn_fwd's bit for bit.  Every copy of the
+ * call is ordered before later work on `stream`: synchronise `stream`
+ * before reading o.  mode may carry SAGE_FLAG_SMOOTH_Q.  Device memory
+ * comes from the same per-(device, stream) workspace as sage_attn_fwd (two
+ * chunks of Q, K, V and O plus one chunk's pipeline); errors as in
+ * sage_attn_fwd (a NULL pointer is SAGE_ERR_INVALID_ARG). */
+int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int dtype,
+                       int64_t B, int64_t H, int64_t N, int64_t d,
+                       int causal, float sm_scale, int mode, sage_stream_t stream);
+
 /* Grouped-query (and multi-query) attention: the kernel-comparison blog
  * ("Attention kernel benchmarks: speed and memory use") notes that
  * grouped-query attention changes the shape of the K/V tensors being

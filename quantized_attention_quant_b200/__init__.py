@@ -17,6 +17,7 @@ Entry points (same names as the C ABI in include/sage.h):
     sage_quant_qk_smooth(q, k, mode)          -> dict, with Q smoothing (q_mean, ds)
     sage_attn_fwd_quantized_smooth(qk, vq, shape, mode, ...) -> O, with Q smoothing
     (sage_attn_fwd(..., smooth_q=True) runs the whole pass with Q smoothing)
+    sage_attn_fwd_host(q, k, v, ...)          -> O  (host tensors in and out, copies overlapped)
 """
 
 import ctypes
@@ -25,7 +26,7 @@ import os
 
 __all__ = ["sage_quant_qk", "sage_quant_v", "sage_quant_qkv", "sage_attn_fwd", "sage_attn_fwd_gqa",
            "sage_attn_fwd_quantized", "sage_attn_fwd_noalloc",
-           "sage_quant_qk_smooth", "sage_attn_fwd_quantized_smooth", "SMOOTH_Q",
+           "sage_quant_qk_smooth", "sage_attn_fwd_quantized_smooth", "SMOOTH_Q", "sage_attn_fwd_host",
            "buffer_bytes", "library", "library_path", "SageError", "MODES", "EXPORTS",
            "selftest_bounded_wait"]
 
@@ -42,7 +43,7 @@ BUF = {name: i for i, name in enumerate(
 # every symbol include/sage.h declares
 EXPORTS = ["sage_buffer_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv",
            "sage_attn_fwd_quantized", "sage_quant_qk_smooth", "sage_attn_fwd_quantized_smooth",
-           "sage_attn_fwd", "sage_attn_fwd_gqa", "sage_attn_fwd_noalloc",
+           "sage_attn_fwd", "sage_attn_fwd_gqa", "sage_attn_fwd_noalloc", "sage_attn_fwd_host",
            "sage_get_last_device_status",
            "sage_selftest_bounded_wait", "sage_status_string", "sage_version",
            "sage_debug_fail_allocations"]
@@ -93,6 +94,9 @@ def library():
     lib.sage_attn_fwd_gqa.restype = i32
     lib.sage_attn_fwd_gqa.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i64, i32,
                                       ctypes.c_float, i32, vp]
+    lib.sage_attn_fwd_host.restype = i32
+    lib.sage_attn_fwd_host.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i32,
+                                       ctypes.c_float, i32, vp]
     lib.sage_attn_fwd_noalloc.restype = i32
     lib.sage_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, i64, i32,
                                           ctypes.c_float, i32, vp]
@@ -297,6 +301,32 @@ def sage_attn_fwd_gqa(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, Hkv, N, d,
         int(bool(causal)), float(sm_scale or 0.0), MODES[mode] | (SMOOTH_Q if smooth_q else 0),
         _stream()))
+    return out
+
+
+def sage_attn_fwd_host(q, k, v, causal=False, sm_scale=None, mode="int8_fp8", out=None,
+                       smooth_q=False):
+    """The whole forward pass on host (CPU) tensors: the library copies the
+    heads in chunks to the device, computes, and copies O back, overlapping
+    the copies with the compute (pinned tensors overlap best).  Returns O on
+    the host once the current CUDA stream has finished it (this call
+    synchronises that stream)."""
+    import torch
+    for t in (q, k, v):
+        if t.dim() != 4 or t.is_cuda or not t.is_contiguous():
+            raise ValueError("expected contiguous host tensors of shape [B, H, N, d]")
+    B, H, N, d = (int(x) for x in q.shape)
+    if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
+        raise ValueError("q, k, v must have the same shape")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must have the same dtype")
+    if out is None:
+        out = torch.empty_like(q, pin_memory=q.is_pinned())
+    _check(library().sage_attn_fwd_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _dtype_code(q), B, H, N, d,
+        int(bool(causal)), float(sm_scale or 0.0), MODES[mode] | (SMOOTH_Q if smooth_q else 0),
+        _stream()))
+    torch.cuda.current_stream().synchronize()
     return out
 
 

@@ -360,6 +360,74 @@ int64_t heads_of(int which, int64_t H, int64_t Hkv) {
 // The whole pipeline (pre-pass, then attention) with every buffer carved
 // from the per-stream workspace. Q and O have H heads, K and V have Hkv heads
 // (Hkv divides H; Hkv == H is plain multi-head attention).
+// Workspace layout of one forward pass (codes, scales, statistics partials,
+// and with Q smoothing the Q means and the score bias), relative to the
+// workspace base.
+struct FwdLayout {
+  size_t off[SAGE_BUF_V_SF + 1];
+  size_t ksum, vmax, qmean, ds, total;
+};
+
+FwdLayout fwd_layout(int mode, bool smooth, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                     int64_t d) {
+  FwdLayout L{};
+  size_t total = 0;
+  for (int w = 0; w <= SAGE_BUF_V_SF; ++w) {
+    L.off[w] = total;
+    total += align_up(sage_buffer_bytes(mode, w, B, heads_of(w, H, Hkv), N, d));
+  }
+  L.ksum = total;
+  total += align_up(ws_ksum_bytes(B * Hkv, N, d));
+  L.vmax = total;
+  total += align_up(ws_vmax_bytes(B * Hkv, N, d));
+  L.qmean = total;
+  if (smooth) total += align_up(sage_buffer_bytes(mode, SAGE_BUF_Q_MEAN, B, H, N, d));
+  L.ds = total;
+  if (smooth) total += align_up(sage_buffer_bytes(mode, SAGE_BUF_DS, B, H, N, d));
+  L.total = total;
+  return L;
+}
+
+// The pre-pass and the attention of one forward pass on `st`, every buffer
+// carved from `base` (laid out by fwd_layout) and the statistics counters
+// `cnt`.  Arguments are already checked.
+int run_fwd(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B, int64_t H,
+            int64_t Hkv, int64_t N, int64_t d, int causal, float sm_scale, int mode, bool smooth,
+            char* base, uint32_t* cnt, uint32_t* status, cudaStream_t st) {
+  const FwdLayout L = fwd_layout(mode, smooth, B, H, Hkv, N, d);
+  auto at = [&](int w) -> void* {
+    return sage_buffer_bytes(mode, w, B, heads_of(w, H, Hkv), N, d) ? base + L.off[w] : nullptr;
+  };
+  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d, Hkv,
+                 at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+                 at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + L.ksum), cnt};
+  QuantVArgs va{v, dtype, mode, B, Hkv, N, d,
+                at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+                reinterpret_cast<double*>(base + L.ksum),
+                reinterpret_cast<float*>(base + L.vmax), cnt};
+  qa.status = status;
+  if (smooth) {
+    qa.q_mean = reinterpret_cast<float*>(base + L.qmean);
+    qa.ds = reinterpret_cast<float*>(base + L.ds);
+  }
+  SAGE_TRY(prepass_forked(qa, va, st));
+  AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
+              at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
+              at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
+              o, dtype, B, H, N, d, Hkv, causal != 0, sm_scale, status};
+  aa.ds = qa.ds;
+  const char* detail = nullptr;
+  const cudaError_t e =
+      mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
+  if (detail) return fail(SAGE_ERR_CUDA, detail);
+  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  return SAGE_OK;
+}
+
+// The whole pipeline (pre-pass, then attention) with every buffer carved
+// from the per-stream workspace. Q and O have H heads, K and V have Hkv heads
+// (Hkv divides H; Hkv == H is plain multi-head attention).
 int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,
                   int64_t H, int64_t Hkv, int64_t N, int64_t d, int causal, float sm_scale,
                   int mode, sage_stream_t stream) {
@@ -378,52 +446,62 @@ int attn_fwd_full(const void* q, const void* k, const void* v, void* o, int dtyp
   DeviceInfo* di = nullptr;
   SAGE_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  size_t off[SAGE_BUF_V_SF + 1];
-  size_t total = 0;
-  for (int w = 0; w <= SAGE_BUF_V_SF; ++w) {
-    off[w] = total;
-    total += align_up(sage_buffer_bytes(mode, w, B, heads_of(w, H, Hkv), N, d));
-  }
-  const size_t off_ksum = total;
-  total += align_up(ws_ksum_bytes(B * Hkv, N, d));
-  const size_t off_vmax = total;
-  total += align_up(ws_vmax_bytes(B * Hkv, N, d));
-  const size_t off_qmean = total;
-  if (smooth) total += align_up(sage_buffer_bytes(mode, SAGE_BUF_Q_MEAN, B, H, N, d));
-  const size_t off_ds = total;
-  if (smooth) total += align_up(sage_buffer_bytes(mode, SAGE_BUF_DS, B, H, N, d));
   void* ws = nullptr;
   uint32_t* cnt = nullptr;
-  SAGE_TRY(workspace(st, total, &ws, &cnt));
-  char* base = static_cast<char*>(ws);
-  auto at = [&](int w) -> void* {
-    return sage_buffer_bytes(mode, w, B, heads_of(w, H, Hkv), N, d) ? base + off[w] : nullptr;
-  };
-  QuantQKArgs qa{q, k, dtype, mode, B, H, N, d, Hkv,
-                 at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
-                 at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
-                 (float*)at(SAGE_BUF_K_MEAN), reinterpret_cast<double*>(base + off_ksum), cnt};
-  QuantVArgs va{v, dtype, mode, B, Hkv, N, d,
-                at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
-                reinterpret_cast<double*>(base + off_ksum),
-                reinterpret_cast<float*>(base + off_vmax), cnt};
-  qa.status = di->status;
-  if (smooth) {
-    qa.q_mean = reinterpret_cast<float*>(base + off_qmean);
-    qa.ds = reinterpret_cast<float*>(base + off_ds);
+  SAGE_TRY(workspace(st, fwd_layout(mode, smooth, B, H, Hkv, N, d).total, &ws, &cnt));
+  return run_fwd(q, k, v, o, dtype, B, H, Hkv, N, d, causal, sm_scale, mode, smooth,
+                 static_cast<char*>(ws), cnt, di->status, st);
+}
+
+// Two more streams per device for sage_attn_fwd_host: host -> device copies
+// of a chunk's Q, K, V and device -> host copies of its O, each ordered
+// against the compute on the caller's stream by events (two slots of staging
+// buffers, so chunk i + 1 is copied in and chunk i - 1 copied out while
+// chunk i computes).
+struct CopyStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t in_ready[2] = {nullptr, nullptr}, done[2] = {nullptr, nullptr},
+              out_read[2] = {nullptr, nullptr};
+  std::mutex mu;  // one pipelined call at a time per device: the events are shared
+};
+std::map<int, CopyStreams*> g_copy;
+
+int copy_streams(CopyStreams** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  CopyStreams*& cs = g_copy[dev];
+  if (!cs) {
+    auto* n = new CopyStreams;
+    e = cudaStreamCreateWithFlags(&n->h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&n->d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n->start, cudaEventDisableTiming);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&n->in_ready[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n->done[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n->out_read[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) {
+      delete n;
+      return fail_cuda(e, "copy stream setup");
+    }
+    cs = n;
   }
-  SAGE_TRY(prepass_forked(qa, va, st));
-  cudaError_t e = cudaSuccess;
-  AttnArgs aa{mode, at(SAGE_BUF_Q_CODES), (float*)at(SAGE_BUF_Q_SCALES), at(SAGE_BUF_Q_SF),
-              at(SAGE_BUF_K_CODES), (float*)at(SAGE_BUF_K_SCALES), at(SAGE_BUF_K_SF),
-              at(SAGE_BUF_V_CODES), (float*)at(SAGE_BUF_V_SCALES), at(SAGE_BUF_V_SF),
-              o, dtype, B, H, N, d, Hkv, causal != 0, sm_scale, di->status};
-  aa.ds = qa.ds;
-  const char* detail = nullptr;
-  e = mode == SAGE_MODE_FP4 ? launch_attn_fp4(aa, st, &detail) : launch_attn_i8f8(aa, st, &detail);
-  if (detail) return fail(SAGE_ERR_CUDA, detail);
-  if (e != cudaSuccess) return fail_cuda(e, "attention launch");
+  *out = cs;
   return SAGE_OK;
+}
+
+// Heads per chunk of sage_attn_fwd_host: about 8 chunks, none smaller than
+// 32 MB of inputs (fewer, larger chunks for small problems).
+int64_t host_chunk_heads(int64_t BH, int64_t N, int64_t d) {
+  const int64_t head_bytes = 3 * N * d * 2;
+  int64_t c = (BH + 7) / 8;
+  const int64_t min_heads = (int64_t(32) << 20) / (head_bytes > 0 ? head_bytes : 1);
+  if (c < min_heads) c = min_heads;
+  if (c > BH) c = BH;
+  return c < 1 ? 1 : c;
 }
 
 }  // namespace
@@ -683,6 +761,90 @@ int sage_attn_fwd_quantized_smooth(int mode, const void* q_codes, const float* q
   if (detail) return fail(SAGE_ERR_CUDA, detail);
   if (e != cudaSuccess) return fail_cuda(e, "attention launch");
   return SAGE_OK;
+}
+
+int sage_attn_fwd_host(const void* q, const void* k, const void* v, void* o, int dtype,
+                       int64_t B, int64_t H, int64_t N, int64_t d, int causal, float sm_scale,
+                       int mode, sage_stream_t stream) {
+  const bool smooth = (mode & SAGE_FLAG_SMOOTH_Q) != 0;
+  const int base_mode = mode & ~SAGE_FLAG_SMOOTH_Q;
+  bool empty = false;
+  SAGE_TRY(check_common(dtype, base_mode, B, H, N, d, &empty));
+  if (!q || !k || !v || !o) return fail(SAGE_ERR_INVALID_ARG, "q, k, v and o must not be NULL");
+  if (!(sm_scale > 0.f)) sm_scale = 1.0f / std::sqrt((float)d);
+  if (!std::isfinite(sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale must be finite");
+  if (empty) return SAGE_OK;
+  DeviceInfo* di = nullptr;
+  SAGE_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t BH = B * H;
+  const int64_t ch = host_chunk_heads(BH, N, d);
+  const size_t head_bytes = (size_t)(N * d * 2);
+  const size_t in_bytes = align_up(head_bytes * ch);   // one tensor of a chunk
+  // staging: two slots of Q, K, V and O; then the chunk pipeline's workspace
+  const size_t stage = 2 * 4 * in_bytes;
+  void* ws = nullptr;
+  uint32_t* cnt = nullptr;
+  SAGE_TRY(workspace(st, stage + fwd_layout(base_mode, smooth, 1, ch, ch, N, d).total, &ws, &cnt));
+  char* base = static_cast<char*>(ws);
+  auto slot = [&](int s, int t) { return base + (size_t)(4 * s + t) * in_bytes; };  // t: q k v o
+  CopyStreams* cs = nullptr;
+  SAGE_TRY(copy_streams(&cs));
+  std::lock_guard<std::mutex> lk(cs->mu);
+  cudaError_t e;
+  // the copy streams start after everything already queued on st (the
+  // workspace may have been in use there)
+  if ((e = cudaEventRecord(cs->start, st)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(cs->h2d, cs->start, 0)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(cs->d2h, cs->start, 0)) != cudaSuccess)
+    return fail_cuda(e, "host pipeline fork");
+  const char* hq = static_cast<const char*>(q);
+  const char* hk = static_cast<const char*>(k);
+  const char* hv = static_cast<const char*>(v);
+  char* ho = static_cast<char*>(o);
+  int status = SAGE_OK;
+  const int64_t nchunks = (BH + ch - 1) / ch;
+  for (int64_t i = 0; i < nchunks && status == SAGE_OK; ++i) {
+    const int s = (int)(i & 1);
+    const int64_t h0 = i * ch, nh = (BH - h0 < ch) ? BH - h0 : ch;
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)nh * head_bytes;
+    // copy in (slot s is free once chunk i - 2 has computed)
+    if ((i >= 2 && (e = cudaStreamWaitEvent(cs->h2d, cs->done[s], 0)) != cudaSuccess) ||
+        (e = cudaMemcpyAsync(slot(s, 0), hq + off, bytes, cudaMemcpyDefault, cs->h2d)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(slot(s, 1), hk + off, bytes, cudaMemcpyDefault, cs->h2d)) !=
+            cudaSuccess ||
+        (e = cudaMemcpyAsync(slot(s, 2), hv + off, bytes, cudaMemcpyDefault, cs->h2d)) !=
+            cudaSuccess ||
+        (e = cudaEventRecord(cs->in_ready[s], cs->h2d)) != cudaSuccess) {
+      status = fail_cuda(e, "host pipeline copy in");
+      break;
+    }
+    // compute (O slot s is free once chunk i - 2 has been copied out)
+    if ((e = cudaStreamWaitEvent(st, cs->in_ready[s], 0)) != cudaSuccess ||
+        (i >= 2 && (e = cudaStreamWaitEvent(st, cs->out_read[s], 0)) != cudaSuccess)) {
+      status = fail_cuda(e, "host pipeline order");
+      break;
+    }
+    status = run_fwd(slot(s, 0), slot(s, 1), slot(s, 2), slot(s, 3), dtype, 1, nh, nh, N, d,
+                     causal, sm_scale, base_mode, smooth, base + stage, cnt, di->status, st);
+    if (status != SAGE_OK) break;
+    if ((e = cudaEventRecord(cs->done[s], st)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(cs->d2h, cs->done[s], 0)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(ho + off, slot(s, 3), bytes, cudaMemcpyDefault, cs->d2h)) !=
+            cudaSuccess ||
+        (e = cudaEventRecord(cs->out_read[s], cs->d2h)) != cudaSuccess) {
+      status = fail_cuda(e, "host pipeline copy out");
+      break;
+    }
+  }
+  // st continues after every copy of this call (also when a step failed)
+  for (cudaStream_t cpy : {cs->h2d, cs->d2h}) {
+    if ((e = cudaEventRecord(cs->start, cpy)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(st, cs->start, 0)) != cudaSuccess)
+      return status != SAGE_OK ? status : fail_cuda(e, "host pipeline join");
+  }
+  return status;
 }
 
 int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtype, int64_t B,

@@ -207,3 +207,14 @@ def test_smoothing_buffers_and_argument_errors(lib):
     s = lib.sage_attn_fwd_noalloc(FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 128, 0,
                                   ctypes.c_float(0.0), q.SMOOTH_Q, None)
     assert s == -1 and "mode" in lib.sage_status_string(s).decode()
+
+
+def test_host_pass_argument_errors(lib):
+    s = lib.sage_attn_fwd_host(FAKE, None, FAKE, FAKE, 1, 1, 1, 128, 128, 0, ctypes.c_float(0.0),
+                               0, None)
+    assert s == -1 and "NULL" in lib.sage_status_string(s).decode()
+    assert lib.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 0, 4, 128, 128, 0,
+                                  ctypes.c_float(0.0), 0, None) == 0
+    s = lib.sage_attn_fwd_host(FAKE, FAKE, FAKE, FAKE, 1, 1, 1, 128, 96, 0, ctypes.c_float(0.0),
+                               0, None)
+    assert s == -2 and "head dim" in lib.sage_status_string(s).decode()
