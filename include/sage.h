@@ -226,7 +226,7 @@ int sage_attn_fwd(const void* q, const void* k, const void* v, void* o, int dtyp
 /* The whole forward pass on HOST buffers: q, k, v and o point to host
  * memory holding [B, H, N, d] in `dtype` (any host memory; page-locked
  * memory lets the copies overlap the compute).  The heads are cut into
- * about 8 chunks (none smaller than 32 MB of inputs); chunk i + 1 is copied
+ * about 16 chunks (none smaller than 32 MB of inputs); chunk i + 1 is copied
  * in and chunk i - 1 copied out on two library-owned copy streams (one pair
  * per device, shared by callers, one call at a time) while chunk i runs the
  * pre-pass and attention of sage_attn_fwd on `stream`.  Heads are

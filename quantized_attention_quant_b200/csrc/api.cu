@@ -493,11 +493,13 @@ int copy_streams(CopyStreams** out) {
   return SAGE_OK;
 }
 
-// Heads per chunk of sage_attn_fwd_host: about 8 chunks, none smaller than
-// 32 MB of inputs (fewer, larger chunks for small problems).
+// Heads per chunk of sage_attn_fwd_host: about 16 chunks, none smaller than
+// 32 MB of inputs (fewer, larger chunks for small problems).  The copy in of
+// the first chunk and the compute and copy out of the last are not
+// overlapped, so more chunks shorten the pass while each still fills the GPU.
 int64_t host_chunk_heads(int64_t BH, int64_t N, int64_t d) {
   const int64_t head_bytes = 3 * N * d * 2;
-  int64_t c = (BH + 7) / 8;
+  int64_t c = (BH + 15) / 16;
   const int64_t min_heads = (int64_t(32) << 20) / (head_bytes > 0 ? head_bytes : 1);
   if (c < min_heads) c = min_heads;
   if (c > BH) c = BH;
