@@ -328,7 +328,17 @@ def summarize(w, world, times, sms, dev_name=None):
                      "kernel": attention_kernel(w, sms),
                      "peak_source": f"{src} bf16 burst x{ratio:g} (nominal dense ratio)",
                      "work": "4 d ops per visible (q,k) pair"},
+        # the secondary bound: one exponential per visible (q,k) pair against the
+        # SFU's 16 per clock per SM (at the maximum SM clock)
+        "exp_rate": exp_rate(w, heads, t_attn, sms),
     }
+
+
+def exp_rate(w, heads, t_attn_ms, sms, sm_mhz=None):
+    mhz = float(sm_mhz or measured_peaks()[0].get("sm_max_mhz") or 1965.0)
+    per_clk = visible_pairs(w) * heads / (t_attn_ms * 1e-3) / (sms * mhz * 1e6)
+    return {"exps_per_clk_per_sm": round(per_clk, 2), "sfu_frac": round(per_clk / 16.0, 4),
+            "sm_mhz": mhz}
 
 
 def run_sage(args):
