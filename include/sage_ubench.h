@@ -48,6 +48,13 @@ int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops);
  * exponentials (values, two per FP16x2 instruction) per SM clock cycle. */
 int sage_ubench_exp(int mode, int threads, int iters, double* per_clk_per_sm);
 
+/* The attention kernels' FMA-pipe exponential (a degree-4 polynomial after
+ * a rint split, on the packed FP32 pipe) evaluated on the device at the n
+ * host values t[i] (t <= 128; arguments below -125 are clamped there), the
+ * results copied to out[i], so that a test can hold it to its stated
+ * relative error (2^-18.5) against an exact exponential. */
+int sage_ubench_exp2_poly(const float* t, float* out, int n);
+
 #ifdef __cplusplus
 }
 #endif

@@ -5,7 +5,9 @@
 //     (is an FP16 accumulator faster than FP32 for FP8 P~V, as the
 //     SageAttention2++ page reports for its GPUs; how much narrower is an
 //     N = 128 tile than N = 256);
-//   - SFU exponential throughput, FP32 against packed FP16x2.
+//   - SFU exponential throughput, FP32 against packed FP16x2;
+//   - the FMA-pipe 2^t of the attention kernels on given arguments (for an
+//     accuracy check against an exact exponential).
 // One CTA per SM; every wait is bounded (a timeout sets a flag the host
 // reads and returns as an error).  No other code of the library uses this.
 
@@ -14,6 +16,7 @@
 #include <cstdint>
 
 #include "../../include/sage_ubench.h"
+#include "exp2_poly.cuh"
 #include "sage_ptx.cuh"
 
 namespace sage {
@@ -137,6 +140,17 @@ __global__ void exp_rate_kernel(int iters, float* sink, long long* cycles) {
   if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
 }
 
+// The attention kernels' FMA-pipe 2^t (exp2_poly.cuh) on given arguments,
+// two per thread through the packed path, so the host can check it against
+// an exact exponential.
+__global__ void exp2_poly_kernel(const float* t, float* out, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float2 v = exp2_poly2(make_float2(t[i], i + 1 < n ? t[i + 1] : 0.f));
+  out[i] = v.x;
+  if (i + 1 < n) out[i + 1] = v.y;
+}
+
 int sms_of_device(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -226,6 +240,26 @@ int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops) {
     default:
       return SAGE_UBENCH_ERR_ARG;
   }
+}
+
+int sage_ubench_exp2_poly(const float* t, float* out, int n) {
+  using namespace sage;
+  if (!t || !out || n <= 0) return SAGE_UBENCH_ERR_ARG;
+  float* dt = nullptr;
+  float* dout = nullptr;
+  int status = SAGE_UBENCH_ERR_CUDA;
+  const size_t bytes = (size_t)n * 4;
+  if (cudaMalloc(&dt, bytes) == cudaSuccess && cudaMalloc(&dout, bytes) == cudaSuccess &&
+      cudaMemcpy(dt, t, bytes, cudaMemcpyHostToDevice) == cudaSuccess) {
+    const int pairs = (n + 1) / 2;
+    exp2_poly_kernel<<<(pairs + 255) / 256, 256>>>(dt, dout, n);
+    if (cudaGetLastError() == cudaSuccess &&
+        cudaMemcpy(out, dout, bytes, cudaMemcpyDeviceToHost) == cudaSuccess)
+      status = SAGE_UBENCH_OK;
+  }
+  cudaFree(dt);
+  cudaFree(dout);
+  return status;
 }
 
 int sage_ubench_exp(int mode, int threads, int iters, double* per_clk_per_sm) {
