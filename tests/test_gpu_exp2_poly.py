@@ -23,9 +23,10 @@ def test_exp2_poly_relative_error(cuda_device):
         rng.uniform(-125.0, 9.0, 1 << 20),                    # the range of t - m + log2 448
         np.arange(-125, 10, dtype=np.float64),                # integers
         np.arange(-125, 10, dtype=np.float64) + 0.5,          # split points of rint
-        np.arange(-125, 10, dtype=np.float64) - 0.5,
+        np.arange(-124, 10, dtype=np.float64) - 0.5,
         np.nextafter(np.arange(-124, 10, dtype=np.float32) + np.float32(0.5), np.float32(-1e9)),
     ]).astype(np.float32)
+    assert t.min() >= -125.0                                  # below, the clamp (checked last)
     out = np.empty_like(t)
     assert ub.sage_ubench_exp2_poly(t.ctypes.data, out.ctypes.data, t.size) == 0
     exact = np.exp2(t.astype(np.float64))
