@@ -51,6 +51,11 @@
 // Dequantization: the Q scale is the row's (one per token), the K scale the
 // 32-key chunk's (one per 32 keys), so every thread applies one factor per
 // chunk of 32 scores it holds.
+// Q smoothing (SMOOTH; SageAttention2 abstract, "smooth Q"): every score
+// gains its key's bias qbar . k' of the query block, so the row maximum is
+// no longer a scaled integer maximum; the exp warpgroups then take it on the
+// biased FP32 scores themselves and exchange the halves, and the stats
+// warpgroup only stages the biases and folds (exp_loop_smooth).
 // Every barrier wait is bounded; an expired wait sets the device status
 // word and makes every role leave its loop.
 
@@ -103,9 +108,13 @@ struct Layout {
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
   static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots][4] s_K sm_scale log2 e per 32 keys
   static constexpr int OFF_VS = OFF_C + 128;         // s_V[D] of the head (bulk-copied with Q)
-  // Q smoothing: the score bias of key tile j (log2 units) in slot j % 4
+  // Q smoothing: the score bias of key tile j (log2 units) in slot j % 4;
+  // the two exp warpgroups' partial maxima of tile j in slot j % 2; alpha_j
+  // for the fold in slot j % 4
   static constexpr int OFF_BIAS = OFF_VS + 4 * D;
-  static constexpr int END = OFF_BIAS + 4 * 128 * 4;
+  static constexpr int OFF_PM = OFF_BIAS + 4 * 128 * 4;
+  static constexpr int OFF_A4 = OFF_PM + 2 * 2 * 128 * 4;
+  static constexpr int END = OFF_A4 + 4 * 128 * 4;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t QK_SBO = 8 * D;  // 8 rows of D bytes
@@ -132,7 +141,9 @@ struct Bars {
   uint64_t* pv_empty;  // [PVB] stats -> MMA: PV[b] read
   uint64_t* l_ready;   // [1] exp -> stats: final row sums
   uint64_t* drain;     // MMA drain on abort
-  uint64_t* bias_full; // [2] stats -> stats: a tile's bias is in shared memory (Q smoothing)
+  uint64_t* bias_full; // [2] stats -> stats, exp: a tile's bias is in shared memory (Q smoothing)
+  uint64_t* pm_full;   // [2] exp <-> exp: both partial maxima of a tile written (Q smoothing)
+  uint64_t* a_full;    // [4] exp -> stats: alpha of a tile written (Q smoothing)
 };
 
 template <int D>
@@ -156,13 +167,15 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.l_ready = r.pv_empty + L::PVB;
   r.drain = r.l_ready + 1;
   r.bias_full = r.drain + 1;
+  r.pm_full = r.bias_full + 2;
+  r.a_full = r.pm_full + 2;
   return r;
 }
 
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
 // RAGGED (non-causal launches of a sequence whose last tile is partial): the
 // last key tile masks keys n_tail .. 127.
-template <int D, bool CAUSAL, bool QF8, bool RAGGED, bool SMOOTH>
+template <int D, bool CAUSAL, bool QF8, bool RAGGED>
 __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
                                          const int bh, const int ntiles,
                                          const float* __restrict__ q_scales, const uint32_t tmem,
@@ -224,13 +237,11 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
                                                      kDevTimeoutMma)))
       return;
-    // Q smoothing: this tile's key biases (m_full(j) orders them too)
-    const float* bias = reinterpret_cast<const float*>(smem + L::OFF_BIAS) + (j & 3) * 128 + 64 * h;
-    float sum = masked ? exp_chunk<true, QF8, SMOOTH>(sa, 2 * h, ca, neg, lim, P, bias)
-                       : exp_chunk<false, QF8, SMOOTH>(sa, 2 * h, ca, neg, lim, P, bias);
+    float sum = masked ? exp_chunk<true, QF8>(sa, 2 * h, ca, neg, lim, P)
+                       : exp_chunk<false, QF8>(sa, 2 * h, ca, neg, lim, P);
     if (r == 0 && h == 0) SAGE_TR(14, j);
-    sum += masked ? exp_chunk<true, QF8, SMOOTH>(sb, 2 * h + 1, cb, neg, lim, P + 8, bias + 32)
-                  : exp_chunk<false, QF8, SMOOTH>(sb, 2 * h + 1, cb, neg, lim, P + 8, bias + 32);
+    sum += masked ? exp_chunk<true, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8)
+                  : exp_chunk<false, QF8>(sb, 2 * h + 1, cb, neg, lim, P + 8);
     l = fmaf(alpha, l, sum);
     if (r == 0 && h == 0) SAGE_TR(10, j);
     tmem_wait_st();
@@ -238,6 +249,149 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     if (r == 0) SAGE_TR(2 + h, j);
     mbar_arrive(&bar.p_full[b]);
     if (r == 0 && h == 0) SAGE_TR(11, j);
+  }
+  l_s[h * 128 + r] = l;
+  mbar_arrive(bar.l_ready);
+}
+
+// Q smoothing: the exp warpgroups take the row maximum themselves.  Each
+// turns its 64 scores of tile j into biased log2-domain scores
+// t = A c + bias (in place), takes their maximum, and exchanges it with the
+// other warpgroup through shared memory (pm_full); both then form the same
+// m_j = max(m_{j-1}, both halves) and alpha_j, warpgroup 0 publishes alpha_j
+// for the fold (a_full), and the exponentials take 2^(t - m_j + log2 448).
+// The stats warpgroup only stages the bias and folds, so the exact biased
+// maximum (about 2.5 instructions a score) no longer sits on one warp per
+// SM sub-partition.  Slots: the partial maxima of tile j in j % 2 (a
+// warpgroup writes tile j + 2's only after passing tile j + 1's exchange,
+// which the other enters only after reading tile j's); alpha in j % 4
+// (written for tile j + 4 only after the bias of tile j + 4 is staged, which
+// the stats warpgroup does only after reading alpha_j).
+template <bool MASKED, bool QF8>
+__device__ __forceinline__ float biased32(uint32_t (&s)[32], float c, const float* bias, int col0,
+                                          int lim) {
+  const float2 c2 = make_float2(c, c);
+  const float2 mb = make_float2(-kBias, -kBias);
+  float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    const float4 bv = *reinterpret_cast<const float4*>(bias + i);
+    float2 x01 = make_float2(score<QF8>(s[i]), score<QF8>(s[i + 1]));
+    float2 x23 = make_float2(score<QF8>(s[i + 2]), score<QF8>(s[i + 3]));
+    if (!QF8) {
+      x01 = __fadd2_rn(x01, mb);
+      x23 = __fadd2_rn(x23, mb);
+    }
+    const float2 t01 = __ffma2_rn(x01, c2, make_float2(bv.x, bv.y));
+    const float2 t23 = __ffma2_rn(x23, c2, make_float2(bv.z, bv.w));
+    s[i] = __float_as_uint(t01.x);
+    s[i + 1] = __float_as_uint(t01.y);
+    s[i + 2] = __float_as_uint(t23.x);
+    s[i + 3] = __float_as_uint(t23.y);
+    float v0 = t01.x, v1 = t01.y, v2 = t23.x, v3 = t23.y;
+    if (MASKED) {
+      v0 = (col0 + i + 0 <= lim) ? v0 : -INFINITY;
+      v1 = (col0 + i + 1 <= lim) ? v1 : -INFINITY;
+      v2 = (col0 + i + 2 <= lim) ? v2 : -INFINITY;
+      v3 = (col0 + i + 3 <= lim) ? v3 : -INFINITY;
+    }
+    m0 = fmax3(m0, v0, v1);
+    m1 = fmax3(m1, v2, v3);
+  }
+  return fmaxf(m0, m1);
+}
+
+template <int D, bool CAUSAL, bool QF8, bool RAGGED>
+__device__ __forceinline__ void exp_loop_smooth(const int h, const int qt, const int nkv,
+                                                const int n_tail, const int bh, const int H,
+                                                const int G, const int ntiles,
+                                                const float* __restrict__ q_scales,
+                                                const float* __restrict__ k_scales,
+                                                const float scale_log2, const uint32_t tmem,
+                                                const Bars& bar, uint8_t* smem,
+                                                volatile int* abort_flag, uint32_t* status) {
+  using L = Layout<D>;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+  const float* bias_s = reinterpret_cast<const float*>(smem + L::OFF_BIAS);
+  float* pm_s = reinterpret_cast<float*>(smem + L::OFF_PM);
+  float* a_s = reinterpret_cast<float*>(smem + L::OFF_A4);
+  float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
+  const float qs = __ldg(q_scales + ((int64_t)bh * ntiles + qt) * 128 + r);
+  // this warpgroup's two K scales of every tile (keys 64h .. 64h + 63)
+  const float* ksp = k_scales + (int64_t)kv_head(bh, H, G) * ntiles * 4 + 2 * h;
+
+  tc_fence_before();
+  mbar_arrive(bar.s_init);
+
+  float l = 0.f, m = -INFINITY;
+  float ks0 = ldg_early(ksp), ks1 = ldg_early(ksp + 1);
+  for (int j = 0; j < nkv; ++j) {
+    const int b = j & 1;
+    const uint32_t ph = (j >> 1) & 1;
+    const float ca = qs * (ks0 * scale_log2), cb = qs * (ks1 * scale_log2);
+    float ks0n = 0.f, ks1n = 0.f;
+    if (j + 1 < nkv) {
+      ks0n = ldg_early(ksp + 4 * (j + 1));
+      ks1n = ldg_early(ksp + 4 * (j + 1) + 1);
+    }
+    const int sbuf = j % L::SB;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[sbuf], (j / L::SB) & 1, abort_flag, status,
+                                           kDevTimeoutMma)))
+      return;
+    tc_fence_after();
+    const bool diag = CAUSAL && (j == qt);
+    const bool masked = diag || (RAGGED && j == nkv - 1);
+    const int lim = diag ? r : n_tail - 1;
+    const uint32_t S = tmem + lanes + 128u * sbuf + 64u * h;
+    const uint32_t P = tmem + lanes + L::COL_P + 32u * b + 16u * h;
+    uint32_t sa[32], sb[32];
+    tmem_ld32(S, sa);
+    tmem_ld32(S + 32, sb);
+    tmem_wait_ld_regs(sa);
+    reg_fence(sb);
+    // S read: free for the next Q K^T into it
+    tc_fence_before();
+    mbar_arrive(&bar.s_ready[sbuf]);
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&bar.bias_full[b], ph, abort_flag, status, kDevTimeoutSoftmax)))
+      return;
+    const float* bias = bias_s + (j & 3) * 128 + 64 * h;
+    const float p = masked ? fmaxf(biased32<true, QF8>(sa, ca, bias, 64 * h, lim),
+                                   biased32<true, QF8>(sb, cb, bias + 32, 64 * h + 32, lim))
+                           : fmaxf(biased32<false, QF8>(sa, ca, bias, 64 * h, lim),
+                                   biased32<false, QF8>(sb, cb, bias + 32, 64 * h + 32, lim));
+    pm_s[(2 * b + h) * 128 + r] = p;
+    mbar_arrive(&bar.pm_full[b]);
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&bar.pm_full[b], ph, abort_flag, status, kDevTimeoutSoftmax)))
+      return;
+    const float m_j = fmax3(m, p, pm_s[(2 * b + (h ^ 1)) * 128 + r]);
+    const float alpha = ex2(m - m_j);
+    m = m_j;
+    if (h == 0) {
+      a_s[(j & 3) * 128 + r] = alpha;
+      mbar_arrive(&bar.a_full[j & 3]);
+    }
+    const float neg = kLog2_448 - m_j;  // yields 448 P~ directly
+    // P~[b] is free once the P~V MMA of tile j - 2 has read it
+    if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
+                                                     kDevTimeoutMma)))
+      return;
+    // the biased scores are plain FP32 now: t - m_j + log2 448 by one FMA
+    float sum = masked ? exp_chunk<true, true>(sa, 2 * h, 1.f, neg, lim, P)
+                       : exp_chunk<false, true>(sa, 2 * h, 1.f, neg, lim, P);
+    sum += masked ? exp_chunk<true, true>(sb, 2 * h + 1, 1.f, neg, lim, P + 8)
+                  : exp_chunk<false, true>(sb, 2 * h + 1, 1.f, neg, lim, P + 8);
+    l = fmaf(alpha, l, sum);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&bar.p_full[b]);
+    ks0 = ks0n;
+    ks1 = ks1n;
   }
   l_s[h * 128 + r] = l;
   mbar_arrive(bar.l_ready);
@@ -303,11 +457,10 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float4 ks_cur = ldg4_early(ksp);
   // Q smoothing: this query block's score bias.  Thread r writes key
   // 128 j + r of tile j (log2 units) into slot j % 4 of the shared bias
-  // buffer one tile ahead, after publishing tile j - 1's maximum, and
-  // arrives on bias_full[j % 2]; the whole buffer is then read by every row's
-  // maximum and, after m_full, by the exp warpgroups.  A slot is rewritten
-  // for tile j + 4 only once both exp warpgroups and every stats thread are
-  // past tile j (the s_full wait of tile j + 3 comes first).
+  // buffer one tile ahead, after reading alpha_{j-1}, and arrives on
+  // bias_full[j % 2]; both exp warpgroups read the whole slot.  A slot is
+  // rewritten for tile j + 4 after alpha_{j+3} is published, which both exp
+  // warpgroups do only past their reads of tile j's bias.
   const float* dsr = SMOOTH ? ds + ((int64_t)bh * ntiles + qt) * (int64_t)(ntiles * 128) : nullptr;
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);
   float d_nxt = 0.f;
@@ -316,7 +469,22 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     mbar_arrive(&bar.bias_full[0]);
     if (nkv > 1) d_nxt = ldg_early(dsr + 128 + r);
   }
-  for (int j = 0; j < nkv; ++j) {
+  for (int j = 0; SMOOTH && j < nkv; ++j) {
+    // Q smoothing: the exp warpgroups take the maximum; this warpgroup
+    // stages the next tile's bias and folds with the published alpha_j
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.a_full[j & 3], (j >> 2) & 1, abort_flag, status,
+                                           kDevTimeoutSoftmax)))
+      return;
+    const float alpha = reinterpret_cast<const float*>(smem + L::OFF_A4)[(j & 3) * 128 + r];
+    if (j + 1 < nkv) {
+      bias_s[((j + 1) & 3) * 128 + r] = d_nxt * scale_log2;
+      mbar_arrive(&bar.bias_full[(j + 1) & 1]);
+      if (j + 2 < nkv) d_nxt = ldg_early(dsr + 128 * (j + 2) + r);
+    }
+    if (j >= L::PVB && !fold(j - L::PVB, alpha_hist[j % L::PVB])) return;
+    alpha_hist[j % L::PVB] = alpha;
+  }
+  for (int j = 0; !SMOOTH && j < nkv; ++j) {
     const int b = j & 1;
     // s_K sm_scale log2 e of the tile's four 32-key chunks; a row's factor
     // is its Q scale times that (the exp warpgroups form the same products)
@@ -333,10 +501,6 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     const bool masked = diag || (RAGGED && j == nkv - 1);
     const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes + (uint32_t)sbuf * 128u;
-    const float* bias = bias_s + (j & 3) * 128;
-    if (SMOOTH && !__all_sync(0xffffffffu, mbar_wait(&bar.bias_full[b], (j >> 1) & 1, abort_flag,
-                                                     status, kDevTimeoutSoftmax)))
-      return;
     float mx = -INFINITY;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -345,21 +509,11 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      if (SMOOTH) {
-        // biased scores: the maximum of the sums
-        const float c0 = qs * kl[2 * hh], c1 = qs * kl[2 * hh + 1];
-        mx = masked ? fmax3(mx, max32_biased<true, QF8>(s[0], 64 * hh, lim, c0, bias + 64 * hh),
-                            max32_biased<true, QF8>(s[1], 64 * hh + 32, lim, c1, bias + 64 * hh + 32))
-                    : fmax3(mx, max32_biased<false, QF8>(s[0], 64 * hh, lim, c0, bias + 64 * hh),
-                            max32_biased<false, QF8>(s[1], 64 * hh + 32, lim, c1,
-                                                     bias + 64 * hh + 32));
-      } else {
-        // each chunk's factor is >= 0, so its scaled max is the max scaled
-        mx = masked ? scaled_max64<true, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
-                                              qs * kl[2 * hh + 1], mx)
-                    : scaled_max64<false, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
-                                               qs * kl[2 * hh + 1], mx);
-      }
+      // each chunk's factor is >= 0, so its scaled max is the max scaled
+      mx = masked ? scaled_max64<true, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                            qs * kl[2 * hh + 1], mx)
+                  : scaled_max64<false, QF8>(&s[0][0], hh, lim, qs * kl[2 * hh],
+                                             qs * kl[2 * hh + 1], mx);
     }
     const float m_j = fmaxf(m, mx);
     const float alpha = ex2(m - m_j);
@@ -376,12 +530,6 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     // S[b] has been read: the exp warpgroups may overwrite it with P~ codes
     tc_fence_before();
     mbar_arrive(&bar.m_full[b]);
-    if (SMOOTH && j + 1 < nkv) {
-      // the next tile's bias, and the one after it from global memory
-      bias_s[((j + 1) & 3) * 128 + r] = d_nxt * scale_log2;
-      mbar_arrive(&bar.bias_full[b ^ 1]);
-      if (j + 2 < nkv) d_nxt = ldg_early(dsr + 128 * (j + 2) + r);
-    }
     if (j >= L::PVB && !fold(j - L::PVB, alpha_hist[j % L::PVB])) return;
     alpha_hist[j % L::PVB] = alpha;
     ks_cur = ks_nxt;
@@ -473,6 +621,9 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
     mbar_init(bar.drain, 1);
     mbar_init(&bar.bias_full[0], 128);
     mbar_init(&bar.bias_full[1], 128);
+    mbar_init(&bar.pm_full[0], 256);
+    mbar_init(&bar.pm_full[1], 256);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar.a_full[i], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -607,10 +758,14 @@ __global__ void __launch_bounds__(kThreadsAttn, 1)
       }
       __syncwarp();
     }
+  } else if (wg < 3 && SMOOTH) {
+    exp_loop_smooth<D, CAUSAL, QF8, RAGGED>(wg - 1, qt, nkv, n_tail, bh, H, G, ntiles, q_scales,
+                                            k_scales, scale_log2, tmem, bar, smem, abort_flag,
+                                            status);
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<D, CAUSAL, QF8, RAGGED, SMOOTH>(wg - 1, qt, nkv, n_tail, bh, ntiles, q_scales, tmem, bar,
-                                     smem, abort_flag, status);
+    exp_loop<D, CAUSAL, QF8, RAGGED>(wg - 1, qt, nkv, n_tail, bh, ntiles, q_scales, tmem, bar, smem,
+                                     abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
     stats_loop<D, CAUSAL, OutT, QF8, RAGGED, SMOOTH>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar,

@@ -136,38 +136,6 @@ __device__ __forceinline__ float scaled_max64(const uint32_t* s, int hh, int lim
   return fmax3(acc, v0, v1);
 }
 
-// Q smoothing: the maximum of 32 scores of a row that each gain a per-key
-// bias (log2 units, bias[i] for key col0 + i), dequantized with factor c;
-// masking as above.
-template <bool MASKED, bool QF8>
-__device__ __forceinline__ float max32_biased(const uint32_t* s, int col0, int lim, float c,
-                                              const float* bias) {
-  const float2 c2 = make_float2(c, c);
-  const float2 mb = make_float2(-kBias, -kBias);
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    const float4 bv = *reinterpret_cast<const float4*>(bias + i);
-    float2 x01 = make_float2(score<QF8>(s[i]), score<QF8>(s[i + 1]));
-    float2 x23 = make_float2(score<QF8>(s[i + 2]), score<QF8>(s[i + 3]));
-    if (!QF8) {
-      x01 = __fadd2_rn(x01, mb);
-      x23 = __fadd2_rn(x23, mb);
-    }
-    const float2 t01 = __ffma2_rn(x01, c2, make_float2(bv.x, bv.y));
-    const float2 t23 = __ffma2_rn(x23, c2, make_float2(bv.z, bv.w));
-    float v0 = t01.x, v1 = t01.y, v2 = t23.x, v3 = t23.y;
-    if (MASKED) {
-      v0 = (col0 + i + 0 <= lim) ? v0 : -INFINITY;
-      v1 = (col0 + i + 1 <= lim) ? v1 : -INFINITY;
-      v2 = (col0 + i + 2 <= lim) ? v2 : -INFINITY;
-      v3 = (col0 + i + 3 <= lim) ? v3 : -INFINITY;
-    }
-    m = fmax3(fmax3(m, v0, v1), v2, v3);
-  }
-  return m;
-}
-
 // Whether group g (0..7) of 4 scores takes the FMA-pipe polynomial: the
 // groups are spread evenly over the 32 scores of a chunk.
 __device__ __forceinline__ constexpr bool poly_group(int g) {
@@ -177,11 +145,9 @@ __device__ __forceinline__ constexpr bool poly_group(int g) {
 // 448 P~ for 32 scores of a row -> 8 words of e4m3 codes (key i in byte
 // i % 4 of word i / 4) and the sum of the unquantized values.  QF8: the
 // scores are plain FP32 (no bias to remove).
-// BIAS (Q smoothing): key col0 + i's score gains bias[i] (log2 units).
-template <bool MASKED, bool QF8, bool BIAS = false>
+template <bool MASKED, bool QF8>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
-                                             int lim, uint32_t (&p)[8],
-                                             const float* bias = nullptr) {
+                                             int lim, uint32_t (&p)[8]) {
   const float2 c2 = make_float2(c, c);
   const float2 n2 = make_float2(neg, neg);
   const float2 mb = make_float2(-kBias, -kBias);
@@ -195,14 +161,8 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
       x01 = __fadd2_rn(x01, mb);
       x23 = __fadd2_rn(x23, mb);
     }
-    float2 n01 = n2, n23 = n2;
-    if (BIAS) {
-      const float4 bv = *reinterpret_cast<const float4*>(bias + i);
-      n01 = __fadd2_rn(make_float2(bv.x, bv.y), n2);
-      n23 = __fadd2_rn(make_float2(bv.z, bv.w), n2);
-    }
-    const float2 t01 = __ffma2_rn(x01, c2, n01);
-    const float2 t23 = __ffma2_rn(x23, c2, n23);
+    const float2 t01 = __ffma2_rn(x01, c2, n2);
+    const float2 t23 = __ffma2_rn(x23, c2, n2);
     float f0, f1, f2, f3;
     if (poly_group(i >> 2)) {
       const float2 e01 = exp2_poly2(t01), e23 = exp2_poly2(t23);
@@ -240,11 +200,11 @@ __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
 // One 32-key chunk cc (0..3) of the exp pass: its e4m3 codes go to the 8
 // TMEM columns pcol (four keys per column, the A-operand layout of the
 // P~V MMA); returns the chunk's row sum.
-template <bool MASKED, bool QF8, bool BIAS = false>
+template <bool MASKED, bool QF8>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int cc, float c, float neg,
-                                           int lim, uint32_t pcol, const float* bias = nullptr) {
+                                           int lim, uint32_t pcol) {
   uint32_t p[8];
-  const float sum = exp_quant32<MASKED, QF8, BIAS>(s, c, neg, 32 * cc, lim, p, bias);
+  const float sum = exp_quant32<MASKED, QF8>(s, c, neg, 32 * cc, lim, p);
   tmem_st8(pcol, p);
   return sum;
 }
