@@ -33,7 +33,10 @@
 //     exp warpgroups release it as soon as they hold their 64 scores, and
 //     the MMA thread issues the next Q K^T ahead of the previous tile's
 //     P~V, so the scores the stats warpgroup needs next never queue behind
-//     a partial that is folded two tiles later.
+//     a partial that is folded two tiles later;
+//   - Q smoothing (SMOOTH): the exp warpgroups take the row maximum of the
+//     biased scores themselves and exchange the halves (exp_loop_smooth), as
+//     in the 8-bit kernel.
 // TMEM columns: S 0..127, PV[0] 128..255, PV[1] 256..383, scale factors
 // SFA_Q 384, SFB_K 392, SFA_P 400, SFB_V 408 (8 columns each: two 64-wide
 // K blocks of 4 columns).  Every barrier wait is bounded; an expired wait
@@ -93,9 +96,13 @@ struct Layout {
   static constexpr int OFF_M = OFF_MISC + 1024;      // [2 slots][m, alpha][128]
   static constexpr int OFF_L = OFF_M + 4 * 128 * 4;  // [2 halves][128] row sums
   static constexpr int OFF_C = OFF_L + 2 * 128 * 4;  // [2 slots] dequant factor of the tile
-  // Q smoothing: the score bias of key tile j (log2 units) in slot j % 4
+  // Q smoothing: the score bias of key tile j (log2 units) in slot j % 4;
+  // the two exp warpgroups' partial maxima of tile j in slot j % 2; alpha_j
+  // for the fold in slot j % 4
   static constexpr int OFF_BIAS = OFF_C + 16;
-  static constexpr int END = OFF_BIAS + 4 * 128 * 4;
+  static constexpr int OFF_PM = OFF_BIAS + 4 * 128 * 4;
+  static constexpr int OFF_A4 = OFF_PM + 2 * 2 * 128 * 4;
+  static constexpr int END = OFF_A4 + 4 * 128 * 4;
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) runs per SM
   static constexpr int SMEM = (END + 1024 > 120 * 1024 ? END + 1024 : 120 * 1024);
   static constexpr uint32_t SBO = 8 * 64;  // 8 rows of 64 bytes (64-byte swizzle atom)
@@ -117,7 +124,9 @@ struct Bars {
   uint64_t* pv_empty;  // [2] stats -> MMA: PV[b] read
   uint64_t* l_ready;   // [1] exp -> stats: final row sums
   uint64_t* drain;     // MMA drain on abort
-  uint64_t* bias_full; // [2] stats -> stats: a tile's bias is in shared memory (Q smoothing)
+  uint64_t* bias_full; // [2] stats -> exp: a tile's bias is in shared memory (Q smoothing)
+  uint64_t* pm_full;   // [2] exp <-> exp: both partial maxima of a tile written (Q smoothing)
+  uint64_t* a_full;    // [4] exp -> stats: alpha of a tile written (Q smoothing)
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
@@ -139,6 +148,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.l_ready = r.pv_empty + 2;
   r.drain = r.l_ready + 1;
   r.bias_full = r.drain + 1;
+  r.pm_full = r.bias_full + 2;
+  r.a_full = r.pm_full + 2;
   return r;
 }
 
@@ -231,13 +242,14 @@ __device__ __forceinline__ float max64(const uint32_t* s, int col0, int lim, flo
   return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], acc));
 }
 
-// Q smoothing: the maximum of 32 scores that each gain a per-key bias (log2
-// units, bias[i] for key col0 + i), dequantized with factor c, and a
-// running value; masking as in max64.
+// Q smoothing: 32 scores of a row turned in place into biased log2-domain
+// scores t = A c + bias[i] (key col0 + i); returns their maximum (masking
+// as in max64).
 template <bool MASKED>
-__device__ __forceinline__ float max32_biased(const uint32_t* s, int col0, int lim, float c,
-                                              const float* bias, float acc) {
+__device__ __forceinline__ float biased32(uint32_t (&s)[32], float c, const float* bias, int col0,
+                                          int lim) {
   const float2 c2 = make_float2(c, c);
+  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
     const float4 bv = *reinterpret_cast<const float4*>(bias + i);
@@ -245,6 +257,10 @@ __device__ __forceinline__ float max32_biased(const uint32_t* s, int col0, int l
                                   c2, make_float2(bv.x, bv.y));
     const float2 t23 = __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])),
                                   c2, make_float2(bv.z, bv.w));
+    s[i] = __float_as_uint(t01.x);
+    s[i + 1] = __float_as_uint(t01.y);
+    s[i + 2] = __float_as_uint(t23.x);
+    s[i + 3] = __float_as_uint(t23.y);
     float v0 = t01.x, v1 = t01.y, v2 = t23.x, v3 = t23.y;
     if (MASKED) {
       v0 = (col0 + i + 0 <= lim) ? v0 : -INFINITY;
@@ -252,36 +268,29 @@ __device__ __forceinline__ float max32_biased(const uint32_t* s, int col0, int l
       v2 = (col0 + i + 2 <= lim) ? v2 : -INFINITY;
       v3 = (col0 + i + 3 <= lim) ? v3 : -INFINITY;
     }
-    acc = fmax3(fmax3(acc, v0, v1), v2, v3);
+    m0 = fmax3(m0, v0, v1);
+    m1 = fmax3(m1, v2, v3);
   }
-  return acc;
+  return fmaxf(m0, m1);
 }
 
 // P~ for 32 scores of a row -> 16 bytes of e2m1 codes (key i in nibble i),
 // the two UE4M3 scales of its 16-key groups (bytes 0 and 1 of *sf2), and
 // the sum of the unquantized values.
 //   s16 = ue4m3(448 amax16); code = e2m1(P~ * 2688 / s16) (0 when s16 = 0).
-// BIAS (Q smoothing): key col0 + i's score gains bias[i] (log2 units).
-template <bool MASKED, bool BIAS = false>
+template <bool MASKED>
 __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, float neg, int col0,
-                                             int lim, uint32_t (&p)[4], uint32_t* sf2,
-                                             const float* bias = nullptr) {
+                                             int lim, uint32_t (&p)[4], uint32_t* sf2) {
   const float2 c2 = make_float2(c, c);
   const float2 n2 = make_float2(neg, neg);
   float x[32];
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
-    float2 n01 = n2, n23 = n2;
-    if (BIAS) {
-      const float4 bv = *reinterpret_cast<const float4*>(bias + i);
-      n01 = __fadd2_rn(make_float2(bv.x, bv.y), n2);
-      n23 = __fadd2_rn(make_float2(bv.z, bv.w), n2);
-    }
     const float2 t01 =
-        __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), c2, n01);
+        __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), c2, n2);
     const float2 t23 =
-        __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), c2, n23);
+        __ffma2_rn(make_float2(__uint_as_float(s[i + 2]), __uint_as_float(s[i + 3])), c2, n2);
     float f0, f1, f2, f3;
     if (((i >> 2) * SAGE_FP4_EXP_POLY_GROUPS) % 8 < SAGE_FP4_EXP_POLY_GROUPS) {
       const float2 e01 = exp2_poly2(t01), e23 = exp2_poly2(t23);
@@ -335,12 +344,11 @@ __device__ __forceinline__ float exp_quant32(const uint32_t (&s)[32], float c, f
 // One 32-key chunk q (0..3) of row r: e2m1 codes into the 64-byte-swizzled
 // P~ tile (16-byte chunk q of row r lands at q ^ ((r >> 1) & 3)); returns
 // the chunk's row sum and its two scale bytes.
-template <bool MASKED, bool BIAS = false>
+template <bool MASKED>
 __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int q, float c, float neg,
-                                           int r, int lim, uint32_t prow, uint32_t* sf2,
-                                           const float* bias = nullptr) {
+                                           int r, int lim, uint32_t prow, uint32_t* sf2) {
   uint32_t p[4];
-  const float sum = exp_quant32<MASKED, BIAS>(s, c, neg, 32 * q, lim, p, sf2, bias);
+  const float sum = exp_quant32<MASKED>(s, c, neg, 32 * q, lim, p, sf2);
   st_shared_v4(prow + (((uint32_t)q ^ (uint32_t)((r >> 1) & 3)) << 4), p[0], p[1], p[2], p[3]);
   return sum;
 }
@@ -348,7 +356,7 @@ __device__ __forceinline__ float exp_chunk(const uint32_t (&s)[32], int q, float
 // Exp warpgroup h (0 or 1): key columns 64h .. 64h+63 of every tile.
 // RAGGED (non-causal launches of a sequence whose last tile is partial): the
 // last key tile masks keys n_tail .. 127.
-template <bool CAUSAL, bool RAGGED, bool SMOOTH>
+template <bool CAUSAL, bool RAGGED>
 __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nkv, const int n_tail,
                                          const uint32_t tmem, const Bars& bar, uint8_t* smem,
                                          volatile int* abort_flag, uint32_t* status) {
@@ -396,12 +404,10 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
       return;
     const uint32_t prow = smem_u32(smem + L::OFF_P + b * L::TILE + r * 64);
     uint32_t sf_lo, sf_hi;
-    // Q smoothing: this tile's key biases (m_full(j) orders them too)
-    const float* bias = reinterpret_cast<const float*>(smem + L::OFF_BIAS) + (j & 3) * 128 + 64 * h;
-    float sum = masked ? exp_chunk<true, SMOOTH>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo, bias)
-                       : exp_chunk<false, SMOOTH>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo, bias);
-    sum += masked ? exp_chunk<true, SMOOTH>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi, bias + 32)
-                  : exp_chunk<false, SMOOTH>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi, bias + 32);
+    float sum = masked ? exp_chunk<true>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo)
+                       : exp_chunk<false>(sa, 2 * h, c, neg, r, lim, prow, &sf_lo);
+    sum += masked ? exp_chunk<true>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi)
+                  : exp_chunk<false>(sb, 2 * h + 1, c, neg, r, lim, prow, &sf_hi);
     // the row's four group scales of this 64-key block, in the tensor-core
     // layout: byte 16 (r % 32) + 4 (r / 32) + s of the block's 512 bytes
     st_shared_u32(smem_u32(smem + L::OFF_SFP + b * L::SF + h * 512 + 16 * (r & 31) + 4 * (r >> 5)),
@@ -409,6 +415,105 @@ __device__ __forceinline__ void exp_loop(const int h, const int qt, const int nk
     l = fmaf(alpha, l, sum);
     fence_proxy_async_smem();  // P~ stores visible to the tensor core
     mbar_arrive(&bar.p_full[b]);
+  }
+  l_s[h * 128 + r] = l;
+  mbar_arrive(bar.l_ready);
+}
+
+// Q smoothing: the exp warpgroups take the row maximum themselves, as in the
+// 8-bit kernel.  Each turns its 64 scores of tile j into biased log2-domain
+// scores t = A c + bias in place, takes their maximum, and exchanges it with
+// the other warpgroup through shared memory (pm_full); both form the same
+// m_j and alpha_j, warpgroup 0 publishes alpha_j for the fold (a_full), and
+// P~ = 2^(t - m_j).  The stats warpgroup only stages the biases and folds.
+// Slots: the partial maxima of tile j in j % 2 (a warpgroup writes tile
+// j + 2's only after passing tile j + 1's exchange, which the other enters
+// only after reading tile j's); alpha in j % 4 (written for tile j + 4 only
+// after the bias of tile j + 4 is staged, which the stats warpgroup does
+// only after reading alpha_j).
+template <bool CAUSAL, bool RAGGED>
+__device__ __forceinline__ void exp_loop_smooth(const int h, const int qt, const int nkv,
+                                                const int n_tail, const int bh, const int H,
+                                                const int G, const int ntiles,
+                                                const float* __restrict__ q_scales,
+                                                const float* __restrict__ k_scales,
+                                                const float scale_log2, const uint32_t tmem,
+                                                const Bars& bar, uint8_t* smem,
+                                                volatile int* abort_flag, uint32_t* status) {
+  using L = Layout;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const uint32_t lanes = (uint32_t)(quarter * 32) << 16;
+  const float* bias_s = reinterpret_cast<const float*>(smem + L::OFF_BIAS);
+  float* pm_s = reinterpret_cast<float*>(smem + L::OFF_PM);
+  float* a_s = reinterpret_cast<float*>(smem + L::OFF_A4);
+  float* l_s = reinterpret_cast<float*>(smem + L::OFF_L);
+  // the tile scales g_Q (this query tile) and g_K (one per key tile)
+  const float qs = __ldg(q_scales + (int64_t)bh * ntiles + qt);
+  const float* ksp = k_scales + (int64_t)kv_head(bh, H, G) * ntiles;
+
+  float l = 0.f, m = -INFINITY;
+  float ks = ldg_early(ksp);
+  for (int j = 0; j < nkv; ++j) {
+    const int b = j & 1;
+    const uint32_t ph = (j >> 1) & 1;
+    const float c = qs * ks * scale_log2;
+    const float ks_nxt = j + 1 < nkv ? ldg_early(ksp + j + 1) : 0.f;
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(bar.s_full, j & 1, abort_flag, status, kDevTimeoutMma)))
+      return;
+    tc_fence_after();
+    const bool diag = CAUSAL && (j == qt);
+    const bool masked = diag || (RAGGED && j == nkv - 1);
+    const int lim = diag ? r : n_tail - 1;
+    const uint32_t S = tmem + lanes + 64u * h;
+    uint32_t sa[32], sb[32];
+    tmem_ld32(S, sa);
+    tmem_ld32(S + 32, sb);
+    tmem_wait_ld_regs(sa);
+    reg_fence(sb);
+    // S is in registers: free for Q K_{j+1}^T
+    tc_fence_before();
+    mbar_arrive(bar.s_ready);
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&bar.bias_full[b], ph, abort_flag, status, kDevTimeoutSoftmax)))
+      return;
+    const float* bias = bias_s + (j & 3) * 128 + 64 * h;
+    const float p = masked ? fmaxf(biased32<true>(sa, c, bias, 64 * h, lim),
+                                   biased32<true>(sb, c, bias + 32, 64 * h + 32, lim))
+                           : fmaxf(biased32<false>(sa, c, bias, 64 * h, lim),
+                                   biased32<false>(sb, c, bias + 32, 64 * h + 32, lim));
+    pm_s[(2 * b + h) * 128 + r] = p;
+    mbar_arrive(&bar.pm_full[b]);
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait(&bar.pm_full[b], ph, abort_flag, status, kDevTimeoutSoftmax)))
+      return;
+    const float m_j = fmax3(m, p, pm_s[(2 * b + (h ^ 1)) * 128 + r]);
+    const float alpha = ex2(m - m_j);
+    m = m_j;
+    if (h == 0) {
+      a_s[(j & 3) * 128 + r] = alpha;
+      mbar_arrive(&bar.a_full[j & 3]);
+    }
+    // P~ tile b is free once the P~V MMA of tile j - 2 has read it
+    if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.p_empty[b], ph ^ 1, abort_flag, status,
+                                                     kDevTimeoutMma)))
+      return;
+    const uint32_t prow = smem_u32(smem + L::OFF_P + b * L::TILE + r * 64);
+    uint32_t sf_lo, sf_hi;
+    // the biased scores are plain FP32 now: t - m_j by one FMA
+    float sum = masked ? exp_chunk<true>(sa, 2 * h, 1.f, -m_j, r, lim, prow, &sf_lo)
+                       : exp_chunk<false>(sa, 2 * h, 1.f, -m_j, r, lim, prow, &sf_lo);
+    sum += masked ? exp_chunk<true>(sb, 2 * h + 1, 1.f, -m_j, r, lim, prow, &sf_hi)
+                  : exp_chunk<false>(sb, 2 * h + 1, 1.f, -m_j, r, lim, prow, &sf_hi);
+    st_shared_u32(smem_u32(smem + L::OFF_SFP + b * L::SF + h * 512 + 16 * (r & 31) + 4 * (r >> 5)),
+                  sf_lo | (sf_hi << 16));
+    l = fmaf(alpha, l, sum);
+    fence_proxy_async_smem();  // P~ stores visible to the tensor core
+    mbar_arrive(&bar.p_full[b]);
+    ks = ks_nxt;
   }
   l_s[h * 128 + r] = l;
   mbar_arrive(bar.l_ready);
@@ -476,9 +581,10 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
   float ks_cur = ldg_early(ksp);
   // Q smoothing: this query block's score bias, exchanged through slot j % 4
   // of a shared buffer one tile ahead (as in the 8-bit kernel): thread r
-  // writes key 128 j + r after publishing tile j - 1's maximum and arrives on
-  // bias_full[j % 2]; a slot is rewritten for tile j + 4 only after the
-  // s_full wait of tile j + 3, when every reader is past tile j.
+  // writes key 128 j + r after reading alpha_{j-1} and arrives on
+  // bias_full[j % 2]; a slot is rewritten for tile j + 4 after alpha_{j+3}
+  // is published, which both exp warpgroups do only past their reads of
+  // tile j's bias.
   const float* dsr = SMOOTH ? ds + ((int64_t)bh * ntiles + qt) * (int64_t)(ntiles * 128) : nullptr;
   float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS);
   float d_nxt = 0.f;
@@ -487,7 +593,23 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     mbar_arrive(&bar.bias_full[0]);
     if (nkv > 1) d_nxt = ldg_early(dsr + 128 + r);
   }
-  for (int j = 0; j < nkv; ++j) {
+  for (int j = 0; SMOOTH && j < nkv; ++j) {
+    // Q smoothing: the exp warpgroups take the maximum; this warpgroup
+    // stages the next tile's bias and folds with the published alpha_j
+    const int b = j & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar.a_full[j & 3], (j >> 2) & 1, abort_flag, status,
+                                           kDevTimeoutSoftmax)))
+      return;
+    const float alpha = reinterpret_cast<const float*>(smem + L::OFF_A4)[(j & 3) * 128 + r];
+    if (j + 1 < nkv) {
+      bias_s[((j + 1) & 3) * 128 + r] = d_nxt * scale_log2;
+      mbar_arrive(&bar.bias_full[(j + 1) & 1]);
+      if (j + 2 < nkv) d_nxt = ldg_early(dsr + 128 * (j + 2) + r);
+    }
+    if (j > 1 && !fold(j - 2, alpha_hist[b])) return;
+    alpha_hist[b] = alpha;
+  }
+  for (int j = 0; !SMOOTH && j < nkv; ++j) {
     const int b = j & 1;
     const float c = qs * ks_cur * scale_log2;
     const float ks_nxt = j + 1 < nkv ? ldg_early(ksp + j + 1) : 0.f;
@@ -499,10 +621,6 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     const bool masked = diag || (RAGGED && j == nkv - 1);
     const int lim = diag ? r : n_tail - 1;
     const uint32_t S = tmem + lanes;
-    if (SMOOTH && !__all_sync(0xffffffffu, mbar_wait(&bar.bias_full[b], (j >> 1) & 1, abort_flag,
-                                                     status, kDevTimeoutSoftmax)))
-      return;
-    const float* bias = bias_s + (j & 3) * 128;
     float mx = -INFINITY;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -511,18 +629,10 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
       tmem_ld32(S + 64 * hh + 32, s[1]);
       tmem_wait_ld_regs(s[0]);
       reg_fence(s[1]);
-      if (SMOOTH) {
-        // biased scores, already scaled: the maximum of the sums
-        mx = masked ? max32_biased<true>(s[1], 64 * hh + 32, lim, c, bias + 64 * hh + 32,
-                                         max32_biased<true>(s[0], 64 * hh, lim, c, bias + 64 * hh, mx))
-                    : max32_biased<false>(s[1], 64 * hh + 32, lim, c, bias + 64 * hh + 32,
-                                          max32_biased<false>(s[0], 64 * hh, lim, c, bias + 64 * hh, mx));
-      } else {
-        mx = masked ? max64<true>(&s[0][0], 64 * hh, lim, mx)
-                    : max64<false>(&s[0][0], 64 * hh, lim, mx);
-      }
+      mx = masked ? max64<true>(&s[0][0], 64 * hh, lim, mx)
+                  : max64<false>(&s[0][0], 64 * hh, lim, mx);
     }
-    const float m_j = fmaxf(m, SMOOTH ? mx : mx * c);
+    const float m_j = fmaxf(m, mx * c);
     const float alpha = ex2(m - m_j);
     m = m_j;
     m_s[(2 * b) * 128 + r] = m_j;
@@ -530,12 +640,6 @@ __device__ __forceinline__ void stats_loop(const int qt, const int nkv, const in
     if (r == 0) c_s[b] = c;
     tc_fence_before();
     mbar_arrive(&bar.m_full[b]);
-    if (SMOOTH && j + 1 < nkv) {
-      // the next tile's bias, and the one after it from global memory
-      bias_s[((j + 1) & 3) * 128 + r] = d_nxt * scale_log2;
-      mbar_arrive(&bar.bias_full[b ^ 1]);
-      if (j + 2 < nkv) d_nxt = ldg_early(dsr + 128 * (j + 2) + r);
-    }
     // the fold runs two tiles behind the max
     if (j > 1 && !fold(j - 2, alpha_hist[b])) return;
     alpha_hist[b] = alpha;
@@ -619,6 +723,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar.drain, 1);
     mbar_init(&bar.bias_full[0], 128);
     mbar_init(&bar.bias_full[1], 128);
+    mbar_init(&bar.pm_full[0], 256);
+    mbar_init(&bar.pm_full[1], 256);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar.a_full[i], 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -759,9 +866,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+  } else if (wg < 3 && SMOOTH) {
+    exp_loop_smooth<CAUSAL, RAGGED>(wg - 1, qt, nkv, n_tail, bh, H, G, ntiles, q_scales, k_scales,
+                                    scale_log2, tmem, bar, smem, abort_flag, status);
   } else if (wg < 3) {
     // the exp warpgroups keep the 128 registers they were launched with
-    exp_loop<CAUSAL, RAGGED, SMOOTH>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
+    exp_loop<CAUSAL, RAGGED>(wg - 1, qt, nkv, n_tail, tmem, bar, smem, abort_flag, status);
   } else {
     setmaxnreg_inc<kRegsStats>();
     stats_loop<CAUSAL, OutT, RAGGED, SMOOTH>(qt, nkv, n_tail, bh, H, G, N, ntiles, tmem, bar, smem,
