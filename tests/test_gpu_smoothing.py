@@ -76,10 +76,15 @@ def test_smoothed_prepass_matches_oracle(cuda_device, mode, N, d):
             assert np.array_equal(g.view(np.uint8), arr.view(np.uint8)), name
 
 
+# N = 77 is one key tile; N >= 1100 (9 to 11 tiles, ragged) cycles the
+# exp warpgroups' shared slots (2 for the partial maxima, 4 for alpha and
+# the biases) more than twice
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("mode,N,d", [("int8_fp8", 512, 128), ("int8_fp8", 300, 64),
                                       ("fp8", 640, 128), ("int8_fp8", 77, 128),
-                                      ("fp4", 512, 128), ("fp4", 300, 128)])
+                                      ("fp4", 512, 128), ("fp4", 300, 128),
+                                      ("int8_fp8", 1200, 128), ("fp8", 1300, 64),
+                                      ("fp4", 1100, 128)])
 def test_smoothed_attention_matches_oracle(cuda_device, mode, N, d, causal):
     B, H = 1, 2
     q, k, v = biased_qkv(B, H, N, d, "bf16", seed=10 + N + d + causal)
