@@ -574,8 +574,8 @@ def run_reference(args):
 
 def run_ubench():
     """The microbenchmarks behind the kernels' design (libsage_ubench.so):
-    tcgen05 MMA throughput per kind, accumulator and tile width, and the
-    SFU exponential rate, FP32 against packed FP16x2."""
+    tcgen05 MMA throughput per kind, accumulator and tile width, the SFU
+    exponential rate, FP32 against packed FP16x2, and the FP64 FMA rate."""
     import ctypes
 
     import torch
@@ -588,7 +588,9 @@ def run_ubench():
                                     ctypes.POINTER(ctypes.c_double)]
     lib.sage_ubench_exp.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.POINTER(ctypes.c_double)]
-    out = {"ubench": "tcgen05 MMA and SFU exponential rates", "mma_tops": {}, "exp_per_clk_per_sm": {}}
+    lib.sage_ubench_dfma.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+    out = {"ubench": "tcgen05 MMA, SFU exponential and FP64 FMA rates", "mma_tops": {},
+           "exp_per_clk_per_sm": {}, "dfma_per_clk_per_sm": {}}
     kinds = {"f8f6f4_e4m3_f32acc": (0, 32), "f8f6f4_e4m3_f16acc": (1, 32), "i8_s32acc": (2, 32),
              "mxf4nvf4_e2m1_ue4m3x16_f32acc": (3, 64)}
     for name, (kind, kdim) in kinds.items():
@@ -603,6 +605,11 @@ def run_ubench():
             st = lib.sage_ubench_exp(mode, threads, 4096, ctypes.byref(v))
             out["exp_per_clk_per_sm"][f"{name}_{threads}thr"] = round(v.value, 2) if st == 0 \
                 else f"status {st}"
+    for threads in (256, 512, 1024):
+        v = ctypes.c_double(0.0)
+        st = lib.sage_ubench_dfma(threads, 4096, ctypes.byref(v))
+        out["dfma_per_clk_per_sm"][f"{threads}thr"] = round(v.value, 2) if st == 0 \
+            else f"status {st}"
     out["device"] = torch.cuda.get_device_name(0)
     print(json.dumps(out), flush=True)
 

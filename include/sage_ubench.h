@@ -48,6 +48,11 @@ int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops);
  * exponentials (values, two per FP16x2 instruction) per SM clock cycle. */
 int sage_ubench_exp(int mode, int threads, int iters, double* per_clk_per_sm);
 
+/* FP64 FMA throughput: one CTA of `threads` threads per SM, each with 8
+ * independent chains of `iters` FMAs; *per_clk_per_sm receives the FP64
+ * FMAs per SM clock cycle.  The denominator of the Q smoothing bias
+ * kernel, which sums q-bar . k' in FP64 (sage.h, sage_quant_qk_smooth). */
+int sage_ubench_dfma(int threads, int iters, double* per_clk_per_sm);
 /* The attention kernels' FMA-pipe exponential (a degree-4 polynomial after
  * a rint split, on the packed FP32 pipe) evaluated on the device at the n
  * host values t[i] (t <= 128; arguments below -125 are clamped there), the

@@ -1034,17 +1034,30 @@ cudaError_t dispatch(const PrepassPtrs& p, int dtype, int64_t d, Roles a, Roles 
 // dS[bh, blk, j] = fp32(sum_c qbar[bh, blk, c] * k'[j, c]), k' = fp32(K) -
 // mean_K of the key/value head, the sum in FP64 in channel order (products
 // of FP32 values are exact in FP64, so FMA and multiply-then-add agree):
-// the oracle's arithmetic, bit for bit.  A CTA takes 64 keys and 32 query
-// blocks of one query head; a thread a 4 x 4 register tile (keys tx + 16 i,
-// blocks ty + 8 i), reading two channels of a key or a block per 16-byte
-// shared load.  Keys past N get 0.
-constexpr int kBiasKeys = 64;
-constexpr int kBiasBlocks = 32;
+// the oracle's arithmetic, bit for bit.  The work is B H N^2 d / 128 FP64
+// FMAs, so the kernel is built to keep the FP64 pipe busy: a CTA takes 256
+// keys and 32 query blocks of one query head, a thread two keys (tx and
+// tx + 128) against all 32 blocks (64 FP64 accumulators).  A thread reads
+// its keys' rows itself, 8 channels per 16-byte load issued one step ahead;
+// the block means sit in shared memory as [channel][block] doubles, and
+// every warp reads the same 16 bytes at once (a broadcast), so shared
+// memory serves one load per four FMAs of a warp.  Keys past N get 0.
 constexpr int kBiasThreads = 128;
+constexpr int kBiasKeys = 2 * kBiasThreads;
+constexpr int kBiasBlocks = 32;
 
 template <int D>
 constexpr int bias_smem_bytes() {
-  return (kBiasKeys + kBiasBlocks) * (D / 2) * 16;
+  return D * kBiasBlocks * 8 + D * 4;
+}
+
+// 8 channels of a K row (one 16-byte load, u) as FP32 values minus the mean
+template <typename T>
+__device__ __forceinline__ void k_smoothed8(const uint4 u, const float* mu, float (&kv)[8]) {
+  T v[8];
+  memcpy(v, &u, 16);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) kv[e] = __fsub_rn(static_cast<float>(v[e]), mu[e]);
 }
 
 template <typename T, int D>
@@ -1052,65 +1065,66 @@ __global__ void __launch_bounds__(kBiasThreads)
     smoothing_bias_kernel(const T* __restrict__ k, const float* __restrict__ k_mean,
                           const float* __restrict__ q_mean, float* __restrict__ ds, int N, int Np,
                           int nblk, int H, int G) {
-  extern __shared__ __align__(16) double2 bias_smem[];
-  double2* ks = bias_smem;                              // [D/2][64]: k' of channels 2cp, 2cp+1
-  double2* qs = bias_smem + (D / 2) * kBiasKeys;        // [D/2][32]: qbar likewise
+  extern __shared__ __align__(16) double bias_smem[];
+  double* qs = bias_smem;                                          // [D][32] qbar
+  float* mu = reinterpret_cast<float*>(bias_smem + D * kBiasBlocks);  // [D] K mean
   const int bh = (int)blockIdx.z;
   const int bhk = kv_head(bh, H, G);
   const int j0 = (int)blockIdx.x * kBiasKeys;
   const int b0 = (int)blockIdx.y * kBiasBlocks;
   const int nb = min(kBiasBlocks, nblk - b0);
   const int t = threadIdx.x;
-  for (int i = t; i < kBiasKeys * (D / 2); i += kBiasThreads) {
-    const int key = i / (D / 2), cp = i % (D / 2);
-    const int j = j0 + key;
-    float k0 = 0.f, k1 = 0.f;
-    if (j < N) {
-      const T* row = k + ((int64_t)bhk * N + j) * D + 2 * cp;
-      const float* mu = k_mean + (int64_t)bhk * D + 2 * cp;
-      k0 = __fsub_rn(static_cast<float>(row[0]), mu[0]);
-      k1 = __fsub_rn(static_cast<float>(row[1]), mu[1]);
-    }
-    ks[cp * kBiasKeys + key] = make_double2((double)k0, (double)k1);
+  // block-fastest order: a warp's 32 stores fill one channel's row of 32
+  // doubles (no bank conflicts)
+  for (int i = t; i < kBiasBlocks * D; i += kBiasThreads) {
+    const int blk = i % kBiasBlocks, c = i / kBiasBlocks;
+    qs[c * kBiasBlocks + blk] =
+        blk < nb ? (double)q_mean[((int64_t)bh * nblk + b0 + blk) * D + c] : 0.0;
   }
-  for (int i = t; i < kBiasBlocks * (D / 2); i += kBiasThreads) {
-    const int blk = i / (D / 2), cp = i % (D / 2);
-    const float* qm = q_mean + ((int64_t)bh * nblk + b0 + blk) * D + 2 * cp;
-    qs[cp * kBiasBlocks + blk] =
-        blk < nb ? make_double2((double)qm[0], (double)qm[1]) : make_double2(0.0, 0.0);
-  }
+  for (int c = t; c < D; c += kBiasThreads) mu[c] = k_mean[(int64_t)bhk * D + c];
   __syncthreads();
-  const int tx = t % 16, ty = t / 16;
-  double acc[4][4];
+  // this thread's keys; rows past N read row N - 1 (their sums are not stored)
+  const int ja = j0 + t, jb = j0 + kBiasThreads + t;
+  const T* ra = k + ((int64_t)bhk * N + min(ja, N - 1)) * D;
+  const T* rb = k + ((int64_t)bhk * N + min(jb, N - 1)) * D;
+  double acc[2][kBiasBlocks];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int i = 0; i < kBiasBlocks; ++i) acc[0][i] = acc[1][i] = 0.0;
+  // the next 8 channels of both rows are loaded while these are summed
+  uint4 ua = __ldg(reinterpret_cast<const uint4*>(ra));
+  uint4 ub = __ldg(reinterpret_cast<const uint4*>(rb));
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 8) {
+    float ka[8], kb[8];
+    k_smoothed8<T>(ua, mu + c0, ka);
+    k_smoothed8<T>(ub, mu + c0, kb);
+    if (c0 + 8 < D) {
+      ua = __ldg(reinterpret_cast<const uint4*>(ra + c0 + 8));
+      ub = __ldg(reinterpret_cast<const uint4*>(rb + c0 + 8));
+    }
+    // channels c0 .. c0 + 7 in order: the channel order of every sum
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
-#pragma unroll 2
-  for (int cp = 0; cp < D / 2; ++cp) {
-    double2 kv[4], qv[4];
+    for (int e = 0; e < 8; ++e) {
+      const double da = (double)ka[e], db = (double)kb[e];
+      const double2* q2 = reinterpret_cast<const double2*>(qs + (c0 + e) * kBiasBlocks);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) kv[i] = ks[cp * kBiasKeys + tx + 16 * i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qv[i] = qs[cp * kBiasBlocks + ty + 8 * i];
-    // channel 2cp, then 2cp + 1: the channel order of every sum
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[b].x, kv[a].x, acc[a][b]);
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[b].y, kv[a].y, acc[a][b]);
+      for (int i = 0; i < kBiasBlocks / 2; ++i) {
+        const double2 q = q2[i];
+        acc[0][2 * i] = __fma_rn(q.x, da, acc[0][2 * i]);
+        acc[0][2 * i + 1] = __fma_rn(q.y, da, acc[0][2 * i + 1]);
+        acc[1][2 * i] = __fma_rn(q.x, db, acc[1][2 * i]);
+        acc[1][2 * i + 1] = __fma_rn(q.y, db, acc[1][2 * i + 1]);
+      }
+    }
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int j = j0 + tx + 16 * a;
+  for (int kk = 0; kk < 2; ++kk) {
+    const int j = kk ? jb : ja;
+    if (j >= Np) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int blk = b0 + ty + 8 * b;
-      if (blk < nblk) ds[((int64_t)bh * nblk + blk) * Np + j] = j < N ? __double2float_rn(acc[a][b]) : 0.f;
-    }
+    for (int i = 0; i < kBiasBlocks; ++i)
+      if (i < nb)
+        ds[((int64_t)bh * nblk + b0 + i) * Np + j] = j < N ? __double2float_rn(acc[kk][i]) : 0.f;
   }
 }
 
@@ -1122,8 +1136,8 @@ cudaError_t run_bias(const QuantQKArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int Np = (int)((a.N + 127) / 128 * 128);
   const int nblk = Np / 128;
-  const dim3 grid((unsigned)(Np / kBiasKeys), (unsigned)((nblk + kBiasBlocks - 1) / kBiasBlocks),
-                  (unsigned)(a.B * a.H));
+  const dim3 grid((unsigned)((Np + kBiasKeys - 1) / kBiasKeys),
+                  (unsigned)((nblk + kBiasBlocks - 1) / kBiasBlocks), (unsigned)(a.B * a.H));
   kern<<<grid, kBiasThreads, bias_smem_bytes<D>(), st>>>(
       static_cast<const T*>(a.k), a.k_mean, a.q_mean, a.ds, (int)a.N, Np, nblk, (int)a.H,
       (int)(a.H / a.Hkv));

@@ -140,6 +140,25 @@ __global__ void exp_rate_kernel(int iters, float* sink, long long* cycles) {
   if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
 }
 
+// FP64 FMA throughput: 8 independent chains per thread (the Q smoothing
+// bias kernel's arithmetic); cycles as in exp_rate_kernel.
+__global__ void dfma_rate_kernel(int iters, double* sink, long long* cycles) {
+  const long long t0 = clock64();
+  double y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = 1e-3 * (double)(threadIdx.x + i);
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fma_rn(y[i], 1.0000001, 1e-9);
+  }
+  double acc = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc += y[i];
+  const long long t1 = clock64();
+  sink[blockIdx.x * blockDim.x + threadIdx.x] = acc;
+  if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
+}
+
 // The attention kernels' FMA-pipe 2^t (exp2_poly.cuh) on given arguments,
 // two per thread through the packed path, so the host can check it against
 // an exact exponential.
@@ -216,10 +235,42 @@ int run_exp(int threads, int iters, double* per_clk) {
   return status;
 }
 
+int run_dfma(int threads, int iters, double* per_clk) {
+  int sms = 0;
+  if (sms_of_device(&sms) != 0) return SAGE_UBENCH_ERR_CUDA;
+  double* sink = nullptr;
+  long long* cyc = nullptr;
+  int status = SAGE_UBENCH_ERR_CUDA;
+  if (cudaMalloc(&sink, (size_t)sms * threads * 8) == cudaSuccess &&
+      cudaMalloc(&cyc, (size_t)sms * 8) == cudaSuccess) {
+    dfma_rate_kernel<<<sms, threads>>>(iters, sink, cyc);  // warm-up
+    dfma_rate_kernel<<<sms, threads>>>(iters, sink, cyc);
+    long long* h = new long long[sms];
+    if (cudaMemcpy(h, cyc, (size_t)sms * 8, cudaMemcpyDeviceToHost) == cudaSuccess) {
+      double c = 0;
+      for (int i = 0; i < sms; ++i) c += (double)h[i];
+      c /= sms;
+      *per_clk = (double)threads * 8 * iters / c;
+      status = SAGE_UBENCH_OK;
+    }
+    delete[] h;
+  }
+  cudaFree(sink);
+  cudaFree(cyc);
+  return status;
+}
+
 }  // namespace
 }  // namespace sage
 
 extern "C" {
+
+int sage_ubench_dfma(int threads, int iters, double* per_clk_per_sm) {
+  using namespace sage;
+  if (!per_clk_per_sm || iters <= 0 || threads <= 0 || threads > 1024 || threads % 32)
+    return SAGE_UBENCH_ERR_ARG;
+  return run_dfma(threads, iters, per_clk_per_sm);
+}
 
 int sage_ubench_mma(int kind, int n, int iters, int reps, double* tops) {
   using namespace sage;

@@ -45,7 +45,8 @@ def test_ubench_library_exports_its_header():
     text = open(os.path.join(ROOT, "include", "sage_ubench.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
-    assert names == ["sage_ubench_exp", "sage_ubench_exp2_poly", "sage_ubench_mma"]
+    assert names == ["sage_ubench_dfma", "sage_ubench_exp", "sage_ubench_exp2_poly",
+                     "sage_ubench_mma"]
     ub = ctypes.CDLL(qb.UBENCH_LIB)
     for n in names:
         assert hasattr(ub, n), n
@@ -57,6 +58,9 @@ def test_ubench_library_exports_its_header():
     assert ub.sage_ubench_mma(3, 64, 10, 1, ctypes.byref(v)) == -1      # FP4 kind: N 128 or 256 too
     assert ub.sage_ubench_exp(0, 100, 10, ctypes.byref(v)) == -1        # not whole warps
     assert ub.sage_ubench_exp(5, 128, 10, ctypes.byref(v)) == -1        # unknown mode
+    ub.sage_ubench_dfma.argtypes = [ctypes.c_int] * 2 + [ctypes.POINTER(ctypes.c_double)]
+    assert ub.sage_ubench_dfma(100, 10, ctypes.byref(v)) == -1          # not whole warps
+    assert ub.sage_ubench_dfma(128, 0, ctypes.byref(v)) == -1           # no rounds
     ub.sage_ubench_exp2_poly.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     assert ub.sage_ubench_exp2_poly(None, None, 4) == -1               # null buffers
 
