@@ -110,11 +110,6 @@ __device__ __forceinline__ void load8(const T* p, float (&f)[8]) {
   }
 }
 
-template <typename T>
-__device__ __forceinline__ float load1(const T* p) {
-  return static_cast<float>(*p);
-}
-
 // Division-free quotient for code decisions.  With rs = fp32(1/s) (correctly
 // rounded), q = fp32(x * rs) lies within 3 * 2^-24 |x/s| of fp32(x / s), so
 // the interval [q (1 - 2^-20), q (1 + 2^-20)] (each end rounded to fp32)

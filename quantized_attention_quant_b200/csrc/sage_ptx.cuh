@@ -152,10 +152,6 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// Barrier among `count` threads (a multiple of 32) on hardware barrier `id`.
-__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 // Plain (untiled) bulk copy global -> shared, completing on `bar` as
 // transaction bytes.  Both addresses 16-byte aligned, bytes a multiple of 16.
@@ -295,9 +291,6 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 // tcgen05.wait::ld that also names the destination registers of the loads
 // it waits for as read-write operands, so the compiler cannot move a use of
 // them above the wait.
