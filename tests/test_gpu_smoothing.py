@@ -110,15 +110,17 @@ def test_smoothed_one_call_equals_split_calls(cuda_device, mode):
     assert torch.equal(one, two)
 
 
-def test_smoothed_gqa_equals_repeated_heads(cuda_device):
+@pytest.mark.parametrize("mode", ["int8_fp8", "fp8", "fp4"])
+def test_smoothed_gqa_equals_repeated_heads(cuda_device, mode):
     # grouped-query attention with Q smoothing: the bias pairs each query
-    # head's block means with its key/value head's smoothed keys
+    # head's block means with its key/value head's smoothed keys, and the
+    # exp warpgroups read the K scales of the key/value head
     B, H, Hkv, N, d = 1, 4, 2, 384, 128
     q, k, v = (t.cuda() for t in biased_qkv(B, H, N, d, "bf16", seed=43, Hkv=Hkv))
-    o = sage.sage_attn_fwd_gqa(q, k, v, mode="int8_fp8", smooth_q=True)
+    o = sage.sage_attn_fwd_gqa(q, k, v, mode=mode, smooth_q=True)
     rep = H // Hkv
     o2 = sage.sage_attn_fwd(q, k.repeat_interleave(rep, 1).contiguous(),
-                            v.repeat_interleave(rep, 1).contiguous(), mode="int8_fp8",
+                            v.repeat_interleave(rep, 1).contiguous(), mode=mode,
                             smooth_q=True)
     torch.cuda.synchronize()
     assert torch.equal(o, o2)
